@@ -1,0 +1,336 @@
+"""Python binding of the plain C oracle (``fp4q_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by the package smoke check in
+``__graft_entry__.smoke()`` and by the CPU-baseline leg of ``bench.py``.  The
+CUDA library and its Python binding never import this package; the two share no
+code.  Arrays are numpy; bf16 tensors travel as ``uint16`` bit patterns.
+
+Each helper below composes the scalar C steps in the order the pages give them;
+the C file's header states the numeric rules and where they come from.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_LIB = None
+
+
+def lib() -> C.CDLL:
+    global _LIB
+    if _LIB is None:
+        path = _build.build()
+        L = C.CDLL(path)
+        i64, f32, f64 = C.c_int64, C.c_float, C.c_double
+        p = C.c_void_p
+        sig = {
+            "orc_bf16_to_f32": (f32, [C.c_uint16]),
+            "orc_f32_to_bf16": (C.c_uint16, [f32]),
+            "orc_bf16_array_to_f32": (None, [p, i64, p]),
+            "orc_f32_array_to_bf16": (None, [p, i64, p]),
+            "orc_e2m1_decode": (f32, [C.c_uint8]),
+            "orc_e2m1_encode": (C.c_uint8, [f32]),
+            "orc_e4m3_decode": (f32, [C.c_uint8]),
+            "orc_e4m3_encode": (C.c_uint8, [f32]),
+            "orc_floor_log2": (C.c_int, [f32]),
+            "orc_e8m0_encode": (C.c_uint8, [f32]),
+            "orc_e8m0_decode": (f32, [C.c_uint8]),
+            "orc_swizzle_offset": (i64, [i64, i64, i64]),
+            "orc_swizzle_scales": (None, [p, i64, i64, p]),
+            "orc_amax": (f32, [p, i64, i64, i64]),
+            "orc_tensor_scale": (f32, [f32]),
+            "orc_nvfp4_quantize": (None, [p, i64, i64, i64, f32, p, p]),
+            "orc_mxfp4_quantize": (None, [p, i64, i64, i64, p, p]),
+            "orc_dual_quantize": (None, [p, i64, i64, i64, p, p, p]),
+            "orc_nvfp4_dequantize": (None, [p, p, f32, i64, i64, p]),
+            "orc_dual_dequantize": (None, [p, p, p, i64, i64, p]),
+            "orc_mxfp4_dequantize": (None, [p, p, i64, i64, p]),
+            "orc_hadamard_entry": (C.c_int, [C.c_int, C.c_int]),
+            "orc_hadamard": (None, [p, i64, i64, i64, C.c_int, p]),
+            "orc_rmsnorm_permute": (None, [p, i64, i64, i64, p, p, f64, p]),
+            "orc_arc_quantize": (None, [p, i64, i64, i64, p, f32, p, p]),
+            "orc_e2m1_encode_array": (None, [p, i64, p]),
+            "orc_e4m3_encode_array": (None, [p, i64, p]),
+            "orc_e4m3_decode_array": (None, [p, i64, p]),
+            "orc_e8m0_encode_array": (None, [p, i64, p]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = L
+    return _LIB
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data
+
+
+def _f32(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+# --------------------------------------------------------------------------- formats
+
+def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    out = np.empty(bits.shape, np.float32)
+    lib().orc_bf16_array_to_f32(_ptr(bits), bits.size, _ptr(out))
+    return out
+
+
+def f32_to_bf16(x: np.ndarray) -> np.ndarray:
+    x = _f32(x)
+    out = np.empty(x.shape, np.uint16)
+    lib().orc_f32_array_to_bf16(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def e2m1_encode(v) -> np.ndarray:
+    v = _f32(v)
+    out = np.empty(v.shape, np.uint8)
+    lib().orc_e2m1_encode_array(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    codes = np.asarray(codes, dtype=np.uint8)
+    table = np.array([lib().orc_e2m1_decode(c) for c in range(16)], np.float32)
+    return table[codes & 15]
+
+
+def e4m3_encode(v) -> np.ndarray:
+    v = _f32(v)
+    out = np.empty(v.shape, np.uint8)
+    lib().orc_e4m3_encode_array(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def e4m3_decode(b) -> np.ndarray:
+    b = np.ascontiguousarray(b, dtype=np.uint8)
+    out = np.empty(b.shape, np.float32)
+    lib().orc_e4m3_decode_array(_ptr(b), b.size, _ptr(out))
+    return out
+
+
+def e8m0_encode(amax) -> np.ndarray:
+    v = _f32(amax)
+    out = np.empty(v.shape, np.uint8)
+    lib().orc_e8m0_encode_array(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def e8m0_decode(b) -> np.ndarray:
+    b = np.asarray(b, dtype=np.uint8)
+    return np.array([lib().orc_e8m0_decode(int(x)) for x in b.reshape(-1)],
+                    np.float32).reshape(b.shape)
+
+
+def floor_log2(a: float) -> int:
+    return int(lib().orc_floor_log2(float(a)))
+
+
+def unpack_codes(codes: np.ndarray) -> np.ndarray:
+    """[M, K/2] packed bytes -> [M, K] 4-bit codes (low nibble = even index)."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    out = np.empty(codes.shape[:-1] + (codes.shape[-1] * 2,), np.uint8)
+    out[..., 0::2] = codes & 15
+    out[..., 1::2] = codes >> 4
+    return out
+
+
+# --------------------------------------------------------------------------- layouts
+
+def swizzle_offset(r: int, c: int, n_cols: int) -> int:
+    return int(lib().orc_swizzle_offset(r, c, (n_cols + 3) // 4))
+
+
+def swizzled_size(M: int, n_cols: int) -> int:
+    return ((M + 127) // 128 * 128) * ((n_cols + 3) // 4 * 4)
+
+
+def swizzle_scales(lin: np.ndarray) -> np.ndarray:
+    lin = np.ascontiguousarray(lin, dtype=np.uint8)
+    M, n = lin.shape
+    out = np.empty(swizzled_size(M, n), np.uint8)
+    lib().orc_swizzle_scales(_ptr(lin), M, n, _ptr(out))
+    return out
+
+
+# --------------------------------------------------------------------------- steps
+
+def amax(y: np.ndarray) -> float:
+    y = _f32(y)
+    M, K = y.shape
+    return float(lib().orc_amax(_ptr(y), M, K, K))
+
+
+def tensor_scale(a: float) -> float:
+    return float(lib().orc_tensor_scale(float(a)))
+
+
+def nvfp4_quantize(y: np.ndarray, s_t: float):
+    y = _f32(y)
+    M, K = y.shape
+    assert K % 16 == 0
+    codes = np.empty((M, K // 2), np.uint8)
+    scales = np.empty((M, K // 16), np.uint8)
+    lib().orc_nvfp4_quantize(_ptr(y), M, K, K, float(s_t), _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def mxfp4_quantize(y: np.ndarray):
+    y = _f32(y)
+    M, K = y.shape
+    assert K % 32 == 0
+    codes = np.empty((M, K // 2), np.uint8)
+    scales = np.empty((M, K // 32), np.uint8)
+    lib().orc_mxfp4_quantize(_ptr(y), M, K, K, _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def dual_quantize(y: np.ndarray):
+    y = _f32(y)
+    M, K = y.shape
+    assert K % 128 == 0
+    codes = np.empty((M, K // 2), np.uint8)
+    scales = np.empty((M, K // 16), np.uint8)
+    g = np.empty((M, K // 128), np.float32)
+    lib().orc_dual_quantize(_ptr(y), M, K, K, _ptr(codes), _ptr(scales), _ptr(g))
+    return codes, scales, g
+
+
+def nvfp4_dequantize(codes, scales, s_t: float) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    M, K = codes.shape[0], codes.shape[1] * 2
+    out = np.empty((M, K), np.float32)
+    lib().orc_nvfp4_dequantize(_ptr(codes), _ptr(scales), float(s_t), M, K, _ptr(out))
+    return out
+
+
+def dual_dequantize(codes, scales, gscales) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    g = _f32(gscales)
+    M, K = codes.shape[0], codes.shape[1] * 2
+    out = np.empty((M, K), np.float32)
+    lib().orc_dual_dequantize(_ptr(codes), _ptr(scales), _ptr(g), M, K, _ptr(out))
+    return out
+
+
+def mxfp4_dequantize(codes, scales) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    M, K = codes.shape[0], codes.shape[1] * 2
+    out = np.empty((M, K), np.float32)
+    lib().orc_mxfp4_dequantize(_ptr(codes), _ptr(scales), M, K, _ptr(out))
+    return out
+
+
+def hadamard_entry(i: int, j: int) -> int:
+    return int(lib().orc_hadamard_entry(i, j))
+
+
+def hadamard(x: np.ndarray, n: int) -> np.ndarray:
+    x = _f32(x)
+    M, K = x.shape
+    assert K % n == 0
+    y = np.empty((M, K), np.float32)
+    lib().orc_hadamard(_ptr(x), M, K, K, int(n), _ptr(y))
+    return y
+
+
+def rmsnorm_permute(x: np.ndarray, gamma: np.ndarray, perm, eps: float) -> np.ndarray:
+    x = _f32(x)
+    g = _f32(gamma)
+    M, K = x.shape
+    y = np.empty((M, K), np.float32)
+    pp = None if perm is None else np.ascontiguousarray(perm, np.int32)
+    lib().orc_rmsnorm_permute(_ptr(x), M, K, K, _ptr(g), None if pp is None else _ptr(pp),
+                              float(eps), _ptr(y))
+    return y
+
+
+def arc_quantize(y: np.ndarray, outliers, s_t: float):
+    y = _f32(y)
+    M, K = y.shape
+    o = np.ascontiguousarray(outliers, np.int32)
+    S = o.size
+    assert K % 16 == 0 and S % 16 == 0
+    codes = np.empty((M, (K + S) // 2), np.uint8)
+    scales = np.empty((M, (K + S) // 16), np.uint8)
+    lib().orc_arc_quantize(_ptr(y), M, K, S, _ptr(o) if S else None, float(s_t), _ptr(codes),
+                           _ptr(scales))
+    return codes, scales
+
+
+# --------------------------------------------------------------------------- workloads
+
+def quantize_nvfp4(x_bits: np.ndarray, s_t: float | None = None):
+    """NVFP4 of a bf16 matrix.  ``s_t=None``: dynamic, s_t = amax/2688 of x."""
+    y = bf16_to_f32(x_bits)
+    if s_t is None:
+        s_t = tensor_scale(amax(y))
+    codes, scales = nvfp4_quantize(y, s_t)
+    return codes, scales, np.float32(s_t)
+
+
+def quantize_mxfp4(x_bits: np.ndarray):
+    return mxfp4_quantize(bf16_to_f32(x_bits))
+
+
+def hadamard_quantize(x_bits: np.ndarray, n: int, fmt: str = "nvfp4", s_t: float | None = None):
+    """Block-Hadamard (size n, normalised) then NVFP4 / MXFP4 / dual quantization.
+
+    Returns (codes, scales, s_t_or_gscales, y) with y the rotated fp32 matrix."""
+    y = hadamard(bf16_to_f32(x_bits), n)
+    if fmt == "nvfp4":
+        if s_t is None:
+            s_t = tensor_scale(amax(y))
+        c, s = nvfp4_quantize(y, s_t)
+        return c, s, np.float32(s_t), y
+    if fmt == "mxfp4":
+        c, s = mxfp4_quantize(y)
+        return c, s, None, y
+    if fmt == "dual":
+        c, s, g = dual_quantize(y)
+        return c, s, g, y
+    raise ValueError(fmt)
+
+
+def arc_prepare(x_bits, gamma_bits, perm, eps: float = 1e-6) -> np.ndarray:
+    """Reordered + RMS-normalised fp32 matrix y[M, K] of the ARCQuant path."""
+    return rmsnorm_permute(bf16_to_f32(x_bits), bf16_to_f32(gamma_bits), perm, eps)
+
+
+def arc(x_bits, gamma_bits, perm, outliers, eps: float = 1e-6, s_t: float | None = None):
+    y = arc_prepare(x_bits, gamma_bits, perm, eps)
+    if s_t is None:
+        s_t = tensor_scale(amax(y))
+    c, s = arc_quantize(y, outliers, s_t)
+    return c, s, np.float32(s_t), y
+
+
+def dequantize(fmt: str, codes, scales, scale=None, inv_had: int = 0) -> np.ndarray:
+    """Dequantize to fp32 (then optionally inverse block Hadamard); returns fp32."""
+    if fmt == "nvfp4":
+        y = nvfp4_dequantize(codes, scales, float(scale))
+    elif fmt == "mxfp4":
+        y = mxfp4_dequantize(codes, scales)
+    elif fmt == "dual":
+        y = dual_dequantize(codes, scales, scale)
+    else:
+        raise ValueError(fmt)
+    if inv_had:
+        y = hadamard(y, inv_had)  # the normalised Sylvester matrix is its own inverse
+    return y
+
+
+def dequantize_bf16(fmt: str, codes, scales, scale=None, inv_had: int = 0) -> np.ndarray:
+    return f32_to_bf16(dequantize(fmt, codes, scales, scale, inv_had))
