@@ -1,0 +1,454 @@
+// fp4q.cu -- the extern "C" boundary of the quantizer library: host-side
+// argument validation, TMA descriptor encoding and kernel launches.  All
+// arithmetic runs in the kernels included below.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/fp4q.h"
+#include "fp4q_arc.cuh"
+#include "fp4q_dequant.cuh"
+#include "fp4q_device.cuh"
+#include "fp4q_quant.cuh"
+
+#define FP4Q_API extern "C" __attribute__((visibility("default")))
+
+namespace {
+
+using namespace fp4q;
+
+constexpr int kMaxGrid = 4096;  // partial maxima fit FP4Q_WORKSPACE_BYTES
+static_assert(kMaxGrid * sizeof(float) <= FP4Q_WORKSPACE_BYTES, "workspace too small");
+
+// ---------------------------------------------------------------- device info
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+
+fp4q_status sm_count(int* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FP4Q_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return FP4Q_ERR_UNSUPPORTED;
+    int n = g_sm_count[dev].load(std::memory_order_relaxed);
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return FP4Q_ERR_CUDA;
+        g_sm_count[dev].store(n, std::memory_order_relaxed);
+    }
+    *out = n;
+    return FP4Q_OK;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::atomic<EncodeTiledFn> g_encode{nullptr};
+
+fp4q_status encode_fn(EncodeTiledFn* out) {
+    EncodeTiledFn fn = g_encode.load(std::memory_order_acquire);
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !p)
+            return FP4Q_ERR_CUDA;
+        fn = reinterpret_cast<EncodeTiledFn>(p);
+        g_encode.store(fn, std::memory_order_release);
+    }
+    *out = fn;
+    return FP4Q_OK;
+}
+
+// bf16 [M, K] with row stride ldx elements; boxes of 64 columns x 16 rows,
+// 128-byte swizzle, zero fill outside the matrix.
+fp4q_status make_x_map(CUtensorMap* map, const void* x, int64_t M, int64_t K, int64_t ldx) {
+    EncodeTiledFn enc;
+    fp4q_status st = encode_fn(&enc);
+    if (st != FP4Q_OK) return st;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kBoxCols, (cuuint32_t)kTileRows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FP4Q_OK : FP4Q_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- validation
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+constexpr int64_t kMaxDim = (int64_t)1 << 31;
+
+fp4q_status check_x(const void* x, int64_t M, int64_t K, int64_t ldx) {
+    if (M < 0 || K <= 0 || ldx < K) return FP4Q_ERR_INVALID_ARG;
+    if (M >= kMaxDim || K >= kMaxDim || ldx >= kMaxDim) return FP4Q_ERR_UNSUPPORTED;
+    if (K < 64) return FP4Q_ERR_UNSUPPORTED;
+    if (M > 0 && !x) return FP4Q_ERR_INVALID_ARG;
+    if (ldx % 8 != 0 || !aligned(x, 16)) return FP4Q_ERR_ALIGNMENT;
+    return FP4Q_OK;
+}
+
+fp4q_status check_out(const uint8_t* codes, const uint8_t* scales) {
+    if (!codes || !scales) return FP4Q_ERR_INVALID_ARG;
+    if (!aligned(codes, 16) || !aligned(scales, 4)) return FP4Q_ERR_ALIGNMENT;
+    return FP4Q_OK;
+}
+
+bool valid_had(int n) {
+    return n == 0 || n == 16 || n == 32 || n == 64 || n == 128 || n == 256 || n == 512;
+}
+
+fp4q_status launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? FP4Q_OK : FP4Q_ERR_CUDA;
+}
+
+// Raises a kernel's dynamic shared-memory limit once per device (the attribute
+// is per function and device; setting it again is harmless but costs host time).
+template <typename Kern>
+fp4q_status ensure_smem(Kern kern, int bytes, std::atomic<uint64_t>& done) {
+    if (bytes <= 48 * 1024) return FP4Q_OK;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FP4Q_ERR_CUDA;
+    const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return FP4Q_OK;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return FP4Q_ERR_CUDA;
+    done.fetch_or(bit, std::memory_order_acq_rel);
+    return FP4Q_OK;
+}
+
+// ---------------------------------------------------------------- quantizer launch
+template <int FMT, int HAD, bool AMAX>
+fp4q_status launch_quant_t(const CUtensorMap& map, const QuantParams& p, int grid, cudaStream_t s) {
+    auto kern = quant_kernel<FMT, HAD, AMAX>;
+    constexpr int smem = quant_smem_bytes<HAD>();
+    static std::atomic<uint64_t> done{0};
+    fp4q_status st = ensure_smem(kern, smem, done);
+    if (st != FP4Q_OK) return st;
+    kern<<<grid, kThreads, smem, s>>>(map, p);
+    return launch_status();
+}
+
+template <int FMT, bool AMAX>
+fp4q_status launch_quant_h(int had, const CUtensorMap& map, const QuantParams& p, int grid,
+                           cudaStream_t s) {
+    switch (had) {
+        case 0: return launch_quant_t<FMT, 0, AMAX>(map, p, grid, s);
+        case 16: return launch_quant_t<FMT, 16, AMAX>(map, p, grid, s);
+        case 32: return launch_quant_t<FMT, 32, AMAX>(map, p, grid, s);
+        case 64: return launch_quant_t<FMT, 64, AMAX>(map, p, grid, s);
+        case 128: return launch_quant_t<FMT, 128, AMAX>(map, p, grid, s);
+        case 256: return launch_quant_t<FMT, 256, AMAX>(map, p, grid, s);
+        case 512: return launch_quant_t<FMT, 512, AMAX>(map, p, grid, s);
+        default: return FP4Q_ERR_INVALID_ARG;
+    }
+}
+
+float had_norm(int n) { return n > 0 ? (float)(1.0 / std::sqrt((double)n)) : 1.0f; }
+
+fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, int had,
+                            int fmt, uint8_t* codes, uint8_t* scales, float* scale_fp32,
+                            fp4q_tscale_mode mode, fp4q_scale_layout layout, void* ws,
+                            size_t ws_bytes, cudaStream_t stream) {
+    fp4q_status st = check_x(x, M, K, ldx);
+    if (st != FP4Q_OK) return st;
+    if (!valid_had(had)) return FP4Q_ERR_INVALID_ARG;
+    if (layout != FP4Q_SCALES_LINEAR && layout != FP4Q_SCALES_SWIZZLED) return FP4Q_ERR_INVALID_ARG;
+    const int B = fmt == FMT_MXFP4 ? 32 : 16;
+    if (K % B != 0 || (had && K % had != 0)) return FP4Q_ERR_INVALID_ARG;
+    if (fmt == FMT_DUAL && K % 128 != 0) return FP4Q_ERR_INVALID_ARG;
+    const bool dynamic = fmt == FMT_NVFP4 && mode == FP4Q_TSCALE_DYNAMIC;
+    if (fmt == FMT_NVFP4 && mode != FP4Q_TSCALE_DYNAMIC && mode != FP4Q_TSCALE_STATIC)
+        return FP4Q_ERR_INVALID_ARG;
+    if (M == 0) return FP4Q_OK;
+    if ((st = check_out(codes, scales)) != FP4Q_OK) return st;
+    if (fmt != FMT_MXFP4) {
+        if (!scale_fp32) return FP4Q_ERR_INVALID_ARG;
+        if (!aligned(scale_fp32, 4)) return FP4Q_ERR_ALIGNMENT;
+    }
+    if (dynamic) {
+        if (!ws) return FP4Q_ERR_INVALID_ARG;
+        if (ws_bytes < FP4Q_WORKSPACE_BYTES) return FP4Q_ERR_INVALID_ARG;
+        if (!aligned(ws, 4)) return FP4Q_ERR_ALIGNMENT;
+    }
+
+    int sms = 0;
+    if ((st = sm_count(&sms)) != FP4Q_OK) return st;
+    CUtensorMap map;
+    if ((st = make_x_map(&map, x, M, K, ldx)) != FP4Q_OK) return st;
+
+    QuantParams p{};
+    p.M = M;
+    p.K = K;
+    p.n_row_tiles = (M + kTileRows - 1) / kTileRows;
+    p.n_col_tiles = (K + kTileCols - 1) / kTileCols;
+    p.n_tiles = p.n_row_tiles * p.n_col_tiles;
+    p.codes = codes;
+    p.scales = scales;
+    p.scale_fp32 = scale_fp32;
+    p.partials = static_cast<float*>(ws);
+    p.swizzled = layout == FP4Q_SCALES_SWIZZLED;
+    p.dynamic = dynamic;
+    p.had_norm = had_norm(had);
+    const int grid = (int)std::min<int64_t>({p.n_tiles, (int64_t)2 * sms, (int64_t)kMaxGrid});
+    p.n_partials = grid;
+
+    if (p.swizzled) {  // padding rows/columns of the tiled layout read as zero
+        const int64_t ncols = K / B;
+        const int64_t bytes = fp4q_scales_bytes(M, ncols, FP4Q_SCALES_SWIZZLED);
+        if (bytes != M * ncols && cudaMemsetAsync(scales, 0, (size_t)bytes, stream) != cudaSuccess)
+            return FP4Q_ERR_CUDA;
+    }
+    if (dynamic) {
+        st = fmt == FMT_NVFP4 ? launch_quant_h<FMT_NVFP4, true>(had, map, p, grid, stream)
+                              : FP4Q_ERR_INVALID_ARG;
+        if (st != FP4Q_OK) return st;
+    }
+    switch (fmt) {
+        case FMT_NVFP4: return launch_quant_h<FMT_NVFP4, false>(had, map, p, grid, stream);
+        case FMT_MXFP4: return launch_quant_h<FMT_MXFP4, false>(had, map, p, grid, stream);
+        case FMT_DUAL: return launch_quant_h<FMT_DUAL, false>(had, map, p, grid, stream);
+        default: return FP4Q_ERR_INVALID_ARG;
+    }
+}
+
+// ---------------------------------------------------------------- dequantizer launch
+template <int FMT, int HAD>
+fp4q_status launch_dequant_t(const DequantParams& p, int grid, cudaStream_t s) {
+    auto kern = dequant_kernel<FMT, HAD>;
+    constexpr int smem = dequant_smem_bytes<HAD>();
+    static std::atomic<uint64_t> done{0};
+    fp4q_status st = ensure_smem(kern, smem, done);
+    if (st != FP4Q_OK) return st;
+    kern<<<grid, kThreads, smem, s>>>(p);
+    return launch_status();
+}
+
+template <int FMT>
+fp4q_status launch_dequant_h(int had, const DequantParams& p, int grid, cudaStream_t s) {
+    switch (had) {
+        case 0: return launch_dequant_t<FMT, 0>(p, grid, s);
+        case 16: return launch_dequant_t<FMT, 16>(p, grid, s);
+        case 32: return launch_dequant_t<FMT, 32>(p, grid, s);
+        case 64: return launch_dequant_t<FMT, 64>(p, grid, s);
+        case 128: return launch_dequant_t<FMT, 128>(p, grid, s);
+        case 256: return launch_dequant_t<FMT, 256>(p, grid, s);
+        case 512: return launch_dequant_t<FMT, 512>(p, grid, s);
+        default: return FP4Q_ERR_INVALID_ARG;
+    }
+}
+
+// ---------------------------------------------------------------- self-test kernel
+__global__ void selftest_div_kernel(const float* x, const float* d, int64_t n, float* qf,
+                                    float* qi) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float dv = d[i], xv = x[i];
+        qi[i] = __fdiv_rn(xv, dv);
+        qf[i] = div_fast_ok(dv, fabsf(xv)) ? div_rn(xv, dv, __frcp_rn(dv)) : __fdiv_rn(xv, dv);
+    }
+}
+
+}  // namespace
+
+// ==================================================================== C ABI
+
+FP4Q_API size_t fp4q_workspace_bytes(int64_t M, int64_t K) {
+    (void)M;
+    (void)K;
+    return FP4Q_WORKSPACE_BYTES;
+}
+
+FP4Q_API int64_t fp4q_scales_bytes(int64_t M, int64_t ncols, fp4q_scale_layout layout) {
+    if (M < 0 || ncols < 0) return -1;
+    if (layout == FP4Q_SCALES_LINEAR) return M * ncols;
+    if (layout == FP4Q_SCALES_SWIZZLED) return ((M + 127) / 128 * 128) * ((ncols + 3) / 4 * 4);
+    return -1;
+}
+
+FP4Q_API fp4q_status fp4q_quantize_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                         uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                                         fp4q_tscale_mode mode, fp4q_scale_layout layout,
+                                         void* workspace, size_t workspace_bytes,
+                                         fp4q_stream_t stream) {
+    return quantize_common(x, M, K, ldx, 0, FMT_NVFP4, codes, scales, tensor_scale, mode, layout,
+                           workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+FP4Q_API fp4q_status fp4q_quantize_mxfp4(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                         uint8_t* codes, uint8_t* scales,
+                                         fp4q_scale_layout layout, fp4q_stream_t stream) {
+    return quantize_common(x, M, K, ldx, 0, FMT_MXFP4, codes, scales, nullptr,
+                           FP4Q_TSCALE_STATIC, layout, nullptr, 0, (cudaStream_t)stream);
+}
+
+FP4Q_API fp4q_status fp4q_hadamard_quantize(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                            int had_size, fp4q_format format, uint8_t* codes,
+                                            uint8_t* scales, float* scale_fp32,
+                                            fp4q_tscale_mode mode, fp4q_scale_layout layout,
+                                            void* workspace, size_t workspace_bytes,
+                                            fp4q_stream_t stream) {
+    int fmt;
+    switch (format) {
+        case FP4Q_NVFP4: fmt = FMT_NVFP4; break;
+        case FP4Q_MXFP4: fmt = FMT_MXFP4; break;
+        case FP4Q_NVFP4_DUAL: fmt = FMT_DUAL; break;
+        default: return FP4Q_ERR_INVALID_ARG;
+    }
+    return quantize_common(x, M, K, ldx, had_size, fmt, codes, scales, scale_fp32, mode, layout,
+                           workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+FP4Q_API fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                       const void* gamma, float eps, const int32_t* perm,
+                                       const int32_t* outliers, int64_t S, uint8_t* codes,
+                                       uint8_t* scales, float* tensor_scale,
+                                       fp4q_tscale_mode mode, fp4q_scale_layout layout,
+                                       void* workspace, size_t workspace_bytes,
+                                       fp4q_stream_t stream) {
+    fp4q_status st = check_x(x, M, K, ldx);
+    if (st != FP4Q_OK) return st;
+    if (K % 16 != 0 || S < 0 || S % 16 != 0 || S > K) return FP4Q_ERR_INVALID_ARG;
+    if (K > 16384) return FP4Q_ERR_UNSUPPORTED;
+    if (!(eps >= 0.0f) || !std::isfinite(eps)) return FP4Q_ERR_INVALID_ARG;
+    if (mode != FP4Q_TSCALE_DYNAMIC && mode != FP4Q_TSCALE_STATIC) return FP4Q_ERR_INVALID_ARG;
+    if (layout != FP4Q_SCALES_LINEAR && layout != FP4Q_SCALES_SWIZZLED) return FP4Q_ERR_INVALID_ARG;
+    if (M == 0) return FP4Q_OK;
+    if ((st = check_out(codes, scales)) != FP4Q_OK) return st;
+    if (!gamma || !perm || !tensor_scale || (S > 0 && !outliers)) return FP4Q_ERR_INVALID_ARG;
+    if (!aligned(gamma, 2) || !aligned(perm, 4) || !aligned(tensor_scale, 4) ||
+        (S > 0 && !aligned(outliers, 4)))
+        return FP4Q_ERR_ALIGNMENT;
+    const bool dynamic = mode == FP4Q_TSCALE_DYNAMIC;
+    if (dynamic && (!workspace || workspace_bytes < FP4Q_WORKSPACE_BYTES)) return FP4Q_ERR_INVALID_ARG;
+    if (dynamic && !aligned(workspace, 4)) return FP4Q_ERR_ALIGNMENT;
+
+    int sms = 0;
+    if ((st = sm_count(&sms)) != FP4Q_OK) return st;
+    ArcParams p{};
+    p.M = M;
+    p.K = K;
+    p.S = S;
+    p.perm = perm;
+    p.outliers = outliers;
+    p.gamma = static_cast<const uint16_t*>(gamma);
+    p.x = static_cast<const uint8_t*>(x);
+    p.ldx_bytes = ldx * 2;
+    p.eps = eps;
+    p.codes = codes;
+    p.scales = scales;
+    p.tensor_scale = tensor_scale;
+    p.partials = static_cast<float*>(workspace);
+    p.swizzled = layout == FP4Q_SCALES_SWIZZLED;
+    p.dynamic = dynamic;
+    const int threads = (int)std::max<int64_t>(32, ((K / 16) + 31) / 32 * 32);
+    const int smem = arc_smem_bytes(K);
+    const int per_sm = threads <= 256 ? 2 : 1;
+    const int grid = (int)std::min<int64_t>({M, (int64_t)per_sm * sms, (int64_t)kMaxGrid});
+    p.n_partials = grid;
+    if (p.swizzled) {
+        const int64_t ncols = (K + S) / 16;
+        const int64_t bytes = fp4q_scales_bytes(M, ncols, FP4Q_SCALES_SWIZZLED);
+        if (bytes != M * ncols && cudaMemsetAsync(scales, 0, (size_t)bytes, (cudaStream_t)stream) != cudaSuccess)
+            return FP4Q_ERR_CUDA;
+    }
+    // The shared-memory size depends on K, so the attribute is set on every call.
+    auto run = [&](auto kern) -> fp4q_status {
+        if (smem > 48 * 1024 &&
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return FP4Q_ERR_CUDA;
+        kern<<<grid, threads, smem, (cudaStream_t)stream>>>(p);
+        return launch_status();
+    };
+    if (threads <= 256) {
+        if (dynamic && (st = run(arc_kernel<true, 256>)) != FP4Q_OK) return st;
+        return run(arc_kernel<false, 256>);
+    }
+    if (dynamic && (st = run(arc_kernel<true, 1024>)) != FP4Q_OK) return st;
+    return run(arc_kernel<false, 1024>);
+}
+
+FP4Q_API fp4q_status fp4q_dequantize(fp4q_format format, const uint8_t* codes,
+                                     const uint8_t* scales, const float* scale_fp32, int64_t M,
+                                     int64_t K, fp4q_scale_layout layout, int inv_had_size,
+                                     void* y, fp4q_stream_t stream) {
+    if (M < 0 || K <= 0) return FP4Q_ERR_INVALID_ARG;
+    if (M >= kMaxDim || K >= kMaxDim) return FP4Q_ERR_UNSUPPORTED;
+    if (K < 64) return FP4Q_ERR_UNSUPPORTED;
+    if (!valid_had(inv_had_size)) return FP4Q_ERR_INVALID_ARG;
+    if (layout != FP4Q_SCALES_LINEAR && layout != FP4Q_SCALES_SWIZZLED) return FP4Q_ERR_INVALID_ARG;
+    int fmt;
+    switch (format) {
+        case FP4Q_NVFP4: fmt = FMT_NVFP4; break;
+        case FP4Q_MXFP4: fmt = FMT_MXFP4; break;
+        case FP4Q_NVFP4_DUAL: fmt = FMT_DUAL; break;
+        default: return FP4Q_ERR_INVALID_ARG;
+    }
+    const int B = fmt == FMT_MXFP4 ? 32 : 16;
+    if (K % B != 0 || (inv_had_size && K % inv_had_size != 0)) return FP4Q_ERR_INVALID_ARG;
+    if (fmt == FMT_DUAL && K % 128 != 0) return FP4Q_ERR_INVALID_ARG;
+    if (M == 0) return FP4Q_OK;
+    if (!codes || !scales || !y || (fmt != FMT_MXFP4 && !scale_fp32)) return FP4Q_ERR_INVALID_ARG;
+    if (!aligned(codes, 16) || !aligned(y, 16) || (scale_fp32 && !aligned(scale_fp32, 4)))
+        return FP4Q_ERR_ALIGNMENT;
+    int sms = 0;
+    fp4q_status st;
+    if ((st = sm_count(&sms)) != FP4Q_OK) return st;
+    DequantParams p{};
+    p.M = M;
+    p.K = K;
+    p.n_col_tiles = (K + kTileCols - 1) / kTileCols;
+    p.n_tiles = ((M + kTileRows - 1) / kTileRows) * p.n_col_tiles;
+    p.codes = codes;
+    p.scales = scales;
+    p.scale_fp32 = scale_fp32;
+    p.y = static_cast<uint16_t*>(y);
+    p.swizzled = layout == FP4Q_SCALES_SWIZZLED;
+    p.had_norm = had_norm(inv_had_size);
+    const int grid = (int)std::min<int64_t>({p.n_tiles, (int64_t)4 * sms, (int64_t)kMaxGrid});
+    cudaStream_t s = (cudaStream_t)stream;
+    switch (fmt) {
+        case FMT_NVFP4: return launch_dequant_h<FMT_NVFP4>(inv_had_size, p, grid, s);
+        case FMT_MXFP4: return launch_dequant_h<FMT_MXFP4>(inv_had_size, p, grid, s);
+        default: return launch_dequant_h<FMT_DUAL>(inv_had_size, p, grid, s);
+    }
+}
+
+FP4Q_API const char* fp4q_status_string(fp4q_status status) {
+    switch (status) {
+        case FP4Q_OK: return "FP4Q_OK";
+        case FP4Q_ERR_INVALID_ARG: return "FP4Q_ERR_INVALID_ARG: invalid argument";
+        case FP4Q_ERR_UNSUPPORTED: return "FP4Q_ERR_UNSUPPORTED: unsupported size or option";
+        case FP4Q_ERR_ALIGNMENT: return "FP4Q_ERR_ALIGNMENT: misaligned pointer or stride";
+        case FP4Q_ERR_CUDA: return "FP4Q_ERR_CUDA: CUDA call failed";
+        case FP4Q_ERR_DEVICE: return "FP4Q_ERR_DEVICE: device-side wait timed out";
+        default: return "FP4Q: unknown status";
+    }
+}
+
+FP4Q_API int fp4q_device_error(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return -1;
+    if (v && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return -1;
+    return (int)v;
+}
+
+FP4Q_API fp4q_status fp4q_selftest_div(const float* x, const float* d, int64_t n, float* q_fast,
+                                       float* q_ieee, fp4q_stream_t stream) {
+    if (n < 0) return FP4Q_ERR_INVALID_ARG;
+    if (n == 0) return FP4Q_OK;
+    if (!x || !d || !q_fast || !q_ieee) return FP4Q_ERR_INVALID_ARG;
+    const int grid = (int)std::min<int64_t>((n + 255) / 256, 4096);
+    selftest_div_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(x, d, n, q_fast, q_ieee);
+    return launch_status();
+}

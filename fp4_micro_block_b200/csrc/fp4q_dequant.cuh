@@ -1,0 +1,216 @@
+// fp4q_dequant.cuh -- dequantization kernels for sm_100a: packed E2M1 codes +
+// block scales back to bf16, optionally followed by the inverse block Hadamard
+// (the normalised Sylvester matrix is its own inverse).  This is the receiving
+// side of FP4-compressed activations (FP4Quant abstract).
+//
+// Same tile geometry and thread -> unit map as the quantizer (16 rows x 512
+// columns per tile, one 32-column unit per thread).  Codes and scales are read
+// straight from global memory (0.5-0.6 byte per element); the bf16 output is
+// written with 16-byte stores.  For Hadamard sizes >= 64 the unit first gets
+// H_32 in registers, then the threads of one n-block exchange through a
+// swizzled fp32 scratch, apply H_n2 across the 32-column rows, and store their
+// column slices.
+#pragma once
+
+#include "fp4q_quant.cuh"
+
+namespace fp4q {
+
+struct DequantParams {
+    int64_t M, K;
+    int64_t n_col_tiles, n_tiles;
+    const uint8_t* codes;
+    const uint8_t* scales;
+    const float* scale_fp32;
+    uint16_t* y;
+    int swizzled;
+    float had_norm;
+};
+
+template <int FMT>
+__device__ __forceinline__ void decode_unit(const DequantParams& p, int64_t row, int64_t col,
+                                            int nval, float* v) {
+    const uint8_t* cp = p.codes + row * (p.K / 2) + col / 2;
+    uint32_t w[4];
+    if ((p.K & 31) == 0) {
+        uint4 q = __ldg(reinterpret_cast<const uint4*>(cp));
+        w[0] = q.x; w[1] = q.y; w[2] = q.z; w[3] = q.w;
+    } else {
+        uint2 q = __ldg(reinterpret_cast<const uint2*>(cp));
+        w[0] = q.x; w[1] = q.y;
+        if (nval > 16) {
+            uint2 q2 = __ldg(reinterpret_cast<const uint2*>(cp + 8));
+            w[2] = q2.x; w[3] = q2.y;
+        } else {
+            w[2] = 0u; w[3] = 0u;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        float2 c = e2m1x2_decode((w[i >> 2] >> (8 * (i & 3))) & 0xffu);
+        v[2 * i] = c.x;
+        v[2 * i + 1] = c.y;
+    }
+    if constexpr (FMT == FMT_MXFP4) {
+        const int64_t nsc = p.K / 32, c0 = col / 32;
+        const uint32_t b = p.swizzled ? p.scales[swizzle_offset(row, c0, (nsc + 3) / 4)]
+                                      : p.scales[row * nsc + c0];
+        const float sc = b ? __uint_as_float(b << 23) : __uint_as_float(0x00400000u);  // 2^(b-127)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= sc;
+    } else {
+        const int64_t nsc = p.K / 16, c0 = col / 16;
+        uint32_t e0, e1 = 0;
+        if (p.swizzled) {
+            const int64_t nC = (nsc + 3) / 4;
+            e0 = p.scales[swizzle_offset(row, c0, nC)];
+            if (nval > 16) e1 = p.scales[swizzle_offset(row, c0 + 1, nC)];
+        } else {
+            e0 = p.scales[row * nsc + c0];
+            if (nval > 16) e1 = p.scales[row * nsc + c0 + 1];
+        }
+        const float s = (FMT == FMT_DUAL) ? p.scale_fp32[row * (p.K / 128) + col / 128]
+                                          : p.scale_fp32[0];
+        const float ev0 = e4m3_decode(e0), ev1 = e4m3_decode(e1);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = (v[i] * ev0) * s;
+#pragma unroll
+        for (int i = 16; i < 32; ++i) v[i] = (v[i] * ev1) * s;
+    }
+}
+
+template <int FMT, int HAD>
+__global__ void __launch_bounds__(kThreads, 2) dequant_kernel(const DequantParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    float* scratch = reinterpret_cast<float*>(smem_raw);
+    const uint32_t tid = threadIdx.x;
+    const uint32_t lane = tid & 31, warp = tid >> 5;
+    const uint32_t r = (lane & 7) + 8 * (warp & 1);
+    const uint32_t j = (lane >> 3) + 4 * (warp >> 1);
+
+    for (int64_t t = blockIdx.x; t < p.n_tiles; t += gridDim.x) {
+        const int64_t rt = t / p.n_col_tiles, ct = t % p.n_col_tiles;
+        const int64_t row = rt * kTileRows + r;
+        const int64_t col = ct * kTileCols + 32 * (int64_t)j;
+        const bool live = row < p.M && col < p.K;
+        const int nval = live ? (int)min64(32, p.K - col) : 0;
+        float v[32];
+        if (live) {
+            decode_unit<FMT>(p, row, col, nval, v);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+        }
+        uint16_t* yrow = p.y + row * p.K;
+
+        if constexpr (HAD <= 32) {
+            if constexpr (HAD == 16) {
+                fwht_reg<16>(v);
+                fwht_reg<16>(v + 16);
+            } else if constexpr (HAD == 32) {
+                fwht_reg<32>(v);
+            }
+            if constexpr (HAD > 0) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] *= p.had_norm;
+            }
+            if (live) {
+                uint32_t o[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) o[i] = bf16x2_pack(v[2 * i], v[2 * i + 1]);
+                uint4* dst = reinterpret_cast<uint4*>(yrow + col);
+                dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+                dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+                if (nval > 16) {
+                    dst[2] = make_uint4(o[8], o[9], o[10], o[11]);
+                    dst[3] = make_uint4(o[12], o[13], o[14], o[15]);
+                }
+            }
+        } else {
+            constexpr int n2 = HadShape<HAD>::n2;
+            constexpr int k1w = HadShape<HAD>::k1w;
+            const uint32_t tau = j % n2, blk = j / n2;
+            fwht_reg<32>(v);
+            uint8_t* sb = reinterpret_cast<uint8_t*>(scratch) +
+                          (r * (kTileCols / HAD) + blk) * (uint32_t)(n2 * 128);
+            const bool cross_warp = n2 > 4;
+            if (cross_warp) bar_sync(2, kThreads);
+            else __syncwarp();
+            {
+                uint8_t* rowp = sb + tau * 128;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<float4*>(rowp + (((ch ^ r) & 7u) << 4)) =
+                        make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
+            }
+            if (cross_warp) bar_sync(2, kThreads);
+            else __syncwarp();
+            float a[n2][k1w];
+            const uint32_t k1 = k1w * tau;
+#pragma unroll
+            for (int k2 = 0; k2 < n2; ++k2) {
+                const uint8_t* rowp = sb + k2 * 128;
+                if constexpr (k1w == 2) {
+                    float2 q = *reinterpret_cast<const float2*>(
+                        rowp + ((((k1 >> 2) ^ r) & 7u) << 4) + (k1 & 3u) * 4u);
+                    a[k2][0] = q.x;
+                    a[k2][1] = q.y;
+                } else {
+#pragma unroll
+                    for (int h = 0; h < k1w / 4; ++h) {
+                        float4 q = *reinterpret_cast<const float4*>(
+                            rowp + (((((k1 >> 2) + h) ^ r) & 7u) << 4));
+                        a[k2][4 * h] = q.x;
+                        a[k2][4 * h + 1] = q.y;
+                        a[k2][4 * h + 2] = q.z;
+                        a[k2][4 * h + 3] = q.w;
+                    }
+                }
+            }
+#pragma unroll
+            for (int s = 1; s < n2; s <<= 1) {
+#pragma unroll
+                for (int k2 = 0; k2 < n2; ++k2) {
+                    if ((k2 & s) == 0) {
+#pragma unroll
+                        for (int i = 0; i < k1w; ++i) {
+                            float x0 = a[k2][i], x1 = a[k2 + s][i];
+                            a[k2][i] = x0 + x1;
+                            a[k2 + s][i] = x0 - x1;
+                        }
+                    }
+                }
+            }
+            if (live) {
+                const int64_t cb = ct * kTileCols + (int64_t)blk * HAD + k1;
+#pragma unroll
+                for (int k2 = 0; k2 < n2; ++k2) {
+                    uint16_t* dst = yrow + cb + 32 * k2;
+                    if constexpr (k1w == 2) {
+                        *reinterpret_cast<uint32_t*>(dst) =
+                            bf16x2_pack(a[k2][0] * p.had_norm, a[k2][1] * p.had_norm);
+                    } else if constexpr (k1w == 4) {
+                        *reinterpret_cast<uint2*>(dst) =
+                            make_uint2(bf16x2_pack(a[k2][0] * p.had_norm, a[k2][1] * p.had_norm),
+                                       bf16x2_pack(a[k2][2] * p.had_norm, a[k2][3] * p.had_norm));
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < k1w / 8; ++h)
+                            reinterpret_cast<uint4*>(dst)[h] = make_uint4(
+                                bf16x2_pack(a[k2][8 * h + 0] * p.had_norm, a[k2][8 * h + 1] * p.had_norm),
+                                bf16x2_pack(a[k2][8 * h + 2] * p.had_norm, a[k2][8 * h + 3] * p.had_norm),
+                                bf16x2_pack(a[k2][8 * h + 4] * p.had_norm, a[k2][8 * h + 5] * p.had_norm),
+                                bf16x2_pack(a[k2][8 * h + 6] * p.had_norm, a[k2][8 * h + 7] * p.had_norm));
+                    }
+                }
+            }
+        }
+    }
+}
+
+template <int HAD>
+constexpr int dequant_smem_bytes() {
+    return HAD >= 64 ? kScratchBytes : 0;
+}
+
+}  // namespace fp4q

@@ -1,0 +1,220 @@
+/*
+ * fp4q.h -- C ABI of the B200 (sm_100a) micro-block FP4 activation quantizer.
+ *
+ * The library turns bf16 activations [M tokens x K channels] into 4-bit E2M1
+ * codes plus block scales, in the two hardware micro-scaling formats and a
+ * dual-scale variant, optionally after a block Hadamard rotation or the
+ * ARCQuant reorder + RMSNorm + residual path, and back again.
+ *
+ * Common conventions
+ * ------------------
+ *  - Every pointer argument is a DEVICE pointer to memory the caller allocated
+ *    and owns (unless stated otherwise).  The library allocates nothing, holds
+ *    no pointer after a call returns, and enqueues its kernels on `stream` only
+ *    (NULL = the legacy default stream).  Calls are asynchronous.
+ *  - bf16 matrices are row-major with a row stride `ld*` given in ELEMENTS.
+ *  - Packed codes are row-major uint8 [M, K/2]: two E2M1 codes per byte, the
+ *    code of the even column in the LOW nibble.  E2M1 code c: bit 3 = sign,
+ *    magnitude (c & 7) -> {0, 0.5, 1, 1.5, 2, 3, 4, 6}.
+ *  - Scale matrices are uint8 [M, K/B] row-major (FP4Q_SCALES_LINEAR) or the
+ *    128x4-tiled layout of block-scaled tensor-core GEMMs
+ *    (FP4Q_SCALES_SWIZZLED, see fp4q_scales_bytes): rows padded to a multiple
+ *    of 128, scale columns to a multiple of 4, padding written as zero.
+ *  - Validation happens on the host before anything is launched.  On any
+ *    error the call returns a status != FP4Q_OK and launches nothing.
+ *    Requirements shared by the quantizers: M >= 0, K >= 64, ldx >= K,
+ *    ldx % 8 == 0, x 16-byte aligned; M == 0 is a no-op returning FP4Q_OK.
+ *  - Kernel launch failures return FP4Q_ERR_CUDA.  Faults that happen later on
+ *    the device surface through the CUDA error state of the stream.  A device-
+ *    side bounded wait that runs out records a code read by fp4q_device_error().
+ *  - The library is reentrant: it keeps no state between calls apart from the
+ *    device error word described at fp4q_device_error().
+ *
+ * Numeric rules (identical in every entry point):
+ *  - E2M1 rounding: nearest grid value, ties to the even code, saturation at
+ *    +-6, sign kept (a negative value rounding to zero gives code 0x8).
+ *  - NVFP4 (16-element blocks; ARCQuant summary, "Enonce du Probleme": NVFP4
+ *    needs block size 16; E4M3 scales with an FP32 per-tensor scale, the usual
+ *    NVFP4 recipe named in the nGPT abstract "Normalized Architectures are
+ *    Natively 4-Bit"):  s_t = amax/2688;  per block r = (amax_b/6)/s_t,
+ *    e = E4M3 round-to-nearest-even saturating at 448, d = E4M3(e)*s_t,
+ *    code = E2M1(y/d) with y/d correctly rounded.  d == 0 gives zero codes.
+ *  - MXFP4 (32-element blocks, power-of-two scale; MR-GPTQ abstract, point
+ *    (2)): scale byte b = clamp(floor(log2 amax_b) - 2 + 127, 0, 254),
+ *    code = E2M1(y * 2^(127-b)) (exact scaling); amax_b == 0 gives b = 0 and
+ *    zero codes.
+ *  - Dual scale (FP4Quant abstract, "micro-grouped dual-scale FP4"): an FP32
+ *    group scale G = amax_128/2688 per 128 contiguous elements, then the NVFP4
+ *    rule per 16-block with G in place of s_t.
+ */
+#ifndef FP4Q_H
+#define FP4Q_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st* fp4q_stream_t;
+
+typedef enum fp4q_status {
+    FP4Q_OK = 0,
+    FP4Q_ERR_INVALID_ARG = 1, /* null pointer, bad size or enum value          */
+    FP4Q_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. K too large)  */
+    FP4Q_ERR_ALIGNMENT = 3,   /* pointer or row stride misaligned              */
+    FP4Q_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed             */
+    FP4Q_ERR_DEVICE = 5       /* a kernel's bounded wait ran out (see below)   */
+} fp4q_status;
+
+typedef enum fp4q_format {
+    FP4Q_NVFP4 = 0,      /* B = 16, E4M3 block scale, FP32 tensor scale          */
+    FP4Q_MXFP4 = 1,      /* B = 32, E8M0 shared exponent                          */
+    FP4Q_NVFP4_DUAL = 2  /* B = 16, E4M3 micro-scale, FP32 scale per 128 elements */
+} fp4q_format;
+
+typedef enum fp4q_scale_layout {
+    FP4Q_SCALES_LINEAR = 0,   /* uint8 [M, K/B] row-major                            */
+    FP4Q_SCALES_SWIZZLED = 1  /* 128x4 tiles: byte of (r, c) at
+                                 ((r/128)*nC + c/4)*512 + (r%32)*16 + ((r%128)/32)*4 + c%4,
+                                 nC = ceil((K/B)/4)                                   */
+} fp4q_scale_layout;
+
+typedef enum fp4q_tscale_mode {
+    FP4Q_TSCALE_DYNAMIC = 0, /* compute s_t = amax/2688 of the quantized tensor and
+                                WRITE it to *tensor_scale (two passes over x)        */
+    FP4Q_TSCALE_STATIC = 1   /* READ s_t from *tensor_scale (a calibrated scale;
+                                one pass).  s_t <= 0 gives zero scales and codes.    */
+} fp4q_tscale_mode;
+
+/* Bytes of scratch the DYNAMIC tensor-scale mode needs (per-CTA partial maxima).
+ * A constant; any M, K.  The workspace may be reused as soon as the call's
+ * kernels have finished on the stream. */
+#define FP4Q_WORKSPACE_BYTES ((size_t)16384)
+size_t fp4q_workspace_bytes(int64_t M, int64_t K);
+
+/* Size in bytes of the scale buffer a quantizer writes for an [M, ncols]
+ * matrix of ncols = K/B blocks (ARC: (K+S)/16) in the given layout.  The
+ * SWIZZLED size is ceil(M/128)*128 * ceil(ncols/4)*4.  Returns -1 on bad args. */
+int64_t fp4q_scales_bytes(int64_t M, int64_t ncols, fp4q_scale_layout layout);
+
+/* fp4q_quantize_nvfp4 -- NVFP4 quantization of a bf16 matrix.
+ *   x            bf16 [M, ldx], K columns used.          (read)
+ *   codes        uint8 [M, K/2].                         (written)
+ *   scales       E4M3 bytes, [M, K/16] or swizzled.      (written)
+ *   tensor_scale 1 float: written (DYNAMIC) or read (STATIC).
+ *   workspace    >= fp4q_workspace_bytes() device bytes, DYNAMIC mode only
+ *                (may be NULL in STATIC mode).
+ * Requires K % 16 == 0.
+ * Defined by: ARCQuant summary, "Methodologie" item 2 (primary stage: standard
+ * block NVFP4 quantization) and "Enonce du Probleme" (block size 16). */
+fp4q_status fp4q_quantize_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                                fp4q_tscale_mode mode, fp4q_scale_layout layout,
+                                void* workspace, size_t workspace_bytes,
+                                fp4q_stream_t stream);
+
+/* fp4q_quantize_mxfp4 -- MXFP4 quantization of a bf16 matrix.
+ *   x       bf16 [M, ldx].                     (read)
+ *   codes   uint8 [M, K/2].                    (written)
+ *   scales  E8M0 bytes, [M, K/32] or swizzled. (written)
+ * Requires K % 32 == 0.
+ * Defined by: MR-GPTQ abstract (MXFP4 and its power-of-two scale). */
+fp4q_status fp4q_quantize_mxfp4(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                uint8_t* codes, uint8_t* scales, fp4q_scale_layout layout,
+                                fp4q_stream_t stream);
+
+/* fp4q_hadamard_quantize -- block Hadamard rotation, then quantization.
+ *   y[r, b*n + i] = (1/sqrt(n)) * sum_j H_n[i][j] x[r, b*n + j]  for every
+ *   contiguous n-block along K, H_n the Sylvester matrix
+ *   H_n[i][j] = (-1)^popcount(i & j); then `format` quantization of y.
+ *   had_size   n in {0 (no rotation), 16, 32, 64, 128, 256, 512}.
+ *   format     FP4Q_NVFP4: scale_fp32 = 1 float tensor scale (DYNAMIC: written,
+ *              STATIC: read).  FP4Q_MXFP4: scale_fp32 unused (may be NULL).
+ *              FP4Q_NVFP4_DUAL: scale_fp32 = float [M, K/128] group scales,
+ *              written; `mode` ignored.
+ *   codes/scales as above; workspace as for fp4q_quantize_nvfp4.
+ * Requires K % n == 0 and K % B == 0 (K % 128 == 0 for the dual format).
+ * Defined by: MR-GPTQ abstract (block-wise Hadamard transforms, computed on the
+ * fly for activations) and FP4Quant abstract (two-level FWHT, micro-grouped
+ * dual-scale quantization). */
+fp4q_status fp4q_hadamard_quantize(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                   int had_size, fp4q_format format,
+                                   uint8_t* codes, uint8_t* scales, float* scale_fp32,
+                                   fp4q_tscale_mode mode, fp4q_scale_layout layout,
+                                   void* workspace, size_t workspace_bytes,
+                                   fp4q_stream_t stream);
+
+/* fp4q_arc_quantize -- ARCQuant fused reorder + RMSNorm + primary NVFP4 +
+ * residual NVFP4 of the outlier channels.
+ *   For each row: y[p] = x[perm[p]] / sqrt(mean_k x[k]^2 + eps) * gamma[perm[p]]
+ *   (p = 0..K-1), primary = NVFP4(y) with tensor scale s_t; for j < S, the
+ *   residual res[j] = y[outliers[j]] - dq(outliers[j]) with
+ *   dq = (E2M1 value * E4M3 value) * s_t, quantized NVFP4 with the same s_t.
+ *   Output row = [primary K columns | residual S columns]:
+ *   codes uint8 [M, (K+S)/2], scales [M, (K+S)/16] (or swizzled).
+ *   gamma     bf16 [K], indexed by ORIGINAL channel.
+ *   perm      int32 [K], perm[p] = original channel placed at position p
+ *             (a permutation of 0..K-1; entries outside [0, K) are replaced
+ *             by 0 and reported through fp4q_device_error(), code 2).
+ *   outliers  int32 [S], positions in the REORDERED order (0 <= o < K, same
+ *             out-of-range handling as perm); the
+ *             calibrated choice is 0..S-1 (channels sorted by descending
+ *             calibration absmax).  May be NULL when S == 0.
+ *   tensor_scale / mode / workspace as for fp4q_quantize_nvfp4; DYNAMIC uses the
+ *   amax of y.
+ * Requires K % 16 == 0, S % 16 == 0, 0 <= S <= K, K <= 16384, eps >= 0.
+ * Defined by: ARCQuant summary, "Methodologie" items 1 (reorder by absolute
+ * maximum, subset S), 2 (two-stage quantization), 3 (residual channels
+ * concatenated along K) and 5 (one fused kernel: reorder, RMSNorm, primary and
+ * residual quantization, GEMM-ready channel layout). */
+fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int64_t ldx,
+                              const void* gamma, float eps, const int32_t* perm,
+                              const int32_t* outliers, int64_t S,
+                              uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                              fp4q_tscale_mode mode, fp4q_scale_layout layout,
+                              void* workspace, size_t workspace_bytes,
+                              fp4q_stream_t stream);
+
+/* fp4q_dequantize -- codes + scales back to bf16, optionally followed by the
+ * inverse block Hadamard (the normalised Sylvester matrix is its own inverse).
+ *   value = (E2M1 value * E4M3 value) * s (s = *scale_fp32 for NVFP4, the
+ *   group scale for the dual format) or E2M1 value * 2^(b-127) for MXFP4,
+ *   computed in FP32, then (if inv_had_size) rotated, then rounded to bf16
+ *   (nearest even).
+ *   codes      uint8 [M, K/2]; scales [M, K/B] or swizzled, per `layout`.
+ *   scale_fp32 NVFP4: 1 float; dual: float [M, K/128]; MXFP4: unused.
+ *   y          bf16 [M, K] (row stride K).  (written)
+ *   inv_had_size 0 or n in {16, 32, 64, 128, 256, 512}, K % n == 0.
+ * Requires K % B == 0 (K % 128 for dual), K >= 64, 16-byte aligned codes and y.
+ * Defined by: FP4Quant abstract (the receiving side of FP4-compressed
+ * activations: unpack, rescale, inverse FWHT). */
+fp4q_status fp4q_dequantize(fp4q_format format, const uint8_t* codes, const uint8_t* scales,
+                            const float* scale_fp32, int64_t M, int64_t K,
+                            fp4q_scale_layout layout, int inv_had_size, void* y,
+                            fp4q_stream_t stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fp4q_status_string(fp4q_status status);
+
+/* Reads and clears the device error word of the CURRENT device: 0 if no kernel
+ * recorded an error since the last read, else a bit mask (1 = a bounded wait
+ * on a tile's arrival barrier ran out; 2 = an index argument of
+ * fp4q_arc_quantize was outside [0, K) and was clamped).  Synchronizes the
+ * device.  Returns -1 if the read itself failed. */
+int fp4q_device_error(void);
+
+/* Self-check of the division used by the quantizers (no page counterpart: it
+ * exists so that tests can compare the kernels' correctly rounded quotient
+ * against CUDA's IEEE division).  For i < n: q_fast[i] = x[i]/d[i] by the
+ * kernels' method, q_ieee[i] = the IEEE quotient.  All device pointers. */
+fp4q_status fp4q_selftest_div(const float* x, const float* d, int64_t n, float* q_fast,
+                              float* q_ieee, fp4q_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4Q_H */

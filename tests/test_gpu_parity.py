@@ -1,0 +1,365 @@
+"""GPU parity: the sm_100a kernels, called through the C ABI, against the oracle.
+
+Small cases run element by element (several tiles, ragged tails in M and K,
+strided rows, both scale layouts, both tensor-scale modes); the five workload
+shapes run at full size, compared on every element where the oracle is cheap
+(quantize-only) and on sampled rows where it is not (Hadamard, RMSNorm).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity import (assert_bitexact, assert_tolerant, bf16_torch_to_bits, bits_to_torch_cuda,
+                    to_np, unswizzle)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fq():
+    from fp4_micro_block_b200 import build
+    build.build()
+    import fp4_micro_block_b200 as m
+    assert m.fp4q_device_error() == 0
+    yield m
+    assert m.fp4q_device_error() == 0
+
+
+def linear_scales(fq, scales_t, M, ncols, layout):
+    s = to_np(scales_t)
+    if layout == fq.FP4Q_SCALES_SWIZZLED:
+        assert s.size == fq.fp4q_scales_bytes(M, ncols, layout)
+        lin = unswizzle(s, M, ncols)
+        # every byte outside the (r, c) positions is padding and must be zero
+        assert_bitexact("tiled scale buffer", s, oracle.swizzle_scales(lin))
+        return lin
+    return s.reshape(M, ncols)
+
+
+# ----------------------------------------------------------------------------- division
+
+def test_division_is_correctly_rounded(fq):
+    rng = np.random.default_rng(100)
+    n = 1 << 20
+    d = (oracle.e4m3_decode(rng.integers(1, 127, n).astype(np.uint8)).astype(np.float64) *
+         np.exp(rng.uniform(-30, 30, n))).astype(np.float32)
+    x = (rng.standard_normal(n) * d * rng.uniform(0, 7, n)).astype(np.float32)
+    # quotients placed within a few ulps of every E2M1 decision point
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0], np.float32)
+    k = n // 4
+    q = mids[rng.integers(0, len(mids), k)]
+    q = (q.view(np.int32) + rng.integers(-3, 4, k).astype(np.int32)).view(np.float32)
+    x[:k] = (q.astype(np.float64) * d[:k]).astype(np.float32) * np.where(rng.random(k) < .5, -1, 1)
+    x[k] = -0.0
+    x[k + 1] = 0.0
+    xt, dt = torch.from_numpy(x).cuda(), torch.from_numpy(d).cuda()
+    qf, qi = torch.empty_like(xt), torch.empty_like(xt)
+    fq.fp4q_selftest_div(xt, dt, qf, qi)
+    torch.cuda.synchronize()
+    assert_bitexact("markstein vs IEEE", to_np(qf), to_np(qi))
+    # and the IEEE quotient is the host's binary32 quotient
+    assert_bitexact("IEEE vs host", to_np(qi), x / d)
+
+
+# ----------------------------------------------------------------------------- formats
+
+def test_mxfp4_format_conformance(fq):
+    """Blocks whose amax is exactly 4 * 2^E, elements at and around every E2M1
+    decision point, negative values that round to zero, signed zeros."""
+    pts = np.array([0, .25, .5, .75, 1, 1.25, 1.5, 1.75, 2, 2.5, 3, 3.5, 4, 5, 6, 7, 8], np.float64)
+    rng = np.random.default_rng(101)
+    vals = []
+    for p in pts:
+        for u in (-2, -1, 0, 1, 2):
+            v = np.float32(p)
+            if p > 0:
+                v = (np.array([p], np.float32).view(np.int32) + u).view(np.float32)[0]
+            vals += [v, -v]
+    vals = np.array(vals, np.float32)
+    M, K = 64, 256
+    y = np.empty((M, K), np.float32)
+    for r in range(M):
+        y[r] = rng.choice(vals, K)
+        y[r, ::32] = 4.0  # amax = 4 -> E = 0 for every block... and 2^E scaling below
+    y *= np.exp2(rng.integers(-20, 20, (M, 1))).astype(np.float32)
+    y[0, 1] = -0.0
+    x_bits = oracle.f32_to_bf16(y)
+    y = oracle.bf16_to_f32(x_bits)
+    codes_o, scales_o = oracle.mxfp4_quantize(y)
+    x = bits_to_torch_cuda(x_bits)
+    codes, scales = fq.quantize_mxfp4(x)
+    torch.cuda.synchronize()
+    assert_bitexact("codes", to_np(codes), codes_o)
+    assert_bitexact("scales", to_np(scales), scales_o)
+
+
+# ----------------------------------------------------------------------------- NVFP4
+
+NV_SHAPES = [(256, 1024), (37, 1040), (16, 64), (1, 512), (130, 1536), (300, 4096)]
+
+
+@pytest.mark.parametrize("shape", NV_SHAPES)
+@pytest.mark.parametrize("layout", [0, 1])
+@pytest.mark.parametrize("mode", ["dynamic", "static"])
+def test_nvfp4_bitexact(fq, shape, layout, mode):
+    M, K = shape
+    x_bits = workloads.nvfp4_outliers(M, K, seed=M * 7 + K)
+    st = None
+    if mode == "static":
+        st = np.float32(oracle.tensor_scale(oracle.amax(oracle.bf16_to_f32(x_bits))) * np.float32(0.75))
+    codes_o, scales_o, st_o = oracle.quantize_nvfp4(x_bits, st)
+    x = bits_to_torch_cuda(x_bits)
+    codes, scales, sf = fq.quantize_nvfp4(
+        x, None if st is None else torch.tensor([st], device="cuda"), layout)
+    torch.cuda.synchronize()
+    assert_bitexact("tensor scale", to_np(sf)[:1], np.array([st_o], np.float32))
+    assert_bitexact("codes", to_np(codes), codes_o)
+    assert_bitexact("scales", linear_scales(fq, scales, M, K // 16, layout), scales_o)
+
+
+def test_nvfp4_strided_rows_and_zero_tensor(fq):
+    M, K, ld = 40, 512, 640
+    full = workloads.nvfp4_outliers(M, ld, seed=5)
+    x_bits = np.ascontiguousarray(full[:, :K])
+    codes_o, scales_o, st_o = oracle.quantize_nvfp4(x_bits)
+    xt = bits_to_torch_cuda(full)[:, :K]
+    assert xt.stride(0) == ld
+    codes, scales, sf = fq.quantize_nvfp4(xt)
+    torch.cuda.synchronize()
+    assert_bitexact("codes", to_np(codes), codes_o)
+    assert_bitexact("scales", to_np(scales), scales_o)
+    z = torch.zeros((32, 128), dtype=torch.bfloat16, device="cuda")
+    codes, scales, sf = fq.quantize_nvfp4(z)
+    torch.cuda.synchronize()
+    assert to_np(sf)[0] == 0 and not to_np(codes).any() and not to_np(scales).any()
+
+
+# ----------------------------------------------------------------------------- MXFP4
+
+MX_SHAPES = [(4096, 4096), (37, 1056), (16, 64), (129, 2048)]
+
+
+@pytest.mark.parametrize("shape", MX_SHAPES)
+@pytest.mark.parametrize("layout", [0, 1])
+def test_mxfp4_bitexact(fq, shape, layout):
+    M, K = shape
+    x_bits = workloads.mxfp4_student_t(M, K, seed=2 if shape == (4096, 4096) else M + K)
+    codes_o, scales_o = oracle.quantize_mxfp4(x_bits)
+    x = bits_to_torch_cuda(x_bits)
+    codes, scales = fq.quantize_mxfp4(x, layout)
+    torch.cuda.synchronize()
+    assert_bitexact("codes", to_np(codes), codes_o)
+    assert_bitexact("scales", linear_scales(fq, scales, M, K // 32, layout), scales_o)
+
+
+# ----------------------------------------------------------------------------- dual scale
+
+@pytest.mark.parametrize("shape", [(64, 1024), (33, 4096), (16, 128)])
+def test_dual_bitexact(fq, shape):
+    M, K = shape
+    x_bits = workloads.dual_gain(M, K, seed=M + K)
+    codes_o, scales_o, g_o = oracle.dual_quantize(oracle.bf16_to_f32(x_bits))
+    x = bits_to_torch_cuda(x_bits)
+    codes, scales, g = fq.hadamard_quantize(x, 0, fq.FP4Q_NVFP4_DUAL)
+    torch.cuda.synchronize()
+    assert_bitexact("codes", to_np(codes), codes_o)
+    assert_bitexact("scales", to_np(scales), scales_o)
+    assert_bitexact("group scales", to_np(g), g_o)
+
+
+# ----------------------------------------------------------------------------- dequantize
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4", "dual"])
+@pytest.mark.parametrize("layout", [0, 1])
+def test_dequantize_bitexact(fq, fmt, layout):
+    M, K = 70, 2048
+    x_bits = workloads.dual_gain(M, K, seed=9)
+    if fmt == "nvfp4":
+        c, s, sc = oracle.quantize_nvfp4(x_bits)
+        sct = torch.tensor([sc], device="cuda")
+        f, ncols = fq.FP4Q_NVFP4, K // 16
+    elif fmt == "mxfp4":
+        c, s = oracle.quantize_mxfp4(x_bits)
+        sc, sct = None, None
+        f, ncols = fq.FP4Q_MXFP4, K // 32
+    else:
+        c, s, sc = oracle.dual_quantize(oracle.bf16_to_f32(x_bits))
+        sct = torch.from_numpy(sc).cuda()
+        f, ncols = fq.FP4Q_NVFP4_DUAL, K // 16
+    want = oracle.dequantize_bf16(fmt, c, s, sc)
+    s_dev = s if layout == 0 else oracle.swizzle_scales(s)
+    y = fq.dequantize(f, torch.from_numpy(c).cuda(), torch.from_numpy(s_dev).cuda(), sct, K, layout)
+    torch.cuda.synchronize()
+    assert_bitexact("dequant", bf16_torch_to_bits(y), want)
+
+
+# ----------------------------------------------------------------------------- Hadamard
+
+@pytest.mark.parametrize("n", [16, 32, 64, 128, 256, 512])
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4", "dual"])
+def test_hadamard_quantize_tolerance(fq, n, fmt):
+    M, K = 40, 2048
+    x_bits = workloads.hadamard_channels(M, K, seed=n)
+    fcode = {"nvfp4": fq.FP4Q_NVFP4, "mxfp4": fq.FP4Q_MXFP4, "dual": fq.FP4Q_NVFP4_DUAL}[fmt]
+    codes, scales, sf = fq.hadamard_quantize(bits_to_torch_cuda(x_bits), n, fcode)
+    torch.cuda.synchronize()
+    c_o, s_o, sc_o, y_o = oracle.hadamard_quantize(x_bits, n, fmt)
+    if fmt == "nvfp4":
+        # tensor scale: amax of the rotated tensor / 2688, GPU rotation in fp32
+        assert abs(float(to_np(sf)[0]) - float(sc_o)) <= 4e-7 * float(sc_o)
+        gpu = (to_np(codes), to_np(scales), to_np(sf))
+    elif fmt == "dual":
+        g = to_np(sf)
+        np.testing.assert_allclose(g, sc_o, rtol=4e-7)
+        gpu = (to_np(codes), to_np(scales), g)
+    else:
+        gpu = (to_np(codes), to_np(scales), None)
+    assert_tolerant(fmt, K, gpu, (c_o, s_o, sc_o), y_o, name=f"had{n}-{fmt}")
+
+
+def test_hadamard_static_scale(fq):
+    M, K, n = 48, 1024, 128
+    x_bits = workloads.hadamard_channels(M, K, seed=77)
+    ts = np.float32(0.05)
+    codes, scales, sf = fq.hadamard_quantize(bits_to_torch_cuda(x_bits), n, fq.FP4Q_NVFP4,
+                                             torch.tensor([ts], device="cuda"))
+    torch.cuda.synchronize()
+    c_o, s_o, sc_o, y_o = oracle.hadamard_quantize(x_bits, n, "nvfp4", s_t=ts)
+    assert to_np(sf)[0] == ts
+    assert_tolerant("nvfp4", K, (to_np(codes), to_np(scales), to_np(sf)), (c_o, s_o, sc_o), y_o)
+
+
+@pytest.mark.parametrize("n", [16, 32, 64, 128, 256, 512])
+@pytest.mark.parametrize("fmt", ["nvfp4", "dual"])
+def test_dequantize_inverse_hadamard(fq, n, fmt):
+    M, K = 33, 1024
+    x_bits = workloads.dual_gain(M, K, seed=n + 1)
+    if fmt == "nvfp4":
+        c, s, sc, _ = oracle.hadamard_quantize(x_bits, n, "nvfp4")
+        sct, f = torch.tensor([sc], device="cuda"), fq.FP4Q_NVFP4
+    else:
+        c, s, sc, _ = oracle.hadamard_quantize(x_bits, n, "dual")
+        sct, f = torch.from_numpy(sc).cuda(), fq.FP4Q_NVFP4_DUAL
+    want = oracle.bf16_to_f32(oracle.dequantize_bf16(fmt, c, s, sc, inv_had=n)).astype(np.float64)
+    y = fq.dequantize(f, torch.from_numpy(c).cuda(), torch.from_numpy(s).cuda(), sct, K, 0, n)
+    torch.cuda.synchronize()
+    got = oracle.bf16_to_f32(bf16_torch_to_bits(y)).astype(np.float64)
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(want), np.abs(got)) + 1e-300)) - 7)
+    diff = np.abs(got - want)
+    assert np.all(diff <= ulp * 1.0001), "more than one bf16 ulp apart"
+    assert (diff > 0).mean() <= 1e-3
+
+
+# ----------------------------------------------------------------------------- ARC
+
+def arc_case(fq, M, K, S, seed, static=False, layout=0):
+    x_bits, gamma, perm, outl = workloads.arc_activations(M, K, seed=seed, S=S)
+    ts = None
+    if static:
+        ts = np.float32(0.01)
+    codes, scales, sf = fq.arc_quantize(
+        bits_to_torch_cuda(x_bits), bits_to_torch_cuda(gamma), torch.from_numpy(perm).cuda(),
+        torch.from_numpy(outl).cuda(), 1e-6, None if ts is None else torch.tensor([ts], device="cuda"),
+        layout)
+    torch.cuda.synchronize()
+    return x_bits, gamma, perm, outl, ts, codes, scales, sf
+
+
+@pytest.mark.parametrize("shape", [(64, 1024, 64), (37, 4096, 256), (20, 512, 0), (16, 8192, 128)])
+@pytest.mark.parametrize("layout", [0, 1])
+def test_arc_tolerance(fq, shape, layout):
+    M, K, S = shape
+    x_bits, gamma, perm, outl, ts, codes, scales, sf = arc_case(fq, M, K, S, seed=K + S, layout=layout)
+    c_o, s_o, sc_o, y_o = oracle.arc(x_bits, gamma, perm, outl)
+    assert abs(float(to_np(sf)[0]) - float(sc_o)) <= 4e-7 * float(sc_o)
+    s_g = linear_scales(fq, scales, M, (K + S) // 16, layout)
+    # y for the comparator: primary columns then the oracle's residuals
+    dq_o = oracle.nvfp4_dequantize(c_o, s_o, sc_o)
+    res_o = y_o[:, outl] - dq_o[:, outl] if S else np.zeros((M, 0), np.float32)
+    y_full = np.concatenate([y_o, res_o], axis=1)
+    assert_tolerant("nvfp4", K + S, (to_np(codes), s_g, to_np(sf)), (c_o, s_o, sc_o), y_full,
+                    name="arc", frac=2e-4)
+
+
+def test_arc_general_outlier_list(fq):
+    """Outlier positions in arbitrary order (not the first S positions)."""
+    M, K, S = 24, 1024, 32
+    x_bits, gamma, perm, _ = workloads.arc_activations(M, K, seed=3, S=S)
+    outl = np.random.default_rng(4).choice(K, S, replace=False).astype(np.int32)
+    codes, scales, sf = fq.arc_quantize(
+        bits_to_torch_cuda(x_bits), bits_to_torch_cuda(gamma), torch.from_numpy(perm).cuda(),
+        torch.from_numpy(outl).cuda(), 1e-6, torch.tensor([0.01], device="cuda"))
+    torch.cuda.synchronize()
+    c_o, s_o, sc_o, y_o = oracle.arc(x_bits, gamma, perm, outl, s_t=0.01)
+    dq_o = oracle.nvfp4_dequantize(c_o, s_o, sc_o)
+    y_full = np.concatenate([y_o, y_o[:, outl] - dq_o[:, outl]], axis=1)
+    assert_tolerant("nvfp4", K + S, (to_np(codes), to_np(scales), to_np(sf)), (c_o, s_o, sc_o),
+                    y_full, name="arc-general", frac=2e-4)
+
+
+# ----------------------------------------------------------------------------- full sizes
+
+def _rows(M, n=64, seed=0):
+    rng = np.random.default_rng(seed)
+    return np.unique(np.concatenate([[0, M - 1], rng.choice(M, n, replace=False)]))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("n", [128, 16, 32])
+def test_full_hadamard_nvfp4_8192x4096(fq, n):
+    x_bits = workloads.hadamard_channels()
+    M, K = x_bits.shape
+    codes, scales, sf = fq.hadamard_quantize(bits_to_torch_cuda(x_bits), n, fq.FP4Q_NVFP4)
+    torch.cuda.synchronize()
+    # exact tensor amax of the rotated tensor (oracle, all rows, in chunks)
+    am = 0.0
+    for r0 in range(0, M, 1024):
+        am = max(am, oracle.amax(oracle.hadamard(oracle.bf16_to_f32(x_bits[r0:r0 + 1024]), n)))
+    st_o = oracle.tensor_scale(am)
+    assert abs(float(to_np(sf)[0]) - st_o) <= 4e-7 * st_o
+    rows = _rows(M, 96, n)
+    c_o, s_o, _, y_o = oracle.hadamard_quantize(x_bits[rows], n, "nvfp4", s_t=st_o)
+    gpu = (to_np(codes)[rows], to_np(scales)[rows], to_np(sf))
+    assert_tolerant("nvfp4", K, gpu, (c_o, s_o, np.float32(st_o)), y_o, name=f"full-had{n}")
+
+
+@pytest.mark.slow
+def test_full_arc_8192x4096(fq):
+    M, K, S = 8192, 4096, 256
+    x_bits, gamma, perm, outl, ts, codes, scales, sf = arc_case(fq, M, K, S, seed=4)
+    am = 0.0
+    for r0 in range(0, M, 2048):
+        am = max(am, oracle.amax(oracle.arc_prepare(x_bits[r0:r0 + 2048], gamma, perm)))
+    st_o = oracle.tensor_scale(am)
+    assert abs(float(to_np(sf)[0]) - st_o) <= 4e-7 * st_o
+    rows = _rows(M, 128, 4)
+    c_o, s_o, _, y_o = oracle.arc(x_bits[rows], gamma, perm, outl, s_t=st_o)
+    dq_o = oracle.nvfp4_dequantize(c_o, s_o, st_o)
+    y_full = np.concatenate([y_o, y_o[:, outl] - dq_o[:, outl]], axis=1)
+    assert_tolerant("nvfp4", K + S, (to_np(codes)[rows], to_np(scales)[rows], to_np(sf)),
+                    (c_o, s_o, np.float32(st_o)), y_full, name="full-arc", frac=2e-4)
+
+
+@pytest.mark.slow
+def test_full_dual_fwht512_round_trip_32768x4096(fq):
+    x_bits = workloads.dual_gain()
+    M, K = x_bits.shape
+    x = bits_to_torch_cuda(x_bits)
+    codes, scales, g = fq.hadamard_quantize(x, 512, fq.FP4Q_NVFP4_DUAL)
+    y = fq.dequantize(fq.FP4Q_NVFP4_DUAL, codes, scales, g, K, 0, 512)
+    torch.cuda.synchronize()
+    rows = _rows(M, 64, 5)
+    c_o, s_o, g_o, y_o = oracle.hadamard_quantize(x_bits[rows], 512, "dual")
+    gg = to_np(g)[rows]
+    np.testing.assert_allclose(gg, g_o, rtol=4e-7)
+    assert_tolerant("dual", K, (to_np(codes)[rows], to_np(scales)[rows], gg), (c_o, s_o, g_o), y_o,
+                    name="full-dual")
+    # round trip of the GPU's own codes against the oracle's dequantizer on them
+    want = oracle.bf16_to_f32(oracle.dequantize_bf16("dual", to_np(codes)[rows], to_np(scales)[rows],
+                                                     gg, inv_had=512)).astype(np.float64)
+    got = oracle.bf16_to_f32(bf16_torch_to_bits(y)[rows]).astype(np.float64)
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(want), np.abs(got)) + 1e-300)) - 7)
+    assert np.all(np.abs(got - want) <= ulp * 1.0001)
+    assert (got != want).mean() <= 1e-3
