@@ -115,3 +115,26 @@ def assert_tolerant(fmt: str, K: int, gpu, orc, y_orc: np.ndarray, *, frac: floa
         bound = np.where(v > 6, (v - 6 + 1e-3) * dg[scale_diff], (step / 2 + 1e-3) * dg[scale_diff])
         assert np.all(err <= bound * (1 + 1e-6)), f"{name}: error bound violated in rescaled blocks"
     return {"codes_off": nbad, "blocks_rescaled": n_blocks_diff, "n": n}
+
+
+def assert_roundtrip_close(got_bits: np.ndarray, want_bits: np.ndarray, n: int, name: str = "",
+                           max_frac: float = 1e-3):
+    """bf16 outputs of an inverse-Hadamard dequantizer against the oracle's.
+
+    The GPU rotates in fp32 butterflies, the oracle in binary64 rounded once;
+    the difference before the final bf16 rounding is a few fp32 ulps of the
+    Hadamard block's magnitude.  So each element may differ by one bf16 ulp of
+    itself (a rounding flip) plus 2^-18 of the block's largest magnitude (a
+    cancelled, near-zero element), and at most `max_frac` of them may differ."""
+    got = oracle.bf16_to_f32(got_bits).astype(np.float64)
+    want = oracle.bf16_to_f32(want_bits).astype(np.float64)
+    M, K = want.shape
+    blk = np.abs(want).reshape(M, K // n, n).max(axis=2)
+    blk = np.repeat(blk, n, axis=1)
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(want), np.abs(got)) + 1e-300)) - 7)
+    diff = np.abs(got - want)
+    bound = ulp + 2.0 ** -18 * blk
+    bad = diff > bound
+    assert not bad.any(), (f"{name}: {int(bad.sum())} elements beyond one bf16 ulp; first "
+                           f"{np.argwhere(bad)[0]}: got {got[bad][0]} want {want[bad][0]}")
+    assert (diff > 0).mean() <= max_frac, f"{name}: {(diff > 0).mean():.2e} of elements differ"

@@ -11,8 +11,8 @@ import torch
 
 import oracle
 import workloads
-from parity import (assert_bitexact, assert_tolerant, bf16_torch_to_bits, bits_to_torch_cuda,
-                    to_np, unswizzle)
+from parity import (assert_bitexact, assert_roundtrip_close, assert_tolerant, bf16_torch_to_bits,
+                    bits_to_torch_cuda, to_np, unswizzle)
 
 pytestmark = pytest.mark.gpu
 
@@ -242,14 +242,10 @@ def test_dequantize_inverse_hadamard(fq, n, fmt):
     else:
         c, s, sc, _ = oracle.hadamard_quantize(x_bits, n, "dual")
         sct, f = torch.from_numpy(sc).cuda(), fq.FP4Q_NVFP4_DUAL
-    want = oracle.bf16_to_f32(oracle.dequantize_bf16(fmt, c, s, sc, inv_had=n)).astype(np.float64)
+    want = oracle.dequantize_bf16(fmt, c, s, sc, inv_had=n)
     y = fq.dequantize(f, torch.from_numpy(c).cuda(), torch.from_numpy(s).cuda(), sct, K, 0, n)
     torch.cuda.synchronize()
-    got = oracle.bf16_to_f32(bf16_torch_to_bits(y)).astype(np.float64)
-    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(want), np.abs(got)) + 1e-300)) - 7)
-    diff = np.abs(got - want)
-    assert np.all(diff <= ulp * 1.0001), "more than one bf16 ulp apart"
-    assert (diff > 0).mean() <= 1e-3
+    assert_roundtrip_close(bf16_torch_to_bits(y), want, n, name=f"inv-had{n}-{fmt}")
 
 
 # ----------------------------------------------------------------------------- ARC
@@ -357,9 +353,5 @@ def test_full_dual_fwht512_round_trip_32768x4096(fq):
     assert_tolerant("dual", K, (to_np(codes)[rows], to_np(scales)[rows], gg), (c_o, s_o, g_o), y_o,
                     name="full-dual")
     # round trip of the GPU's own codes against the oracle's dequantizer on them
-    want = oracle.bf16_to_f32(oracle.dequantize_bf16("dual", to_np(codes)[rows], to_np(scales)[rows],
-                                                     gg, inv_had=512)).astype(np.float64)
-    got = oracle.bf16_to_f32(bf16_torch_to_bits(y)[rows]).astype(np.float64)
-    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(want), np.abs(got)) + 1e-300)) - 7)
-    assert np.all(np.abs(got - want) <= ulp * 1.0001)
-    assert (got != want).mean() <= 1e-3
+    want = oracle.dequantize_bf16("dual", to_np(codes)[rows], to_np(scales)[rows], gg, inv_had=512)
+    assert_roundtrip_close(bf16_torch_to_bits(y)[rows], want, 512, name="full-dual-roundtrip")
