@@ -199,7 +199,8 @@ fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, in
     p.swizzled = layout == FP4Q_SCALES_SWIZZLED;
     p.dynamic = dynamic;
     p.had_norm = had_norm(had);
-    const int grid = (int)std::min<int64_t>({p.n_tiles, (int64_t)2 * sms, (int64_t)kMaxGrid});
+    const int grid =
+        (int)std::min<int64_t>({p.n_tiles, (int64_t)kQuantCtasPerSm * sms, (int64_t)kMaxGrid});
     p.n_partials = grid;
 
     if (p.swizzled) {  // padding rows/columns of the tiled layout read as zero
@@ -414,7 +415,8 @@ FP4Q_API fp4q_status fp4q_dequantize(fp4q_format format, const uint8_t* codes,
     p.y = static_cast<uint16_t*>(y);
     p.swizzled = layout == FP4Q_SCALES_SWIZZLED;
     p.had_norm = had_norm(inv_had_size);
-    const int grid = (int)std::min<int64_t>({p.n_tiles, (int64_t)4 * sms, (int64_t)kMaxGrid});
+    const int grid =
+        (int)std::min<int64_t>({p.n_tiles, (int64_t)kDequantCtasPerSm * sms, (int64_t)kMaxGrid});
     cudaStream_t s = (cudaStream_t)stream;
     switch (fmt) {
         case FMT_NVFP4: return launch_dequant_h<FMT_NVFP4>(inv_had_size, p, grid, s);

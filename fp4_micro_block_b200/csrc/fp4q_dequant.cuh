@@ -27,60 +27,82 @@ struct DequantParams {
     float had_norm;
 };
 
-template <int FMT>
-__device__ __forceinline__ void decode_unit(const DequantParams& p, int64_t row, int64_t col,
-                                            int nval, float* v) {
-    const uint8_t* cp = p.codes + row * (p.K / 2) + col / 2;
+// Raw bytes of one 32-column unit: packed codes, its scale byte(s) and the fp32
+// scale, loaded one tile ahead of their use (software pipelining).
+struct RawUnit {
     uint32_t w[4];
+    uint32_t e0, e1;
+    float s;
+};
+
+template <int FMT>
+__device__ __forceinline__ void load_raw(const DequantParams& p, int64_t row, int64_t col, int nval,
+                                         RawUnit& u) {
+    const uint8_t* cp = p.codes + row * (p.K / 2) + col / 2;
     if ((p.K & 31) == 0) {
         uint4 q = __ldg(reinterpret_cast<const uint4*>(cp));
-        w[0] = q.x; w[1] = q.y; w[2] = q.z; w[3] = q.w;
+        u.w[0] = q.x; u.w[1] = q.y; u.w[2] = q.z; u.w[3] = q.w;
     } else {
         uint2 q = __ldg(reinterpret_cast<const uint2*>(cp));
-        w[0] = q.x; w[1] = q.y;
+        u.w[0] = q.x; u.w[1] = q.y;
         if (nval > 16) {
             uint2 q2 = __ldg(reinterpret_cast<const uint2*>(cp + 8));
-            w[2] = q2.x; w[3] = q2.y;
+            u.w[2] = q2.x; u.w[3] = q2.y;
         } else {
-            w[2] = 0u; w[3] = 0u;
+            u.w[2] = 0u; u.w[3] = 0u;
         }
     }
+    if constexpr (FMT == FMT_MXFP4) {
+        const int64_t nsc = p.K / 32, c0 = col / 32;
+        u.e0 = p.swizzled ? __ldg(p.scales + swizzle_offset(row, c0, (nsc + 3) / 4))
+                          : __ldg(p.scales + row * nsc + c0);
+        u.e1 = 0u;
+        u.s = 0.0f;
+    } else {
+        const int64_t nsc = p.K / 16, c0 = col / 16;
+        u.e1 = 0u;
+        if (p.swizzled) {
+            const int64_t nC = (nsc + 3) / 4;
+            u.e0 = __ldg(p.scales + swizzle_offset(row, c0, nC));
+            if (nval > 16) u.e1 = __ldg(p.scales + swizzle_offset(row, c0 + 1, nC));
+        } else {
+            u.e0 = __ldg(p.scales + row * nsc + c0);
+            if (nval > 16) u.e1 = __ldg(p.scales + row * nsc + c0 + 1);
+        }
+        u.s = (FMT == FMT_DUAL) ? __ldg(p.scale_fp32 + row * (p.K / 128) + col / 128)
+                                : __ldg(p.scale_fp32);
+    }
+}
+
+template <int FMT>
+__device__ __forceinline__ void decode_raw(const RawUnit& u, float* v) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-        float2 c = e2m1x2_decode((w[i >> 2] >> (8 * (i & 3))) & 0xffu);
+        float2 c = e2m1x2_decode((u.w[i >> 2] >> (8 * (i & 3))) & 0xffu);
         v[2 * i] = c.x;
         v[2 * i + 1] = c.y;
     }
     if constexpr (FMT == FMT_MXFP4) {
-        const int64_t nsc = p.K / 32, c0 = col / 32;
-        const uint32_t b = p.swizzled ? p.scales[swizzle_offset(row, c0, (nsc + 3) / 4)]
-                                      : p.scales[row * nsc + c0];
+        const uint32_t b = u.e0;
         const float sc = b ? __uint_as_float(b << 23) : __uint_as_float(0x00400000u);  // 2^(b-127)
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] *= sc;
     } else {
-        const int64_t nsc = p.K / 16, c0 = col / 16;
-        uint32_t e0, e1 = 0;
-        if (p.swizzled) {
-            const int64_t nC = (nsc + 3) / 4;
-            e0 = p.scales[swizzle_offset(row, c0, nC)];
-            if (nval > 16) e1 = p.scales[swizzle_offset(row, c0 + 1, nC)];
-        } else {
-            e0 = p.scales[row * nsc + c0];
-            if (nval > 16) e1 = p.scales[row * nsc + c0 + 1];
-        }
-        const float s = (FMT == FMT_DUAL) ? p.scale_fp32[row * (p.K / 128) + col / 128]
-                                          : p.scale_fp32[0];
-        const float ev0 = e4m3_decode(e0), ev1 = e4m3_decode(e1);
+        const float ev0 = e4m3_decode(u.e0), ev1 = e4m3_decode(u.e1);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = (v[i] * ev0) * s;
+        for (int i = 0; i < 16; ++i) v[i] = (v[i] * ev0) * u.s;
 #pragma unroll
-        for (int i = 16; i < 32; ++i) v[i] = (v[i] * ev1) * s;
+        for (int i = 16; i < 32; ++i) v[i] = (v[i] * ev1) * u.s;
     }
 }
 
+#ifndef FP4Q_DEQUANT_CTAS_PER_SM
+#define FP4Q_DEQUANT_CTAS_PER_SM 4
+#endif
+constexpr int kDequantCtasPerSm = FP4Q_DEQUANT_CTAS_PER_SM;
+
 template <int FMT, int HAD>
-__global__ void __launch_bounds__(kThreads, 2) dequant_kernel(const DequantParams p) {
+__global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_kernel(const DequantParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     float* scratch = reinterpret_cast<float*>(smem_raw);
     const uint32_t tid = threadIdx.x;
@@ -88,19 +110,40 @@ __global__ void __launch_bounds__(kThreads, 2) dequant_kernel(const DequantParam
     const uint32_t r = (lane & 7) + 8 * (warp & 1);
     const uint32_t j = (lane >> 3) + 4 * (warp >> 1);
 
-    for (int64_t t = blockIdx.x; t < p.n_tiles; t += gridDim.x) {
+    // Unit coordinates of tile t for this thread.
+    auto coords = [&](int64_t t, int64_t& row, int64_t& col, int& nval) {
         const int64_t rt = t / p.n_col_tiles, ct = t % p.n_col_tiles;
-        const int64_t row = rt * kTileRows + r;
-        const int64_t col = ct * kTileCols + 32 * (int64_t)j;
-        const bool live = row < p.M && col < p.K;
-        const int nval = live ? (int)min64(32, p.K - col) : 0;
+        row = rt * kTileRows + r;
+        col = ct * kTileCols + 32 * (int64_t)j;
+        nval = (row < p.M && col < p.K) ? (int)min64(32, p.K - col) : 0;
+    };
+    RawUnit cur{};
+    int64_t row, col;
+    int nval;
+    if ((int64_t)blockIdx.x < p.n_tiles) {
+        coords(blockIdx.x, row, col, nval);
+        if (nval) load_raw<FMT>(p, row, col, nval, cur);
+    }
+    for (int64_t t = blockIdx.x; t < p.n_tiles; t += gridDim.x) {
+        coords(t, row, col, nval);
+        const int64_t ct = t % p.n_col_tiles;
+        // issue the next tile's loads before working on this one
+        RawUnit nxt{};
+        if (t + gridDim.x < p.n_tiles) {
+            int64_t row2, col2;
+            int nval2;
+            coords(t + gridDim.x, row2, col2, nval2);
+            if (nval2) load_raw<FMT>(p, row2, col2, nval2, nxt);
+        }
+        const bool live = nval > 0;
         float v[32];
         if (live) {
-            decode_unit<FMT>(p, row, col, nval, v);
+            decode_raw<FMT>(cur, v);
         } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0.0f;
         }
+        cur = nxt;
         uint16_t* yrow = p.y + row * p.K;
 
         if constexpr (HAD <= 32) {

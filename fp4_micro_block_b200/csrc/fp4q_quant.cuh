@@ -24,6 +24,13 @@
 
 namespace fp4q {
 
+#ifndef FP4Q_STAGES
+#define FP4Q_STAGES 4
+#endif
+#ifndef FP4Q_QUANT_CTAS_PER_SM
+#define FP4Q_QUANT_CTAS_PER_SM 2
+#endif
+
 constexpr int kThreads = 256;
 constexpr int kTileRows = 16;
 constexpr int kTileCols = 512;
@@ -31,7 +38,8 @@ constexpr int kBoxCols = 64;
 constexpr int kBoxes = kTileCols / kBoxCols;            // 8
 constexpr int kBoxBytes = kTileRows * kBoxCols * 2;     // 2048
 constexpr int kTileBytes = kTileRows * kTileCols * 2;   // 16384
-constexpr int kStages = 4;
+constexpr int kStages = FP4Q_STAGES;                    // tiles in the shared-memory ring
+constexpr int kQuantCtasPerSm = FP4Q_QUANT_CTAS_PER_SM;
 constexpr int kScratchBytes = kTileRows * kTileCols * 4;  // fp32 exchange, 32 KiB
 
 enum : int { FMT_NVFP4 = 0, FMT_MXFP4 = 1, FMT_DUAL = 2 };
@@ -214,7 +222,7 @@ __device__ __forceinline__ float tensor_scale_from_partials(const float* partial
 }
 
 template <int FMT, int HAD, bool AMAX_ONLY>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, kQuantCtasPerSm)
     quant_kernel(const __grid_constant__ CUtensorMap tmap_x, const QuantParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned stage ring, then the exchange scratch, then barriers.

@@ -118,14 +118,20 @@ def assert_tolerant(fmt: str, K: int, gpu, orc, y_orc: np.ndarray, *, frac: floa
 
 
 def assert_roundtrip_close(got_bits: np.ndarray, want_bits: np.ndarray, n: int, name: str = "",
-                           max_frac: float = 1e-3):
+                           max_frac: float = 3e-2):
     """bf16 outputs of an inverse-Hadamard dequantizer against the oracle's.
 
     The GPU rotates in fp32 butterflies, the oracle in binary64 rounded once;
     the difference before the final bf16 rounding is a few fp32 ulps of the
     Hadamard block's magnitude.  So each element may differ by one bf16 ulp of
     itself (a rounding flip) plus 2^-18 of the block's largest magnitude (a
-    cancelled, near-zero element), and at most `max_frac` of them may differ."""
+    cancelled, near-zero element), and at most `max_frac` of them may differ.
+    The dequantized inputs carry only a few significant bits, so binary64 sums
+    are often exact where fp32 butterflies are not, and single-ulp bf16 flips
+    are far more frequent than for random data: about 1.3% of the outputs for
+    n = 16 when the fp32 butterflies are replayed on the host in numpy.  The
+    element-wise one-ulp bound is the check that catches a wrong sign, index
+    or scale."""
     got = oracle.bf16_to_f32(got_bits).astype(np.float64)
     want = oracle.bf16_to_f32(want_bits).astype(np.float64)
     M, K = want.shape
