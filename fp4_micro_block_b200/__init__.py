@@ -4,8 +4,9 @@ The entry points below carry the C names of ``include/fp4q.h`` and only
 marshal arguments: torch tensors become device pointers, the current torch CUDA
 stream becomes the ``stream`` argument, and a non-zero status raises
 ``Fp4qError``.  Every step of the computation runs in the library's kernels;
-there is no CPU or PyTorch fallback.  Importing this module without the built
-library raises ImportError (build it with ``python -m fp4_micro_block_b200.build``).
+there is no CPU or PyTorch fallback.  The library is loaded on first use; if it
+has not been built, that first call raises ImportError (build it with
+``python -m fp4_micro_block_b200.build``).
 
 Helpers at the bottom (``quantize_nvfp4`` ...) only allocate the output tensors
 with torch and call the entry points.
@@ -29,7 +30,7 @@ FP4Q_TSCALE_DYNAMIC, FP4Q_TSCALE_STATIC = 0, 1
 FP4Q_WORKSPACE_BYTES = 16384
 
 EXPORTED = [
-    "fp4q_quantize_nvfp4", "fp4q_quantize_mxfp4", "fp4q_hadamard_quantize", "fp4q_arc_quantize",
+    "fp4q_quantize_nvfp4", "fp4q_quantize_nvfp4_noalloc", "fp4q_quantize_mxfp4", "fp4q_hadamard_quantize", "fp4q_arc_quantize",
     "fp4q_dequantize", "fp4q_workspace_bytes", "fp4q_scales_bytes", "fp4q_status_string",
     "fp4q_device_error", "fp4q_selftest_div",
 ]
@@ -48,6 +49,7 @@ def _load() -> C.CDLL:
     p, i64, f32, i32, sz = C.c_void_p, C.c_int64, C.c_float, C.c_int, C.c_size_t
     sigs = {
         "fp4q_quantize_nvfp4": (i32, [p, i64, i64, i64, p, p, p, i32, i32, p, sz, p]),
+        "fp4q_quantize_nvfp4_noalloc": (i32, [p, i64, i64, i64, p, p, p, i32, p]),
         "fp4q_quantize_mxfp4": (i32, [p, i64, i64, i64, p, p, i32, p]),
         "fp4q_hadamard_quantize": (i32, [p, i64, i64, i64, i32, i32, p, p, p, i32, i32, p, sz, p]),
         "fp4q_arc_quantize": (i32, [p, i64, i64, i64, p, f32, p, p, i64, p, p, p, i32, i32, p, sz, p]),
@@ -65,10 +67,21 @@ def _load() -> C.CDLL:
     return L
 
 
-_lib = _load()
+class _Lazy:
+    """Loads libfp4q.so on first attribute access."""
+
+    _cdll = None
+
+    def __getattr__(self, name):
+        if _Lazy._cdll is None:
+            _Lazy._cdll = _load()
+        return getattr(_Lazy._cdll, name)
 
 
-def lib() -> C.CDLL:
+_lib = _Lazy()
+
+
+def lib():
     return _lib
 
 
@@ -121,6 +134,14 @@ def fp4q_quantize_nvfp4(x, codes, scales, tensor_scale, mode=FP4Q_TSCALE_DYNAMIC
     return _check(_lib.fp4q_quantize_nvfp4(_ptr(x), M, K, _ld(x), _ptr(codes), _ptr(scales),
                                            _ptr(tensor_scale), mode, layout, _ptr(workspace),
                                            ws_bytes, _stream(stream)), "fp4q_quantize_nvfp4")
+
+
+def fp4q_quantize_nvfp4_noalloc(x, codes, scales, tensor_scale, layout=FP4Q_SCALES_LINEAR,
+                                stream=None):
+    M, K = x.shape
+    return _check(_lib.fp4q_quantize_nvfp4_noalloc(_ptr(x), M, K, _ld(x), _ptr(codes), _ptr(scales),
+                                                   _ptr(tensor_scale), layout, _stream(stream)),
+                  "fp4q_quantize_nvfp4_noalloc")
 
 
 def fp4q_quantize_mxfp4(x, codes, scales, layout=FP4Q_SCALES_LINEAR, stream=None):

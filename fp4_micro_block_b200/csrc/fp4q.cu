@@ -261,6 +261,36 @@ __global__ void selftest_div_kernel(const float* x, const float* d, int64_t n, f
 
 }  // namespace
 
+// ---------------------------------------------------------------- allocation-free variant
+// Scratch of fp4q_quantize_nvfp4_noalloc: the per-CTA partial maxima of the
+// tensor-scale pre-pass, in static device memory instead of a caller-supplied
+// workspace.  Every GPU that loads the library keeps these 16 KiB until the
+// process exits.  In host code the symbol is only a stand-in; the kernels get
+// the device address that cudaGetSymbolAddress returns for the current device.
+constexpr int kNoAllocPartials = 4096;
+static_assert(kNoAllocPartials >= kMaxGrid, "scratch must hold one partial per pre-pass CTA");
+static __device__ __align__(256) float g_noalloc_partials[kNoAllocPartials];
+
+namespace {
+std::atomic<float*> g_noalloc_ptr[kMaxDevices];
+
+// Device address of the scratch on the current device, looked up once per device.
+fp4q_status noalloc_scratch(float** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FP4Q_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return FP4Q_ERR_UNSUPPORTED;
+    float* ptr = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+    if (!ptr) {
+        void* a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_noalloc_partials) != cudaSuccess || !a) return FP4Q_ERR_CUDA;
+        ptr = static_cast<float*>(a);
+        g_noalloc_ptr[dev].store(ptr, std::memory_order_release);
+    }
+    *out = ptr;
+    return FP4Q_OK;
+}
+}  // namespace
+
 // ==================================================================== C ABI
 
 FP4Q_API size_t fp4q_workspace_bytes(int64_t M, int64_t K) {
@@ -283,6 +313,28 @@ FP4Q_API fp4q_status fp4q_quantize_nvfp4(const void* x, int64_t M, int64_t K, in
                                          fp4q_stream_t stream) {
     return quantize_common(x, M, K, ldx, 0, FMT_NVFP4, codes, scales, tensor_scale, mode, layout,
                            workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+FP4Q_API fp4q_status fp4q_quantize_nvfp4_noalloc(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                                 uint8_t* codes, uint8_t* scales,
+                                                 float* tensor_scale, fp4q_scale_layout layout,
+                                                 fp4q_stream_t stream) {
+    fp4q_status st = check_x(x, M, K, ldx);
+    if (st != FP4Q_OK) return st;
+    if (K % 16 != 0) return FP4Q_ERR_INVALID_ARG;
+    if (M == 0) return FP4Q_OK;
+    int sms = 0;
+    if ((st = sm_count(&sms)) != FP4Q_OK) return st;
+    // One partial maximum per pre-pass CTA; the grid is capped below the scratch size,
+    // so this only trips if that cap is ever raised.
+    const int64_t n_tiles = ((M + kTileRows - 1) / kTileRows) * ((K + kTileCols - 1) / kTileCols);
+    const int64_t grid = std::min<int64_t>({n_tiles, (int64_t)kQuantCtasPerSm * sms, (int64_t)kMaxGrid});
+    if (grid > kNoAllocPartials) return FP4Q_ERR_UNSUPPORTED;
+    float* scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != FP4Q_OK) return st;
+    return quantize_common(x, M, K, ldx, 0, FMT_NVFP4, codes, scales, tensor_scale,
+                           FP4Q_TSCALE_DYNAMIC, layout, scratch,
+                           (size_t)kNoAllocPartials * sizeof(float), (cudaStream_t)stream);
 }
 
 FP4Q_API fp4q_status fp4q_quantize_mxfp4(const void* x, int64_t M, int64_t K, int64_t ldx,

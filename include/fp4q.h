@@ -116,6 +116,32 @@ fp4q_status fp4q_quantize_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx
                                 void* workspace, size_t workspace_bytes,
                                 fp4q_stream_t stream);
 
+/* fp4q_quantize_nvfp4_noalloc -- fp4q_quantize_nvfp4 in DYNAMIC tensor-scale
+ * mode for callers that cannot allocate device memory: for example a host
+ * framework that hands the library only its input and output tensors and gives
+ * plugins no device allocator, or a service that fixes its device memory at
+ * start-up and may not grow it afterwards.  Such a caller has no way to provide
+ * the `workspace` of the dynamic mode, so this variant keeps that scratch (the
+ * per-CTA partial maxima of the amax pre-pass) in a 16 KiB array of static
+ * device memory inside the library, which every GPU that loads the library
+ * holds until the process exits.  It calls no cudaMalloc, cudaFree or other
+ * allocating routine.  (Not a method of the pages: they have no counterpart.)
+ *   Arguments and results are those of fp4q_quantize_nvfp4 with
+ *   mode = FP4Q_TSCALE_DYNAMIC: *tensor_scale is written.
+ *   Limit: at most 4096 partial maxima; the pre-pass grid never exceeds 4096
+ *   CTAs, so every M and K accepted by fp4q_quantize_nvfp4 fits, and a grid
+ *   above the limit would return FP4Q_ERR_UNSUPPORTED.
+ *   Set-up: the first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   Sharing: every call on a device uses the same array, which keeps the last
+ *   call's contents.  Nothing in it needs clearing (each call's pre-pass writes
+ *   every entry its quantizer reads), but calls that overlap on the GPU (for
+ *   example on two streams at once) race on it and must be serialised. */
+fp4q_status fp4q_quantize_nvfp4_noalloc(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                        uint8_t* codes, uint8_t* scales, float* tensor_scale,
+                                        fp4q_scale_layout layout, fp4q_stream_t stream);
+
 /* fp4q_quantize_mxfp4 -- MXFP4 quantization of a bf16 matrix.
  *   x       bf16 [M, ldx].                     (read)
  *   codes   uint8 [M, K/2].                    (written)
