@@ -66,15 +66,15 @@ fp4q_status encode_fn(EncodeTiledFn* out) {
     return FP4Q_OK;
 }
 
-// bf16 [M, K] with row stride ldx elements; boxes of 64 columns x 16 rows,
-// 128-byte swizzle, zero fill outside the matrix.
+// bf16 [M, K] with row stride ldx elements; boxes of 64 columns x 8 rows (the
+// G2 warp-tile halves), 128-byte swizzle, zero fill outside the matrix.
 fp4q_status make_x_map(CUtensorMap* map, const void* x, int64_t M, int64_t K, int64_t ldx) {
     EncodeTiledFn enc;
     fp4q_status st = encode_fn(&enc);
     if (st != FP4Q_OK) return st;
     cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
     cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
-    cuuint32_t box[2] = {(cuuint32_t)kBoxCols, (cuuint32_t)kTileRows};
+    cuuint32_t box[2] = {64u, 8u};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -127,28 +127,58 @@ fp4q_status ensure_smem(Kern kern, int bytes, std::atomic<uint64_t>& done) {
 }
 
 // ---------------------------------------------------------------- quantizer launch
+// Resident CTAs per SM of a kernel, looked up once per device.
+template <typename Kern>
+fp4q_status resident_ctas(Kern kern, int smem, std::atomic<int>* cache, int* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FP4Q_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return FP4Q_ERR_UNSUPPORTED;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n <= 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kQuantThreads, smem) != cudaSuccess)
+            return FP4Q_ERR_CUDA;
+        if (n <= 0) return FP4Q_ERR_UNSUPPORTED;
+        cache[dev].store(n, std::memory_order_relaxed);
+    }
+    *out = n;
+    return FP4Q_OK;
+}
+
+// Launches quant_kernel<FMT, HAD, AMAX> persistently (resident CTAs x SMs, at most
+// one warp per warp tile); returns the grid through *grid_out.
 template <int FMT, int HAD, bool AMAX>
-fp4q_status launch_quant_t(const CUtensorMap& map, const QuantParams& p, int grid, cudaStream_t s) {
+fp4q_status launch_quant_t(const CUtensorMap& map, QuantParams p, int sms, cudaStream_t s,
+                           int* grid_out) {
+    using G = Geo<HAD>;
     auto kern = quant_kernel<FMT, HAD, AMAX>;
     constexpr int smem = quant_smem_bytes<HAD>();
     static std::atomic<uint64_t> done{0};
+    static std::atomic<int> occ[kMaxDevices];
     fp4q_status st = ensure_smem(kern, smem, done);
     if (st != FP4Q_OK) return st;
-    kern<<<grid, kThreads, smem, s>>>(map, p);
+    int per_sm = 0;
+    if ((st = resident_ctas(kern, smem, occ, &per_sm)) != FP4Q_OK) return st;
+    p.n_rb = (p.M + G::rows - 1) / G::rows;
+    p.n_cb = (p.K + G::cols - 1) / G::cols;
+    p.n_wt = p.n_rb * p.n_cb;
+    const int grid = (int)std::min<int64_t>(
+        {(p.n_wt + kWarps - 1) / kWarps, (int64_t)per_sm * sms, (int64_t)kMaxGrid});
+    kern<<<grid, kQuantThreads, smem, s>>>(map, p);
+    if (grid_out) *grid_out = grid;
     return launch_status();
 }
 
 template <int FMT, bool AMAX>
-fp4q_status launch_quant_h(int had, const CUtensorMap& map, const QuantParams& p, int grid,
-                           cudaStream_t s) {
+fp4q_status launch_quant_h(int had, const CUtensorMap& map, const QuantParams& p, int sms,
+                           cudaStream_t s, int* grid_out) {
     switch (had) {
-        case 0: return launch_quant_t<FMT, 0, AMAX>(map, p, grid, s);
-        case 16: return launch_quant_t<FMT, 16, AMAX>(map, p, grid, s);
-        case 32: return launch_quant_t<FMT, 32, AMAX>(map, p, grid, s);
-        case 64: return launch_quant_t<FMT, 64, AMAX>(map, p, grid, s);
-        case 128: return launch_quant_t<FMT, 128, AMAX>(map, p, grid, s);
-        case 256: return launch_quant_t<FMT, 256, AMAX>(map, p, grid, s);
-        case 512: return launch_quant_t<FMT, 512, AMAX>(map, p, grid, s);
+        case 0: return launch_quant_t<FMT, 0, AMAX>(map, p, sms, s, grid_out);
+        case 16: return launch_quant_t<FMT, 16, AMAX>(map, p, sms, s, grid_out);
+        case 32: return launch_quant_t<FMT, 32, AMAX>(map, p, sms, s, grid_out);
+        case 64: return launch_quant_t<FMT, 64, AMAX>(map, p, sms, s, grid_out);
+        case 128: return launch_quant_t<FMT, 128, AMAX>(map, p, sms, s, grid_out);
+        case 256: return launch_quant_t<FMT, 256, AMAX>(map, p, sms, s, grid_out);
+        case 512: return launch_quant_t<FMT, 512, AMAX>(map, p, sms, s, grid_out);
         default: return FP4Q_ERR_INVALID_ARG;
     }
 }
@@ -184,14 +214,14 @@ fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, in
     int sms = 0;
     if ((st = sm_count(&sms)) != FP4Q_OK) return st;
     CUtensorMap map;
-    if ((st = make_x_map(&map, x, M, K, ldx)) != FP4Q_OK) return st;
+    std::memset(&map, 0, sizeof(map));
+    if (had < 256 && (st = make_x_map(&map, x, M, K, ldx)) != FP4Q_OK) return st;
 
     QuantParams p{};
     p.M = M;
     p.K = K;
-    p.n_row_tiles = (M + kTileRows - 1) / kTileRows;
-    p.n_col_tiles = (K + kTileCols - 1) / kTileCols;
-    p.n_tiles = p.n_row_tiles * p.n_col_tiles;
+    p.x = static_cast<const uint8_t*>(x);
+    p.ldx_bytes = ldx * 2;
     p.codes = codes;
     p.scales = scales;
     p.scale_fp32 = scale_fp32;
@@ -199,9 +229,6 @@ fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, in
     p.swizzled = layout == FP4Q_SCALES_SWIZZLED;
     p.dynamic = dynamic;
     p.had_norm = had_norm(had);
-    const int grid =
-        (int)std::min<int64_t>({p.n_tiles, (int64_t)kQuantCtasPerSm * sms, (int64_t)kMaxGrid});
-    p.n_partials = grid;
 
     if (p.swizzled) {  // padding rows/columns of the tiled layout read as zero
         const int64_t ncols = K / B;
@@ -209,15 +236,16 @@ fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, in
         if (bytes != M * ncols && cudaMemsetAsync(scales, 0, (size_t)bytes, stream) != cudaSuccess)
             return FP4Q_ERR_CUDA;
     }
-    if (dynamic) {
-        st = fmt == FMT_NVFP4 ? launch_quant_h<FMT_NVFP4, true>(had, map, p, grid, stream)
-                              : FP4Q_ERR_INVALID_ARG;
+    if (dynamic) {  // amax pre-pass: one partial maximum per CTA into the workspace
+        int grid_a = 0;
+        st = launch_quant_h<FMT_NVFP4, true>(had, map, p, sms, stream, &grid_a);
         if (st != FP4Q_OK) return st;
+        p.n_partials = grid_a;
     }
     switch (fmt) {
-        case FMT_NVFP4: return launch_quant_h<FMT_NVFP4, false>(had, map, p, grid, stream);
-        case FMT_MXFP4: return launch_quant_h<FMT_MXFP4, false>(had, map, p, grid, stream);
-        case FMT_DUAL: return launch_quant_h<FMT_DUAL, false>(had, map, p, grid, stream);
+        case FMT_NVFP4: return launch_quant_h<FMT_NVFP4, false>(had, map, p, sms, stream, nullptr);
+        case FMT_MXFP4: return launch_quant_h<FMT_MXFP4, false>(had, map, p, sms, stream, nullptr);
+        case FMT_DUAL: return launch_quant_h<FMT_DUAL, false>(had, map, p, sms, stream, nullptr);
         default: return FP4Q_ERR_INVALID_ARG;
     }
 }
@@ -234,12 +262,23 @@ fp4q_status launch_dequant_t(const DequantParams& p, int grid, cudaStream_t s) {
     return launch_status();
 }
 
+// Rotation sizes 0, 16, 32: the streaming kernel, 4 CTAs of 256 threads per SM.
+template <int FMT, int HAD>
+fp4q_status launch_dequant_stream(const DequantParams& p, int sms, cudaStream_t s) {
+    const int64_t units = p.M * ((p.K + 31) / 32);
+    const int grid = (int)std::min<int64_t>({(units + kThreads - 1) / kThreads, (int64_t)3 * sms,
+                                            (int64_t)kMaxGrid});
+    const int w32 = ((reinterpret_cast<uintptr_t>(p.y) & 31) == 0 && (p.K & 15) == 0) ? 1 : 0;
+    dequant_stream_kernel<FMT, HAD><<<grid, kThreads, 0, s>>>(p, w32);
+    return launch_status();
+}
+
 template <int FMT>
-fp4q_status launch_dequant_h(int had, const DequantParams& p, int grid, cudaStream_t s) {
+fp4q_status launch_dequant_h(int had, const DequantParams& p, int grid, int sms, cudaStream_t s) {
     switch (had) {
-        case 0: return launch_dequant_t<FMT, 0>(p, grid, s);
-        case 16: return launch_dequant_t<FMT, 16>(p, grid, s);
-        case 32: return launch_dequant_t<FMT, 32>(p, grid, s);
+        case 0: return launch_dequant_stream<FMT, 0>(p, sms, s);
+        case 16: return launch_dequant_stream<FMT, 16>(p, sms, s);
+        case 32: return launch_dequant_stream<FMT, 32>(p, sms, s);
         case 64: return launch_dequant_t<FMT, 64>(p, grid, s);
         case 128: return launch_dequant_t<FMT, 128>(p, grid, s);
         case 256: return launch_dequant_t<FMT, 256>(p, grid, s);
@@ -323,12 +362,10 @@ FP4Q_API fp4q_status fp4q_quantize_nvfp4_noalloc(const void* x, int64_t M, int64
     if (st != FP4Q_OK) return st;
     if (K % 16 != 0) return FP4Q_ERR_INVALID_ARG;
     if (M == 0) return FP4Q_OK;
-    int sms = 0;
-    if ((st = sm_count(&sms)) != FP4Q_OK) return st;
-    // One partial maximum per pre-pass CTA; the grid is capped below the scratch size,
-    // so this only trips if that cap is ever raised.
-    const int64_t n_tiles = ((M + kTileRows - 1) / kTileRows) * ((K + kTileCols - 1) / kTileCols);
-    const int64_t grid = std::min<int64_t>({n_tiles, (int64_t)kQuantCtasPerSm * sms, (int64_t)kMaxGrid});
+    // One partial maximum per pre-pass CTA: at most one CTA per 8 warp tiles and
+    // never more than kMaxGrid, so this only trips if that cap is ever raised.
+    const int64_t n_wt = ((M + Geo<0>::rows - 1) / Geo<0>::rows) * ((K + Geo<0>::cols - 1) / Geo<0>::cols);
+    const int64_t grid = std::min<int64_t>((n_wt + kWarps - 1) / kWarps, (int64_t)kMaxGrid);
     if (grid > kNoAllocPartials) return FP4Q_ERR_UNSUPPORTED;
     float* scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != FP4Q_OK) return st;
@@ -471,9 +508,9 @@ FP4Q_API fp4q_status fp4q_dequantize(fp4q_format format, const uint8_t* codes,
         (int)std::min<int64_t>({p.n_tiles, (int64_t)kDequantCtasPerSm * sms, (int64_t)kMaxGrid});
     cudaStream_t s = (cudaStream_t)stream;
     switch (fmt) {
-        case FMT_NVFP4: return launch_dequant_h<FMT_NVFP4>(inv_had_size, p, grid, s);
-        case FMT_MXFP4: return launch_dequant_h<FMT_MXFP4>(inv_had_size, p, grid, s);
-        default: return launch_dequant_h<FMT_DUAL>(inv_had_size, p, grid, s);
+        case FMT_NVFP4: return launch_dequant_h<FMT_NVFP4>(inv_had_size, p, grid, sms, s);
+        case FMT_MXFP4: return launch_dequant_h<FMT_MXFP4>(inv_had_size, p, grid, sms, s);
+        default: return launch_dequant_h<FMT_DUAL>(inv_had_size, p, grid, sms, s);
     }
 }
 

@@ -33,14 +33,6 @@ struct ArcParams {
     int dynamic;
 };
 
-__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes,
-                                             uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-        "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
-}
-
 // Shared-memory layout: [stages: kArcStages * K bf16][res: K fp32][flags: K/32 u32]
 //                       [red: 32 fp32][bars: kArcStages u64]
 template <bool AMAX_ONLY, int MAXT>

@@ -16,6 +16,32 @@
 
 namespace fp4q {
 
+constexpr int kTileRows = 16;   // dequantizer tile: 16 rows x 512 columns
+constexpr int kTileCols = 512;
+constexpr int kDqScratchBytes = kTileRows * kTileCols * 4;
+
+// In-register butterflies over v[0..N) (unnormalised Walsh-Hadamard).
+template <int N>
+__device__ __forceinline__ void fwht_reg(float* v) {
+#pragma unroll
+    for (int s = 1; s < N; s <<= 1) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+            if ((i & s) == 0) {
+                float a = v[i], b = v[i + s];
+                v[i] = a + b;
+                v[i + s] = a - b;
+            }
+        }
+    }
+}
+
+template <int HAD>
+struct HadShape {
+    static constexpr int n2 = HAD >= 64 ? HAD / 32 : 1;  // threads per Hadamard block
+    static constexpr int k1w = 32 / n2;                  // columns per k2 row a thread owns
+};
+
 struct DequantParams {
     int64_t M, K;
     int64_t n_col_tiles, n_tiles;
@@ -31,7 +57,7 @@ struct DequantParams {
 // scale, loaded one tile ahead of their use (software pipelining).
 struct RawUnit {
     uint32_t w[4];
-    uint32_t e0, e1;
+    uint32_t e0, e1;  // scale bytes of the unit's two 16-blocks (MXFP4: e0 only)
     float s;
 };
 
@@ -93,6 +119,96 @@ __device__ __forceinline__ void decode_raw(const RawUnit& u, float* v) {
         for (int i = 0; i < 16; ++i) v[i] = (v[i] * ev0) * u.s;
 #pragma unroll
         for (int i = 16; i < 32; ++i) v[i] = (v[i] * ev1) * u.s;
+    }
+}
+
+// ---------------------------------------------------------------- streaming dequantizer
+// Rotation sizes 0, 16 and 32 need no data from other units: each thread
+// streams units (row-major order, grid-stride) and keeps the codes and scales of
+// kDqDepth units in registers ahead of their use, so that enough small loads
+// stay in flight to cover the memory latency.
+constexpr int kDqDepth = 4;
+
+__device__ __forceinline__ void advance_unit(int32_t& row, int32_t& j, int32_t drow, int32_t dj,
+                                             int32_t upr) {
+    j += dj;
+    row += drow;
+    if (j >= upr) {
+        j -= upr;
+        ++row;
+    }
+}
+
+__device__ __forceinline__ void store_bf16x32(uint16_t* dst, const uint32_t* o, int nval, bool w32) {
+    if (w32 && nval == 32) {  // two 256-bit stores
+        asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst), "r"(o[0]), "r"(o[1]),
+                     "r"(o[2]), "r"(o[3]), "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7])
+                     : "memory");
+        asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst + 16), "r"(o[8]),
+                     "r"(o[9]), "r"(o[10]), "r"(o[11]), "r"(o[12]), "r"(o[13]), "r"(o[14]), "r"(o[15])
+                     : "memory");
+    } else {
+        uint4* d4 = reinterpret_cast<uint4*>(dst);
+        d4[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        d4[1] = make_uint4(o[4], o[5], o[6], o[7]);
+        if (nval > 16) {
+            d4[2] = make_uint4(o[8], o[9], o[10], o[11]);
+            d4[3] = make_uint4(o[12], o[13], o[14], o[15]);
+        }
+    }
+}
+
+template <int FMT, int HAD>
+__global__ void __launch_bounds__(kThreads, 3) dequant_stream_kernel(const DequantParams p, int w32) {
+    // rows < 2^31 and units per row < 2^26: 32-bit unit coordinates
+    const int32_t upr = (int32_t)((p.K + 31) / 32);  // units per row
+    const int32_t M = (int32_t)p.M;
+    const int64_t S = (int64_t)gridDim.x * blockDim.x;
+    const int64_t u0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    const int32_t srow = (int32_t)(S / upr), sj = (int32_t)(S % upr);
+    const int64_t D = kDqDepth * S;
+    const int32_t drow = (int32_t)(D / upr), dj = (int32_t)(D % upr);
+    int32_t row[kDqDepth], jj[kDqDepth];
+    row[0] = (int32_t)min64(u0 / upr, (int64_t)M);
+    jj[0] = (int32_t)(u0 % upr);
+#pragma unroll
+    for (int k = 1; k < kDqDepth; ++k) {
+        row[k] = row[k - 1];
+        jj[k] = jj[k - 1];
+        advance_unit(row[k], jj[k], srow, sj, upr);
+    }
+    RawUnit buf[kDqDepth];
+#pragma unroll
+    for (int k = 0; k < kDqDepth; ++k)
+        if (row[k] < M) load_raw<FMT>(p, row[k], 32 * (int64_t)jj[k], (int)min64(32, p.K - 32 * (int64_t)jj[k]), buf[k]);
+
+    while (row[0] < M) {
+#pragma unroll
+        for (int k = 0; k < kDqDepth; ++k) {
+            if (row[k] >= M) continue;
+            const RawUnit cur = buf[k];
+            const int64_t r = row[k], col = 32 * (int64_t)jj[k];
+            const int nval = (int)min64(32, p.K - col);
+            advance_unit(row[k], jj[k], drow, dj, upr);
+            if (row[k] < M)
+                load_raw<FMT>(p, row[k], 32 * (int64_t)jj[k], (int)min64(32, p.K - 32 * (int64_t)jj[k]), buf[k]);
+            float v[32];
+            decode_raw<FMT>(cur, v);
+            if constexpr (HAD == 16) {
+                fwht_reg<16>(v);
+                fwht_reg<16>(v + 16);
+            } else if constexpr (HAD == 32) {
+                fwht_reg<32>(v);
+            }
+            if constexpr (HAD > 0) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] *= p.had_norm;
+            }
+            uint32_t o[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = bf16x2_pack(v[2 * i], v[2 * i + 1]);
+            store_bf16x32(p.y + r * p.K + col, o, nval, w32 != 0);
+        }
     }
 }
 
@@ -253,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_kernel(co
 
 template <int HAD>
 constexpr int dequant_smem_bytes() {
-    return HAD >= 64 ? kScratchBytes : 0;
+    return HAD >= 64 ? kDqScratchBytes : 0;
 }
 
 }  // namespace fp4q

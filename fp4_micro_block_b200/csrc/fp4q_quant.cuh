@@ -1,208 +1,242 @@
-// fp4q_quant.cuh -- persistent TMA-fed quantizer kernels for sm_100a:
-// optional block Hadamard rotation (sizes 16..512), then NVFP4 / MXFP4 / dual
-// scale quantization, or the amax pre-pass of the dynamic tensor scale.
+// fp4q_quant.cuh -- persistent quantizer kernels for sm_100a: optional block
+// Hadamard rotation (sizes 16..512), then NVFP4 / MXFP4 / dual-scale
+// quantization, or the amax pre-pass of the dynamic tensor scale.
 //
-// Work decomposition
-//   A tile is 16 rows x 512 columns of the bf16 input (16 KiB), brought into
-//   shared memory by eight 2-D TMA box loads of 16 rows x 64 columns each
-//   (128-byte swizzle).  A CTA owns a strided subset of the tiles and keeps
-//   kStages tiles in flight through a ring of mbarrier-tracked stages.
-//   The 256 threads each own one "unit" of 32 consecutive columns of one row:
-//     lane l, warp w  ->  row r = (l & 7) + 8*(w & 1),  unit j = (l >> 3) + 4*(w >> 1)
-//   so the eight lanes of each shared-memory phase read eight different rows
-//   at the same swizzled column: no bank conflicts for any access width.
+// Work decomposition: warp pipelines.
+//   Every warp streams its own "warp tiles" (1024 bf16 elements, 2 KiB)
+//   through a private ring of kStages shared-memory stages with one mbarrier
+//   each; lane 0 issues the copies for the tile kStages ahead as soon as the
+//   warp has read a stage.  Warps never wait for each other, so a CTA needs no
+//   block-wide barrier in its main loop, and the many warps of an SM keep
+//   ~100-200 KiB of loads in flight.  Each lane owns one "unit" of 32
+//   consecutive columns of one row.
+//
+// Warp-tile geometries (each keeps every shared-memory access below free of
+// bank conflicts):
+//   G2 (rotation n <= 128): 8 rows x 128 columns, two 2-D TMA boxes of
+//      64 columns x 8 rows with the 128-byte swizzle.  lane -> row = lane & 7,
+//      unit = lane >> 3, so the 8 lanes of a shared-memory phase are 8 rows.
+//   G3 (rotation n = 256, 512): 1024/n rows x n columns, one 1-D bulk copy
+//      per row into rows padded by 64 bytes.  lane -> row = lane / (n/32),
+//      unit = lane % (n/32).
 //
 // Block Hadamard of size n = n2 * 32 (Sylvester order, H_n = H_n2 (x) H_32):
-//   the n2 threads owning one n-block first read the block "column-major"
-//   (for every k2 < n2 their 32/n2 columns k1), apply H_n2 across k2 in
-//   registers, exchange through a swizzled fp32 scratch so that each thread
-//   holds its 32 contiguous values, then apply H_32 in registers.  n = 16 and
-//   32 need no exchange.  The result is scaled by RN(1/sqrt(n)).
+//   the n2 lanes owning one n-block read it "column-major" (for every k2 < n2
+//   their 32/n2 columns k1), apply H_n2 across k2 in registers, exchange through
+//   a swizzled per-warp fp32 scratch (n = 64: shuffles with the partner lane) so
+//   that each lane holds its 32 contiguous values, and apply H_32 in registers.
+//   n = 16, 32 need no exchange.  The result is scaled by RN(1/sqrt(n)).
 #pragma once
 
-#include "fp4q_device.cuh"
+#include "fp4q_unit.cuh"
 
 namespace fp4q {
 
 #ifndef FP4Q_STAGES
 #define FP4Q_STAGES 4
 #endif
-#ifndef FP4Q_QUANT_CTAS_PER_SM
-#define FP4Q_QUANT_CTAS_PER_SM 2
-#endif
 
-constexpr int kThreads = 256;
-constexpr int kTileRows = 16;
-constexpr int kTileCols = 512;
-constexpr int kBoxCols = 64;
-constexpr int kBoxes = kTileCols / kBoxCols;            // 8
-constexpr int kBoxBytes = kTileRows * kBoxCols * 2;     // 2048
-constexpr int kTileBytes = kTileRows * kTileCols * 2;   // 16384
-constexpr int kStages = FP4Q_STAGES;                    // tiles in the shared-memory ring
-constexpr int kQuantCtasPerSm = FP4Q_QUANT_CTAS_PER_SM;
-constexpr int kScratchBytes = kTileRows * kTileCols * 4;  // fp32 exchange, 32 KiB
+constexpr int kWarps = 8;                     // consumer warps of a quantizer CTA
+constexpr int kQuantThreads = kWarps * 32;
+constexpr int kThreads = 256;                 // CTA size of the other kernels
+constexpr int kStages = FP4Q_STAGES;     // per-warp ring depth
+constexpr int kWtElems = 1024;           // elements of a warp tile
+constexpr int kStageBytesG2 = 2048;      // two 1 KiB TMA boxes
+constexpr int kStageBytesG3 = 2304;      // rows of n*2 bytes + 64 bytes of padding
+constexpr int kScratchBytes = 4096;      // per-warp fp32 exchange (rotations >= 128)
+constexpr int kRowPad = 64;
 
 enum : int { FMT_NVFP4 = 0, FMT_MXFP4 = 1, FMT_DUAL = 2 };
 
 struct QuantParams {
     int64_t M, K;
-    int64_t n_row_tiles, n_col_tiles, n_tiles;
-    uint8_t* codes;       // [M, K/2]
-    uint8_t* scales;      // [M, K/B] or swizzled
-    float* scale_fp32;    // NVFP4: tensor scale; DUAL: [M, K/128]
-    float* partials;      // amax pass: per-CTA maxima out; dynamic quant: in
-    int n_partials;       // number of valid partials (dynamic quant)
-    int swizzled;         // scale layout
-    int dynamic;          // NVFP4: 1 = tensor scale from partials, 0 = read *scale_fp32
-    float had_norm;       // RN(1/sqrt(n))
+    int64_t n_rb, n_cb, n_wt;   // warp-tile grid: row blocks x column blocks
+    const uint8_t* x;           // bf16 rows (bulk-copy geometry)
+    int64_t ldx_bytes;
+    uint8_t* codes;             // [M, K/2]
+    uint8_t* scales;            // [M, K/B] or swizzled
+    float* scale_fp32;          // NVFP4: tensor scale; DUAL: [M, K/128]
+    float* partials;            // amax pass: per-CTA maxima out; dynamic quant: in
+    int n_partials;             // number of valid partials (dynamic quant)
+    int swizzled;               // scale layout
+    int dynamic;                // NVFP4: 1 = tensor scale from partials, 0 = read *scale_fp32
+    float had_norm;             // RN(1/sqrt(n))
 };
 
 template <int HAD>
-struct HadShape {
-    static constexpr int n2 = HAD >= 64 ? HAD / 32 : 1;  // threads per Hadamard block
-    static constexpr int k1w = 32 / n2;                  // columns per k2 row a thread reads
+struct Geo {
+    static constexpr bool bulk = HAD >= 256;
+    static constexpr int cols = bulk ? HAD : 128;             // warp-tile width
+    static constexpr int rows = kWtElems / cols;              // 8, 4 or 2
+    static constexpr int stage_bytes = bulk ? kStageBytesG3 : kStageBytesG2;
+    static constexpr int row_bytes = bulk ? HAD * 2 + kRowPad : 0;
+    static constexpr int lanes_per_row = cols / 32;           // 4, 8 or 16
+    static constexpr int scratch = HAD >= 128 ? kScratchBytes : 0;
+    // every warp's ring starts 1024-byte aligned (TMA swizzle-128 boxes); the
+    // mbarriers of all warps sit after the rings
+    static constexpr int warp_stride = kStages * stage_bytes + scratch;
+    static_assert(bulk || warp_stride % 1024 == 0, "G2 rings must stay 1024-byte aligned");
+    static_assert(warp_stride % 128 == 0, "warp regions must stay 128-byte aligned");
+    static constexpr int min_ctas = HAD >= 128 ? 2 : 3;  // per SM (shared memory)
+    static constexpr int n2 = HAD >= 64 ? HAD / 32 : 1;       // lanes per Hadamard block
+    static constexpr int k1w = 32 / n2;                       // columns per k2 a lane reads
 };
 
-// Physical shared-memory byte offset of (row r, tile column c) in a stage.
-__device__ __forceinline__ uint32_t tile_off(uint32_t r, uint32_t c) {
-    return (c >> 6) * kBoxBytes + swz128(r, (c & 63u) * 2u);
-}
-
-// In-register butterflies over v[0..N) with stride s (unnormalised Walsh-Hadamard).
-template <int N>
-__device__ __forceinline__ void fwht_reg(float* v) {
-#pragma unroll
-    for (int s = 1; s < N; s <<= 1) {
-#pragma unroll
-        for (int i = 0; i < N; ++i) {
-            if ((i & s) == 0) {
-                float a = v[i], b = v[i + s];
-                v[i] = a + b;
-                v[i + s] = a - b;
-            }
-        }
-    }
-}
-
-// Loads this thread's 32 post-rotation values of unit (r, j) of a staged tile.
+// Shared memory: the warps' rings, their mbarriers [kWarps][kStages], the
+// reduction slots and the NVFP4 table.
 template <int HAD>
-__device__ __forceinline__ void load_unit(const uint8_t* stage, float* scratch, uint32_t r,
-                                          uint32_t j, float had_norm, float* v) {
+constexpr int quant_smem_bytes() {
+    return 1024 + kWarps * Geo<HAD>::warp_stride + kWarps * kStages * 8 + (kWarps + 2) * 4 +
+           128 * 8 + 64;
+}
+
+// Stage byte offset of (row, column) in the G2 geometry: two boxes of
+// 64 columns x 8 rows (1 KiB each), 128-byte swizzle.
+__device__ __forceinline__ uint32_t g2_off(uint32_t row, uint32_t c) {
+    return (c >> 6) * 1024u + swz128(row, (c & 63u) * 2u);
+}
+
+// Negated values of 8 consecutive bf16 into two float2 pairs-of-pairs order:
+// out[j] = -x[j] for j < 8.
+__device__ __forceinline__ void nunpack8(uint4 q, float* o) {
+    o[0] = nbf16lo(q.x); o[1] = nbf16hi(q.x); o[2] = nbf16lo(q.y); o[3] = nbf16hi(q.y);
+    o[4] = nbf16lo(q.z); o[5] = nbf16hi(q.z); o[6] = nbf16lo(q.w); o[7] = nbf16hi(q.w);
+}
+
+// 32 contiguous values t[0..31] -> unit pairs n[i] = (t[i], t[16+i]).
+__device__ __forceinline__ void to_pairs(const float* t, float2* n) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) n[i] = make_float2(t[i], t[16 + i]);
+}
+
+// This lane's 32 post-rotation values, negated, as unit pairs (unit `u` of row
+// `row` of the staged tile).  For rotations >= 64 the call exchanges data with
+// other lanes of the warp: every lane must call it.
+template <int HAD>
+__device__ __forceinline__ void load_unit(const uint8_t* stage, uint8_t* scratch, uint32_t lane,
+                                          uint32_t row, uint32_t u, float had_norm, float2* n) {
+    using G = Geo<HAD>;
     if constexpr (HAD <= 32) {
+        float t[32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            uint4 q = *reinterpret_cast<const uint4*>(stage + tile_off(r, 32 * j + 8 * c));
-            v[8 * c + 0] = bf16lo(q.x);
-            v[8 * c + 1] = bf16hi(q.x);
-            v[8 * c + 2] = bf16lo(q.y);
-            v[8 * c + 3] = bf16hi(q.y);
-            v[8 * c + 4] = bf16lo(q.z);
-            v[8 * c + 5] = bf16hi(q.z);
-            v[8 * c + 6] = bf16lo(q.w);
-            v[8 * c + 7] = bf16hi(q.w);
+        for (int c = 0; c < 4; ++c)
+            nunpack8(*reinterpret_cast<const uint4*>(stage + g2_off(row, 32 * u + 8 * c)), t + 8 * c);
+        to_pairs(t, n);
+        if constexpr (HAD == 16) fwht16x2(n);
+        if constexpr (HAD == 32) {
+            fwht32(n);
+            scale_unit(n, had_norm);
         }
-        if constexpr (HAD == 16) {
-            fwht_reg<16>(v);
-            fwht_reg<16>(v + 16);
-        } else if constexpr (HAD == 32) {
-            fwht_reg<32>(v);
-        }
-        if constexpr (HAD > 0) {
+    } else if constexpr (HAD == 64) {
+        // units (2p, 2p+1) of a row = lanes l and l ^ 8; tau = position in the pair
+        const uint32_t tau = u & 1u, c0 = 64u * (u >> 1);
+        float a[2][16];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= had_norm;
+        for (int k2 = 0; k2 < 2; ++k2) {
+            nunpack8(*reinterpret_cast<const uint4*>(stage + g2_off(row, c0 + 32 * k2 + 16 * tau)), a[k2]);
+            nunpack8(*reinterpret_cast<const uint4*>(stage + g2_off(row, c0 + 32 * k2 + 16 * tau + 8)),
+                     a[k2] + 8);
         }
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {  // H_2 across k2
+            const float2 x0 = make_float2(a[0][i], a[0][i + 1]), x1 = make_float2(a[1][i], a[1][i + 1]);
+            const float2 s = add2(x0, x1), d = sub2(x0, x1);
+            a[0][i] = s.x; a[0][i + 1] = s.y;
+            a[1][i] = d.x; a[1][i + 1] = d.y;
+        }
+        // row k2 = tau: my 16 columns of it plus the partner's 16
+        float t[32];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float send = tau ? a[0][i] : a[1][i];
+            const float got = __shfl_xor_sync(0xffffffffu, send, 8);
+            const float mine = tau ? a[1][i] : a[0][i];
+            t[i] = tau ? got : mine;
+            t[16 + i] = tau ? mine : got;
+        }
+        to_pairs(t, n);
+        fwht32(n);  // n = 64: the 1/8 normalisation is folded into the quantizer
     } else {
-        constexpr int n2 = HadShape<HAD>::n2;
-        constexpr int k1w = HadShape<HAD>::k1w;
-        const uint32_t tau = j % n2;           // position inside the Hadamard block
-        const uint32_t blk = j / n2;           // Hadamard block inside the tile row
-        const uint32_t col0 = blk * HAD;       // first tile column of the block
-        // Phase A: a[k2][i] = x[col0 + 32*k2 + k1w*tau + i]
-        float a[n2][k1w];
+        constexpr int n2 = G::n2, k1w = G::k1w, kp = k1w / 2;
+        // A[k2][j] = -x[row, block + 32*k2 + k1w*tau + 2j + (0, 1)]
+        float2 A[n2][kp];
+        uint32_t tau, team;
+        if constexpr (HAD == 128) {
+            tau = u;  // lanes row, row+8, row+16, row+24
+            team = row;
 #pragma unroll
-        for (int k2 = 0; k2 < n2; ++k2) {
-            const uint32_t c = col0 + 32 * k2 + k1w * tau;
-            const uint8_t* p = stage + tile_off(r, c);
-            if constexpr (k1w == 2) {
-                uint32_t u = *reinterpret_cast<const uint32_t*>(p);
-                a[k2][0] = bf16lo(u);
-                a[k2][1] = bf16hi(u);
-            } else if constexpr (k1w == 4) {
-                uint2 u = *reinterpret_cast<const uint2*>(p);
-                a[k2][0] = bf16lo(u.x);
-                a[k2][1] = bf16hi(u.x);
-                a[k2][2] = bf16lo(u.y);
-                a[k2][3] = bf16hi(u.y);
-            } else {
+            for (int k2 = 0; k2 < n2; ++k2) {
+                float o[8];
+                nunpack8(*reinterpret_cast<const uint4*>(stage + g2_off(row, 32 * k2 + 8 * tau)), o);
 #pragma unroll
-                for (int h = 0; h < k1w / 8; ++h) {
-                    uint4 u = *reinterpret_cast<const uint4*>(stage + tile_off(r, c + 8 * h));
-                    a[k2][8 * h + 0] = bf16lo(u.x);
-                    a[k2][8 * h + 1] = bf16hi(u.x);
-                    a[k2][8 * h + 2] = bf16lo(u.y);
-                    a[k2][8 * h + 3] = bf16hi(u.y);
-                    a[k2][8 * h + 4] = bf16lo(u.z);
-                    a[k2][8 * h + 5] = bf16hi(u.z);
-                    a[k2][8 * h + 6] = bf16lo(u.w);
-                    a[k2][8 * h + 7] = bf16hi(u.w);
+                for (int j = 0; j < 4; ++j) A[k2][j] = make_float2(o[2 * j], o[2 * j + 1]);
+            }
+        } else {
+            tau = lane % n2;
+            team = lane / n2;
+            const uint8_t* rp = stage + team * G::row_bytes;
+#pragma unroll
+            for (int k2 = 0; k2 < n2; ++k2) {
+                const uint8_t* q = rp + (32 * k2 + k1w * tau) * 2;
+                if constexpr (k1w == 2) {
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(q);
+                    A[k2][0] = make_float2(nbf16lo(w), nbf16hi(w));
+                } else {
+                    const uint2 w = *reinterpret_cast<const uint2*>(q);
+                    A[k2][0] = make_float2(nbf16lo(w.x), nbf16hi(w.x));
+                    A[k2][1] = make_float2(nbf16lo(w.y), nbf16hi(w.y));
                 }
             }
         }
-        // H_n2 across k2, independently for each of the k1w columns
 #pragma unroll
-        for (int s = 1; s < n2; s <<= 1) {
+        for (int s = 1; s < n2; s <<= 1) {  // H_n2 across k2
 #pragma unroll
             for (int k2 = 0; k2 < n2; ++k2) {
                 if ((k2 & s) == 0) {
 #pragma unroll
-                    for (int i = 0; i < k1w; ++i) {
-                        float x0 = a[k2][i], x1 = a[k2 + s][i];
-                        a[k2][i] = x0 + x1;
-                        a[k2 + s][i] = x0 - x1;
+                    for (int j = 0; j < kp; ++j) {
+                        const float2 x0 = A[k2][j], x1 = A[k2 + s][j];
+                        A[k2][j] = add2(x0, x1);
+                        A[k2 + s][j] = sub2(x0, x1);
                     }
                 }
             }
         }
-        // Exchange: write row k2 of this block's scratch, read back row tau.
-        // Scratch of block (r, blk): n2 rows of 32 floats (128 B), 16-byte chunk
-        // index XORed with r & 7.
-        uint8_t* sb = reinterpret_cast<uint8_t*>(scratch) +
-                      (r * (kTileCols / HAD) + blk) * (uint32_t)(n2 * 128);
-        const bool cross_warp = n2 > 4;  // blocks of 256/512 span several warps
-        if (cross_warp) bar_sync(2, kThreads);
-        else __syncwarp();
+        // Exchange through the warp's scratch: team rows R = team*n2 + k2 of 32
+        // floats (128 B); the 16-byte chunk index is XORed with f(R) = team (n =
+        // 128) or k2 & 7 (n >= 256), which keeps both the writes and the reads
+        // free of bank conflicts.
+        const uint32_t k1 = k1w * tau;
 #pragma unroll
         for (int k2 = 0; k2 < n2; ++k2) {
-            uint8_t* rowp = sb + k2 * 128;
-            const uint32_t k1 = k1w * tau;
+            const uint32_t f = (HAD == 128) ? (team & 7u) : (uint32_t)(k2 & 7);
+            uint8_t* rowp = scratch + (team * n2 + k2) * 128;
             if constexpr (k1w == 2) {
-                uint32_t off = ((((k1 >> 2) ^ r) & 7u) << 4) + (k1 & 3u) * 4u;
-                *reinterpret_cast<float2*>(rowp + off) = make_float2(a[k2][0], a[k2][1]);
+                *reinterpret_cast<float2*>(rowp + ((((k1 >> 2) ^ f) & 7u) << 4) + (k1 & 3u) * 4u) = A[k2][0];
             } else {
 #pragma unroll
-                for (int h = 0; h < k1w / 4; ++h) {
-                    uint32_t chunk = (k1 >> 2) + h;
-                    *reinterpret_cast<float4*>(rowp + (((chunk ^ r) & 7u) << 4)) =
-                        make_float4(a[k2][4 * h], a[k2][4 * h + 1], a[k2][4 * h + 2], a[k2][4 * h + 3]);
-                }
+                for (int h = 0; h < k1w / 4; ++h)
+                    *reinterpret_cast<float4*>(rowp + (((((k1 >> 2) + h) ^ f) & 7u) << 4)) =
+                        make_float4(A[k2][2 * h].x, A[k2][2 * h].y, A[k2][2 * h + 1].x, A[k2][2 * h + 1].y);
             }
         }
-        if (cross_warp) bar_sync(2, kThreads);
-        else __syncwarp();
+        __syncwarp();
         {
-            const uint8_t* rowp = sb + tau * 128;
+            const uint32_t f = (HAD == 128) ? (team & 7u) : (tau & 7u);
+            const uint8_t* rowp = scratch + (team * n2 + tau) * 128;
+            float t[32];
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
-                float4 q = *reinterpret_cast<const float4*>(rowp + (((ch ^ r) & 7u) << 4));
-                v[4 * ch + 0] = q.x;
-                v[4 * ch + 1] = q.y;
-                v[4 * ch + 2] = q.z;
-                v[4 * ch + 3] = q.w;
+                const float4 q = *reinterpret_cast<const float4*>(rowp + (((ch ^ f) & 7u) << 4));
+                t[4 * ch] = q.x;
+                t[4 * ch + 1] = q.y;
+                t[4 * ch + 2] = q.z;
+                t[4 * ch + 3] = q.w;
             }
+            to_pairs(t, n);
         }
-        fwht_reg<32>(v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] *= had_norm;
+        fwht32(n);
+        if constexpr (HAD != 256) scale_unit(n, had_norm);  // 256: 1/16 folded into the quantizer
     }
 }
 
@@ -222,35 +256,25 @@ __device__ __forceinline__ float tensor_scale_from_partials(const float* partial
 }
 
 template <int FMT, int HAD, bool AMAX_ONLY>
-__global__ void __launch_bounds__(kThreads, kQuantCtasPerSm)
+__global__ void __launch_bounds__(kQuantThreads, Geo<HAD>::min_ctas)
     quant_kernel(const __grid_constant__ CUtensorMap tmap_x, const QuantParams p) {
+    using G = Geo<HAD>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    // 1024-byte aligned stage ring, then the exchange scratch, then barriers.
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    uint8_t* stages = smem;
-    float* scratch = reinterpret_cast<float*>(smem + kStages * kTileBytes);
-    constexpr int scratch_bytes = (HAD >= 64) ? kScratchBytes : 0;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kTileBytes + scratch_bytes);
-    float* red = reinterpret_cast<float*>(bars + kStages);
-
     const uint32_t tid = threadIdx.x;
     const uint32_t lane = tid & 31, warp = tid >> 5;
-    const uint32_t r = (lane & 7) + 8 * (warp & 1);
-    const uint32_t j = (lane >> 3) + 4 * (warp >> 1);
-
-    const int64_t n_my = p.n_tiles > (int64_t)blockIdx.x
-                             ? (p.n_tiles - 1 - blockIdx.x) / gridDim.x + 1
-                             : 0;
+    uint64_t* full_bars = reinterpret_cast<uint64_t*>(smem + kWarps * G::warp_stride);
+    float* red = reinterpret_cast<float*>(full_bars + kWarps * kStages);
+    float2* tab = reinterpret_cast<float2*>(red + kWarps + 2);
+    constexpr bool kFold = HAD == 16 || HAD == 64 || HAD == 256;  // 1/sqrt(n) a power of two
 
     if (tid == 0) {
-        prefetch_tmap(&tmap_x);
-        for (int s = 0; s < kStages; ++s) mbar_init(smem_u32(&bars[s]), 1);
+        if constexpr (!G::bulk) prefetch_tmap(&tmap_x);
+        for (int k = 0; k < kWarps * kStages; ++k) mbar_init(smem_u32(&full_bars[k]), 1);
         fence_barrier_init();
     }
-    __syncthreads();
-
-    // Per-CTA scale of the NVFP4 format.
+    // NVFP4: tensor scale, and the per-CTA table of decoded block scales.
     float s_t = 0.0f;
     if constexpr (FMT == FMT_NVFP4 && !AMAX_ONLY) {
         if (p.dynamic) {
@@ -259,113 +283,140 @@ __global__ void __launch_bounds__(kThreads, kQuantCtasPerSm)
         } else {
             s_t = *p.scale_fp32;
         }
+        build_table(tab, s_t);
     }
+    __syncthreads();
 
-    auto issue = [&](int64_t i) {  // tile i of this CTA into stage i % kStages
-        const int64_t t = blockIdx.x + i * (int64_t)gridDim.x;
-        const int64_t rt = t / p.n_col_tiles, ct = t % p.n_col_tiles;
-        const int32_t y = (int32_t)(rt * kTileRows);
-        const int32_t x0 = (int32_t)(ct * kTileCols);
-        const int nb = (int)min64(kBoxes, (p.K - x0 + kBoxCols - 1) / kBoxCols);
-        const uint32_t st = (uint32_t)(i % kStages);
-        const uint32_t bar = smem_u32(&bars[st]);
-        mbar_arrive_expect_tx(bar, (uint32_t)(nb * kBoxBytes));
-        const uint32_t dst = smem_u32(stages + st * kTileBytes);
-        for (int b = 0; b < nb; ++b) tma_load_2d(dst + b * kBoxBytes, &tmap_x, x0 + b * kBoxCols, y, bar);
-    };
-
-    if (tid == 0)
-        for (int64_t i = 0; i < min64(kStages, n_my); ++i) issue(i);
-
-    float my_amax = 0.0f;
-    for (int64_t i = 0; i < n_my; ++i) {
-        const uint32_t st = (uint32_t)(i % kStages);
-        const bool ok = mbar_wait(smem_u32(&bars[st]), (uint32_t)((i / kStages) & 1));
-        if (!bar_and(1, kThreads, ok)) {
-            // A tile never arrived: record it, let the copies still in flight land, leave.
-            if (tid == 0) {
-                atomicOr(&g_device_error, kErrWaitTimeout);
-                for (int64_t k = i; k < min64(n_my, i + kStages); ++k)
-                    (void)mbar_wait(smem_u32(&bars[k % kStages]), (uint32_t)((k / kStages) & 1));
-            }
-            return;
+    const int64_t nw = (int64_t)gridDim.x * kWarps;
+    const int64_t step_rb = nw / p.n_cb, step_cb = nw % p.n_cb;
+    auto advance = [&](int64_t& rb, int64_t& cb) {  // tile t -> t + nw without division
+        cb += step_cb;
+        rb += step_rb;
+        if (cb >= p.n_cb) {
+            cb -= p.n_cb;
+            ++rb;
         }
-        // The previous stage is free once every thread passed the vote above.
-        if (tid == 0 && i >= 1 && i - 1 + kStages < n_my) issue(i - 1 + kStages);
+    };
+    float my_amax = 0.0f;
 
-        const int64_t t = blockIdx.x + i * (int64_t)gridDim.x;
-        const int64_t rt = t / p.n_col_tiles, ct = t % p.n_col_tiles;
-        const int64_t row = rt * kTileRows + r;
-        const int64_t col = ct * kTileCols + 32 * (int64_t)j;
-        const uint8_t* stage = stages + st * kTileBytes;
+    if (warp < kWarps) {
+        // Each warp streams its own tiles t = gw, gw + nw, ... : lane 0 refills a
+        // stage as soon as the warp has read it, kStages tiles ahead.
+        uint8_t* stages = smem + warp * G::warp_stride;
+        uint8_t* scratch = stages + kStages * G::stage_bytes;
+        uint64_t* bars = full_bars + warp * kStages;
+        const uint32_t row = G::bulk ? lane / G::lanes_per_row : (lane & 7u);
+        const uint32_t u = G::bulk ? lane % G::lanes_per_row : (lane >> 3);
+        const int64_t gw = (int64_t)blockIdx.x * kWarps + warp;
+        const int64_t n_my = p.n_wt > gw ? (p.n_wt - 1 - gw) / nw + 1 : 0;
+        int64_t rb = gw / p.n_cb, cb = gw % p.n_cb;  // tile being consumed
+        int64_t irb = rb, icb = cb;                  // next tile to issue (lane 0)
+        const int64_t kc = p.K / 2;
+        ScaleCtx ctx = make_ctx(s_t);
+        const float fold = kFold ? p.had_norm : 1.0f;
+        const float norm = kFold ? 1.0f : p.had_norm;
 
-        // Units entirely past K skip work, but Hadamard blocks of 256/512 still
-        // meet at the exchange barrier: every thread of the CTA calls load_unit.
-        float v[32];
-        load_unit<HAD>(stage, scratch, r, j, p.had_norm, v);
-        const bool live = row < p.M && col < p.K;
-        const int nval = (int)min64(32, p.K - col);  // 16 or 32 when live
+        auto issue = [&](int64_t i) {  // lane 0: tile (irb, icb) into stage i % kStages
+            const uint32_t st = (uint32_t)(i % kStages);
+            const uint32_t bar = smem_u32(&bars[st]);
+            const uint32_t dst = smem_u32(stages + st * G::stage_bytes);
+            if constexpr (G::bulk) {
+                const int64_t r0 = irb * G::rows;
+                const int nr = (int)min64(G::rows, p.M - r0);
+                mbar_arrive_expect_tx(bar, (uint32_t)(nr * HAD * 2));
+                const uint8_t* src = p.x + r0 * p.ldx_bytes + icb * HAD * 2;
+                for (int r = 0; r < nr; ++r)
+                    bulk_load_1d(dst + r * G::row_bytes, src + r * p.ldx_bytes, HAD * 2, bar);
+            } else {
+                const int32_t x0 = (int32_t)(icb * 128), y = (int32_t)(irb * 8);
+                const int nb = (p.K - x0 > 64) ? 2 : 1;
+                mbar_arrive_expect_tx(bar, (uint32_t)(nb * 1024));
+                tma_load_2d(dst, &tmap_x, x0, y, bar);
+                if (nb == 2) tma_load_2d(dst + 1024, &tmap_x, x0 + 64, y, bar);
+            }
+            advance(irb, icb);
+        };
+        if (lane == 0)
+            for (int64_t i = 0; i < min64(kStages, n_my); ++i) issue(i);
 
-        if constexpr (AMAX_ONLY) {
-            if (live) {
-                float m = amax16(v);
-                if (nval > 16) m = fmaxf(m, amax16(v + 16));
-                my_amax = fmaxf(my_amax, m);
-            }
-        } else if constexpr (FMT == FMT_NVFP4) {
-            if (live) {
-                uint32_t w[4];
-                const uint32_t e0 = nvfp4_block16(v, amax16(v), s_t, w[0], w[1]);
-                uint32_t e1 = 0;
-                if (nval > 16) e1 = nvfp4_block16(v + 16, amax16(v + 16), s_t, w[2], w[3]);
-                uint8_t* cp = p.codes + row * (p.K / 2) + col / 2;
-                if ((p.K & 31) == 0) {  // rows of codes are 16-byte aligned
-                    *reinterpret_cast<uint4*>(cp) = make_uint4(w[0], w[1], w[2], w[3]);
-                } else {  // K = 16 (mod 32): rows are only 8-byte aligned
-                    *reinterpret_cast<uint2*>(cp) = make_uint2(w[0], w[1]);
-                    if (nval > 16) *reinterpret_cast<uint2*>(cp + 8) = make_uint2(w[2], w[3]);
+        for (int64_t i = 0; i < n_my; ++i, advance(rb, cb)) {
+            const uint32_t st = (uint32_t)(i % kStages);
+            const bool ok = mbar_wait(smem_u32(&bars[st]), (uint32_t)((i / kStages) & 1));
+            if (!__all_sync(0xffffffffu, ok)) {
+                // A tile never arrived: record it, let this warp's copies land, stop.
+                if (lane == 0) {
+                    atomicOr(&g_device_error, kErrWaitTimeout);
+                    for (int64_t k = i; k < min64(n_my, i + kStages); ++k)
+                        (void)mbar_wait(smem_u32(&bars[k % kStages]), (uint32_t)((k / kStages) & 1));
                 }
-                const int64_t nsc = p.K / 16, c0 = col / 16;
-                if (p.swizzled) {
-                    const int64_t nC = (nsc + 3) / 4;
-                    p.scales[swizzle_offset(row, c0, nC)] = (uint8_t)e0;
-                    if (nval > 16) p.scales[swizzle_offset(row, c0 + 1, nC)] = (uint8_t)e1;
-                } else {
-                    p.scales[row * nsc + c0] = (uint8_t)e0;
-                    if (nval > 16) p.scales[row * nsc + c0 + 1] = (uint8_t)e1;
-                }
+                break;
             }
-        } else if constexpr (FMT == FMT_MXFP4) {
-            if (live) {
-                uint32_t w[4];
-                const uint32_t b = mxfp4_block32(v, w);
-                *reinterpret_cast<uint4*>(p.codes + row * (p.K / 2) + col / 2) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
-                const int64_t nsc = p.K / 32, c0 = col / 32;
-                if (p.swizzled) p.scales[swizzle_offset(row, c0, (nsc + 3) / 4)] = (uint8_t)b;
-                else p.scales[row * nsc + c0] = (uint8_t)b;
-            }
-        } else {  // FMT_DUAL: group of 128 = 4 units = lanes l, l^8, l^16, l^24
-            float a0 = amax16(v), a1 = amax16(v + 16);
-            float g = fmaxf(a0, a1);
-            g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, 8));
-            g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, 16));
-            if (live) {
-                const float G = __fdiv_rn(g, 2688.0f);
-                uint32_t w[4];
-                const uint32_t e0 = nvfp4_block16(v, a0, G, w[0], w[1]);
-                const uint32_t e1 = nvfp4_block16(v + 16, a1, G, w[2], w[3]);
-                *reinterpret_cast<uint4*>(p.codes + row * (p.K / 2) + col / 2) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
-                const int64_t nsc = p.K / 16, c0 = col / 16;
-                if (p.swizzled) {
-                    const int64_t nC = (nsc + 3) / 4;
-                    *reinterpret_cast<uint16_t*>(p.scales + swizzle_offset(row, c0, nC)) =
-                        (uint16_t)(e0 | (e1 << 8));
-                } else {
-                    *reinterpret_cast<uint16_t*>(p.scales + row * nsc + c0) = (uint16_t)(e0 | (e1 << 8));
+            float2 n[16];
+            load_unit<HAD>(stages + st * G::stage_bytes, scratch, lane, row, u, norm, n);
+            __syncwarp();  // every lane has read the stage (and the scratch): refill it
+            if (lane == 0 && i + kStages < n_my) issue(i + kStages);
+
+            const int64_t grow = rb * G::rows + row;
+            const int64_t col = cb * G::cols + 32 * (int64_t)u;
+            const bool live = grow < p.M && col < p.K;
+            const bool full = col + 32 <= p.K;  // else half a unit (NVFP4 with K = 16 mod 32)
+
+            if constexpr (AMAX_ONLY) {
+                if (live) {
+                    const float2 am = mul2(amax_pair(n), dup2(fold));
+                    my_amax = fmaxf(my_amax, full ? fmaxf(am.x, am.y) : am.x);
                 }
-                if ((j & 3) == 0) p.scale_fp32[row * (p.K / 128) + col / 128] = G;
+            } else if constexpr (FMT == FMT_MXFP4) {
+                if (live) {
+                    if constexpr (kFold) scale_unit(n, fold);
+                    uint32_t w[4];
+                    const uint32_t b = mxfp4_unit(n, w);
+                    *reinterpret_cast<uint4*>(p.codes + grow * kc + col / 2) = make_uint4(w[0], w[1], w[2], w[3]);
+                    const int64_t nsc = p.K / 32, c0 = col / 32;
+                    if (p.swizzled) p.scales[swizzle_offset(grow, c0, (nsc + 3) / 4)] = (uint8_t)b;
+                    else p.scales[grow * nsc + c0] = (uint8_t)b;
+                }
+            } else {
+                const float2 am = amax_pair(n);
+                if constexpr (FMT == FMT_DUAL) {  // group scale over 4 units of one row
+                    float g = fmaxf(am.x, am.y) * fold;
+                    if constexpr (G::bulk) {  // the units of a group are 4 consecutive lanes
+                        g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, 1));
+                        g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, 2));
+                    } else {  // lanes row, row+8, row+16, row+24
+                        g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, 8));
+                        g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, 16));
+                    }
+                    const float Gs = (g >= 0x1p-90f) ? div2(make_float2(-g, 0.0f), dup2(2688.0f),
+                                                            dup2(-__uint_as_float(kRcp2688Bits))).x
+                                                     : __fdiv_rn(g, 2688.0f);
+                    ctx = make_ctx(Gs);
+                }
+                if (live) {
+                    uint32_t w[4];
+                    const uint32_t e2 = nvfp4_unit<FMT == FMT_NVFP4>(n, am, ctx, tab, fold, w);
+                    uint8_t* cp = p.codes + grow * kc + col / 2;
+                    const int64_t nsc = p.K / 16, c0 = col / 16;
+                    if ((p.K & 31) == 0) {  // rows of codes are 16-byte aligned
+                        *reinterpret_cast<uint4*>(cp) = make_uint4(w[0], w[1], w[2], w[3]);
+                    } else {  // K = 16 (mod 32): rows are only 8-byte aligned
+                        *reinterpret_cast<uint2*>(cp) = make_uint2(w[0], w[1]);
+                        if (full) *reinterpret_cast<uint2*>(cp + 8) = make_uint2(w[2], w[3]);
+                    }
+                    if (p.swizzled) {
+                        const int64_t nC = (nsc + 3) / 4;
+                        p.scales[swizzle_offset(grow, c0, nC)] = (uint8_t)(e2 & 0xffu);
+                        if (full) p.scales[swizzle_offset(grow, c0 + 1, nC)] = (uint8_t)(e2 >> 8);
+                    } else if (full && ((grow * nsc + c0) & 1) == 0) {
+                        *reinterpret_cast<uint16_t*>(p.scales + grow * nsc + c0) = (uint16_t)e2;
+                    } else {
+                        p.scales[grow * nsc + c0] = (uint8_t)(e2 & 0xffu);
+                        if (full) p.scales[grow * nsc + c0 + 1] = (uint8_t)(e2 >> 8);
+                    }
+                    if constexpr (FMT == FMT_DUAL) {
+                        if ((col & 127) == 0) p.scale_fp32[grow * (p.K / 128) + col / 128] = ctx.s;
+                    }
+                }
             }
         }
     }
@@ -373,20 +424,14 @@ __global__ void __launch_bounds__(kThreads, kQuantCtasPerSm)
     if constexpr (AMAX_ONLY) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) my_amax = fmaxf(my_amax, __shfl_xor_sync(0xffffffffu, my_amax, o));
-        __syncthreads();
         if (lane == 0) red[warp] = my_amax;
         __syncthreads();
         if (tid == 0) {
             float m = 0.0f;
-            for (int w = 0; w < kThreads / 32; ++w) m = fmaxf(m, red[w]);
+            for (int w = 0; w < kWarps; ++w) m = fmaxf(m, red[w]);
             p.partials[blockIdx.x] = m;
         }
     }
-}
-
-template <int HAD>
-constexpr int quant_smem_bytes() {
-    return 1024 + kStages * kTileBytes + (HAD >= 64 ? kScratchBytes : 0) + kStages * 8 + 64;
 }
 
 }  // namespace fp4q

@@ -1,0 +1,254 @@
+// fp4q_unit.cuh -- quantization of one 32-value "unit" with the packed
+// two-wide fp32 instructions of sm_100a (FADD2 / FMUL2 / FFMA2).
+//
+// A unit holds 32 consecutive values v[0..31] of one row.  They are kept
+// NEGATED, as 16 pairs n[i] = (-v[i], -v[16+i]): the first component belongs
+// to block 0 (v[0..15]), the second to block 1 (v[16..31]), so the two
+// 16-element NVFP4 blocks of a unit are always processed side by side, and
+// Walsh-Hadamard stages of stride 1..8 are "vertical" pair operations.
+// Carrying -v costs nothing (the bf16 unpack flips the sign for free) and
+// gives the correctly rounded division below the -x operand it needs.
+#pragma once
+
+#include "fp4q_device.cuh"
+
+namespace fp4q {
+
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);  // RN(a - b)
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 dup2(float a) { return make_float2(a, a); }
+
+// Negated bf16 -> binary32 (exact): w = (lo, hi) bf16 pair.  w * 2^16 + 2^31
+// (mod 2^32) is the low half moved up with its sign bit flipped.
+__device__ __forceinline__ float nbf16lo(uint32_t w) { return __uint_as_float(w * 65536u + 0x80000000u); }
+__device__ __forceinline__ float nbf16hi(uint32_t w) {
+    return __uint_as_float((w & 0xffff0000u) ^ 0x80000000u);
+}
+
+// RN(1/6) and RN(1/2688) as binary32 (checked against exact rationals).
+constexpr uint32_t kRcp6Bits = 0x3e2aaaabu;
+constexpr uint32_t kRcp2688Bits = 0x39c30c31u;
+
+// Correctly rounded quotient x/d for both lanes, from nx = -x, d and
+// ny = -RN(1/d): two Markstein corrections of x*RN(1/d) (see div_rn in
+// fp4q_device.cuh for the argument and the preconditions).  The remainder is
+// formed as q*d - x so that a zero quotient carries the sign of x.
+__device__ __forceinline__ float2 div2(float2 nx, float2 d, float2 ny) {
+    float2 q = mul2(nx, ny);
+    float2 e = fma2(q, d, nx);
+    q = fma2(e, ny, q);
+    e = fma2(q, d, nx);
+    q = fma2(e, ny, q);
+    return q;
+}
+
+// ---------------------------------------------------------------- Walsh-Hadamard
+template <int S>
+__device__ __forceinline__ void vstage(float2* n) {  // stride S < 16: pairs i, i+S
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        if ((i & S) == 0) {
+            const float2 a = n[i], b = n[i + S];
+            n[i] = add2(a, b);
+            n[i + S] = sub2(a, b);
+        }
+}
+__device__ __forceinline__ void hstage(float2* n) {  // stride 16: within each pair
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float a = n[i].x, b = n[i].y;
+        n[i] = make_float2(a + b, a - b);
+    }
+}
+// H_16 on both blocks (v[0..15], v[16..31]) / H_32 on the whole unit (unnormalised).
+__device__ __forceinline__ void fwht16x2(float2* n) { vstage<1>(n); vstage<2>(n); vstage<4>(n); vstage<8>(n); }
+__device__ __forceinline__ void fwht32(float2* n) { fwht16x2(n); hstage(n); }
+
+__device__ __forceinline__ void scale_unit(float2* n, float c) {
+    const float2 c2 = dup2(c);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) n[i] = mul2(n[i], c2);
+}
+
+// ---------------------------------------------------------------- amax
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+// Block maxima |v| of the two blocks of a unit.
+__device__ __forceinline__ float2 amax_pair(const float2* n) {
+    float a0 = fmaxf(fabsf(n[0].x), fabsf(n[1].x)), a1 = fmaxf(fabsf(n[0].y), fabsf(n[1].y));
+#pragma unroll
+    for (int i = 2; i < 16; i += 2) {
+        a0 = max3(a0, fabsf(n[i].x), fabsf(n[i + 1].x));
+        a1 = max3(a1, fabsf(n[i].y), fabsf(n[i + 1].y));
+    }
+    return make_float2(a0, a1);
+}
+
+// ---------------------------------------------------------------- packing
+// Packed E2M1 codes of the quotients q (x/d, both blocks): w[0..1] block 0,
+// w[2..3] block 1, low nibble = even index.
+__device__ __forceinline__ void pack_codes(const float2* q, uint32_t (&w)[4]) {
+    float b0[16], b1[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        b0[i] = q[i].x;
+        b1[i] = q[i].y;
+    }
+    w[0] = e2m1_pack8(b0);
+    w[1] = e2m1_pack8(b0 + 8);
+    w[2] = e2m1_pack8(b1);
+    w[3] = e2m1_pack8(b1 + 8);
+}
+
+// Two E4M3 bytes (lo = block 0) of the non-negative pair r, and their values.
+__device__ __forceinline__ uint32_t e4m3x2_encode(float2 r) {
+    uint16_t h;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(r.y), "f"(r.x));
+    return h;
+}
+__device__ __forceinline__ float2 e4m3x2_decode(uint32_t e2) {
+    uint32_t h2;
+    const uint16_t in = (uint16_t)e2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+    return make_float2(__half2float(__ushort_as_half((unsigned short)(h2 & 0xffffu))),
+                       __half2float(__ushort_as_half((unsigned short)(h2 >> 16))));
+}
+
+// Constants of the NVFP4 rule for one FP32 scale s (the tensor scale, or a
+// group scale of the dual format).  The fast path needs s in [2^-90, 2^90] and,
+// per block, 2^-90 <= amax <= 2^62 * s (or amax = 0): then every quotient below
+// stays in the normal range, (amax/6)/s <= 2^60, and each decoded block scale
+// d = E4M3(e) * s is either 0 or in [2^-99, 2^99], which are the preconditions
+// of the packed division.
+struct ScaleCtx {
+    float s;       // the FP32 scale
+    float nrs;     // -RN(1/s)
+    float am_max;  // 2^62 * s
+    bool fast;
+};
+
+__device__ __forceinline__ ScaleCtx make_ctx(float s) {
+    ScaleCtx c;
+    c.s = s;
+    c.fast = s >= 0x1p-90f && s <= 0x1p90f;
+    c.nrs = c.fast ? -__frcp_rn(s) : 0.0f;
+    c.am_max = s * 0x1p62f;
+    return c;
+}
+
+// Per-CTA table of the NVFP4 decoded scales for a fixed s: t[e] = (d, ny) with
+// d = E4M3(e) * s and ny = -RN(1/d) (0 when d == 0), for the 128 non-negative
+// E4M3 bytes.
+__device__ __forceinline__ void build_table(float2* t, float s) {
+    for (int e = threadIdx.x; e < 128; e += blockDim.x) {
+        const float d = (e < 127) ? e4m3_decode((uint32_t)e) * s : 0.0f;
+        t[e] = make_float2(d, (d >= 0x1p-100f && d <= 0x1p100f) ? -__frcp_rn(d) : 0.0f);
+    }
+}
+
+// The NVFP4 rule with IEEE divisions, for units outside the fast range.
+__device__ __noinline__ uint32_t nvfp4_unit_ieee(const float2* n, float2 am, float s, float fold,
+                                                 uint32_t* w) {
+    float q0[16], q1[16];
+    uint32_t e[2];
+    const float a[2] = {am.x, am.y};
+    for (int b = 0; b < 2; ++b) {
+        float d = 0.0f;
+        e[b] = 0;
+        if (s > 0.0f) {
+            const float r = __fdiv_rn(__fdiv_rn(a[b], 6.0f), s);  // a[] already folded
+            e[b] = e4m3_encode(r);
+            d = e4m3_decode(e[b]) * s;
+        }
+        float* q = b ? q1 : q0;
+        for (int i = 0; i < 16; ++i) {
+            const float x = -(b ? n[i].y : n[i].x) * fold;
+            q[i] = d != 0.0f ? __fdiv_rn(x, d) : 0.0f;
+        }
+        if (d == 0.0f)
+            for (int i = 0; i < 16; ++i) q[i] = 0.0f;
+    }
+    w[0] = e2m1_pack8(q0);
+    w[1] = e2m1_pack8(q0 + 8);
+    w[2] = e2m1_pack8(q1);
+    w[3] = e2m1_pack8(q1 + 8);
+    return e[0] | (e[1] << 8);
+}
+
+// NVFP4 rule for the two blocks of a unit against the FP32 scale of `c`:
+//   r = (amax_b / 6) / s,  e = E4M3(r),  d = E4M3(e) * s,  code = E2M1(v / d).
+// `fold` = 2^-k > 0 means the unit holds z with v = z * 2^-k (a Hadamard
+// normalisation by a power of two, applied exactly here instead of per element);
+// am is then the amax of z.  Returns the two scale bytes (block 0 low) and
+// writes the codes to w.
+template <bool TABLE>
+__device__ __forceinline__ uint32_t nvfp4_unit(const float2* n, float2 am, const ScaleCtx& c,
+                                               const float2* tab, float fold, uint32_t (&w)[4]) {
+    am = mul2(am, dup2(fold));
+    const uint32_t b0 = __float_as_uint(am.x), b1 = __float_as_uint(am.y);
+    const uint32_t tiny = __float_as_uint(0x1p-90f);  // amax == 0 passes, 0 < amax < 2^-90 fails
+    const bool in_range = c.fast && (b0 - 1u) >= tiny - 1u && (b1 - 1u) >= tiny - 1u &&
+                          fmaxf(am.x, am.y) <= c.am_max;
+    if (!in_range) return nvfp4_unit_ieee(n, am, c.s, fold, w);
+    const float r6 = __uint_as_float(kRcp6Bits);
+    const float2 bs = div2(make_float2(-am.x, -am.y), dup2(6.0f), dup2(-r6));
+    const float2 r = div2(make_float2(-bs.x, -bs.y), dup2(c.s), dup2(c.nrs));
+    const uint32_t e2 = e4m3x2_encode(r);
+    float2 d, ny;
+    if constexpr (TABLE) {
+        const float2 t0 = tab[e2 & 0xffu], t1 = tab[e2 >> 8];
+        d = make_float2(t0.x, t1.x);
+        ny = make_float2(t0.y, t1.y);
+    } else {
+        d = mul2(e4m3x2_decode(e2), dup2(c.s));
+        ny = make_float2(d.x != 0.0f ? -__frcp_rn(d.x) : 0.0f, d.y != 0.0f ? -__frcp_rn(d.y) : 0.0f);
+    }
+    if (fold != 1.0f) {  // divide z by d / 2^-k
+        const float inv = 1.0f / fold;  // exact: a power of two
+        d = mul2(d, dup2(inv));
+        ny = mul2(ny, dup2(fold));
+    }
+    float2 q[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q[i] = div2(n[i], d, ny);
+    pack_codes(q, w);
+    if (d.x == 0.0f) w[0] = w[1] = 0u;  // zero block scale: all codes +0
+    if (d.y == 0.0f) w[2] = w[3] = 0u;
+    return e2;
+}
+
+// MXFP4 of a whole unit (one 32-block): byte = clamp(floor(log2 amax) - 2 + 127,
+// 0, 254) from the exponent field, codes = E2M1(v * 2^(127-byte)) (exact).
+__device__ __forceinline__ uint32_t mxfp4_unit(const float2* n, uint32_t (&w)[4]) {
+    const float2 a = amax_pair(n);
+    const float am = fmaxf(a.x, a.y);
+    if (am == 0.0f) {
+        w[0] = w[1] = w[2] = w[3] = 0u;
+        return 0u;
+    }
+    const uint32_t ef = __float_as_uint(am) >> 23;
+    const uint32_t b = ef >= 2u ? ef - 2u : 0u;
+    const float2 nm = dup2(-__uint_as_float((254u - b) << 23));  // -2^(127-b), normal for b <= 252
+    float2 q[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q[i] = mul2(n[i], nm);
+    // q[i] = (v[i], v[16+i]) * 2^(127-b): codes in element order
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        v[i] = q[i].x;
+        v[16 + i] = q[i].y;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = e2m1_pack8(v + 8 * i);
+    return b;
+}
+
+}  // namespace fp4q
