@@ -14,6 +14,7 @@
 #include "fp4q_arc.cuh"
 #include "fp4q_dequant.cuh"
 #include "fp4q_device.cuh"
+#include "fp4q_mma.cuh"
 #include "fp4q_quant.cuh"
 
 #define FP4Q_API extern "C" __attribute__((visibility("default")))
@@ -66,15 +67,17 @@ fp4q_status encode_fn(EncodeTiledFn* out) {
     return FP4Q_OK;
 }
 
-// bf16 [M, K] with row stride ldx elements; boxes of 64 columns x 8 rows (the
-// G2 warp-tile halves), 128-byte swizzle, zero fill outside the matrix.
-fp4q_status make_x_map(CUtensorMap* map, const void* x, int64_t M, int64_t K, int64_t ldx) {
+// bf16 [M, K] with row stride ldx elements; boxes of 64 columns x box_rows rows
+// (8: the G2 warp-tile halves; 128: the tensor-core tile halves), 128-byte
+// swizzle, zero fill outside the matrix.
+fp4q_status make_x_map(CUtensorMap* map, const void* x, int64_t M, int64_t K, int64_t ldx,
+                       uint32_t box_rows = 8) {
     EncodeTiledFn enc;
     fp4q_status st = encode_fn(&enc);
     if (st != FP4Q_OK) return st;
     cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
     cuuint64_t strides[1] = {(cuuint64_t)ldx * 2};
-    cuuint32_t box[2] = {64u, 8u};
+    cuuint32_t box[2] = {64u, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -183,6 +186,32 @@ fp4q_status launch_quant_h(int had, const CUtensorMap& map, const QuantParams& p
     }
 }
 
+// ---------------------------------------------------------------- tensor-core rotation launch
+// Rotation sizes 16..128 on K a multiple of the 128-column tile go through the
+// tcgen05 kernel; other shapes use the register-FWHT warp pipelines.
+bool use_mma(int had, int64_t K) { return had >= 16 && had <= 128 && K % kMmaTile == 0; }
+
+template <int FMT, int HAD, bool AMAX>
+fp4q_status launch_mma_t(const CUtensorMap& map, const MmaParams& p, int grid, cudaStream_t s) {
+    auto kern = had_mma_kernel<FMT, HAD, AMAX>;
+    static std::atomic<uint64_t> done{0};
+    fp4q_status st = ensure_smem(kern, kMmaSmemBytes, done);
+    if (st != FP4Q_OK) return st;
+    kern<<<grid, kMmaThreads, kMmaSmemBytes, s>>>(map, p);
+    return launch_status();
+}
+
+template <int FMT, bool AMAX>
+fp4q_status launch_mma_h(int had, const CUtensorMap& map, const MmaParams& p, int grid, cudaStream_t s) {
+    switch (had) {
+        case 16: return launch_mma_t<FMT, 16, AMAX>(map, p, grid, s);
+        case 32: return launch_mma_t<FMT, 32, AMAX>(map, p, grid, s);
+        case 64: return launch_mma_t<FMT, 64, AMAX>(map, p, grid, s);
+        case 128: return launch_mma_t<FMT, 128, AMAX>(map, p, grid, s);
+        default: return FP4Q_ERR_INVALID_ARG;
+    }
+}
+
 float had_norm(int n) { return n > 0 ? (float)(1.0 / std::sqrt((double)n)) : 1.0f; }
 
 fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, int had,
@@ -215,7 +244,8 @@ fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, in
     if ((st = sm_count(&sms)) != FP4Q_OK) return st;
     CUtensorMap map;
     std::memset(&map, 0, sizeof(map));
-    if (had < 256 && (st = make_x_map(&map, x, M, K, ldx)) != FP4Q_OK) return st;
+    const bool mma = use_mma(had, K);
+    if (had < 256 && (st = make_x_map(&map, x, M, K, ldx, mma ? kMmaTile : 8)) != FP4Q_OK) return st;
 
     QuantParams p{};
     p.M = M;
@@ -235,6 +265,30 @@ fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, in
         const int64_t bytes = fp4q_scales_bytes(M, ncols, FP4Q_SCALES_SWIZZLED);
         if (bytes != M * ncols && cudaMemsetAsync(scales, 0, (size_t)bytes, stream) != cudaSuccess)
             return FP4Q_ERR_CUDA;
+    }
+    if (mma) {
+        MmaParams q{};
+        q.M = M;
+        q.K = K;
+        q.n_ct = K / kMmaTile;
+        q.n_tiles = (M + kMmaTile - 1) / kMmaTile * q.n_ct;
+        q.codes = codes;
+        q.scales = scales;
+        q.scale_fp32 = scale_fp32;
+        q.partials = static_cast<float*>(ws);
+        q.swizzled = p.swizzled;
+        q.dynamic = dynamic;
+        const int grid = (int)std::min<int64_t>({q.n_tiles, (int64_t)sms, (int64_t)kMaxGrid});
+        if (dynamic) {
+            if ((st = launch_mma_h<FMT_NVFP4, true>(had, map, q, grid, stream)) != FP4Q_OK) return st;
+            q.n_partials = grid;
+        }
+        switch (fmt) {
+            case FMT_NVFP4: return launch_mma_h<FMT_NVFP4, false>(had, map, q, grid, stream);
+            case FMT_MXFP4: return launch_mma_h<FMT_MXFP4, false>(had, map, q, grid, stream);
+            case FMT_DUAL: return launch_mma_h<FMT_DUAL, false>(had, map, q, grid, stream);
+            default: return FP4Q_ERR_INVALID_ARG;
+        }
     }
     if (dynamic) {  // amax pre-pass: one partial maximum per CTA into the workspace
         int grid_a = 0;

@@ -1,0 +1,428 @@
+// fp4q_mma.cuh -- block Hadamard rotation on the 5th-generation tensor cores
+// (tcgen05), fused with NVFP4 / MXFP4 / dual-scale quantization.
+//
+// For rotation sizes n <= 128 the rotated tile is a dense product: a tile X of
+// 128 rows x 128 columns times B = -2^-f * blockdiag(H_n, ..., H_n) (128 x 128,
+// Sylvester order, f = floor(log2(n) / 2)).  Every product of a bf16 input with
+// +-2^-f is exact and the sums accumulate in fp32 in tensor memory, so the tile
+// arrives in TMEM as the negated, (partly) normalised rotation; odd log2(n)
+// leaves a factor RN(1/sqrt(2)) for the epilogue.  (MR-GPTQ applies the
+// Hadamard as a matrix product on the activations; FP4Quant notes the FWHT as
+// one of the costs of the format.)
+//
+// CTA roles (one persistent CTA per SM):
+//   warp 0     lane 0 streams X tiles by TMA into a ring of kMmaStages stages;
+//   warp 1     allocates TMEM; lane 0 issues 8 UMMAs (K = 16 each) per tile
+//              into one of kEpiGroups fp32 accumulators (128 columns each)
+//              and commits them to the tile's barriers;
+//   warps 2..  kEpiGroups warpgroups of epilogue: warpgroup g takes the CTA's
+//              tiles j = g (mod kEpiGroups); thread = one row of the tile
+//              (TMEM lane), reading 32 columns at a time with tcgen05.ld and
+//              quantizing them in registers (two 16-blocks or one 32-block).
+// Every wait is bounded: a wait that runs out sets g_device_error and the role
+// stops; the CTA then drains its own copies and MMAs (bounded again) and frees
+// its TMEM before it exits.
+#pragma once
+
+#include "fp4q_quant.cuh"
+
+namespace fp4q {
+
+#ifndef FP4Q_MMA_STAGES
+#define FP4Q_MMA_STAGES 5
+#endif
+#ifndef FP4Q_EPI_GROUPS
+#define FP4Q_EPI_GROUPS 3
+#endif
+
+constexpr int kMmaTile = 128;                         // tile rows = tile columns
+constexpr int kMmaStages = FP4Q_MMA_STAGES;           // X ring depth
+constexpr int kEpiGroups = FP4Q_EPI_GROUPS;           // epilogue warpgroups = accumulators
+constexpr int kMmaThreads = 64 + 128 * kEpiGroups;
+constexpr int kTileBytes = kMmaTile * kMmaTile * 2;   // 32 KiB of bf16
+constexpr int kHalfBytes = kTileBytes / 2;            // one TMA box: 64 columns x 128 rows
+constexpr uint32_t kTmemCols = kEpiGroups * kMmaTile <= 256 ? (kEpiGroups * kMmaTile <= 128 ? 128u : 256u) : 512u;
+static_assert(kEpiGroups * kMmaTile <= 512, "accumulators exceed TMEM");
+
+// UMMA instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major,
+// M = 128, N = 128 (fields: D format [4,6), A format [7,10), B format [10,13),
+// N >> 3 at [17,23), M >> 4 at [24,29)).
+constexpr uint32_t kIdescBf16M128N128 =
+    (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kMmaTile >> 3) << 17) | ((uint32_t)(kMmaTile >> 4) << 24);
+
+// Shared-memory matrix descriptor of a K-major operand stored as rows of 128
+// bytes with the 128-byte swizzle, 8-row groups 1024 bytes apart: start address
+// >> 4 at [0,14), leading byte offset 16 >> 4 at [16,30) (unused by this
+// swizzle), stride byte offset 1024 >> 4 at [32,46), descriptor version 1 at
+// [46,48), layout "128-byte swizzle" (2) at [61,64).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3fffu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
+           ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+
+// ---------------------------------------------------------------- tcgen05 wrappers
+__device__ __forceinline__ void tmem_alloc(uint32_t slot_saddr, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_saddr),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// The barrier receives one arrival when every tcgen05 operation this thread
+// issued before has completed.
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]^T, M = N = 128, K = 16.
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// 32 consecutive fp32 columns of this thread's TMEM lane (shape 32x32b, x32).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Orders the computation of x before any later volatile asm (the next TMEM
+// load), so that chunks reduced in a loop do not stay live in registers.
+__device__ __forceinline__ void pin(float x) { asm volatile("" ::"f"(x)); }
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// ---------------------------------------------------------------- shared memory
+// [B 32 KiB][X ring kMmaStages x 32 KiB][barriers][tmem slot][NVFP4 table][reduction]
+constexpr int kMmaBOff = 0;
+constexpr int kMmaRingOff = kTileBytes;
+constexpr int kMmaBarOff = kMmaRingOff + kMmaStages * kTileBytes;
+constexpr int kMmaNumBars = 2 * kMmaStages + 2 * kEpiGroups + 1;
+constexpr int kMmaSlotOff = kMmaBarOff + kMmaNumBars * 8;
+constexpr int kMmaTabOff = (kMmaSlotOff + 4 + 15) / 16 * 16;
+constexpr int kMmaRedOff = kMmaTabOff + 128 * 8;
+constexpr int kMmaSmemBytes = 1024 + kMmaRedOff + (kMmaThreads / 32) * 4;
+static_assert(kMmaSmemBytes <= 227 * 1024, "shared memory");
+
+// B = -2^-f * blockdiag(H_n) in the K-major 128-byte-swizzled layout of the
+// tile: element (row nn, column k) of half h = k / 64 lives at byte
+// h * 16 KiB + nn * 128 + ((k % 64) / 8 ^ nn % 8) * 16 + (k % 8) * 2.
+template <int HAD>
+__device__ __forceinline__ void build_hadamard_b(uint8_t* b) {
+    constexpr int lg = HAD == 16 ? 4 : HAD == 32 ? 5 : HAD == 64 ? 6 : 7;
+    const uint32_t mag = 0x3f80u - (uint32_t)(lg / 2) * 0x80u;  // bf16 bits of 2^-f
+    for (int chunk = threadIdx.x; chunk < kTileBytes / 16; chunk += blockDim.x) {
+        const int h = chunk / 1024, nn = (chunk / 8) % 128, cp = chunk % 8;  // physical chunk cp
+        const int c = cp ^ (nn & 7);                                          // logical 16-byte chunk
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+            uint32_t pair = 0;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const int k = h * 64 + c * 8 + e + t;
+                uint32_t bits = 0;
+                if (k / HAD == nn / HAD) {
+                    const int par = __popc((uint32_t)((k % HAD) & (nn % HAD))) & 1;
+                    bits = mag | (par ? 0u : 0x8000u);  // -(+-1) * 2^-f
+                }
+                pair |= bits << (16 * t);
+            }
+            w[e / 2] = pair;
+        }
+        *reinterpret_cast<uint4*>(b + chunk * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+struct MmaParams {
+    int64_t M, K;
+    int64_t n_ct, n_tiles;       // column tiles per row band, tiles
+    uint8_t* codes;
+    uint8_t* scales;
+    float* scale_fp32;
+    float* partials;
+    int n_partials;
+    int swizzled;
+    int dynamic;
+};
+
+// Quantize the 32 values of one chunk (negated pairs n) and store codes and
+// scale bytes.  Returns the scale bytes of the chunk (NVFP4/dual: two).
+template <int FMT>
+__device__ __forceinline__ uint32_t quant_chunk(const float2* n, const ScaleCtx& ctx, const float2* tab,
+                                                uint8_t* cp) {
+    uint32_t w[4], e;
+    if constexpr (FMT == FMT_MXFP4) {
+        e = mxfp4_unit(n, w);
+    } else {
+        const float2 am = amax_pair(n);
+        e = nvfp4_unit<FMT == FMT_NVFP4>(n, am, ctx, tab, 1.0f, w);
+    }
+    *reinterpret_cast<uint4*>(cp) = make_uint4(w[0], w[1], w[2], w[3]);
+    return e;
+}
+
+template <int FMT, int HAD, bool AMAX_ONLY>
+__global__ void __launch_bounds__(kMmaThreads, 1)
+    had_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, const MmaParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    const uint32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kMmaBarOff);
+    const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * kMmaStages;
+    const uint32_t accf0 = empty0 + 8 * kMmaStages, acce0 = accf0 + 8 * kEpiGroups;
+    const uint32_t done_bar = acce0 + 8 * kEpiGroups;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kMmaSlotOff);
+    float2* tab = reinterpret_cast<float2*>(smem + kMmaTabOff);
+    float* red = reinterpret_cast<float*>(smem + kMmaRedOff);
+    constexpr bool kOddLog = HAD == 32 || HAD == 128;  // RN(1/sqrt(2)) left for the epilogue
+
+    if (tid == 0) {
+        prefetch_tmap(&tmap_x);
+        for (int s = 0; s < kMmaStages; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, 1);
+        }
+        for (int g = 0; g < kEpiGroups; ++g) {
+            mbar_init(accf0 + 8 * g, 1);
+            mbar_init(acce0 + 8 * g, 4);  // one arrival per epilogue warp
+        }
+        mbar_init(done_bar, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    build_hadamard_b<HAD>(smem + kMmaBOff);
+    fence_proxy_async_smem();  // B is read by the tensor cores (async proxy)
+    float s_t = 0.0f;
+    if constexpr (FMT == FMT_NVFP4 && !AMAX_ONLY) {
+        if (p.dynamic) {
+            s_t = tensor_scale_from_partials(p.partials, p.n_partials, red);
+            if (blockIdx.x == 0 && tid == 0) *p.scale_fp32 = s_t;
+        } else {
+            s_t = *p.scale_fp32;
+        }
+        build_table(tab, s_t);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int64_t n_my = p.n_tiles > (int64_t)blockIdx.x ? (p.n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    float my_amax = 0.0f;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int64_t j = 0;
+            for (; j < n_my; ++j) {
+                const int s = (int)(j % kMmaStages);
+                if (j >= kMmaStages &&
+                    !mbar_wait(empty0 + 8 * s, (uint32_t)((j / kMmaStages - 1) & 1))) {
+                    atomicOr(&g_device_error, kErrWaitTimeout);
+                    break;
+                }
+                const int64_t t = blockIdx.x + j * gridDim.x;
+                const int32_t x0 = (int32_t)((t % p.n_ct) * kMmaTile), y0 = (int32_t)((t / p.n_ct) * kMmaTile);
+                const uint32_t dst = smem_u32(smem + kMmaRingOff + s * kTileBytes);
+                mbar_arrive_expect_tx(full0 + 8 * s, kTileBytes);
+                tma_load_2d(dst, &tmap_x, x0, y0, full0 + 8 * s);
+                tma_load_2d(dst + kHalfBytes, &tmap_x, x0 + 64, y0, full0 + 8 * s);
+            }
+            // Every issued copy must have landed before the CTA may exit: the
+            // MMA warp waited for all of them unless something ran out.
+            for (int64_t k = j > kMmaStages ? j - kMmaStages : 0; k < j; ++k)
+                (void)mbar_wait(full0 + 8 * (int)(k % kMmaStages), (uint32_t)((k / kMmaStages) & 1));
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t b_addr = smem_u32(smem + kMmaBOff);
+            for (int64_t j = 0; j < n_my; ++j) {
+                const int s = (int)(j % kMmaStages), a = (int)(j % kEpiGroups);
+                bool ok = mbar_wait(full0 + 8 * s, (uint32_t)((j / kMmaStages) & 1));
+                if (ok && j >= kEpiGroups)
+                    ok = mbar_wait(acce0 + 8 * a, (uint32_t)((j / kEpiGroups - 1) & 1));
+                if (!ok) {
+                    atomicOr(&g_device_error, kErrWaitTimeout);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_addr = smem_u32(smem + kMmaRingOff + s * kTileBytes);
+                const uint32_t d = tmem_base + (uint32_t)(a * kMmaTile);
+#pragma unroll
+                for (int k = 0; k < kMmaTile / 16; ++k) {
+                    const uint32_t off = (uint32_t)((k / 4) * kHalfBytes + (k % 4) * 32);
+                    umma_bf16(d, sw128_desc(a_addr + off), sw128_desc(b_addr + off), kIdescBf16M128N128,
+                              k > 0 ? 1u : 0u);
+                }
+                tc_commit(empty0 + 8 * s);
+                tc_commit(accf0 + 8 * a);
+            }
+            // all MMAs of this CTA complete before TMEM is freed
+            tc_commit(done_bar);
+            if (!mbar_wait(done_bar, 0)) atomicOr(&g_device_error, kErrWaitTimeout);
+        }
+    } else {
+        // ------------------------------------------------ epilogue
+        const uint32_t ew = warp - 2, g = ew / 4, quarter = warp & 3;
+        const uint32_t lane_base = (quarter * 32u) << 16;
+        ScaleCtx ctx = make_ctx(s_t);
+        const float2 rs2 = dup2(__uint_as_float(0x3f3504f3u));  // RN(1/sqrt(2))
+        const int64_t kc = p.K / 2;
+#pragma unroll 1
+        for (int64_t j = g; j < n_my; j += kEpiGroups) {
+            const bool ok = mbar_wait(accf0 + 8 * g, (uint32_t)((j / kEpiGroups) & 1));
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) atomicOr(&g_device_error, kErrWaitTimeout);
+                break;
+            }
+            tc_fence_after();
+            const int64_t t = blockIdx.x + j * gridDim.x;
+            const int64_t ct = t % p.n_ct, rt = t / p.n_ct;
+            const int64_t row = rt * kMmaTile + quarter * 32 + lane;
+            const bool live = row < p.M;
+            const uint32_t tacc = tmem_base + lane_base + g * kMmaTile;
+
+            auto load_chunk = [&](int c, float2* n) {
+                float v[32];
+                tmem_ld32(tacc + 32u * c, v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) n[i] = make_float2(v[i], v[16 + i]);
+                if constexpr (kOddLog) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) n[i] = mul2(n[i], rs2);
+                }
+            };
+            auto release = [&]() {  // every lane's loads of this accumulator are done
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acce0 + 8 * g);
+            };
+
+            if constexpr (AMAX_ONLY) {
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float v[32];
+                    tmem_ld32(tacc + 32u * c, v);
+                    if (c == 3) release();
+                    float m0 = fmaxf(fabsf(v[0]), fabsf(v[1]));
+#pragma unroll
+                    for (int i = 2; i < 32; i += 2) m0 = max3(m0, fabsf(v[i]), fabsf(v[i + 1]));
+                    if constexpr (kOddLog) m0 *= rs2.x;  // RN is monotone: max of the scaled values
+                    const float2 am = make_float2(m0, m0);
+                    if (live) my_amax = fmaxf(my_amax, fmaxf(am.x, am.y));
+                    pin(my_amax);
+                }
+            } else {
+                if constexpr (FMT == FMT_DUAL) {  // group scale: amax over the 128 columns
+                    float gm = 0.0f;
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {
+                        float2 n[16];
+                        load_chunk(c, n);
+                        const float2 am = amax_pair(n);
+                        gm = fmaxf(gm, fmaxf(am.x, am.y));
+                        pin(gm);
+                    }
+                    const float Gs = (gm >= 0x1p-90f) ? div2(make_float2(-gm, 0.0f), dup2(2688.0f),
+                                                             dup2(-__uint_as_float(kRcp2688Bits))).x
+                                                      : __fdiv_rn(gm, 2688.0f);
+                    ctx = make_ctx(Gs);
+                    if (live) p.scale_fp32[row * (p.K / 128) + ct] = Gs;
+                }
+                uint8_t* cp = p.codes + row * kc + ct * (kMmaTile / 2);
+                uint32_t sc0 = 0u, sc1 = 0u;  // scale bytes of blocks 0-3 / 4-7 (MXFP4: sc0)
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float2 n[16];
+                    load_chunk(c, n);
+                    if (c == 3) release();
+                    if (live) {
+                        const uint32_t e = quant_chunk<FMT>(n, ctx, tab, cp + 16 * c);
+                        if constexpr (FMT == FMT_MXFP4) {
+                            sc0 |= e << (8 * c);
+                        } else {
+                            const uint32_t sh = e << (16 * (c & 1));
+                            if (c < 2) sc0 |= sh;
+                            else sc1 |= sh;
+                        }
+                    }
+                }
+                if (live) {
+                    if constexpr (FMT == FMT_MXFP4) {
+                        const int64_t nsc = p.K / 32;
+                        uint8_t* sp = p.swizzled ? p.scales + swizzle_offset(row, ct * 4, (nsc + 3) / 4)
+                                                 : p.scales + row * nsc + ct * 4;
+                        *reinterpret_cast<uint32_t*>(sp) = sc0;
+                    } else {
+                        const int64_t nsc = p.K / 16;
+                        if (p.swizzled) {
+                            const int64_t nC = (nsc + 3) / 4;
+                            *reinterpret_cast<uint32_t*>(p.scales + swizzle_offset(row, ct * 8, nC)) = sc0;
+                            *reinterpret_cast<uint32_t*>(p.scales + swizzle_offset(row, ct * 8 + 4, nC)) = sc1;
+                        } else {
+                            uint32_t* sp = reinterpret_cast<uint32_t*>(p.scales + row * nsc + ct * 8);
+                            sp[0] = sc0;
+                            sp[1] = sc1;
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    if constexpr (AMAX_ONLY) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) my_amax = fmaxf(my_amax, __shfl_xor_sync(0xffffffffu, my_amax, o));
+        if (lane == 0) red[warp] = my_amax;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if constexpr (AMAX_ONLY) {
+        if (tid == 0) {
+            float m = 0.0f;
+            for (int w = 0; w < kMmaThreads / 32; ++w) m = fmaxf(m, red[w]);
+            p.partials[blockIdx.x] = m;
+        }
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+}  // namespace fp4q

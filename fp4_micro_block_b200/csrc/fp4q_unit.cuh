@@ -153,33 +153,35 @@ __device__ __forceinline__ void build_table(float2* t, float s) {
     }
 }
 
-// The NVFP4 rule with IEEE divisions, for units outside the fast range.
-__device__ __noinline__ uint32_t nvfp4_unit_ieee(const float2* n, float2 am, float s, float fold,
-                                                 uint32_t* w) {
-    float q0[16], q1[16];
-    uint32_t e[2];
-    const float a[2] = {am.x, am.y};
-    for (int b = 0; b < 2; ++b) {
-        float d = 0.0f;
-        e[b] = 0;
-        if (s > 0.0f) {
-            const float r = __fdiv_rn(__fdiv_rn(a[b], 6.0f), s);  // a[] already folded
-            e[b] = e4m3_encode(r);
-            d = e4m3_decode(e[b]) * s;
-        }
-        float* q = b ? q1 : q0;
-        for (int i = 0; i < 16; ++i) {
-            const float x = -(b ? n[i].y : n[i].x) * fold;
-            q[i] = d != 0.0f ? __fdiv_rn(x, d) : 0.0f;
-        }
-        if (d == 0.0f)
-            for (int i = 0; i < 16; ++i) q[i] = 0.0f;
+// The NVFP4 rule with IEEE divisions for one block of a unit (component Y of
+// the pairs), for units outside the fast range.  Writes two code words and
+// returns the scale byte.
+template <bool Y>
+__device__ __forceinline__ uint32_t nvfp4_block_ieee(const float2* n, float a, float s, float fold,
+                                                     uint32_t& w0, uint32_t& w1) {
+    float d = 0.0f;
+    uint32_t e = 0;
+    if (s > 0.0f) {
+        const float r = __fdiv_rn(__fdiv_rn(a, 6.0f), s);  // a already folded
+        e = e4m3_encode(r);
+        d = e4m3_decode(e) * s;
     }
-    w[0] = e2m1_pack8(q0);
-    w[1] = e2m1_pack8(q0 + 8);
-    w[2] = e2m1_pack8(q1);
-    w[3] = e2m1_pack8(q1 + 8);
-    return e[0] | (e[1] << 8);
+    float q[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float x = -(Y ? n[i].y : n[i].x) * fold;
+        q[i] = d != 0.0f ? __fdiv_rn(x, d) : 0.0f;
+    }
+    w0 = d != 0.0f ? e2m1_pack8(q) : 0u;
+    w1 = d != 0.0f ? e2m1_pack8(q + 8) : 0u;
+    return e;
+}
+
+__device__ __forceinline__ uint32_t nvfp4_unit_ieee(const float2* n, float2 am, float s, float fold,
+                                                    uint32_t (&w)[4]) {
+    const uint32_t e0 = nvfp4_block_ieee<false>(n, am.x, s, fold, w[0], w[1]);
+    const uint32_t e1 = nvfp4_block_ieee<true>(n, am.y, s, fold, w[2], w[3]);
+    return e0 | (e1 << 8);
 }
 
 // NVFP4 rule for the two blocks of a unit against the FP32 scale of `c`:
