@@ -15,6 +15,7 @@
 #include "fp4q_dequant.cuh"
 #include "fp4q_device.cuh"
 #include "fp4q_mma.cuh"
+#include "fp4q_mma_wide.cuh"
 #include "fp4q_quant.cuh"
 
 #define FP4Q_API extern "C" __attribute__((visibility("default")))
@@ -187,17 +188,27 @@ fp4q_status launch_quant_h(int had, const CUtensorMap& map, const QuantParams& p
 }
 
 // ---------------------------------------------------------------- tensor-core rotation launch
-// Rotation sizes 16..128 on K a multiple of the 128-column tile go through the
-// tcgen05 kernel; other shapes use the register-FWHT warp pipelines.
-bool use_mma(int had, int64_t K) { return had >= 16 && had <= 128 && K % kMmaTile == 0; }
+// Rotations on K a multiple of the 128-column tile go through the tcgen05
+// kernels (sizes 16..128: one UMMA tile per block group; 256, 512: H_128 on
+// the tensor cores and the cross-group butterfly in the epilogue); other
+// shapes use the register-FWHT warp pipelines.
+bool use_mma(int had, int64_t K) { return had >= 16 && K % kMmaTile == 0; }
 
 template <int FMT, int HAD, bool AMAX>
 fp4q_status launch_mma_t(const CUtensorMap& map, const MmaParams& p, int grid, cudaStream_t s) {
-    auto kern = had_mma_kernel<FMT, HAD, AMAX>;
     static std::atomic<uint64_t> done{0};
-    fp4q_status st = ensure_smem(kern, kMmaSmemBytes, done);
-    if (st != FP4Q_OK) return st;
-    kern<<<grid, kMmaThreads, kMmaSmemBytes, s>>>(map, p);
+    if constexpr (HAD <= kMmaTile) {
+        auto kern = had_mma_kernel<FMT, HAD, AMAX>;
+        fp4q_status st = ensure_smem(kern, kMmaSmemBytes, done);
+        if (st != FP4Q_OK) return st;
+        kern<<<grid, kMmaThreads, kMmaSmemBytes, s>>>(map, p);
+    } else {
+        auto kern = had_mma_wide_kernel<FMT, HAD, AMAX>;
+        constexpr int smem = Wide<HAD>::smem;
+        fp4q_status st = ensure_smem(kern, smem, done);
+        if (st != FP4Q_OK) return st;
+        kern<<<grid, kWideThreads, smem, s>>>(map, p);
+    }
     return launch_status();
 }
 
@@ -208,6 +219,8 @@ fp4q_status launch_mma_h(int had, const CUtensorMap& map, const MmaParams& p, in
         case 32: return launch_mma_t<FMT, 32, AMAX>(map, p, grid, s);
         case 64: return launch_mma_t<FMT, 64, AMAX>(map, p, grid, s);
         case 128: return launch_mma_t<FMT, 128, AMAX>(map, p, grid, s);
+        case 256: return launch_mma_t<FMT, 256, AMAX>(map, p, grid, s);
+        case 512: return launch_mma_t<FMT, 512, AMAX>(map, p, grid, s);
         default: return FP4Q_ERR_INVALID_ARG;
     }
 }
@@ -245,7 +258,8 @@ fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, in
     CUtensorMap map;
     std::memset(&map, 0, sizeof(map));
     const bool mma = use_mma(had, K);
-    if (had < 256 && (st = make_x_map(&map, x, M, K, ldx, mma ? kMmaTile : 8)) != FP4Q_OK) return st;
+    if ((mma || had < 256) && (st = make_x_map(&map, x, M, K, ldx, mma ? kMmaTile : 8)) != FP4Q_OK)
+        return st;
 
     QuantParams p{};
     p.M = M;
@@ -270,7 +284,7 @@ fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, in
         MmaParams q{};
         q.M = M;
         q.K = K;
-        q.n_ct = K / kMmaTile;
+        q.n_ct = K / std::max(had, kMmaTile);
         q.n_tiles = (M + kMmaTile - 1) / kMmaTile * q.n_ct;
         q.codes = codes;
         q.scales = scales;
@@ -348,7 +362,7 @@ __global__ void selftest_div_kernel(const float* x, const float* d, int64_t n, f
          i += (int64_t)gridDim.x * blockDim.x) {
         const float dv = d[i], xv = x[i];
         qi[i] = __fdiv_rn(xv, dv);
-        qf[i] = div_fast_ok(dv, fabsf(xv)) ? div_rn(xv, dv, __frcp_rn(dv)) : __fdiv_rn(xv, dv);
+        qf[i] = div_fast_ok(dv, fabsf(xv)) ? div_split(-xv, dv, make_rcp(dv)) : __fdiv_rn(xv, dv);
     }
 }
 

@@ -108,7 +108,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
           "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr)
         : "memory");
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    // The wait takes the destination registers as operands, so no use of them
+    // can be scheduled before the asynchronous load has completed.
+    asm volatile(
+        "tcgen05.wait::ld.sync.aligned;"
+        : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+          "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+          "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+          "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+          "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+        :
+        : "memory");
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
@@ -129,7 +139,7 @@ constexpr int kMmaBarOff = kMmaRingOff + kMmaStages * kTileBytes;
 constexpr int kMmaNumBars = 2 * kMmaStages + 2 * kEpiGroups + 1;
 constexpr int kMmaSlotOff = kMmaBarOff + kMmaNumBars * 8;
 constexpr int kMmaTabOff = (kMmaSlotOff + 4 + 15) / 16 * 16;
-constexpr int kMmaRedOff = kMmaTabOff + 128 * 8;
+constexpr int kMmaRedOff = kMmaTabOff + 128 * 16;
 constexpr int kMmaSmemBytes = 1024 + kMmaRedOff + (kMmaThreads / 32) * 4;
 static_assert(kMmaSmemBytes <= 227 * 1024, "shared memory");
 
@@ -178,7 +188,7 @@ struct MmaParams {
 // Quantize the 32 values of one chunk (negated pairs n) and store codes and
 // scale bytes.  Returns the scale bytes of the chunk (NVFP4/dual: two).
 template <int FMT>
-__device__ __forceinline__ uint32_t quant_chunk(const float2* n, const ScaleCtx& ctx, const float2* tab,
+__device__ __forceinline__ uint32_t quant_chunk(const float2* n, const ScaleCtx& ctx, const float4* tab,
                                                 uint8_t* cp) {
     uint32_t w[4], e;
     if constexpr (FMT == FMT_MXFP4) {
@@ -203,7 +213,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     const uint32_t accf0 = empty0 + 8 * kMmaStages, acce0 = accf0 + 8 * kEpiGroups;
     const uint32_t done_bar = acce0 + 8 * kEpiGroups;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kMmaSlotOff);
-    float2* tab = reinterpret_cast<float2*>(smem + kMmaTabOff);
+    float4* tab = reinterpret_cast<float4*>(smem + kMmaTabOff);
     float* red = reinterpret_cast<float*>(smem + kMmaRedOff);
     constexpr bool kOddLog = HAD == 32 || HAD == 128;  // RN(1/sqrt(2)) left for the epilogue
 
@@ -358,9 +368,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
                         gm = fmaxf(gm, fmaxf(am.x, am.y));
                         pin(gm);
                     }
-                    const float Gs = (gm >= 0x1p-90f) ? div2(make_float2(-gm, 0.0f), dup2(2688.0f),
-                                                             dup2(-__uint_as_float(kRcp2688Bits))).x
-                                                      : __fdiv_rn(gm, 2688.0f);
+                    const float Gs = (gm >= 0x1p-90f) ? div_split(-gm, 2688.0f, rcp2688()) : __fdiv_rn(gm, 2688.0f);
                     ctx = make_ctx(Gs);
                     if (live) p.scale_fp32[row * (p.K / 128) + ct] = Gs;
                 }

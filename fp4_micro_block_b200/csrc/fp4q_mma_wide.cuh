@@ -1,0 +1,382 @@
+// fp4q_mma_wide.cuh -- tensor-core block Hadamard of size n = 256 or 512 fused
+// with NVFP4 / MXFP4 / dual-scale quantization.
+//
+// Sylvester's matrix factors as H_n = H_G (x) H_128 (G = n / 128): with the
+// column index i = 128 a + b of an n-block,
+//     y[128 a + b] = sum_a' H_G[a][a'] * z[128 a' + b],   z = H_128 applied to
+//     each 128-column group of the block.
+// The tensor cores compute every z group as a 128 x 128 x 128 UMMA (the B
+// operand is -2^-4 H_128, so TMEM receives negated, partly normalised values);
+// the epilogue applies the G-point butterfly across the groups in registers.
+// (FP4Quant builds its 512-point FWHT the same way, as a small transform
+// inside a level of size 32 plus a level across it; here the inner level is a
+// dense product on the tensor cores.)
+//
+// A tile is 128 rows x n columns: G accumulators of 128 TMEM columns, all 512
+// columns for n = 512 (two tiles in flight for n = 256).  All four epilogue
+// warpgroups work on the same tile, warpgroup w on the columns
+// b in [32 w, 32 w + 32) of every group:
+//   pass 1  reads z in steps of 8 columns of every group, applies H_G (and
+//           RN(1/sqrt 2) for n = 512), takes the per-group maxima and writes
+//           y back into TMEM in place;
+//   (dual)  the group maxima of the four warpgroups meet in shared memory;
+//   pass 2  reads y group by group (32 columns = one quantization unit), hands
+//           each group's columns back to the MMA warp as soon as every warp has
+//           read them (the next tile's UMMAs then overlap the rest of pass 2),
+//           and quantizes.
+#pragma once
+
+#include "fp4q_mma.cuh"
+
+namespace fp4q {
+
+constexpr int kWideEpiWarps = 16;                    // four warpgroups
+constexpr int kWideThreads = 64 + 32 * kWideEpiWarps;
+constexpr int kWideRedBytes = 2 * 4 * 4 * kMmaTile * 4;  // [parity][warpgroup][group][row] fp32
+
+template <int HAD>
+struct Wide {
+    static constexpr int G = HAD / kMmaTile;           // 128-column groups per block
+    static constexpr int NBUF = 4 / G;                 // tiles in TMEM
+    static constexpr int bars = 2 * kMmaStages + NBUF + NBUF * G + 2 + 1;
+    static constexpr int ring_off = kTileBytes;
+    static constexpr int red_off = ring_off + kMmaStages * kTileBytes;
+    static constexpr int bar_off = red_off + kWideRedBytes;
+    static constexpr int slot_off = bar_off + bars * 8;
+    static constexpr int tab_off = (slot_off + 4 + 15) / 16 * 16;
+    static constexpr int misc_off = tab_off + 128 * 16;
+    static constexpr int smem = 1024 + misc_off + (kWideThreads / 32) * 4;
+    static_assert(smem <= 227 * 1024, "shared memory");
+};
+
+// Issues the load of 8 fp32 columns; the values are valid only after
+// tmem_wait_ld8x(), which takes them as operands so that no use is scheduled
+// before the wait.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]),
+                   "=f"(v[7])
+                 : "r"(taddr)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld8x2(float (&a)[8], float (&b)[8]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+f"(a[0]), "+f"(a[1]), "+f"(a[2]), "+f"(a[3]), "+f"(a[4]), "+f"(a[5]), "+f"(a[6]), "+f"(a[7]),
+                   "+f"(b[0]), "+f"(b[1]), "+f"(b[2]), "+f"(b[3]), "+f"(b[4]), "+f"(b[5]), "+f"(b[6]), "+f"(b[7])
+                 :
+                 : "memory");
+}
+template <int G>
+__device__ __forceinline__ void tmem_wait_ld8x(float (&z)[G][8]) {
+    if constexpr (G == 2) {
+        tmem_wait_ld8x2(z[0], z[1]);
+    } else {
+        asm volatile("tcgen05.wait::ld.sync.aligned;"
+                     : "+f"(z[0][0]), "+f"(z[0][1]), "+f"(z[0][2]), "+f"(z[0][3]), "+f"(z[0][4]), "+f"(z[0][5]),
+                       "+f"(z[0][6]), "+f"(z[0][7]), "+f"(z[1][0]), "+f"(z[1][1]), "+f"(z[1][2]), "+f"(z[1][3]),
+                       "+f"(z[1][4]), "+f"(z[1][5]), "+f"(z[1][6]), "+f"(z[1][7]), "+f"(z[2][0]), "+f"(z[2][1]),
+                       "+f"(z[2][2]), "+f"(z[2][3]), "+f"(z[2][4]), "+f"(z[2][5]), "+f"(z[2][6]), "+f"(z[2][7]),
+                       "+f"(z[3][0]), "+f"(z[3][1]), "+f"(z[3][2]), "+f"(z[3][3]), "+f"(z[3][4]), "+f"(z[3][5]),
+                       "+f"(z[3][6]), "+f"(z[3][7])
+                     :
+                     : "memory");
+    }
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+                 "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+                 "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// B = -2^-4 * H_128 (K-major, 128-byte swizzle) for n = 256 and 512.
+__device__ __forceinline__ void build_h128_b(uint8_t* b) {
+    const uint32_t mag = 0x3f80u - 4u * 0x80u;  // bf16 bits of 2^-4
+    for (int chunk = threadIdx.x; chunk < kTileBytes / 16; chunk += blockDim.x) {
+        const int h = chunk / 1024, nn = (chunk / 8) % 128, cp = chunk % 8;
+        const int c = cp ^ (nn & 7);
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+            uint32_t pair = 0;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const int k = h * 64 + c * 8 + e + t;
+                const int par = __popc((uint32_t)(k & nn)) & 1;
+                pair |= (mag | (par ? 0u : 0x8000u)) << (16 * t);
+            }
+            w[e / 2] = pair;
+        }
+        *reinterpret_cast<uint4*>(b + chunk * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+template <int FMT, int HAD, bool AMAX_ONLY>
+__global__ void __launch_bounds__(kWideThreads, 1)
+    had_mma_wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const MmaParams p) {
+    using W = Wide<HAD>;
+    constexpr int G = W::G, NBUF = W::NBUF;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    const uint32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t full0 = smem_u32(smem + W::bar_off), empty0 = full0 + 8 * kMmaStages;
+    const uint32_t accf0 = empty0 + 8 * kMmaStages, relg0 = accf0 + 8 * NBUF;
+    const uint32_t redb0 = relg0 + 8 * NBUF * G;  // [2] dual: the four warpgroups' group maxima
+    const uint32_t done_bar = redb0 + 16;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + W::slot_off);
+    float4* tab = reinterpret_cast<float4*>(smem + W::tab_off);
+    float* red = reinterpret_cast<float*>(smem + W::misc_off);
+    float* red2 = reinterpret_cast<float*>(smem + W::red_off);
+    constexpr bool kOddLog = HAD == 512;
+
+    if (tid == 0) {
+        prefetch_tmap(&tmap_x);
+        for (int s = 0; s < kMmaStages; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, 1);
+        }
+        for (int b = 0; b < NBUF; ++b) mbar_init(accf0 + 8 * b, 1);
+        for (int k = 0; k < NBUF * G; ++k) mbar_init(relg0 + 8 * k, kWideEpiWarps);
+        for (int k = 0; k < 2; ++k) mbar_init(redb0 + 8 * k, kWideEpiWarps);
+        mbar_init(done_bar, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), 512u);
+        tmem_relinquish();
+    }
+    build_h128_b(smem);
+    fence_proxy_async_smem();
+    float s_t = 0.0f;
+    if constexpr (FMT == FMT_NVFP4 && !AMAX_ONLY) {
+        if (p.dynamic) {
+            s_t = tensor_scale_from_partials(p.partials, p.n_partials, red);
+            if (blockIdx.x == 0 && tid == 0) *p.scale_fp32 = s_t;
+        } else {
+            s_t = *p.scale_fp32;
+        }
+        build_table(tab, s_t);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int64_t n_my = p.n_tiles > (int64_t)blockIdx.x ? (p.n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    float my_amax = 0.0f;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer: G sub-tiles per tile
+        if (lane == 0) {
+            const int64_t n_sub = n_my * G;
+            int64_t u = 0;
+            for (; u < n_sub; ++u) {
+                const int s = (int)(u % kMmaStages);
+                if (u >= kMmaStages && !mbar_wait(empty0 + 8 * s, (uint32_t)((u / kMmaStages - 1) & 1))) {
+                    atomicOr(&g_device_error, kErrWaitTimeout);
+                    break;
+                }
+                const int64_t t = blockIdx.x + (u / G) * gridDim.x;
+                const int32_t x0 = (int32_t)((t % p.n_ct) * HAD + (u % G) * kMmaTile);
+                const int32_t y0 = (int32_t)((t / p.n_ct) * kMmaTile);
+                const uint32_t dst = smem_u32(smem + W::ring_off + s * kTileBytes);
+                mbar_arrive_expect_tx(full0 + 8 * s, kTileBytes);
+                tma_load_2d(dst, &tmap_x, x0, y0, full0 + 8 * s);
+                tma_load_2d(dst + kHalfBytes, &tmap_x, x0 + 64, y0, full0 + 8 * s);
+            }
+            for (int64_t k = u > kMmaStages ? u - kMmaStages : 0; k < u; ++k)
+                (void)mbar_wait(full0 + 8 * (int)(k % kMmaStages), (uint32_t)((k / kMmaStages) & 1));
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t b_addr = smem_u32(smem);
+            bool ok = true;
+            for (int64_t j = 0; ok && j < n_my; ++j) {
+                const int b = (int)(j % NBUF);
+                for (int a = 0; a < G; ++a) {
+                    const int64_t u = j * G + a;
+                    const int s = (int)(u % kMmaStages);
+                    ok = mbar_wait(full0 + 8 * s, (uint32_t)((u / kMmaStages) & 1));
+                    if (ok && j >= NBUF)
+                        ok = mbar_wait(relg0 + 8 * (b * G + a), (uint32_t)((j / NBUF - 1) & 1));
+                    if (!ok) {
+                        atomicOr(&g_device_error, kErrWaitTimeout);
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + W::ring_off + s * kTileBytes);
+                    const uint32_t d = tmem_base + (uint32_t)((b * G + a) * kMmaTile);
+#pragma unroll
+                    for (int k = 0; k < kMmaTile / 16; ++k) {
+                        const uint32_t off = (uint32_t)((k / 4) * kHalfBytes + (k % 4) * 32);
+                        umma_bf16(d, sw128_desc(a_addr + off), sw128_desc(b_addr + off), kIdescBf16M128N128,
+                                  k > 0 ? 1u : 0u);
+                    }
+                    tc_commit(empty0 + 8 * s);
+                }
+                if (ok) tc_commit(accf0 + 8 * b);
+            }
+            tc_commit(done_bar);
+            if (!mbar_wait(done_bar, 0)) atomicOr(&g_device_error, kErrWaitTimeout);
+        }
+    } else {
+        // ------------------------------------------------ epilogue
+        const uint32_t ew = warp - 2, wg = ew >> 2, quarter = warp & 3;
+        const uint32_t rowt = quarter * 32 + lane;
+        const uint32_t lane_base = (quarter * 32u) << 16;
+        const float rs2 = __uint_as_float(0x3f3504f3u);  // RN(1/sqrt(2))
+        const ScaleCtx ctx_t = make_ctx(s_t);
+        const int64_t kc = p.K / 2;
+#pragma unroll 1
+        for (int64_t j = 0; j < n_my; ++j) {
+            const int b = (int)(j % NBUF);
+            const bool ok = mbar_wait(accf0 + 8 * b, (uint32_t)((j / NBUF) & 1));
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) atomicOr(&g_device_error, kErrWaitTimeout);
+                break;
+            }
+            tc_fence_after();
+            const int64_t t = blockIdx.x + j * gridDim.x;
+            const int64_t ct = t % p.n_ct, rt = t / p.n_ct;
+            const int64_t row = rt * kMmaTile + rowt;
+            const bool live = row < p.M;
+            const uint32_t tbuf = tmem_base + lane_base + (uint32_t)(b * G * kMmaTile);
+
+            // ---- pass 1: y = H_G z, group maxima, y back into TMEM
+            float m[G];
+#pragma unroll
+            for (int a = 0; a < G; ++a) m[a] = 0.0f;
+#pragma unroll 1
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t pos = 32u * wg + 8u * k;
+                float z[G][8];
+#pragma unroll
+                for (int a = 0; a < G; ++a) tmem_ld8(tbuf + a * kMmaTile + pos, z[a]);
+                tmem_wait_ld8x<G>(z);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if constexpr (G == 2) {
+                        const float s0 = z[0][i] + z[1][i], d0 = z[0][i] - z[1][i];
+                        z[0][i] = s0;
+                        z[1][i] = d0;
+                    } else {
+                        const float s01 = z[0][i] + z[1][i], d01 = z[0][i] - z[1][i];
+                        const float s23 = z[2][i] + z[3][i], d23 = z[2][i] - z[3][i];
+                        z[0][i] = s01 + s23;
+                        z[1][i] = d01 + d23;
+                        z[2][i] = s01 - s23;
+                        z[3][i] = d01 - d23;
+                    }
+                }
+#pragma unroll
+                for (int a = 0; a < G; ++a) {
+                    if constexpr (kOddLog) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) z[a][i] *= rs2;
+                    }
+                    float mm = fmaxf(fabsf(z[a][0]), fabsf(z[a][1]));
+#pragma unroll
+                    for (int i = 2; i < 8; i += 2) mm = max3(mm, fabsf(z[a][i]), fabsf(z[a][i + 1]));
+                    m[a] = fmaxf(m[a], mm);
+                    if constexpr (!AMAX_ONLY) tmem_st8(tbuf + a * kMmaTile + pos, z[a]);
+                }
+            }
+            if constexpr (AMAX_ONLY) {
+                if (live) {
+#pragma unroll
+                    for (int a = 0; a < G; ++a) my_amax = fmaxf(my_amax, m[a]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    for (int a = 0; a < G; ++a) mbar_arrive(relg0 + 8 * (b * G + a));
+                continue;
+            } else {
+                tmem_wait_st();
+                float gs[G];
+                if constexpr (FMT == FMT_DUAL) {  // group maxima over the four warpgroups
+                    float* rp = red2 + (j & 1) * (4 * 4 * kMmaTile);
+#pragma unroll
+                    for (int a = 0; a < G; ++a) rp[(wg * 4 + a) * kMmaTile + rowt] = m[a];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(redb0 + 8 * (uint32_t)(j & 1));
+                    const bool rok = mbar_wait(redb0 + 8 * (uint32_t)(j & 1), (uint32_t)((j >> 1) & 1));
+                    if (!__all_sync(0xffffffffu, rok)) {
+                        if (lane == 0) atomicOr(&g_device_error, kErrWaitTimeout);
+                        break;
+                    }
+#pragma unroll
+                    for (int a = 0; a < G; ++a) {
+                        float gm = rp[a * kMmaTile + rowt];
+#pragma unroll
+                        for (int w = 1; w < 4; ++w) gm = fmaxf(gm, rp[(w * 4 + a) * kMmaTile + rowt]);
+                        gs[a] = (gm >= 0x1p-90f) ? div_split(-gm, 2688.0f, rcp2688()) : __fdiv_rn(gm, 2688.0f);
+                    }
+                }
+                // ---- pass 2: quantize group by group
+#pragma unroll 1
+                for (int a = 0; a < G; ++a) {
+                    float v[32];
+                    tmem_ld32(tbuf + a * kMmaTile + 32u * wg, v);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(relg0 + 8 * (b * G + a));
+                    if (live) {
+                        float2 n[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) n[i] = make_float2(v[i], v[16 + i]);
+                        const int64_t col = ct * HAD + a * kMmaTile + 32 * wg;
+                        uint32_t w[4], e;
+                        if constexpr (FMT == FMT_MXFP4) {
+                            e = mxfp4_unit(n, w);
+                        } else if constexpr (FMT == FMT_DUAL) {
+                            float g = gs[0];
+#pragma unroll
+                            for (int q = 1; q < G; ++q) g = a == q ? gs[q] : g;
+                            e = nvfp4_unit<false>(n, amax_pair(n), make_ctx(g), tab, 1.0f, w);
+                            if (wg == 0) p.scale_fp32[row * (p.K / 128) + col / 128] = g;
+                        } else {
+                            e = nvfp4_unit<true>(n, amax_pair(n), ctx_t, tab, 1.0f, w);
+                        }
+                        *reinterpret_cast<uint4*>(p.codes + row * kc + col / 2) = make_uint4(w[0], w[1], w[2], w[3]);
+                        if constexpr (FMT == FMT_MXFP4) {
+                            const int64_t nsc = p.K / 32, c0 = col / 32;
+                            if (p.swizzled) p.scales[swizzle_offset(row, c0, (nsc + 3) / 4)] = (uint8_t)e;
+                            else p.scales[row * nsc + c0] = (uint8_t)e;
+                        } else {
+                            const int64_t nsc = p.K / 16, c0 = col / 16;  // c0 even
+                            uint8_t* sp = p.swizzled ? p.scales + swizzle_offset(row, c0, (nsc + 3) / 4)
+                                                     : p.scales + row * nsc + c0;
+                            *reinterpret_cast<uint16_t*>(sp) = (uint16_t)e;
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    if constexpr (AMAX_ONLY) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) my_amax = fmaxf(my_amax, __shfl_xor_sync(0xffffffffu, my_amax, o));
+        if (lane == 0) red[warp] = my_amax;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if constexpr (AMAX_ONLY) {
+        if (tid == 0) {
+            float mx = 0.0f;
+            for (int w = 0; w < kWideThreads / 32; ++w) mx = fmaxf(mx, red[w]);
+            p.partials[blockIdx.x] = mx;
+        }
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512u);
+    }
+}
+
+}  // namespace fp4q

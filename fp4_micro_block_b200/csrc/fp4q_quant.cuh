@@ -86,8 +86,8 @@ struct Geo {
 // reduction slots and the NVFP4 table.
 template <int HAD>
 constexpr int quant_smem_bytes() {
-    return 1024 + kWarps * Geo<HAD>::warp_stride + kWarps * kStages * 8 + (kWarps + 2) * 4 +
-           128 * 8 + 64;
+    return 1024 + kWarps * Geo<HAD>::warp_stride + kWarps * kStages * 8 + (kWarps + 2) * 4 + 16 +
+           128 * 16 + 64;
 }
 
 // Stage byte offset of (row, column) in the G2 geometry: two boxes of
@@ -266,7 +266,8 @@ __global__ void __launch_bounds__(kQuantThreads, Geo<HAD>::min_ctas)
     const uint32_t lane = tid & 31, warp = tid >> 5;
     uint64_t* full_bars = reinterpret_cast<uint64_t*>(smem + kWarps * G::warp_stride);
     float* red = reinterpret_cast<float*>(full_bars + kWarps * kStages);
-    float2* tab = reinterpret_cast<float2*>(red + kWarps + 2);
+    float4* tab = reinterpret_cast<float4*>((reinterpret_cast<uintptr_t>(red + kWarps + 2) + 15) &
+                                            ~uintptr_t(15));
     constexpr bool kFold = HAD == 16 || HAD == 64 || HAD == 256;  // 1/sqrt(n) a power of two
 
     if (tid == 0) {
@@ -387,9 +388,7 @@ __global__ void __launch_bounds__(kQuantThreads, Geo<HAD>::min_ctas)
                         g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, 8));
                         g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, 16));
                     }
-                    const float Gs = (g >= 0x1p-90f) ? div2(make_float2(-g, 0.0f), dup2(2688.0f),
-                                                            dup2(-__uint_as_float(kRcp2688Bits))).x
-                                                     : __fdiv_rn(g, 2688.0f);
+                    const float Gs = (g >= 0x1p-90f) ? div_split(-g, 2688.0f, rcp2688()) : __fdiv_rn(g, 2688.0f);
                     ctx = make_ctx(Gs);
                 }
                 if (live) {

@@ -1,25 +1,26 @@
-// fp4q_unit.cuh -- quantization of one 32-value "unit" with the packed
-// two-wide fp32 instructions of sm_100a (FADD2 / FMUL2 / FFMA2).
+// fp4q_unit.cuh -- quantization of one 32-value "unit" of a row.
 //
 // A unit holds 32 consecutive values v[0..31] of one row.  They are kept
 // NEGATED, as 16 pairs n[i] = (-v[i], -v[16+i]): the first component belongs
 // to block 0 (v[0..15]), the second to block 1 (v[16..31]), so the two
 // 16-element NVFP4 blocks of a unit are always processed side by side, and
 // Walsh-Hadamard stages of stride 1..8 are "vertical" pair operations.
-// Carrying -v costs nothing (the bf16 unpack flips the sign for free) and
-// gives the correctly rounded division below the -x operand it needs.
+// Carrying -v costs nothing (the bf16 unpack and the tensor-core rotation flip
+// the sign for free) and gives the divisions below the -x operand they use.
+//
+// The per-element arithmetic is scalar fp32: on sm_100a the packed FFMA2 /
+// FMUL2 forms save issue slots but run at half the FMA-pipe rate of scalar
+// FFMA, and the quantizer is bound by that pipe.
 #pragma once
 
 #include "fp4q_device.cuh"
 
 namespace fp4q {
 
-__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
-__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
-    return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);  // RN(a - b)
-}
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+// Component-wise pair arithmetic (scalar instructions, see above).
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return make_float2(a.x - b.x, a.y - b.y); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return make_float2(a.x * b.x, a.y * b.y); }
 __device__ __forceinline__ float2 dup2(float a) { return make_float2(a, a); }
 
 // Negated bf16 -> binary32 (exact): w = (lo, hi) bf16 pair.  w * 2^16 + 2^31
@@ -29,21 +30,48 @@ __device__ __forceinline__ float nbf16hi(uint32_t w) {
     return __uint_as_float((w & 0xffff0000u) ^ 0x80000000u);
 }
 
-// RN(1/6) and RN(1/2688) as binary32 (checked against exact rationals).
-constexpr uint32_t kRcp6Bits = 0x3e2aaaabu;
-constexpr uint32_t kRcp2688Bits = 0x39c30c31u;
+// ------------------------------------------------------------------------------
+// Division with a split reciprocal (4 FMA-pipe operations per quotient).
+//
+// For a divisor d > 0 keep rn = RN(1/d), rz = RZ(1/d) (largest float <= 1/d)
+// and lo = RN((1 - d*rz) * rz) >= 0, so that rz + lo = 1/d within 2^-45
+// relative (1 - d*rz is exact by FMA).  Then
+//     q0 = RN(x*rz + RN(x*lo))
+// is within (1/2 + 2^-21) ulp of x/d, hence faithful, and Markstein's
+// correction theorem (P. Markstein, IBM J. Res. Dev. 34, 1990: with rn within
+// half an ulp of 1/d and q0 faithful, the remainder x - q0*d is exact and
+// RN(q0 + (x - q0*d)*rn) = RN(x/d)) gives the correctly rounded quotient in one
+// step.  lo >= 0 makes x*rz and x*lo carry the sign of x, so a zero x keeps its
+// sign through every step.  Preconditions as for div_rn: d in [2^-100, 2^100],
+// |x|/d <= 2^100; quotients below 2^-100 may be off by an ulp and still encode
+// to a zero E2M1 code of the right sign.
+// ------------------------------------------------------------------------------
+struct Rcp {
+    float rn, rz, lo;
+};
 
-// Correctly rounded quotient x/d for both lanes, from nx = -x, d and
-// ny = -RN(1/d): two Markstein corrections of x*RN(1/d) (see div_rn in
-// fp4q_device.cuh for the argument and the preconditions).  The remainder is
-// formed as q*d - x so that a zero quotient carries the sign of x.
-__device__ __forceinline__ float2 div2(float2 nx, float2 d, float2 ny) {
-    float2 q = mul2(nx, ny);
-    float2 e = fma2(q, d, nx);
-    q = fma2(e, ny, q);
-    e = fma2(q, d, nx);
-    q = fma2(e, ny, q);
-    return q;
+__device__ __forceinline__ Rcp make_rcp(float d) {  // d > 0, normal
+    Rcp c;
+    c.rn = __frcp_rn(d);
+    c.rz = fmaf(-d, c.rn, 1.0f) < 0.0f ? __uint_as_float(__float_as_uint(c.rn) - 1u) : c.rn;
+    c.lo = fmaf(-d, c.rz, 1.0f) * c.rz;
+    return c;
+}
+
+// x/d from nx = -x.
+__device__ __forceinline__ float div_split(float nx, float d, const Rcp& c) {
+    const float t = nx * -c.lo;           // x*lo
+    const float q0 = fmaf(nx, -c.rz, t);  // x*rz + x*lo: faithful
+    const float e = fmaf(q0, d, nx);      // q0*d - x, exact
+    return fmaf(-e, c.rn, q0);            // q0 - e*rn
+}
+
+// Split reciprocals of 6 and 2688 (RN, RZ, lo; checked against exact rationals).
+__device__ __forceinline__ Rcp rcp6() {
+    return Rcp{__uint_as_float(0x3e2aaaabu), __uint_as_float(0x3e2aaaaau), __uint_as_float(0x322aaaaau)};
+}
+__device__ __forceinline__ Rcp rcp2688() {
+    return Rcp{__uint_as_float(0x39c30c31u), __uint_as_float(0x39c30c30u), __uint_as_float(0x2dc30c30u)};
 }
 
 // ---------------------------------------------------------------- Walsh-Hadamard
@@ -126,10 +154,10 @@ __device__ __forceinline__ float2 e4m3x2_decode(uint32_t e2) {
 // per block, 2^-90 <= amax <= 2^62 * s (or amax = 0): then every quotient below
 // stays in the normal range, (amax/6)/s <= 2^60, and each decoded block scale
 // d = E4M3(e) * s is either 0 or in [2^-99, 2^99], which are the preconditions
-// of the packed division.
+// of the split-reciprocal division.
 struct ScaleCtx {
     float s;       // the FP32 scale
-    float nrs;     // -RN(1/s)
+    Rcp rs;        // split reciprocal of s
     float am_max;  // 2^62 * s
     bool fast;
 };
@@ -138,18 +166,20 @@ __device__ __forceinline__ ScaleCtx make_ctx(float s) {
     ScaleCtx c;
     c.s = s;
     c.fast = s >= 0x1p-90f && s <= 0x1p90f;
-    c.nrs = c.fast ? -__frcp_rn(s) : 0.0f;
+    c.rs = c.fast ? make_rcp(s) : Rcp{0.0f, 0.0f, 0.0f};
     c.am_max = s * 0x1p62f;
     return c;
 }
 
-// Per-CTA table of the NVFP4 decoded scales for a fixed s: t[e] = (d, ny) with
-// d = E4M3(e) * s and ny = -RN(1/d) (0 when d == 0), for the 128 non-negative
-// E4M3 bytes.
-__device__ __forceinline__ void build_table(float2* t, float s) {
+// Per-CTA table of the NVFP4 decoded scales for a fixed s: t[e] = (d, rn, rz,
+// lo) with d = E4M3(e) * s and the split reciprocal of d (zeros when d == 0 or
+// d is outside [2^-100, 2^100]), for the 128 non-negative E4M3 bytes.
+__device__ __forceinline__ void build_table(float4* t, float s) {
     for (int e = threadIdx.x; e < 128; e += blockDim.x) {
         const float d = (e < 127) ? e4m3_decode((uint32_t)e) * s : 0.0f;
-        t[e] = make_float2(d, (d >= 0x1p-100f && d <= 0x1p100f) ? -__frcp_rn(d) : 0.0f);
+        const bool ok = d >= 0x1p-100f && d <= 0x1p100f;
+        const Rcp c = ok ? make_rcp(d) : Rcp{0.0f, 0.0f, 0.0f};
+        t[e] = make_float4(d, c.rn, c.rz, c.lo);
     }
 }
 
@@ -192,37 +222,50 @@ __device__ __forceinline__ uint32_t nvfp4_unit_ieee(const float2* n, float2 am, 
 // writes the codes to w.
 template <bool TABLE>
 __device__ __forceinline__ uint32_t nvfp4_unit(const float2* n, float2 am, const ScaleCtx& c,
-                                               const float2* tab, float fold, uint32_t (&w)[4]) {
-    am = mul2(am, dup2(fold));
+                                               const float4* tab, float fold, uint32_t (&w)[4]) {
+    am.x *= fold;
+    am.y *= fold;
     const uint32_t b0 = __float_as_uint(am.x), b1 = __float_as_uint(am.y);
     const uint32_t tiny = __float_as_uint(0x1p-90f);  // amax == 0 passes, 0 < amax < 2^-90 fails
     const bool in_range = c.fast && (b0 - 1u) >= tiny - 1u && (b1 - 1u) >= tiny - 1u &&
                           fmaxf(am.x, am.y) <= c.am_max;
     if (!in_range) return nvfp4_unit_ieee(n, am, c.s, fold, w);
-    const float r6 = __uint_as_float(kRcp6Bits);
-    const float2 bs = div2(make_float2(-am.x, -am.y), dup2(6.0f), dup2(-r6));
-    const float2 r = div2(make_float2(-bs.x, -bs.y), dup2(c.s), dup2(c.nrs));
-    const uint32_t e2 = e4m3x2_encode(r);
-    float2 d, ny;
+    const Rcp r6 = rcp6();
+    const float bs0 = div_split(-am.x, 6.0f, r6), bs1 = div_split(-am.y, 6.0f, r6);
+    const float r0 = div_split(-bs0, c.s, c.rs), r1 = div_split(-bs1, c.s, c.rs);
+    const uint32_t e2 = e4m3x2_encode(make_float2(r0, r1));
+    float d0, d1;
+    Rcp c0, c1;
     if constexpr (TABLE) {
-        const float2 t0 = tab[e2 & 0xffu], t1 = tab[e2 >> 8];
-        d = make_float2(t0.x, t1.x);
-        ny = make_float2(t0.y, t1.y);
+        const float4 t0 = tab[e2 & 0xffu], t1 = tab[e2 >> 8];
+        d0 = t0.x; c0 = Rcp{t0.y, t0.z, t0.w};
+        d1 = t1.x; c1 = Rcp{t1.y, t1.z, t1.w};
     } else {
-        d = mul2(e4m3x2_decode(e2), dup2(c.s));
-        ny = make_float2(d.x != 0.0f ? -__frcp_rn(d.x) : 0.0f, d.y != 0.0f ? -__frcp_rn(d.y) : 0.0f);
+        const float2 dd = e4m3x2_decode(e2);
+        d0 = dd.x * c.s;
+        d1 = dd.y * c.s;
+        c0 = d0 != 0.0f ? make_rcp(d0) : Rcp{0.0f, 0.0f, 0.0f};
+        c1 = d1 != 0.0f ? make_rcp(d1) : Rcp{0.0f, 0.0f, 0.0f};
     }
     if (fold != 1.0f) {  // divide z by d / 2^-k
         const float inv = 1.0f / fold;  // exact: a power of two
-        d = mul2(d, dup2(inv));
-        ny = mul2(ny, dup2(fold));
+        d0 *= inv;
+        d1 *= inv;
+        c0 = Rcp{c0.rn * fold, c0.rz * fold, c0.lo * fold};
+        c1 = Rcp{c1.rn * fold, c1.rz * fold, c1.lo * fold};
     }
-    float2 q[16];
+    float q0[16], q1[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) q[i] = div2(n[i], d, ny);
-    pack_codes(q, w);
-    if (d.x == 0.0f) w[0] = w[1] = 0u;  // zero block scale: all codes +0
-    if (d.y == 0.0f) w[2] = w[3] = 0u;
+    for (int i = 0; i < 16; ++i) {
+        q0[i] = div_split(n[i].x, d0, c0);
+        q1[i] = div_split(n[i].y, d1, c1);
+    }
+    w[0] = e2m1_pack8(q0);
+    w[1] = e2m1_pack8(q0 + 8);
+    w[2] = e2m1_pack8(q1);
+    w[3] = e2m1_pack8(q1 + 8);
+    if (d0 == 0.0f) w[0] = w[1] = 0u;  // zero block scale: all codes +0
+    if (d1 == 0.0f) w[2] = w[3] = 0u;
     return e2;
 }
 
@@ -237,16 +280,13 @@ __device__ __forceinline__ uint32_t mxfp4_unit(const float2* n, uint32_t (&w)[4]
     }
     const uint32_t ef = __float_as_uint(am) >> 23;
     const uint32_t b = ef >= 2u ? ef - 2u : 0u;
-    const float2 nm = dup2(-__uint_as_float((254u - b) << 23));  // -2^(127-b), normal for b <= 252
-    float2 q[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) q[i] = mul2(n[i], nm);
-    // q[i] = (v[i], v[16+i]) * 2^(127-b): codes in element order
+    const float nm = -__uint_as_float((254u - b) << 23);  // -2^(127-b), normal for b <= 252
+    // codes in element order: v[i] = -n[i].x * 2^(127-b), v[16+i] = -n[i].y * ...
     float v[32];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-        v[i] = q[i].x;
-        v[16 + i] = q[i].y;
+        v[i] = n[i].x * nm;
+        v[16 + i] = n[i].y * nm;
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) w[i] = e2m1_pack8(v + 8 * i);

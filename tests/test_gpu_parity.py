@@ -52,6 +52,11 @@ def test_division_is_correctly_rounded(fq):
     q = mids[rng.integers(0, len(mids), k)]
     q = (q.view(np.int32) + rng.integers(-3, 4, k).astype(np.int32)).view(np.float32)
     x[:k] = (q.astype(np.float64) * d[:k]).astype(np.float32) * np.where(rng.random(k) < .5, -1, 1)
+    # quotients next to midpoints between adjacent binary32 values (rounding ties
+    # of the quotient itself): x = RN(m * d) for m = (2j + 1) * 2^-25 * 2^E in [2^(E-1), 2^E)
+    m = ((2 * rng.integers(1 << 23, 1 << 24, k) + 1).astype(np.float64) * 2.0 ** -25 *
+         np.exp2(rng.integers(-4, 3, k)))
+    x[k + 2:2 * k + 2] = (m * d[k + 2:2 * k + 2].astype(np.float64)).astype(np.float32)
     x[k] = -0.0
     x[k + 1] = 0.0
     xt, dt = torch.from_numpy(x).cuda(), torch.from_numpy(d).cuda()
