@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <utility>
 
 #include "../../include/fp4q.h"
 #include "fp4q_arc.cuh"
@@ -110,6 +111,24 @@ bool valid_had(int n) {
     return n == 0 || n == 16 || n == 32 || n == 64 || n == 128 || n == 256 || n == 512;
 }
 
+// Launches kern on stream s with programmatic stream serialization, so the
+// kernel's prologue may overlap the end of the previous kernel in the stream
+// (each kernel waits in pdl_wait() before it touches global memory).
+template <typename... KArgs, typename... Args>
+fp4q_status launch(void (*kern)(KArgs...), int grid, int threads, int smem, cudaStream_t s, Args&&... args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess ? FP4Q_OK : FP4Q_ERR_CUDA;
+}
+
 fp4q_status launch_status() {
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? FP4Q_OK : FP4Q_ERR_CUDA;
@@ -167,9 +186,9 @@ fp4q_status launch_quant_t(const CUtensorMap& map, QuantParams p, int sms, cudaS
     p.n_wt = p.n_rb * p.n_cb;
     const int grid = (int)std::min<int64_t>(
         {(p.n_wt + kWarps - 1) / kWarps, (int64_t)per_sm * sms, (int64_t)kMaxGrid});
-    kern<<<grid, kQuantThreads, smem, s>>>(map, p);
+    st = launch(kern, grid, kQuantThreads, smem, s, map, p);
     if (grid_out) *grid_out = grid;
-    return launch_status();
+    return st;
 }
 
 template <int FMT, bool AMAX>
@@ -201,15 +220,14 @@ fp4q_status launch_mma_t(const CUtensorMap& map, const MmaParams& p, int grid, c
         auto kern = had_mma_kernel<FMT, HAD, AMAX>;
         fp4q_status st = ensure_smem(kern, kMmaSmemBytes, done);
         if (st != FP4Q_OK) return st;
-        kern<<<grid, kMmaThreads, kMmaSmemBytes, s>>>(map, p);
+        return launch(kern, grid, kMmaThreads, kMmaSmemBytes, s, map, p);
     } else {
         auto kern = had_mma_wide_kernel<FMT, HAD, AMAX>;
         constexpr int smem = Wide<HAD>::smem;
         fp4q_status st = ensure_smem(kern, smem, done);
         if (st != FP4Q_OK) return st;
-        kern<<<grid, kWideThreads, smem, s>>>(map, p);
+        return launch(kern, grid, kWideThreads, smem, s, map, p);
     }
-    return launch_status();
 }
 
 template <int FMT, bool AMAX>
@@ -326,8 +344,7 @@ fp4q_status launch_dequant_t(const DequantParams& p, int grid, cudaStream_t s) {
     static std::atomic<uint64_t> done{0};
     fp4q_status st = ensure_smem(kern, smem, done);
     if (st != FP4Q_OK) return st;
-    kern<<<grid, kThreads, smem, s>>>(p);
-    return launch_status();
+    return launch(kern, grid, kThreads, smem, s, p);
 }
 
 // Rotation sizes 0, 16, 32: the streaming kernel, 4 CTAs of 256 threads per SM.
@@ -337,8 +354,7 @@ fp4q_status launch_dequant_stream(const DequantParams& p, int sms, cudaStream_t 
     const int grid = (int)std::min<int64_t>({(units + kThreads - 1) / kThreads, (int64_t)3 * sms,
                                             (int64_t)kMaxGrid});
     const int w32 = ((reinterpret_cast<uintptr_t>(p.y) & 31) == 0 && (p.K & 15) == 0) ? 1 : 0;
-    dequant_stream_kernel<FMT, HAD><<<grid, kThreads, 0, s>>>(p, w32);
-    return launch_status();
+    return launch(dequant_stream_kernel<FMT, HAD>, grid, kThreads, 0, s, p, w32);
 }
 
 template <int FMT>
@@ -524,8 +540,7 @@ FP4Q_API fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int6
         if (smem > 48 * 1024 &&
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return FP4Q_ERR_CUDA;
-        kern<<<grid, threads, smem, (cudaStream_t)stream>>>(p);
-        return launch_status();
+        return launch(kern, grid, threads, smem, (cudaStream_t)stream, p);
     };
     if (threads <= 256) {
         if (dynamic && (st = run(arc_kernel<true, 256>)) != FP4Q_OK) return st;

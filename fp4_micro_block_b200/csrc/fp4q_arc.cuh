@@ -37,6 +37,8 @@ struct ArcParams {
 //                       [red: 32 fp32][bars: kArcStages u64]
 template <bool AMAX_ONLY, int MAXT>
 __global__ void __launch_bounds__(MAXT, MAXT <= 256 ? 2 : 1) arc_kernel(const ArcParams p) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                                ~uintptr_t(127));

@@ -160,6 +160,8 @@ __device__ __forceinline__ void store_bf16x32(uint16_t* dst, const uint32_t* o, 
 
 template <int FMT, int HAD>
 __global__ void __launch_bounds__(kThreads, 3) dequant_stream_kernel(const DequantParams p, int w32) {
+    pdl_wait();
+    pdl_trigger();
     // rows < 2^31 and units per row < 2^26: 32-bit unit coordinates
     const int32_t upr = (int32_t)((p.K + 31) / 32);  // units per row
     const int32_t M = (int32_t)p.M;
@@ -219,6 +221,8 @@ constexpr int kDequantCtasPerSm = FP4Q_DEQUANT_CTAS_PER_SM;
 
 template <int FMT, int HAD>
 __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_kernel(const DequantParams p) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     float* scratch = reinterpret_cast<float*>(smem_raw);
     const uint32_t tid = threadIdx.x;

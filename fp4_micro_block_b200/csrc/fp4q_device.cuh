@@ -279,6 +279,14 @@ __device__ __forceinline__ void bar_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+// Programmatic dependent launch: every kernel is launched so that it may start
+// while the previous kernel of the stream is finishing.  pdl_wait() blocks
+// until that kernel has completed and its writes are visible, and comes before
+// the first global read or write; pdl_trigger() lets the next kernel launch
+// (it still waits for this one to complete before touching memory).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // 128-byte TMA swizzle: the 16-byte chunk index inside a 128-byte row is XORed
 // with the row index modulo 8 (box bases are 1024-byte aligned).
 __device__ __forceinline__ uint32_t swz128(uint32_t row, uint32_t byte_in_row) {

@@ -38,7 +38,7 @@ namespace fp4q {
 constexpr int kMmaTile = 128;                         // tile rows = tile columns
 constexpr int kMmaStages = FP4Q_MMA_STAGES;           // X ring depth
 constexpr int kEpiGroups = FP4Q_EPI_GROUPS;           // epilogue warpgroups = accumulators
-constexpr int kMmaThreads = 64 + 128 * kEpiGroups;
+constexpr int kMmaThreads = 96 + 128 * kEpiGroups;  // 2 producer warps, the MMA warp, epilogue
 constexpr int kTileBytes = kMmaTile * kMmaTile * 2;   // 32 KiB of bf16
 constexpr int kHalfBytes = kTileBytes / 2;            // one TMA box: 64 columns x 128 rows
 constexpr uint32_t kTmemCols = kEpiGroups * kMmaTile <= 256 ? (kEpiGroups * kMmaTile <= 128 ? 128u : 256u) : 512u;
@@ -189,13 +189,13 @@ struct MmaParams {
 // scale bytes.  Returns the scale bytes of the chunk (NVFP4/dual: two).
 template <int FMT>
 __device__ __forceinline__ uint32_t quant_chunk(const float2* n, const ScaleCtx& ctx, const float4* tab,
-                                                uint8_t* cp) {
+                                                float fold, uint8_t* cp) {
     uint32_t w[4], e;
     if constexpr (FMT == FMT_MXFP4) {
-        e = mxfp4_unit(n, w);
+        e = mxfp4_unit(n, fold, w);
     } else {
         const float2 am = amax_pair(n);
-        e = nvfp4_unit<FMT == FMT_NVFP4>(n, am, ctx, tab, 1.0f, w);
+        e = nvfp4_unit<FMT == FMT_NVFP4, false>(n, am, ctx, tab, fold, w);
     }
     *reinterpret_cast<uint4*>(cp) = make_uint4(w[0], w[1], w[2], w[3]);
     return e;
@@ -236,6 +236,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     }
     build_hadamard_b<HAD>(smem + kMmaBOff);
     fence_proxy_async_smem();  // B is read by the tensor cores (async proxy)
+    pdl_wait();
+    pdl_trigger();
     float s_t = 0.0f;
     if constexpr (FMT == FMT_NVFP4 && !AMAX_ONLY) {
         if (p.dynamic) {
@@ -254,11 +256,15 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     const int64_t n_my = p.n_tiles > (int64_t)blockIdx.x ? (p.n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     float my_amax = 0.0f;
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+    if (warp == 0 || warp == 2) {
+        // ------------------------------------------------ TMA producers
+        // Two warps issue alternate tiles: the copies of one issuing thread are
+        // handled one after the other, and two streams of 16 KiB boxes keep an
+        // SM's share of HBM bandwidth busy where one does not.
         if (lane == 0) {
-            int64_t j = 0;
-            for (; j < n_my; ++j) {
+            const int64_t pj = warp >> 1;
+            int64_t j = pj;
+            for (; j < n_my; j += 2) {
                 const int s = (int)(j % kMmaStages);
                 if (j >= kMmaStages &&
                     !mbar_wait(empty0 + 8 * s, (uint32_t)((j / kMmaStages - 1) & 1))) {
@@ -274,8 +280,9 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
             }
             // Every issued copy must have landed before the CTA may exit: the
             // MMA warp waited for all of them unless something ran out.
-            for (int64_t k = j > kMmaStages ? j - kMmaStages : 0; k < j; ++k)
-                (void)mbar_wait(full0 + 8 * (int)(k % kMmaStages), (uint32_t)((k / kMmaStages) & 1));
+            for (int64_t k = pj; k < j; k += 2)
+                if (k + kMmaStages >= j)
+                    (void)mbar_wait(full0 + 8 * (int)(k % kMmaStages), (uint32_t)((k / kMmaStages) & 1));
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
@@ -308,10 +315,11 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         }
     } else {
         // ------------------------------------------------ epilogue
-        const uint32_t ew = warp - 2, g = ew / 4, quarter = warp & 3;
+        const uint32_t ew = warp - 3, g = ew / 4, quarter = warp & 3;
         const uint32_t lane_base = (quarter * 32u) << 16;
         ScaleCtx ctx = make_ctx(s_t);
-        const float2 rs2 = dup2(__uint_as_float(0x3f3504f3u));  // RN(1/sqrt(2))
+        // odd log2 n: the remaining RN(1/sqrt 2) is applied per block by the quantizer
+        const float fold = kOddLog ? __uint_as_float(0x3f3504f3u) : 1.0f;
         const int64_t kc = p.K / 2;
 #pragma unroll 1
         for (int64_t j = g; j < n_my; j += kEpiGroups) {
@@ -332,10 +340,6 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
                 tmem_ld32(tacc + 32u * c, v);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) n[i] = make_float2(v[i], v[16 + i]);
-                if constexpr (kOddLog) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) n[i] = mul2(n[i], rs2);
-                }
             };
             auto release = [&]() {  // every lane's loads of this accumulator are done
                 tc_fence_before();
@@ -352,7 +356,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
                     float m0 = fmaxf(fabsf(v[0]), fabsf(v[1]));
 #pragma unroll
                     for (int i = 2; i < 32; i += 2) m0 = max3(m0, fabsf(v[i]), fabsf(v[i + 1]));
-                    if constexpr (kOddLog) m0 *= rs2.x;  // RN is monotone: max of the scaled values
+                    m0 *= fold;  // RN is monotone: the max of the scaled values
                     const float2 am = make_float2(m0, m0);
                     if (live) my_amax = fmaxf(my_amax, fmaxf(am.x, am.y));
                     pin(my_amax);
@@ -368,6 +372,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
                         gm = fmaxf(gm, fmaxf(am.x, am.y));
                         pin(gm);
                     }
+                    gm *= fold;
                     const float Gs = (gm >= 0x1p-90f) ? div_split(-gm, 2688.0f, rcp2688()) : __fdiv_rn(gm, 2688.0f);
                     ctx = make_ctx(Gs);
                     if (live) p.scale_fp32[row * (p.K / 128) + ct] = Gs;
@@ -380,7 +385,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
                     load_chunk(c, n);
                     if (c == 3) release();
                     if (live) {
-                        const uint32_t e = quant_chunk<FMT>(n, ctx, tab, cp + 16 * c);
+                        const uint32_t e = quant_chunk<FMT>(n, ctx, tab, fold, cp + 16 * c);
                         if constexpr (FMT == FMT_MXFP4) {
                             sc0 |= e << (8 * c);
                         } else {

@@ -31,7 +31,7 @@
 namespace fp4q {
 
 constexpr int kWideEpiWarps = 16;                    // four warpgroups
-constexpr int kWideThreads = 64 + 32 * kWideEpiWarps;
+constexpr int kWideThreads = 96 + 32 * kWideEpiWarps;  // 2 producer warps, the MMA warp, epilogue
 constexpr int kWideRedBytes = 2 * 4 * 4 * kMmaTile * 4;  // [parity][warpgroup][group][row] fp32
 
 template <int HAD>
@@ -150,6 +150,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     }
     build_h128_b(smem);
     fence_proxy_async_smem();
+    pdl_wait();
+    pdl_trigger();
     float s_t = 0.0f;
     if constexpr (FMT == FMT_NVFP4 && !AMAX_ONLY) {
         if (p.dynamic) {
@@ -168,12 +170,13 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     const int64_t n_my = p.n_tiles > (int64_t)blockIdx.x ? (p.n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     float my_amax = 0.0f;
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer: G sub-tiles per tile
+    if (warp == 0 || warp == 2) {
+        // ------------------------------------------------ TMA producers: G sub-tiles per tile,
+        // alternate sub-tiles from two warps (see had_mma_kernel)
         if (lane == 0) {
-            const int64_t n_sub = n_my * G;
-            int64_t u = 0;
-            for (; u < n_sub; ++u) {
+            const int64_t n_sub = n_my * G, pu = warp >> 1;
+            int64_t u = pu;
+            for (; u < n_sub; u += 2) {
                 const int s = (int)(u % kMmaStages);
                 if (u >= kMmaStages && !mbar_wait(empty0 + 8 * s, (uint32_t)((u / kMmaStages - 1) & 1))) {
                     atomicOr(&g_device_error, kErrWaitTimeout);
@@ -187,8 +190,9 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                 tma_load_2d(dst, &tmap_x, x0, y0, full0 + 8 * s);
                 tma_load_2d(dst + kHalfBytes, &tmap_x, x0 + 64, y0, full0 + 8 * s);
             }
-            for (int64_t k = u > kMmaStages ? u - kMmaStages : 0; k < u; ++k)
-                (void)mbar_wait(full0 + 8 * (int)(k % kMmaStages), (uint32_t)((k / kMmaStages) & 1));
+            for (int64_t k = pu; k < u; k += 2)
+                if (k + kMmaStages >= u)
+                    (void)mbar_wait(full0 + 8 * (int)(k % kMmaStages), (uint32_t)((k / kMmaStages) & 1));
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
@@ -225,10 +229,11 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         }
     } else {
         // ------------------------------------------------ epilogue
-        const uint32_t ew = warp - 2, wg = ew >> 2, quarter = warp & 3;
+        const uint32_t ew = warp - 3, wg = ew >> 2, quarter = warp & 3;
         const uint32_t rowt = quarter * 32 + lane;
         const uint32_t lane_base = (quarter * 32u) << 16;
-        const float rs2 = __uint_as_float(0x3f3504f3u);  // RN(1/sqrt(2))
+        // n = 512: the remaining RN(1/sqrt 2) is applied per block by the quantizer
+        const float fold = kOddLog ? __uint_as_float(0x3f3504f3u) : 1.0f;
         const ScaleCtx ctx_t = make_ctx(s_t);
         const int64_t kc = p.K / 2;
 #pragma unroll 1
@@ -274,10 +279,6 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                 }
 #pragma unroll
                 for (int a = 0; a < G; ++a) {
-                    if constexpr (kOddLog) {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) z[a][i] *= rs2;
-                    }
                     float mm = fmaxf(fabsf(z[a][0]), fabsf(z[a][1]));
 #pragma unroll
                     for (int i = 2; i < 8; i += 2) mm = max3(mm, fabsf(z[a][i]), fabsf(z[a][i + 1]));
@@ -288,7 +289,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             if constexpr (AMAX_ONLY) {
                 if (live) {
 #pragma unroll
-                    for (int a = 0; a < G; ++a) my_amax = fmaxf(my_amax, m[a]);
+                    for (int a = 0; a < G; ++a) my_amax = fmaxf(my_amax, m[a] * fold);
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -314,6 +315,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                         float gm = rp[a * kMmaTile + rowt];
 #pragma unroll
                         for (int w = 1; w < 4; ++w) gm = fmaxf(gm, rp[(w * 4 + a) * kMmaTile + rowt]);
+                        gm *= fold;
                         gs[a] = (gm >= 0x1p-90f) ? div_split(-gm, 2688.0f, rcp2688()) : __fdiv_rn(gm, 2688.0f);
                     }
                 }
@@ -332,15 +334,15 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                         const int64_t col = ct * HAD + a * kMmaTile + 32 * wg;
                         uint32_t w[4], e;
                         if constexpr (FMT == FMT_MXFP4) {
-                            e = mxfp4_unit(n, w);
+                            e = mxfp4_unit(n, fold, w);
                         } else if constexpr (FMT == FMT_DUAL) {
                             float g = gs[0];
 #pragma unroll
                             for (int q = 1; q < G; ++q) g = a == q ? gs[q] : g;
-                            e = nvfp4_unit<false>(n, amax_pair(n), make_ctx(g), tab, 1.0f, w);
+                            e = nvfp4_unit<false, false>(n, amax_pair(n), make_ctx(g), tab, fold, w);
                             if (wg == 0) p.scale_fp32[row * (p.K / 128) + col / 128] = g;
                         } else {
-                            e = nvfp4_unit<true>(n, amax_pair(n), ctx_t, tab, 1.0f, w);
+                            e = nvfp4_unit<true, false>(n, amax_pair(n), ctx_t, tab, fold, w);
                         }
                         *reinterpret_cast<uint4*>(p.codes + row * kc + col / 2) = make_uint4(w[0], w[1], w[2], w[3]);
                         if constexpr (FMT == FMT_MXFP4) {

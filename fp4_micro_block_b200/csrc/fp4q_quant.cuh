@@ -109,12 +109,12 @@ __device__ __forceinline__ void to_pairs(const float* t, float2* n) {
     for (int i = 0; i < 16; ++i) n[i] = make_float2(t[i], t[16 + i]);
 }
 
-// This lane's 32 post-rotation values, negated, as unit pairs (unit `u` of row
-// `row` of the staged tile).  For rotations >= 64 the call exchanges data with
+// This lane's 32 rotated (unnormalised) values, negated, as unit pairs (unit
+// `u` of row `row` of the staged tile).  For rotations >= 64 the call exchanges data with
 // other lanes of the warp: every lane must call it.
 template <int HAD>
 __device__ __forceinline__ void load_unit(const uint8_t* stage, uint8_t* scratch, uint32_t lane,
-                                          uint32_t row, uint32_t u, float had_norm, float2* n) {
+                                          uint32_t row, uint32_t u, float2* n) {
     using G = Geo<HAD>;
     if constexpr (HAD <= 32) {
         float t[32];
@@ -123,10 +123,7 @@ __device__ __forceinline__ void load_unit(const uint8_t* stage, uint8_t* scratch
             nunpack8(*reinterpret_cast<const uint4*>(stage + g2_off(row, 32 * u + 8 * c)), t + 8 * c);
         to_pairs(t, n);
         if constexpr (HAD == 16) fwht16x2(n);
-        if constexpr (HAD == 32) {
-            fwht32(n);
-            scale_unit(n, had_norm);
-        }
+        if constexpr (HAD == 32) fwht32(n);
     } else if constexpr (HAD == 64) {
         // units (2p, 2p+1) of a row = lanes l and l ^ 8; tau = position in the pair
         const uint32_t tau = u & 1u, c0 = 64u * (u >> 1);
@@ -155,7 +152,7 @@ __device__ __forceinline__ void load_unit(const uint8_t* stage, uint8_t* scratch
             t[16 + i] = tau ? mine : got;
         }
         to_pairs(t, n);
-        fwht32(n);  // n = 64: the 1/8 normalisation is folded into the quantizer
+        fwht32(n);
     } else {
         constexpr int n2 = G::n2, k1w = G::k1w, kp = k1w / 2;
         // A[k2][j] = -x[row, block + 32*k2 + k1w*tau + 2j + (0, 1)]
@@ -236,7 +233,6 @@ __device__ __forceinline__ void load_unit(const uint8_t* stage, uint8_t* scratch
             to_pairs(t, n);
         }
         fwht32(n);
-        if constexpr (HAD != 256) scale_unit(n, had_norm);  // 256: 1/16 folded into the quantizer
     }
 }
 
@@ -268,13 +264,19 @@ __global__ void __launch_bounds__(kQuantThreads, Geo<HAD>::min_ctas)
     float* red = reinterpret_cast<float*>(full_bars + kWarps * kStages);
     float4* tab = reinterpret_cast<float4*>((reinterpret_cast<uintptr_t>(red + kWarps + 2) + 15) &
                                             ~uintptr_t(15));
-    constexpr bool kFold = HAD == 16 || HAD == 64 || HAD == 256;  // 1/sqrt(n) a power of two
+    // The rotation's normalisation RN(1/sqrt n) is applied per block by the
+    // quantizer (nvfp4_unit / mxfp4_unit); only the unrotated path needs the
+    // correctly rounded quotient of the bit-exact acceptance.
+    constexpr bool kFold = HAD > 0;
+    constexpr bool kExact = HAD == 0;
 
     if (tid == 0) {
         if constexpr (!G::bulk) prefetch_tmap(&tmap_x);
         for (int k = 0; k < kWarps * kStages; ++k) mbar_init(smem_u32(&full_bars[k]), 1);
         fence_barrier_init();
     }
+    pdl_wait();
+    pdl_trigger();
     // NVFP4: tensor scale, and the per-CTA table of decoded block scales.
     float s_t = 0.0f;
     if constexpr (FMT == FMT_NVFP4 && !AMAX_ONLY) {
@@ -315,7 +317,6 @@ __global__ void __launch_bounds__(kQuantThreads, Geo<HAD>::min_ctas)
         const int64_t kc = p.K / 2;
         ScaleCtx ctx = make_ctx(s_t);
         const float fold = kFold ? p.had_norm : 1.0f;
-        const float norm = kFold ? 1.0f : p.had_norm;
 
         auto issue = [&](int64_t i) {  // lane 0: tile (irb, icb) into stage i % kStages
             const uint32_t st = (uint32_t)(i % kStages);
@@ -353,7 +354,7 @@ __global__ void __launch_bounds__(kQuantThreads, Geo<HAD>::min_ctas)
                 break;
             }
             float2 n[16];
-            load_unit<HAD>(stages + st * G::stage_bytes, scratch, lane, row, u, norm, n);
+            load_unit<HAD>(stages + st * G::stage_bytes, scratch, lane, row, u, n);
             __syncwarp();  // every lane has read the stage (and the scratch): refill it
             if (lane == 0 && i + kStages < n_my) issue(i + kStages);
 
@@ -369,9 +370,8 @@ __global__ void __launch_bounds__(kQuantThreads, Geo<HAD>::min_ctas)
                 }
             } else if constexpr (FMT == FMT_MXFP4) {
                 if (live) {
-                    if constexpr (kFold) scale_unit(n, fold);
                     uint32_t w[4];
-                    const uint32_t b = mxfp4_unit(n, w);
+                    const uint32_t b = mxfp4_unit(n, fold, w);
                     *reinterpret_cast<uint4*>(p.codes + grow * kc + col / 2) = make_uint4(w[0], w[1], w[2], w[3]);
                     const int64_t nsc = p.K / 32, c0 = col / 32;
                     if (p.swizzled) p.scales[swizzle_offset(grow, c0, (nsc + 3) / 4)] = (uint8_t)b;
@@ -393,7 +393,7 @@ __global__ void __launch_bounds__(kQuantThreads, Geo<HAD>::min_ctas)
                 }
                 if (live) {
                     uint32_t w[4];
-                    const uint32_t e2 = nvfp4_unit<FMT == FMT_NVFP4>(n, am, ctx, tab, fold, w);
+                    const uint32_t e2 = nvfp4_unit<FMT == FMT_NVFP4, kExact>(n, am, ctx, tab, fold, w);
                     uint8_t* cp = p.codes + grow * kc + col / 2;
                     const int64_t nsc = p.K / 16, c0 = col / 16;
                     if ((p.K & 31) == 0) {  // rows of codes are 16-byte aligned

@@ -216,11 +216,16 @@ __device__ __forceinline__ uint32_t nvfp4_unit_ieee(const float2* n, float2 am, 
 
 // NVFP4 rule for the two blocks of a unit against the FP32 scale of `c`:
 //   r = (amax_b / 6) / s,  e = E4M3(r),  d = E4M3(e) * s,  code = E2M1(v / d).
-// `fold` = 2^-k > 0 means the unit holds z with v = z * 2^-k (a Hadamard
-// normalisation by a power of two, applied exactly here instead of per element);
-// am is then the amax of z.  Returns the two scale bytes (block 0 low) and
-// writes the codes to w.
-template <bool TABLE>
+// The unit holds z with v = z * fold (fold > 0: a Hadamard normalisation
+// applied here per block instead of per element); am is the amax of z.
+// EXACT: v / d is the correctly rounded quotient (div_split), and fold must be
+//        a power of two so that the folding is exact (the quantize-only paths,
+//        whose codes are bit-exact).
+// !EXACT: the quotient is z * RN(RN(1/d) * fold), within 2 ulp of v / d
+//        (the rotated paths, whose inputs are themselves fp32 approximations
+//        of the rotation and whose acceptance is a tolerance).
+// Returns the two scale bytes (block 0 low) and writes the codes to w.
+template <bool TABLE, bool EXACT>
 __device__ __forceinline__ uint32_t nvfp4_unit(const float2* n, float2 am, const ScaleCtx& c,
                                                const float4* tab, float fold, uint32_t (&w)[4]) {
     am.x *= fold;
@@ -244,21 +249,35 @@ __device__ __forceinline__ uint32_t nvfp4_unit(const float2* n, float2 am, const
         const float2 dd = e4m3x2_decode(e2);
         d0 = dd.x * c.s;
         d1 = dd.y * c.s;
-        c0 = d0 != 0.0f ? make_rcp(d0) : Rcp{0.0f, 0.0f, 0.0f};
-        c1 = d1 != 0.0f ? make_rcp(d1) : Rcp{0.0f, 0.0f, 0.0f};
-    }
-    if (fold != 1.0f) {  // divide z by d / 2^-k
-        const float inv = 1.0f / fold;  // exact: a power of two
-        d0 *= inv;
-        d1 *= inv;
-        c0 = Rcp{c0.rn * fold, c0.rz * fold, c0.lo * fold};
-        c1 = Rcp{c1.rn * fold, c1.rz * fold, c1.lo * fold};
+        if constexpr (EXACT) {
+            c0 = d0 != 0.0f ? make_rcp(d0) : Rcp{0.0f, 0.0f, 0.0f};
+            c1 = d1 != 0.0f ? make_rcp(d1) : Rcp{0.0f, 0.0f, 0.0f};
+        } else {
+            c0.rn = d0 != 0.0f ? __frcp_rn(d0) : 0.0f;
+            c1.rn = d1 != 0.0f ? __frcp_rn(d1) : 0.0f;
+        }
     }
     float q0[16], q1[16];
+    if constexpr (EXACT) {
+        if (fold != 1.0f) {  // divide z by d / 2^-k
+            const float inv = 1.0f / fold;  // exact: a power of two
+            d0 *= inv;
+            d1 *= inv;
+            c0 = Rcp{c0.rn * fold, c0.rz * fold, c0.lo * fold};
+            c1 = Rcp{c1.rn * fold, c1.rz * fold, c1.lo * fold};
+        }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        q0[i] = div_split(n[i].x, d0, c0);
-        q1[i] = div_split(n[i].y, d1, c1);
+        for (int i = 0; i < 16; ++i) {
+            q0[i] = div_split(n[i].x, d0, c0);
+            q1[i] = div_split(n[i].y, d1, c1);
+        }
+    } else {
+        const float m0 = -(c0.rn * fold), m1 = -(c1.rn * fold);  // n holds -z
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            q0[i] = n[i].x * m0;
+            q1[i] = n[i].y * m1;
+        }
     }
     w[0] = e2m1_pack8(q0);
     w[1] = e2m1_pack8(q0 + 8);
@@ -269,18 +288,21 @@ __device__ __forceinline__ uint32_t nvfp4_unit(const float2* n, float2 am, const
     return e2;
 }
 
-// MXFP4 of a whole unit (one 32-block): byte = clamp(floor(log2 amax) - 2 + 127,
-// 0, 254) from the exponent field, codes = E2M1(v * 2^(127-byte)) (exact).
-__device__ __forceinline__ uint32_t mxfp4_unit(const float2* n, uint32_t (&w)[4]) {
+// MXFP4 of a whole unit (one 32-block) of v = z * fold (fold > 0, see
+// nvfp4_unit; am of v = RN(amax(z) * fold) since rounding is monotone):
+// byte = clamp(floor(log2 amax) - 2 + 127, 0, 254) from the exponent field,
+// codes = E2M1(z * RN(fold * 2^(127-byte))), which is RN(v * 2^(127-byte))
+// exactly when fold = 1 and within an ulp otherwise.
+__device__ __forceinline__ uint32_t mxfp4_unit(const float2* n, float fold, uint32_t (&w)[4]) {
     const float2 a = amax_pair(n);
-    const float am = fmaxf(a.x, a.y);
+    const float am = fmaxf(a.x, a.y) * fold;
     if (am == 0.0f) {
         w[0] = w[1] = w[2] = w[3] = 0u;
         return 0u;
     }
     const uint32_t ef = __float_as_uint(am) >> 23;
     const uint32_t b = ef >= 2u ? ef - 2u : 0u;
-    const float nm = -__uint_as_float((254u - b) << 23);  // -2^(127-b), normal for b <= 252
+    const float nm = -__uint_as_float((254u - b) << 23) * fold;  // -2^(127-b) * fold
     // codes in element order: v[i] = -n[i].x * 2^(127-b), v[16+i] = -n[i].y * ...
     float v[32];
 #pragma unroll
