@@ -150,43 +150,20 @@ fp4q_status ensure_smem(Kern kern, int bytes, std::atomic<uint64_t>& done) {
 }
 
 // ---------------------------------------------------------------- quantizer launch
-// Resident CTAs per SM of a kernel, looked up once per device.
-template <typename Kern>
-fp4q_status resident_ctas(Kern kern, int smem, std::atomic<int>* cache, int* out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return FP4Q_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return FP4Q_ERR_UNSUPPORTED;
-    int n = cache[dev].load(std::memory_order_relaxed);
-    if (n <= 0) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kQuantThreads, smem) != cudaSuccess)
-            return FP4Q_ERR_CUDA;
-        if (n <= 0) return FP4Q_ERR_UNSUPPORTED;
-        cache[dev].store(n, std::memory_order_relaxed);
-    }
-    *out = n;
-    return FP4Q_OK;
-}
-
-// Launches quant_kernel<FMT, HAD, AMAX> persistently (resident CTAs x SMs, at most
-// one warp per warp tile); returns the grid through *grid_out.
+// Launches quant_kernel<FMT, HAD, AMAX> persistently (one CTA per SM, at most
+// one per tile); returns the grid through *grid_out.
 template <int FMT, int HAD, bool AMAX>
 fp4q_status launch_quant_t(const CUtensorMap& map, QuantParams p, int sms, cudaStream_t s,
                            int* grid_out) {
-    using G = Geo<HAD>;
+    using G = QGeo<FMT, HAD>;
     auto kern = quant_kernel<FMT, HAD, AMAX>;
-    constexpr int smem = quant_smem_bytes<HAD>();
     static std::atomic<uint64_t> done{0};
-    static std::atomic<int> occ[kMaxDevices];
-    fp4q_status st = ensure_smem(kern, smem, done);
+    fp4q_status st = ensure_smem(kern, G::smem, done);
     if (st != FP4Q_OK) return st;
-    int per_sm = 0;
-    if ((st = resident_ctas(kern, smem, occ, &per_sm)) != FP4Q_OK) return st;
-    p.n_rb = (p.M + G::rows - 1) / G::rows;
-    p.n_cb = (p.K + G::cols - 1) / G::cols;
-    p.n_wt = p.n_rb * p.n_cb;
-    const int grid = (int)std::min<int64_t>(
-        {(p.n_wt + kWarps - 1) / kWarps, (int64_t)per_sm * sms, (int64_t)kMaxGrid});
-    st = launch(kern, grid, kQuantThreads, smem, s, map, p);
+    p.n_cs = (p.K + G::tc - 1) / G::tc;
+    p.n_tiles = (p.M + kQBoxRows - 1) / kQBoxRows * p.n_cs;
+    const int grid = (int)std::min<int64_t>({p.n_tiles, (int64_t)sms, (int64_t)kMaxGrid});
+    st = launch(kern, grid, G::threads, G::smem, s, map, p);
     if (grid_out) *grid_out = grid;
     return st;
 }
@@ -194,17 +171,21 @@ fp4q_status launch_quant_t(const CUtensorMap& map, QuantParams p, int sms, cudaS
 template <int FMT, bool AMAX>
 fp4q_status launch_quant_h(int had, const CUtensorMap& map, const QuantParams& p, int sms,
                            cudaStream_t s, int* grid_out) {
-    switch (had) {
-        case 0: return launch_quant_t<FMT, 0, AMAX>(map, p, sms, s, grid_out);
-        case 16: return launch_quant_t<FMT, 16, AMAX>(map, p, sms, s, grid_out);
-        case 32: return launch_quant_t<FMT, 32, AMAX>(map, p, sms, s, grid_out);
-        case 64: return launch_quant_t<FMT, 64, AMAX>(map, p, sms, s, grid_out);
-        case 128: return launch_quant_t<FMT, 128, AMAX>(map, p, sms, s, grid_out);
-        case 256: return launch_quant_t<FMT, 256, AMAX>(map, p, sms, s, grid_out);
-        case 512: return launch_quant_t<FMT, 512, AMAX>(map, p, sms, s, grid_out);
-        default: return FP4Q_ERR_INVALID_ARG;
+    if constexpr (FMT == FMT_DUAL) {  // K % 128 == 0: every rotation takes the tensor cores
+        if (had != 0) return FP4Q_ERR_INVALID_ARG;
+        return launch_quant_t<FMT, 0, AMAX>(map, p, sms, s, grid_out);
+    } else {
+        switch (had) {
+            case 0: return launch_quant_t<FMT, 0, AMAX>(map, p, sms, s, grid_out);
+            case 16: return launch_quant_t<FMT, 16, AMAX>(map, p, sms, s, grid_out);
+            case 32: return launch_quant_t<FMT, 32, AMAX>(map, p, sms, s, grid_out);
+            case 64: return launch_quant_t<FMT, 64, AMAX>(map, p, sms, s, grid_out);
+            default: return FP4Q_ERR_INVALID_ARG;  // 128 and up: tensor cores (K % 128 == 0)
+        }
     }
 }
+
+float had_norm(int n) { return n > 0 ? (float)(1.0 / std::sqrt((double)n)) : 1.0f; }
 
 // ---------------------------------------------------------------- tensor-core rotation launch
 // Rotations on K a multiple of the 128-column tile go through the tcgen05
@@ -243,7 +224,6 @@ fp4q_status launch_mma_h(int had, const CUtensorMap& map, const MmaParams& p, in
     }
 }
 
-float had_norm(int n) { return n > 0 ? (float)(1.0 / std::sqrt((double)n)) : 1.0f; }
 
 fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, int had,
                             int fmt, uint8_t* codes, uint8_t* scales, float* scale_fp32,
@@ -276,14 +256,11 @@ fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, in
     CUtensorMap map;
     std::memset(&map, 0, sizeof(map));
     const bool mma = use_mma(had, K);
-    if ((mma || had < 256) && (st = make_x_map(&map, x, M, K, ldx, mma ? kMmaTile : 8)) != FP4Q_OK)
-        return st;
+    if ((st = make_x_map(&map, x, M, K, ldx, mma ? kMmaTile : kQBoxRows)) != FP4Q_OK) return st;
 
     QuantParams p{};
     p.M = M;
     p.K = K;
-    p.x = static_cast<const uint8_t*>(x);
-    p.ldx_bytes = ldx * 2;
     p.codes = codes;
     p.scales = scales;
     p.scale_fp32 = scale_fp32;
@@ -446,11 +423,11 @@ FP4Q_API fp4q_status fp4q_quantize_nvfp4_noalloc(const void* x, int64_t M, int64
     if (st != FP4Q_OK) return st;
     if (K % 16 != 0) return FP4Q_ERR_INVALID_ARG;
     if (M == 0) return FP4Q_OK;
-    // One partial maximum per pre-pass CTA: at most one CTA per 8 warp tiles and
-    // never more than kMaxGrid, so this only trips if that cap is ever raised.
-    const int64_t n_wt = ((M + Geo<0>::rows - 1) / Geo<0>::rows) * ((K + Geo<0>::cols - 1) / Geo<0>::cols);
-    const int64_t grid = std::min<int64_t>((n_wt + kWarps - 1) / kWarps, (int64_t)kMaxGrid);
-    if (grid > kNoAllocPartials) return FP4Q_ERR_UNSUPPORTED;
+    // One partial maximum per pre-pass CTA: the pre-pass runs one CTA per SM
+    // and never more than kMaxGrid, so this only trips if that cap is ever raised.
+    int sms = 0;
+    if ((st = sm_count(&sms)) != FP4Q_OK) return st;
+    if (std::min(sms, kMaxGrid) > kNoAllocPartials) return FP4Q_ERR_UNSUPPORTED;
     float* scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != FP4Q_OK) return st;
     return quantize_common(x, M, K, ldx, 0, FMT_NVFP4, codes, scales, tensor_scale,

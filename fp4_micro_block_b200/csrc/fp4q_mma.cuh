@@ -123,13 +123,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Orders the computation of x before any later volatile asm (the next TMEM
-// load), so that chunks reduced in a loop do not stay live in registers.
-__device__ __forceinline__ void pin(float x) { asm volatile("" ::"f"(x)); }
 
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
 
 // ---------------------------------------------------------------- shared memory
 // [B 32 KiB][X ring kMmaStages x 32 KiB][barriers][tmem slot][NVFP4 table][reduction]
@@ -185,20 +179,38 @@ struct MmaParams {
     int dynamic;
 };
 
-// Quantize the 32 values of one chunk (negated pairs n) and store codes and
-// scale bytes.  Returns the scale bytes of the chunk (NVFP4/dual: two).
+// Quantize the 32 values of one chunk (negated pairs n): codes into w, returns
+// the scale bytes of the chunk (NVFP4 / dual: two, MXFP4: one).
 template <int FMT>
 __device__ __forceinline__ uint32_t quant_chunk(const float2* n, const ScaleCtx& ctx, const float4* tab,
-                                                float fold, uint8_t* cp) {
-    uint32_t w[4], e;
+                                                float fold, uint32_t (&w)[4]) {
     if constexpr (FMT == FMT_MXFP4) {
-        e = mxfp4_unit(n, fold, w);
+        return mxfp4_unit(n, fold, w);
     } else {
         const float2 am = amax_pair(n);
-        e = nvfp4_unit<FMT == FMT_NVFP4, false>(n, am, ctx, tab, fold, w);
+        return nvfp4_unit<FMT == FMT_NVFP4, false>(n, am, ctx, tab, fold, w);
     }
-    *reinterpret_cast<uint4*>(cp) = make_uint4(w[0], w[1], w[2], w[3]);
-    return e;
+}
+
+// Stores the codes of two adjacent 16-byte chunks (wa: chunk c, wb: chunk c + 1)
+// of the rows held by a lane pair (2i, 2i + 1; lane = row): the two lanes swap
+// halves so that each store instruction writes whole 32-byte sectors (16 rows
+// x 32 bytes) instead of 16-byte halves of 32 rows.  mine = this lane's row at
+// chunk c; stride = bytes between rows; live_even / live_odd: the pair's rows
+// exist.  Every lane of the warp must call it.
+__device__ __forceinline__ void store_chunk_pair(uint8_t* mine, int64_t stride, bool live_even, bool live_odd,
+                                                 uint32_t lane, const uint32_t (&wa)[4], const uint32_t (&wb)[4]) {
+    const bool odd = lane & 1u;
+    uint32_t d1[4], d2[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t got = __shfl_xor_sync(0xffffffffu, odd ? wa[k] : wb[k], 1);
+        d1[k] = odd ? got : wa[k];  // row 2i: chunk c (even lane), c + 1 (odd lane)
+        d2[k] = odd ? wb[k] : got;  // row 2i + 1
+    }
+    uint8_t* p1 = mine - (odd ? stride : 0) + (odd ? 16 : 0);
+    if (live_even) *reinterpret_cast<uint4*>(p1) = make_uint4(d1[0], d1[1], d1[2], d1[3]);
+    if (live_odd) *reinterpret_cast<uint4*>(p1 + stride) = make_uint4(d2[0], d2[1], d2[2], d2[3]);
 }
 
 template <int FMT, int HAD, bool AMAX_ONLY>
@@ -378,21 +390,24 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
                     if (live) p.scale_fp32[row * (p.K / 128) + ct] = Gs;
                 }
                 uint8_t* cp = p.codes + row * kc + ct * (kMmaTile / 2);
+                const int64_t row_even = row - (lane & 1u);
+                const bool live_even = row_even < p.M, live_odd = row_even + 1 < p.M;
                 uint32_t sc0 = 0u, sc1 = 0u;  // scale bytes of blocks 0-3 / 4-7 (MXFP4: sc0)
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 4; c += 2) {
+                    uint32_t wa[4], wb[4];
                     float2 n[16];
                     load_chunk(c, n);
-                    if (c == 3) release();
-                    if (live) {
-                        const uint32_t e = quant_chunk<FMT>(n, ctx, tab, fold, cp + 16 * c);
-                        if constexpr (FMT == FMT_MXFP4) {
-                            sc0 |= e << (8 * c);
-                        } else {
-                            const uint32_t sh = e << (16 * (c & 1));
-                            if (c < 2) sc0 |= sh;
-                            else sc1 |= sh;
-                        }
+                    const uint32_t ea = quant_chunk<FMT>(n, ctx, tab, fold, wa);
+                    load_chunk(c + 1, n);
+                    if (c + 1 == 3) release();
+                    const uint32_t eb = quant_chunk<FMT>(n, ctx, tab, fold, wb);
+                    store_chunk_pair(cp + 16 * c, kc, live_even, live_odd, lane, wa, wb);
+                    if constexpr (FMT == FMT_MXFP4) {
+                        sc0 |= (ea | (eb << 8)) << (8 * c);
+                    } else {
+                        if (c == 0) sc0 = ea | (eb << 16);
+                        else sc1 = ea | (eb << 16);
                     }
                 }
                 if (live) {

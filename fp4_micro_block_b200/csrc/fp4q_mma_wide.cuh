@@ -19,11 +19,14 @@
 //   pass 1  reads z in steps of 8 columns of every group, applies H_G (and
 //           RN(1/sqrt 2) for n = 512), takes the per-group maxima and writes
 //           y back into TMEM in place;
-//   (dual)  the group maxima of the four warpgroups meet in shared memory;
-//   pass 2  reads y group by group (32 columns = one quantization unit), hands
-//           each group's columns back to the MMA warp as soon as every warp has
-//           read them (the next tile's UMMAs then overlap the rest of pass 2),
-//           and quantizes.
+//   (sync)  the epilogue warps meet (their pass-2 columns were written by
+//           other warpgroups), and the dual format's group maxima of the four
+//           warpgroups meet in shared memory;
+//   pass 2  warpgroup w quantizes output group w % G (columns [32 c, 32 c + 32)
+//           for its G chunks c), so that each lane writes whole 32-byte sectors
+//           of its row, and hands the group's TMEM columns back to the MMA warp
+//           as soon as its warps have read them (the next tile's UMMAs then
+//           overlap the rest of pass 2).
 #pragma once
 
 #include "fp4q_mma.cuh"
@@ -124,7 +127,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     const uint32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t full0 = smem_u32(smem + W::bar_off), empty0 = full0 + 8 * kMmaStages;
     const uint32_t accf0 = empty0 + 8 * kMmaStages, relg0 = accf0 + 8 * NBUF;
-    const uint32_t redb0 = relg0 + 8 * NBUF * G;  // [2] dual: the four warpgroups' group maxima
+    const uint32_t redb0 = relg0 + 8 * NBUF * G;  // [2] all epilogue warps between the two passes
     const uint32_t done_bar = redb0 + 16;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + W::slot_off);
     float4* tab = reinterpret_cast<float4*>(smem + W::tab_off);
@@ -139,7 +142,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             mbar_init(empty0 + 8 * s, 1);
         }
         for (int b = 0; b < NBUF; ++b) mbar_init(accf0 + 8 * b, 1);
-        for (int k = 0; k < NBUF * G; ++k) mbar_init(relg0 + 8 * k, kWideEpiWarps);
+        for (int k = 0; k < NBUF * G; ++k) mbar_init(relg0 + 8 * k, kWideEpiWarps / G);  // its group's warps
         for (int k = 0; k < 2; ++k) mbar_init(redb0 + 8 * k, kWideEpiWarps);
         mbar_init(done_bar, 1);
         fence_barrier_init();
@@ -294,22 +297,30 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0)
-                    for (int a = 0; a < G; ++a) mbar_arrive(relg0 + 8 * (b * G + a));
+                    mbar_arrive(relg0 + 8 * (b * G + (int)(wg % G)));
                 continue;
             } else {
+                // Pass 2 reads columns that other warpgroups wrote in pass 1: every
+                // epilogue warp meets the others here (bounded mbarrier wait), with
+                // the tcgen05 fences that order their TMEM stores before our loads.
+                // The dual format also exchanges its group maxima here.
                 tmem_wait_st();
                 float gs[G];
-                if constexpr (FMT == FMT_DUAL) {  // group maxima over the four warpgroups
-                    float* rp = red2 + (j & 1) * (4 * 4 * kMmaTile);
+                float* rp = red2 + (j & 1) * (4 * 4 * kMmaTile);
+                if constexpr (FMT == FMT_DUAL) {
 #pragma unroll
                     for (int a = 0; a < G; ++a) rp[(wg * 4 + a) * kMmaTile + rowt] = m[a];
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(redb0 + 8 * (uint32_t)(j & 1));
-                    const bool rok = mbar_wait(redb0 + 8 * (uint32_t)(j & 1), (uint32_t)((j >> 1) & 1));
-                    if (!__all_sync(0xffffffffu, rok)) {
-                        if (lane == 0) atomicOr(&g_device_error, kErrWaitTimeout);
-                        break;
-                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(redb0 + 8 * (uint32_t)(j & 1));
+                const bool rok = mbar_wait(redb0 + 8 * (uint32_t)(j & 1), (uint32_t)((j >> 1) & 1));
+                if (!__all_sync(0xffffffffu, rok)) {
+                    if (lane == 0) atomicOr(&g_device_error, kErrWaitTimeout);
+                    break;
+                }
+                tc_fence_after();
+                if constexpr (FMT == FMT_DUAL) {  // group maxima over the four warpgroups
 #pragma unroll
                     for (int a = 0; a < G; ++a) {
                         float gm = rp[a * kMmaTile + rowt];
@@ -319,41 +330,53 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                         gs[a] = (gm >= 0x1p-90f) ? div_split(-gm, 2688.0f, rcp2688()) : __fdiv_rn(gm, 2688.0f);
                     }
                 }
-                // ---- pass 2: quantize group by group
+                // ---- pass 2: warpgroup wg quantizes output group a = wg % G, chunks
+                // [c0, c0 + G) of its 4 (all of them for n = 512), so that a lane
+                // writes 64 consecutive columns of its row; the group's TMEM
+                // columns go back to the MMA warp once its warps have read them.
+                const int a = (int)(wg % G), c0 = (int)(wg / G) * G;
+                float g = 0.0f;
+                if constexpr (FMT == FMT_DUAL) {
+                    g = gs[0];
+#pragma unroll
+                    for (int q = 1; q < G; ++q) g = a == q ? gs[q] : g;
+                    if (live && c0 == 0) p.scale_fp32[row * (p.K / 128) + ct * G + a] = g;
+                }
+                const ScaleCtx ctx = FMT == FMT_DUAL ? make_ctx(g) : ctx_t;
+                const int64_t row_even = row - (lane & 1u);
+                const bool live_even = row_even < p.M, live_odd = row_even + 1 < p.M;
+                const int64_t colg = ct * HAD + a * kMmaTile;  // first column of the group
 #pragma unroll 1
-                for (int a = 0; a < G; ++a) {
+                for (int c = c0; c < c0 + G; c += 2) {
+                    uint32_t wa[4], wb[4];
+                    float2 n[16];
                     float v[32];
-                    tmem_ld32(tbuf + a * kMmaTile + 32u * wg, v);
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(relg0 + 8 * (b * G + a));
+                    tmem_ld32(tbuf + a * kMmaTile + 32u * c, v);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) n[i] = make_float2(v[i], v[16 + i]);
+                    const uint32_t ea = quant_chunk<FMT>(n, ctx, tab, fold, wa);
+                    tmem_ld32(tbuf + a * kMmaTile + 32u * (c + 1), v);
+                    if (c + 2 == c0 + G) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(relg0 + 8 * (b * G + a));
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) n[i] = make_float2(v[i], v[16 + i]);
+                    const uint32_t eb = quant_chunk<FMT>(n, ctx, tab, fold, wb);
+                    const int64_t col = colg + 32 * c;
+                    store_chunk_pair(p.codes + row * kc + col / 2, kc, live_even, live_odd, lane, wa, wb);
                     if (live) {
-                        float2 n[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) n[i] = make_float2(v[i], v[16 + i]);
-                        const int64_t col = ct * HAD + a * kMmaTile + 32 * wg;
-                        uint32_t w[4], e;
-                        if constexpr (FMT == FMT_MXFP4) {
-                            e = mxfp4_unit(n, fold, w);
-                        } else if constexpr (FMT == FMT_DUAL) {
-                            float g = gs[0];
-#pragma unroll
-                            for (int q = 1; q < G; ++q) g = a == q ? gs[q] : g;
-                            e = nvfp4_unit<false, false>(n, amax_pair(n), make_ctx(g), tab, fold, w);
-                            if (wg == 0) p.scale_fp32[row * (p.K / 128) + col / 128] = g;
-                        } else {
-                            e = nvfp4_unit<true, false>(n, amax_pair(n), ctx_t, tab, fold, w);
-                        }
-                        *reinterpret_cast<uint4*>(p.codes + row * kc + col / 2) = make_uint4(w[0], w[1], w[2], w[3]);
-                        if constexpr (FMT == FMT_MXFP4) {
-                            const int64_t nsc = p.K / 32, c0 = col / 32;
-                            if (p.swizzled) p.scales[swizzle_offset(row, c0, (nsc + 3) / 4)] = (uint8_t)e;
-                            else p.scales[row * nsc + c0] = (uint8_t)e;
-                        } else {
-                            const int64_t nsc = p.K / 16, c0 = col / 16;  // c0 even
-                            uint8_t* sp = p.swizzled ? p.scales + swizzle_offset(row, c0, (nsc + 3) / 4)
-                                                     : p.scales + row * nsc + c0;
-                            *reinterpret_cast<uint16_t*>(sp) = (uint16_t)e;
+                        if constexpr (FMT == FMT_MXFP4) {  // two E8M0 bytes, 2-byte aligned
+                            const int64_t nsc = p.K / 32, cb = col / 32;
+                            uint8_t* sp = p.swizzled ? p.scales + swizzle_offset(row, cb, (nsc + 3) / 4)
+                                                     : p.scales + row * nsc + cb;
+                            *reinterpret_cast<uint16_t*>(sp) = (uint16_t)(ea | (eb << 8));
+                        } else {  // four E4M3 bytes, 4-byte aligned
+                            const int64_t nsc = p.K / 16, cb = col / 16;
+                            uint8_t* sp = p.swizzled ? p.scales + swizzle_offset(row, cb, (nsc + 3) / 4)
+                                                     : p.scales + row * nsc + cb;
+                            *reinterpret_cast<uint32_t*>(sp) = ea | (eb << 16);
                         }
                     }
                 }

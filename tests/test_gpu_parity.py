@@ -224,6 +224,25 @@ def test_hadamard_quantize_tolerance(fq, n, fmt):
     assert_tolerant(fmt, K, gpu, (c_o, s_o, sc_o), y_o, name=f"had{n}-{fmt}")
 
 
+@pytest.mark.parametrize("n,K,fmt", [(16, 1040, "nvfp4"), (32, 1056, "nvfp4"), (64, 1088, "nvfp4"),
+                                     (32, 1056, "mxfp4"), (64, 1088, "mxfp4"), (16, 1120, "mxfp4")])
+def test_hadamard_quantize_ragged_rows(fq, n, K, fmt):
+    """Row lengths that are not a multiple of 128 take the register-FWHT path
+    (ragged last column strip, rows not a multiple of the 128-row tile)."""
+    M = 131
+    x_bits = workloads.hadamard_channels(M, K, seed=n + K)
+    fcode = {"nvfp4": fq.FP4Q_NVFP4, "mxfp4": fq.FP4Q_MXFP4}[fmt]
+    codes, scales, sf = fq.hadamard_quantize(bits_to_torch_cuda(x_bits), n, fcode)
+    torch.cuda.synchronize()
+    c_o, s_o, sc_o, y_o = oracle.hadamard_quantize(x_bits, n, fmt)
+    if fmt == "nvfp4":
+        assert abs(float(to_np(sf)[0]) - float(sc_o)) <= 4e-7 * float(sc_o)
+        gpu = (to_np(codes), to_np(scales), to_np(sf))
+    else:
+        gpu = (to_np(codes), to_np(scales), None)
+    assert_tolerant(fmt, K, gpu, (c_o, s_o, sc_o), y_o, name=f"ragged-had{n}-{fmt}-K{K}")
+
+
 def test_hadamard_static_scale(fq):
     M, K, n = 48, 1024, 128
     x_bits = workloads.hadamard_channels(M, K, seed=77)
