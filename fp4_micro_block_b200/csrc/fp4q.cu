@@ -162,7 +162,7 @@ fp4q_status launch_quant_t(const CUtensorMap& map, QuantParams p, int sms, cudaS
     if (st != FP4Q_OK) return st;
     p.n_cs = (p.K + G::tc - 1) / G::tc;
     p.n_tiles = (p.M + kQBoxRows - 1) / kQBoxRows * p.n_cs;
-    const int grid = (int)std::min<int64_t>({p.n_tiles, (int64_t)sms, (int64_t)kMaxGrid});
+    const int grid = (int)std::min<int64_t>({p.n_tiles, (int64_t)kQCtas * sms, (int64_t)kMaxGrid});
     st = launch(kern, grid, G::threads, G::smem, s, map, p);
     if (grid_out) *grid_out = grid;
     return st;

@@ -260,6 +260,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         }
         build_table(tab, s_t);
     }
+    if constexpr (FMT == FMT_DUAL && !AMAX_ONLY) build_table(tab, 1.0f);  // per-group s: RN(1/E4M3(e))
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

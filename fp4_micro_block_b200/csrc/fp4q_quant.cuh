@@ -36,7 +36,11 @@ constexpr int kQBoxRows = FP4Q_QBOX_ROWS;   // TMA box: 64 columns x kQBoxRows r
 constexpr int kQBoxBytes = kQBoxRows * 128;
 constexpr int kQWarpsPerTile = kQBoxRows / 32;
 constexpr int kQProducers = FP4Q_QPRODUCERS;
-constexpr int kQRingBytes = 192 * 1024;
+#ifndef FP4Q_QCTAS
+#define FP4Q_QCTAS 1
+#endif
+constexpr int kQCtas = FP4Q_QCTAS;             // CTAs per SM
+constexpr int kQRingBytes = 192 * 1024 / kQCtas;
 
 enum : int { FMT_NVFP4 = 0, FMT_MXFP4 = 1, FMT_DUAL = 2 };
 
@@ -62,7 +66,7 @@ struct QGeo {
     static constexpr int units = tc / 32;                       // units per lane per tile
     // consumer warpgroups: three where a lane holds 64 values at once (n = 64)
     // or reduces a dual-scale group, so that 128 registers per thread fit
-    static constexpr int cwarps = (HAD == 64 || FMT == FMT_DUAL) ? 12 : 16;
+    static constexpr int cwarps = ((HAD == 64 || FMT == FMT_DUAL) ? 12 : 16) / kQCtas;
     static_assert(cwarps % kQWarpsPerTile == 0, "consumer warps form whole tile groups");
     static constexpr int groups = cwarps / kQWarpsPerTile;
     static constexpr int threads = 32 * (kQProducers + cwarps);
@@ -116,7 +120,7 @@ __device__ __forceinline__ void read_unit(const uint8_t* row_base, uint32_t row,
 }
 
 template <int FMT, int HAD, bool AMAX_ONLY>
-__global__ void __launch_bounds__(QGeo<FMT, HAD>::threads, 1)
+__global__ void __launch_bounds__(QGeo<FMT, HAD>::threads, kQCtas)
     quant_kernel(const __grid_constant__ CUtensorMap tmap_x, const QuantParams p) {
     using G = QGeo<FMT, HAD>;
     static_assert(FMT != FMT_DUAL || HAD == 0, "dual scale needs K % 128 == 0: rotations go to the tensor cores");

@@ -221,9 +221,10 @@ __device__ __forceinline__ uint32_t nvfp4_unit_ieee(const float2* n, float2 am, 
 // EXACT: v / d is the correctly rounded quotient (div_split), and fold must be
 //        a power of two so that the folding is exact (the quantize-only paths,
 //        whose codes are bit-exact).
-// !EXACT: the quotient is z * RN(RN(1/d) * fold), within 2 ulp of v / d
-//        (the rotated paths, whose inputs are themselves fp32 approximations
-//        of the rotation and whose acceptance is a tolerance).
+// !EXACT: scale and quotient are products with rounded reciprocals (below),
+//        within a few ulp of the exact ones (the rotated paths, whose inputs are
+//        themselves fp32 approximations of the rotation and whose acceptance
+//        is a tolerance).  `tab` must be the table of c.s (TABLE) or of s = 1.
 // Returns the two scale bytes (block 0 low) and writes the codes to w.
 template <bool TABLE, bool EXACT>
 __device__ __forceinline__ uint32_t nvfp4_unit(const float2* n, float2 am, const ScaleCtx& c,
@@ -235,6 +236,33 @@ __device__ __forceinline__ uint32_t nvfp4_unit(const float2* n, float2 am, const
     const bool in_range = c.fast && (b0 - 1u) >= tiny - 1u && (b1 - 1u) >= tiny - 1u &&
                           fmaxf(am.x, am.y) <= c.am_max;
     if (!in_range) return nvfp4_unit_ieee(n, am, c.s, fold, w);
+    if constexpr (!EXACT) {
+        // Scale bytes from RN(RN(amax * RN(1/6)) * RN(1/s)), within 3 ulp of
+        // (amax/6)/s: a byte can differ only for r within 3 ulp of an E4M3
+        // rounding boundary.  Quotients z * RN(rn * fold), rn = RN(1/d) from the
+        // table (TABLE: d = E4M3(e) * s) or RN(1/E4M3(e)) * RN(1/s) from a
+        // table built for s = 1 (the dual format's per-group s).
+        const float k6 = __uint_as_float(0x3e2aaaabu);  // RN(1/6)
+        const float r0 = (am.x * k6) * c.rs.rn, r1 = (am.y * k6) * c.rs.rn;
+        const uint32_t e2 = e4m3x2_encode(make_float2(r0, r1));
+        const float4 t0 = tab[e2 & 0xffu], t1 = tab[e2 >> 8];
+        const float g = TABLE ? fold : c.rs.rn * fold;
+        const float2 m = make_float2(-(t0.y * g), -(t1.y * g));  // n holds -z
+        float q0[16], q1[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float2 q = __fmul2_rn(n[i], m);
+            q0[i] = q.x;
+            q1[i] = q.y;
+        }
+        w[0] = e2m1_pack8(q0);
+        w[1] = e2m1_pack8(q0 + 8);
+        w[2] = e2m1_pack8(q1);
+        w[3] = e2m1_pack8(q1 + 8);
+        if (t0.x == 0.0f) w[0] = w[1] = 0u;  // zero block scale: all codes +0
+        if (t1.x == 0.0f) w[2] = w[3] = 0u;
+        return e2;
+    }
     const Rcp r6 = rcp6();
     const float bs0 = div_split(-am.x, 6.0f, r6), bs1 = div_split(-am.y, 6.0f, r6);
     const float r0 = div_split(-bs0, c.s, c.rs), r1 = div_split(-bs1, c.s, c.rs);
@@ -249,35 +277,21 @@ __device__ __forceinline__ uint32_t nvfp4_unit(const float2* n, float2 am, const
         const float2 dd = e4m3x2_decode(e2);
         d0 = dd.x * c.s;
         d1 = dd.y * c.s;
-        if constexpr (EXACT) {
-            c0 = d0 != 0.0f ? make_rcp(d0) : Rcp{0.0f, 0.0f, 0.0f};
-            c1 = d1 != 0.0f ? make_rcp(d1) : Rcp{0.0f, 0.0f, 0.0f};
-        } else {
-            c0.rn = d0 != 0.0f ? __frcp_rn(d0) : 0.0f;
-            c1.rn = d1 != 0.0f ? __frcp_rn(d1) : 0.0f;
-        }
+        c0 = d0 != 0.0f ? make_rcp(d0) : Rcp{0.0f, 0.0f, 0.0f};
+        c1 = d1 != 0.0f ? make_rcp(d1) : Rcp{0.0f, 0.0f, 0.0f};
+    }
+    if (fold != 1.0f) {  // divide z by d / 2^-k
+        const float inv = 1.0f / fold;  // exact: a power of two
+        d0 *= inv;
+        d1 *= inv;
+        c0 = Rcp{c0.rn * fold, c0.rz * fold, c0.lo * fold};
+        c1 = Rcp{c1.rn * fold, c1.rz * fold, c1.lo * fold};
     }
     float q0[16], q1[16];
-    if constexpr (EXACT) {
-        if (fold != 1.0f) {  // divide z by d / 2^-k
-            const float inv = 1.0f / fold;  // exact: a power of two
-            d0 *= inv;
-            d1 *= inv;
-            c0 = Rcp{c0.rn * fold, c0.rz * fold, c0.lo * fold};
-            c1 = Rcp{c1.rn * fold, c1.rz * fold, c1.lo * fold};
-        }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            q0[i] = div_split(n[i].x, d0, c0);
-            q1[i] = div_split(n[i].y, d1, c1);
-        }
-    } else {
-        const float m0 = -(c0.rn * fold), m1 = -(c1.rn * fold);  // n holds -z
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            q0[i] = n[i].x * m0;
-            q1[i] = n[i].y * m1;
-        }
+    for (int i = 0; i < 16; ++i) {
+        q0[i] = div_split(n[i].x, d0, c0);
+        q1[i] = div_split(n[i].y, d1, c1);
     }
     w[0] = e2m1_pack8(q0);
     w[1] = e2m1_pack8(q0 + 8);
