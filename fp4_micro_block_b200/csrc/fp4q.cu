@@ -501,10 +501,24 @@ FP4Q_API fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int6
     p.partials = static_cast<float*>(workspace);
     p.swizzled = layout == FP4Q_SCALES_SWIZZLED;
     p.dynamic = dynamic;
-    const int threads = (int)std::max<int64_t>(32, ((K / 16) + 31) / 32 * 32);
-    const int smem = arc_smem_bytes(K);
-    const int per_sm = threads <= 256 ? 2 : 1;
-    const int grid = (int)std::min<int64_t>({M, (int64_t)per_sm * sms, (int64_t)kMaxGrid});
+    // Warps per CTA (one row each) and row buffers per warp: as many warps as
+    // fit with two buffers each, else one buffer each.
+    constexpr int kSmemMax = 227 * 1024;
+    int W = 0, SR = 2;
+    for (int w = 12; w >= 1 && !W; --w)  // at most 384 threads (the kernel's launch bound)
+        if (arc_layout(K, S, w, 2).total <= kSmemMax) W = w;
+    if (W < 4) {
+        SR = 1;
+        W = 0;
+        for (int w = 12; w >= 1 && !W; --w)
+            if (arc_layout(K, S, w, 1).total <= kSmemMax) W = w;
+    }
+    if (W == 0) return FP4Q_ERR_UNSUPPORTED;
+    p.warps = W;
+    p.stages = SR;
+    const int threads = 32 * W;
+    const int smem = arc_layout(K, S, W, SR).total;
+    const int grid = (int)std::min<int64_t>({(M + W - 1) / W, (int64_t)sms, (int64_t)kMaxGrid});
     p.n_partials = grid;
     if (p.swizzled) {
         const int64_t ncols = (K + S) / 16;
@@ -512,19 +526,15 @@ FP4Q_API fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int6
         if (bytes != M * ncols && cudaMemsetAsync(scales, 0, (size_t)bytes, (cudaStream_t)stream) != cudaSuccess)
             return FP4Q_ERR_CUDA;
     }
-    // The shared-memory size depends on K, so the attribute is set on every call.
+    // The shared-memory size depends on K and S, so the attribute is set on every call.
     auto run = [&](auto kern) -> fp4q_status {
         if (smem > 48 * 1024 &&
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return FP4Q_ERR_CUDA;
         return launch(kern, grid, threads, smem, (cudaStream_t)stream, p);
     };
-    if (threads <= 256) {
-        if (dynamic && (st = run(arc_kernel<true, 256>)) != FP4Q_OK) return st;
-        return run(arc_kernel<false, 256>);
-    }
-    if (dynamic && (st = run(arc_kernel<true, 1024>)) != FP4Q_OK) return st;
-    return run(arc_kernel<false, 1024>);
+    if (dynamic && (st = run(arc_kernel<true>)) != FP4Q_OK) return st;
+    return run(arc_kernel<false>);
 }
 
 FP4Q_API fp4q_status fp4q_dequantize(fp4q_format format, const uint8_t* codes,
