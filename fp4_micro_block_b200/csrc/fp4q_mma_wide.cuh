@@ -16,9 +16,9 @@
 // columns for n = 512 (two tiles in flight for n = 256).  All four epilogue
 // warpgroups work on the same tile, warpgroup w on the columns
 // b in [32 w, 32 w + 32) of every group:
-//   pass 1  reads z in steps of 8 columns of every group, applies H_G (and
-//           RN(1/sqrt 2) for n = 512), takes the per-group maxima and writes
-//           y back into TMEM in place;
+//   pass 1  reads z in steps of 8 columns of every group, applies H_G, takes
+//           the per-group maxima and writes y back into TMEM in place (the
+//           remaining RN(1/sqrt 2) of n = 512 is folded into the quantizer);
 //   (sync)  the epilogue warps meet (their pass-2 columns were written by
 //           other warpgroups), and the dual format's group maxima of the four
 //           warpgroups meet in shared memory;
@@ -266,19 +266,30 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 #pragma unroll
                 for (int a = 0; a < G; ++a) tmem_ld8(tbuf + a * kMmaTile + pos, z[a]);
                 tmem_wait_ld8x<G>(z);
+                // butterflies on pairs of columns: the packed f32x2 adds halve the
+                // issue slots (the FMA pipe has room to spare in this kernel)
+                const float2 m1 = make_float2(-1.0f, -1.0f);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
+                for (int i = 0; i < 8; i += 2) {
+                    float2 v[G];
+#pragma unroll
+                    for (int a = 0; a < G; ++a) v[a] = make_float2(z[a][i], z[a][i + 1]);
                     if constexpr (G == 2) {
-                        const float s0 = z[0][i] + z[1][i], d0 = z[0][i] - z[1][i];
-                        z[0][i] = s0;
-                        z[1][i] = d0;
+                        const float2 s0 = __fadd2_rn(v[0], v[1]), d0 = __ffma2_rn(v[1], m1, v[0]);
+                        v[0] = s0;
+                        v[1] = d0;
                     } else {
-                        const float s01 = z[0][i] + z[1][i], d01 = z[0][i] - z[1][i];
-                        const float s23 = z[2][i] + z[3][i], d23 = z[2][i] - z[3][i];
-                        z[0][i] = s01 + s23;
-                        z[1][i] = d01 + d23;
-                        z[2][i] = s01 - s23;
-                        z[3][i] = d01 - d23;
+                        const float2 s01 = __fadd2_rn(v[0], v[1]), d01 = __ffma2_rn(v[1], m1, v[0]);
+                        const float2 s23 = __fadd2_rn(v[2], v[3]), d23 = __ffma2_rn(v[3], m1, v[2]);
+                        v[0] = __fadd2_rn(s01, s23);
+                        v[1] = __fadd2_rn(d01, d23);
+                        v[2] = __ffma2_rn(s23, m1, s01);
+                        v[3] = __ffma2_rn(d23, m1, d01);
+                    }
+#pragma unroll
+                    for (int a = 0; a < G; ++a) {
+                        z[a][i] = v[a].x;
+                        z[a][i + 1] = v[a].y;
                     }
                 }
 #pragma unroll

@@ -224,6 +224,24 @@ def test_hadamard_quantize_tolerance(fq, n, fmt):
     assert_tolerant(fmt, K, gpu, (c_o, s_o, sc_o), y_o, name=f"had{n}-{fmt}")
 
 
+@pytest.mark.parametrize("n", [32, 128, 512])
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4", "dual"])
+def test_hadamard_quantize_swizzled_scales(fq, n, fmt):
+    """Tensor-core paths writing the 128x4 tiled scale layout; 130 rows leave a
+    ragged second row tile whose padding must stay zero."""
+    M, K = 130, 1024
+    x_bits = workloads.hadamard_channels(M, K, seed=5 * n + len(fmt))
+    fcode = {"nvfp4": fq.FP4Q_NVFP4, "mxfp4": fq.FP4Q_MXFP4, "dual": fq.FP4Q_NVFP4_DUAL}[fmt]
+    codes, scales, sf = fq.hadamard_quantize(bits_to_torch_cuda(x_bits), n, fcode, None,
+                                             fq.FP4Q_SCALES_SWIZZLED)
+    torch.cuda.synchronize()
+    c_o, s_o, sc_o, y_o = oracle.hadamard_quantize(x_bits, n, fmt)
+    ncols = K // (32 if fmt == "mxfp4" else 16)
+    s_lin = linear_scales(fq, scales, M, ncols, fq.FP4Q_SCALES_SWIZZLED)
+    sfv = None if fmt == "mxfp4" else to_np(sf)
+    assert_tolerant(fmt, K, (to_np(codes), s_lin, sfv), (c_o, s_o, sc_o), y_o, name=f"swz-had{n}-{fmt}")
+
+
 @pytest.mark.parametrize("n,K,fmt", [(16, 1040, "nvfp4"), (32, 1056, "nvfp4"), (64, 1088, "nvfp4"),
                                      (32, 1056, "mxfp4"), (64, 1088, "mxfp4"), (16, 1120, "mxfp4")])
 def test_hadamard_quantize_ragged_rows(fq, n, K, fmt):
