@@ -21,6 +21,13 @@
 
 #define FP4Q_API extern "C" __attribute__((visibility("default")))
 
+#ifndef FP4Q_DQ_WARP
+#define FP4Q_DQ_WARP 0
+#endif
+#ifndef FP4Q_ARC_STAGES
+#define FP4Q_ARC_STAGES 2  // row buffers per ARC warp, where they cost no warp
+#endif
+
 namespace {
 
 using namespace fp4q;
@@ -316,8 +323,15 @@ fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, in
 // ---------------------------------------------------------------- dequantizer launch
 template <int FMT, int HAD>
 fp4q_status launch_dequant_t(const DequantParams& p, int grid, cudaStream_t s) {
+#if FP4Q_DQ_WARP
+    auto kern = dequant_warp_kernel<FMT, HAD>;
+    constexpr int smem = (kThreads / 32) * kDqWarpSmem;
+    const int64_t units = ((p.M + 1) / 2) * p.n_col_tiles;
+    grid = (int)std::min<int64_t>({(units + kThreads / 32 - 1) / (kThreads / 32), (int64_t)grid, (int64_t)kMaxGrid});
+#else
     auto kern = dequant_kernel<FMT, HAD>;
     constexpr int smem = dequant_smem_bytes<HAD>();
+#endif
     static std::atomic<uint64_t> done{0};
     fp4q_status st = ensure_smem(kern, smem, done);
     if (st != FP4Q_OK) return st;
@@ -501,17 +515,20 @@ FP4Q_API fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int6
     p.partials = static_cast<float*>(workspace);
     p.swizzled = layout == FP4Q_SCALES_SWIZZLED;
     p.dynamic = dynamic;
-    // Warps per CTA (one row each) and row buffers per warp: as many warps as
-    // fit with two buffers each, else one buffer each.
+    // Warps per CTA (one row each) and row buffers per warp.  The kernel is
+    // bound by issue latency, not by the row copies: more warps beat a second
+    // buffer (K = 4096: 12 warps with one buffer run 8% faster than 11 with
+    // two), so two buffers are taken only where they cost no warp.
     constexpr int kSmemMax = 227 * 1024;
-    int W = 0, SR = 2;
-    for (int w = 12; w >= 1 && !W; --w)  // at most 384 threads (the kernel's launch bound)
-        if (arc_layout(K, S, w, 2).total <= kSmemMax) W = w;
-    if (W < 4) {
+    auto max_warps = [&](int sr) {
+        for (int w = 12; w >= 1; --w)  // at most 384 threads (the kernel's launch bound)
+            if (arc_layout(K, S, w, sr).total <= kSmemMax) return w;
+        return 0;
+    };
+    int SR = FP4Q_ARC_STAGES, W = max_warps(SR);
+    if (SR > 1 && max_warps(1) > W) {
         SR = 1;
-        W = 0;
-        for (int w = 12; w >= 1 && !W; --w)
-            if (arc_layout(K, S, w, 1).total <= kSmemMax) W = w;
+        W = max_warps(1);
     }
     if (W == 0) return FP4Q_ERR_UNSUPPORTED;
     p.warps = W;

@@ -20,17 +20,48 @@ constexpr int kTileRows = 16;   // dequantizer tile: 16 rows x 512 columns
 constexpr int kTileCols = 512;
 constexpr int kDqScratchBytes = kTileRows * kTileCols * 4;
 
-// In-register butterflies over v[0..N) (unnormalised Walsh-Hadamard).
-template <int N>
+// In-register butterflies over v[0..N) (unnormalised Walsh-Hadamard).  With
+// PACKED the adds run on pairs of columns with the packed f32x2 add (half the
+// issue slots; the tile dequantizer has FMA-pipe capacity to spare, the
+// streaming one has no registers to spare): stride 1 pairs (v[i], v[i+2]) with
+// (v[i+1], v[i+3]); strides >= 2 pair (v[i], v[i+1]) with (v[i+s], v[i+s+1]).
+template <int N, bool PACKED = false>
 __device__ __forceinline__ void fwht_reg(float* v) {
+    if constexpr (!PACKED) {
 #pragma unroll
-    for (int s = 1; s < N; s <<= 1) {
+        for (int s = 1; s < N; s <<= 1) {
 #pragma unroll
-        for (int i = 0; i < N; ++i) {
-            if ((i & s) == 0) {
-                float a = v[i], b = v[i + s];
-                v[i] = a + b;
-                v[i + s] = a - b;
+            for (int i = 0; i < N; ++i) {
+                if ((i & s) == 0) {
+                    float a = v[i], b = v[i + s];
+                    v[i] = a + b;
+                    v[i + s] = a - b;
+                }
+            }
+        }
+        return;
+    }
+    const float2 m1 = make_float2(-1.0f, -1.0f);
+#pragma unroll
+    for (int i = 0; i < N; i += 4) {
+        const float2 a = make_float2(v[i], v[i + 2]), b = make_float2(v[i + 1], v[i + 3]);
+        const float2 s = __fadd2_rn(a, b), d = __ffma2_rn(b, m1, a);
+        v[i] = s.x;
+        v[i + 2] = s.y;
+        v[i + 1] = d.x;
+        v[i + 3] = d.y;
+    }
+#pragma unroll
+    for (int st = 2; st < N; st <<= 1) {
+#pragma unroll
+        for (int i = 0; i < N; i += 2) {
+            if ((i & st) == 0) {
+                const float2 a = make_float2(v[i], v[i + 1]), b = make_float2(v[i + st], v[i + st + 1]);
+                const float2 s = __fadd2_rn(a, b), d = __ffma2_rn(b, m1, a);
+                v[i] = s.x;
+                v[i + 1] = s.y;
+                v[i + st] = d.x;
+                v[i + st + 1] = d.y;
             }
         }
     }
@@ -255,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_kernel(co
             coords(t + gridDim.x, row2, col2, nval2);
             if (nval2) load_raw<FMT>(p, row2, col2, nval2, nxt);
         }
-        const bool live = nval > 0;
+        bool live = nval > 0;
         float v[32];
         if (live) {
             decode_raw<FMT>(cur, v);
@@ -265,6 +296,7 @@ __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_kernel(co
         }
         cur = nxt;
         uint16_t* yrow = p.y + row * p.K;
+        const bool nval_tile = ct * kTileCols < p.K;  // the tile's columns exist
 
         if constexpr (HAD <= 32) {
             if constexpr (HAD == 16) {
@@ -292,15 +324,14 @@ __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_kernel(co
         } else {
             constexpr int n2 = HadShape<HAD>::n2;
             constexpr int k1w = HadShape<HAD>::k1w;
-            const uint32_t tau = j % n2, blk = j / n2;
-            fwht_reg<32>(v);
-            uint8_t* sb = reinterpret_cast<uint8_t*>(scratch) +
-                          (r * (kTileCols / HAD) + blk) * (uint32_t)(n2 * 128);
+            fwht_reg<32, true>(v);
+            uint8_t* const sc = reinterpret_cast<uint8_t*>(scratch);
             const bool cross_warp = n2 > 4;
             if (cross_warp) bar_sync(2, kThreads);
             else __syncwarp();
             {
-                uint8_t* rowp = sb + tau * 128;
+                uint8_t* rowp = sc + (r * (kTileCols / HAD) + j / n2) * (uint32_t)(n2 * 128) +
+                                (j % n2) * 128;
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch)
                     *reinterpret_cast<float4*>(rowp + (((ch ^ r) & 7u) << 4)) =
@@ -308,6 +339,24 @@ __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_kernel(co
             }
             if (cross_warp) bar_sync(2, kThreads);
             else __syncwarp();
+            // Second half: thread (r2, blk, tau) combines columns k1w*tau .. +k1w
+            // of the n2 sub-rows of block blk of tile row r2.  It is the first
+            // half's thread except for n = 512 (two columns per sub-row), where
+            // 16 lanes take consecutive tau of one row so that a store
+            // instruction writes whole 32-byte sectors (it has crossed the CTA
+            // barrier, so any thread may take any row).
+            uint32_t r2 = r, tau = j % n2, blk = j / n2;
+            if constexpr (k1w == 2) {
+                r2 = (lane >> 4) + 2 * warp;
+                tau = lane & 15;
+                blk = 0;
+            }
+            const uint8_t* sb = sc + (r2 * (kTileCols / HAD) + blk) * (uint32_t)(n2 * 128);
+            if constexpr (k1w == 2) {
+                row = (t / p.n_col_tiles) * kTileRows + r2;
+                yrow = p.y + row * p.K;
+                live = row < p.M && nval_tile;
+            }
             float a[n2][k1w];
             const uint32_t k1 = k1w * tau;
 #pragma unroll
@@ -315,14 +364,14 @@ __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_kernel(co
                 const uint8_t* rowp = sb + k2 * 128;
                 if constexpr (k1w == 2) {
                     float2 q = *reinterpret_cast<const float2*>(
-                        rowp + ((((k1 >> 2) ^ r) & 7u) << 4) + (k1 & 3u) * 4u);
+                        rowp + ((((k1 >> 2) ^ r2) & 7u) << 4) + (k1 & 3u) * 4u);
                     a[k2][0] = q.x;
                     a[k2][1] = q.y;
                 } else {
 #pragma unroll
                     for (int h = 0; h < k1w / 4; ++h) {
                         float4 q = *reinterpret_cast<const float4*>(
-                            rowp + (((((k1 >> 2) + h) ^ r) & 7u) << 4));
+                            rowp + (((((k1 >> 2) + h) ^ r2) & 7u) << 4));
                         a[k2][4 * h] = q.x;
                         a[k2][4 * h + 1] = q.y;
                         a[k2][4 * h + 2] = q.z;
@@ -330,16 +379,21 @@ __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_kernel(co
                     }
                 }
             }
+            const float2 m1 = make_float2(-1.0f, -1.0f);
 #pragma unroll
             for (int s = 1; s < n2; s <<= 1) {
 #pragma unroll
                 for (int k2 = 0; k2 < n2; ++k2) {
                     if ((k2 & s) == 0) {
 #pragma unroll
-                        for (int i = 0; i < k1w; ++i) {
-                            float x0 = a[k2][i], x1 = a[k2 + s][i];
-                            a[k2][i] = x0 + x1;
-                            a[k2 + s][i] = x0 - x1;
+                        for (int i = 0; i < k1w; i += 2) {  // k1w is even: packed pairs
+                            const float2 x0 = make_float2(a[k2][i], a[k2][i + 1]);
+                            const float2 x1 = make_float2(a[k2 + s][i], a[k2 + s][i + 1]);
+                            const float2 sm = __fadd2_rn(x0, x1), df = __ffma2_rn(x1, m1, x0);
+                            a[k2][i] = sm.x;
+                            a[k2][i + 1] = sm.y;
+                            a[k2 + s][i] = df.x;
+                            a[k2 + s][i + 1] = df.y;
                         }
                     }
                 }
@@ -365,6 +419,141 @@ __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_kernel(co
                                 bf16x2_pack(a[k2][8 * h + 4] * p.had_norm, a[k2][8 * h + 5] * p.had_norm),
                                 bf16x2_pack(a[k2][8 * h + 6] * p.had_norm, a[k2][8 * h + 7] * p.had_norm));
                     }
+                }
+            }
+        }
+    }
+}
+
+// Hadamard sizes 64..512 without CTA barriers: a warp owns a unit of two rows
+// x 512 columns.  Lane (r2 = lane / 16, l = lane % 16) decodes columns
+// [32 l, 32 l + 32) of row r2 and applies H_32 in registers; the warp then
+// exchanges through its own 4 KiB of shared memory (a warp barrier), and lane
+// (r2, m) applies H_n2 across the n2 sub-rows of 32 columns of block
+// b = m / n2 to its k1w = 32 / n2 columns, tau = m % n2.  For a fixed k2 the
+// n2 lanes of a block store 64 consecutive bytes of the row.  The next unit's
+// codes and scales are loaded before the current one is worked on.
+constexpr int kDqWarpSmem = 4096;  // per warp: 2 rows x 16 sub-rows x 32 fp32
+
+// 16-byte chunk c of sub-row l sits at chunk c ^ dq_swz(l): conflict-free for
+// the row writes and for the column reads of every n2.
+__device__ __forceinline__ uint32_t dq_swz(uint32_t l) { return (l & 7u) ^ ((l >> 2) & 1u); }
+
+template <int FMT, int HAD>
+__global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_warp_kernel(const DequantParams p) {
+    pdl_wait();
+    pdl_trigger();
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    constexpr int n2 = HadShape<HAD>::n2, k1w = HadShape<HAD>::k1w;
+    static_assert(HAD >= 64 && n2 * k1w == 32, "block sizes 64..512");
+    const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint8_t* const ws = smem_raw + warp * kDqWarpSmem;
+    const uint32_t r2 = lane >> 4, l = lane & 15;
+    const uint32_t m = l, b = m / n2, tau = m % n2, k1 = k1w * tau;
+    const int64_t n_ct = p.n_col_tiles;  // 512-column tiles per row
+    const int64_t n_units = ((p.M + 1) / 2) * n_ct;
+    const int64_t stride = (int64_t)gridDim.x * (kThreads / 32);
+    int64_t u = (int64_t)blockIdx.x * (kThreads / 32) + warp;
+
+    auto valid = [&](int64_t uu, int64_t& row, int64_t& col) {
+        row = (uu / n_ct) * 2 + r2;
+        col = (uu % n_ct) * kTileCols + 32 * (int64_t)l;
+        return row < p.M && col < p.K;  // K % 64 == 0: whole 32-column pieces
+    };
+    RawUnit cur{};
+    {
+        int64_t row, col;
+        if (u < n_units && valid(u, row, col)) load_raw<FMT>(p, row, col, 32, cur);
+    }
+    for (; u < n_units; u += stride) {
+        int64_t row, col;
+        const bool live = valid(u, row, col);
+        RawUnit nxt{};
+        {
+            int64_t row2, col2;
+            if (u + stride < n_units && valid(u + stride, row2, col2)) load_raw<FMT>(p, row2, col2, 32, nxt);
+        }
+        float v[32];
+        if (live) {
+            decode_raw<FMT>(cur, v);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+        }
+        cur = nxt;
+        fwht_reg<32, true>(v);
+        __syncwarp();  // the previous unit's reads of this warp's scratch are done
+        {
+            uint8_t* rowp = ws + r2 * 2048u + l * 128u;
+            const uint32_t z = dq_swz(l);
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<float4*>(rowp + ((ch ^ z) << 4)) =
+                    make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
+        }
+        __syncwarp();
+        float a[n2][k1w];
+#pragma unroll
+        for (int k2 = 0; k2 < n2; ++k2) {
+            const uint32_t sl = b * n2 + k2;  // sub-row of this block
+            const uint8_t* rowp = ws + r2 * 2048u + sl * 128u;
+            const uint32_t z = dq_swz(sl);
+            if constexpr (k1w == 2) {
+                const float2 q = *reinterpret_cast<const float2*>(rowp + (((k1 >> 2) ^ z) << 4) + (k1 & 3u) * 4u);
+                a[k2][0] = q.x;
+                a[k2][1] = q.y;
+            } else {
+#pragma unroll
+                for (int h = 0; h < k1w / 4; ++h) {
+                    const float4 q = *reinterpret_cast<const float4*>(rowp + ((((k1 >> 2) + h) ^ z) << 4));
+                    a[k2][4 * h] = q.x;
+                    a[k2][4 * h + 1] = q.y;
+                    a[k2][4 * h + 2] = q.z;
+                    a[k2][4 * h + 3] = q.w;
+                }
+            }
+        }
+        const float2 m1 = make_float2(-1.0f, -1.0f);
+#pragma unroll
+        for (int st = 1; st < n2; st <<= 1) {
+#pragma unroll
+            for (int k2 = 0; k2 < n2; ++k2) {
+                if ((k2 & st) == 0) {
+#pragma unroll
+                    for (int i = 0; i < k1w; i += 2) {
+                        const float2 x0 = make_float2(a[k2][i], a[k2][i + 1]);
+                        const float2 x1 = make_float2(a[k2 + st][i], a[k2 + st][i + 1]);
+                        const float2 sm = __fadd2_rn(x0, x1), df = __ffma2_rn(x1, m1, x0);
+                        a[k2][i] = sm.x;
+                        a[k2][i + 1] = sm.y;
+                        a[k2 + st][i] = df.x;
+                        a[k2 + st][i + 1] = df.y;
+                    }
+                }
+            }
+        }
+        // output row of this lane's block: the row of its half-warp, the
+        // block's columns exist when its first column does (K % n == 0)
+        const int64_t cb = (u % n_ct) * kTileCols + (int64_t)b * HAD + k1;
+        if (row < p.M && cb < p.K) {
+            uint16_t* yrow = p.y + row * p.K;
+            const float hn = p.had_norm;
+#pragma unroll
+            for (int k2 = 0; k2 < n2; ++k2) {
+                uint16_t* dst = yrow + cb + 32 * k2;
+                if constexpr (k1w == 2) {
+                    *reinterpret_cast<uint32_t*>(dst) = bf16x2_pack(a[k2][0] * hn, a[k2][1] * hn);
+                } else if constexpr (k1w == 4) {
+                    *reinterpret_cast<uint2*>(dst) =
+                        make_uint2(bf16x2_pack(a[k2][0] * hn, a[k2][1] * hn), bf16x2_pack(a[k2][2] * hn, a[k2][3] * hn));
+                } else {
+#pragma unroll
+                    for (int h = 0; h < k1w / 8; ++h)
+                        reinterpret_cast<uint4*>(dst)[h] = make_uint4(
+                            bf16x2_pack(a[k2][8 * h + 0] * hn, a[k2][8 * h + 1] * hn),
+                            bf16x2_pack(a[k2][8 * h + 2] * hn, a[k2][8 * h + 3] * hn),
+                            bf16x2_pack(a[k2][8 * h + 4] * hn, a[k2][8 * h + 5] * hn),
+                            bf16x2_pack(a[k2][8 * h + 6] * hn, a[k2][8 * h + 7] * hn));
                 }
             }
         }

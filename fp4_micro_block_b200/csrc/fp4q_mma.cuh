@@ -6,7 +6,9 @@
 // Sylvester order, f = floor(log2(n) / 2)).  Every product of a bf16 input with
 // +-2^-f is exact and the sums accumulate in fp32 in tensor memory, so the tile
 // arrives in TMEM as the negated, (partly) normalised rotation; odd log2(n)
-// leaves a factor RN(1/sqrt(2)) for the epilogue.  (MR-GPTQ applies the
+// leaves a factor RN(1/sqrt(2)) for the epilogue.  B's columns come in the
+// acc_col order, which puts the two 16-column blocks of a 32-column chunk in
+// alternate accumulator columns.  (MR-GPTQ applies the
 // Hadamard as a matrix product on the activations; FP4Quant notes the FWHT as
 // one of the costs of the format.)
 //
@@ -137,9 +139,16 @@ constexpr int kMmaRedOff = kMmaTabOff + 128 * 16;
 constexpr int kMmaSmemBytes = 1024 + kMmaRedOff + (kMmaThreads / 32) * 4;
 static_assert(kMmaSmemBytes <= 227 * 1024, "shared memory");
 
+// Output column held by accumulator column j.  Within each 32-column chunk,
+// accumulator columns 2i and 2i+1 hold output columns i and 16 + i, so that a
+// 32-column TMEM load lands the quantizer's pairs (one column of each 16-column
+// block) in adjacent registers.
+__host__ __device__ constexpr int acc_col(int j) { return (j & ~31) | ((j & 1) << 4) | ((j >> 1) & 15); }
+
 // B = -2^-f * blockdiag(H_n) in the K-major 128-byte-swizzled layout of the
 // tile: element (row nn, column k) of half h = k / 64 lives at byte
-// h * 16 KiB + nn * 128 + ((k % 64) / 8 ^ nn % 8) * 16 + (k % 8) * 2.
+// h * 16 KiB + nn * 128 + ((k % 64) / 8 ^ nn % 8) * 16 + (k % 8) * 2; row nn
+// holds the Hadamard entries of output column acc_col(nn).
 template <int HAD>
 __device__ __forceinline__ void build_hadamard_b(uint8_t* b) {
     constexpr int lg = HAD == 16 ? 4 : HAD == 32 ? 5 : HAD == 64 ? 6 : 7;
@@ -147,6 +156,7 @@ __device__ __forceinline__ void build_hadamard_b(uint8_t* b) {
     for (int chunk = threadIdx.x; chunk < kTileBytes / 16; chunk += blockDim.x) {
         const int h = chunk / 1024, nn = (chunk / 8) % 128, cp = chunk % 8;  // physical chunk cp
         const int c = cp ^ (nn & 7);                                          // logical 16-byte chunk
+        const int oc = acc_col(nn);  // B row nn (accumulator column nn) is output column oc
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 8; e += 2) {
@@ -155,8 +165,8 @@ __device__ __forceinline__ void build_hadamard_b(uint8_t* b) {
             for (int t = 0; t < 2; ++t) {
                 const int k = h * 64 + c * 8 + e + t;
                 uint32_t bits = 0;
-                if (k / HAD == nn / HAD) {
-                    const int par = __popc((uint32_t)((k % HAD) & (nn % HAD))) & 1;
+                if (k / HAD == oc / HAD) {
+                    const int par = __popc((uint32_t)((k % HAD) & (oc % HAD))) & 1;
                     bits = mag | (par ? 0u : 0x8000u);  // -(+-1) * 2^-f
                 }
                 pair |= bits << (16 * t);
@@ -352,7 +362,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
                 float v[32];
                 tmem_ld32(tacc + 32u * c, v);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) n[i] = make_float2(v[i], v[16 + i]);
+                for (int i = 0; i < 16; ++i) n[i] = make_float2(v[2 * i], v[2 * i + 1]);
             };
             auto release = [&]() {  // every lane's loads of this accumulator are done
                 tc_fence_before();

@@ -94,12 +94,13 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// B = -2^-4 * H_128 (K-major, 128-byte swizzle) for n = 256 and 512.
+// B = -2^-4 * H_128 (K-major, 128-byte swizzle) for n = 256 and 512, its rows
+// (accumulator columns) in the acc_col order of the 128-column kernel.
 __device__ __forceinline__ void build_h128_b(uint8_t* b) {
     const uint32_t mag = 0x3f80u - 4u * 0x80u;  // bf16 bits of 2^-4
     for (int chunk = threadIdx.x; chunk < kTileBytes / 16; chunk += blockDim.x) {
         const int h = chunk / 1024, nn = (chunk / 8) % 128, cp = chunk % 8;
-        const int c = cp ^ (nn & 7);
+        const int c = cp ^ (nn & 7), oc = acc_col(nn);
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 8; e += 2) {
@@ -107,7 +108,7 @@ __device__ __forceinline__ void build_h128_b(uint8_t* b) {
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
                 const int k = h * 64 + c * 8 + e + t;
-                const int par = __popc((uint32_t)(k & nn)) & 1;
+                const int par = __popc((uint32_t)(k & oc)) & 1;
                 pair |= (mag | (par ? 0u : 0x8000u)) << (16 * t);
             }
             w[e / 2] = pair;
@@ -365,7 +366,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                     float v[32];
                     tmem_ld32(tbuf + a * kMmaTile + 32u * c, v);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) n[i] = make_float2(v[i], v[16 + i]);
+                    for (int i = 0; i < 16; ++i) n[i] = make_float2(v[2 * i], v[2 * i + 1]);
                     const uint32_t ea = quant_chunk<FMT>(n, ctx, tab, fold, wa);
                     tmem_ld32(tbuf + a * kMmaTile + 32u * (c + 1), v);
                     if (c + 2 == c0 + G) {
@@ -374,7 +375,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                         if (lane == 0) mbar_arrive(relg0 + 8 * (b * G + a));
                     }
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) n[i] = make_float2(v[i], v[16 + i]);
+                    for (int i = 0; i < 16; ++i) n[i] = make_float2(v[2 * i], v[2 * i + 1]);
                     const uint32_t eb = quant_chunk<FMT>(n, ctx, tab, fold, wb);
                     const int64_t col = colg + 32 * c;
                     store_chunk_pair(p.codes + row * kc + col / 2, kc, live_even, live_odd, lane, wa, wb);
