@@ -21,9 +21,6 @@
 
 #define FP4Q_API extern "C" __attribute__((visibility("default")))
 
-#ifndef FP4Q_DQ_WARP
-#define FP4Q_DQ_WARP 0
-#endif
 #ifndef FP4Q_ARC_STAGES
 #define FP4Q_ARC_STAGES 2  // row buffers per ARC warp, where they cost no warp
 #endif
@@ -322,16 +319,13 @@ fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, in
 
 // ---------------------------------------------------------------- dequantizer launch
 template <int FMT, int HAD>
-fp4q_status launch_dequant_t(const DequantParams& p, int grid, cudaStream_t s) {
-#if FP4Q_DQ_WARP
+fp4q_status launch_dequant_t(const DequantParams& p, int sms, cudaStream_t s) {
     auto kern = dequant_warp_kernel<FMT, HAD>;
-    constexpr int smem = (kThreads / 32) * kDqWarpSmem;
-    const int64_t units = ((p.M + 1) / 2) * p.n_col_tiles;
-    grid = (int)std::min<int64_t>({(units + kThreads / 32 - 1) / (kThreads / 32), (int64_t)grid, (int64_t)kMaxGrid});
-#else
-    auto kern = dequant_kernel<FMT, HAD>;
-    constexpr int smem = dequant_smem_bytes<HAD>();
-#endif
+    constexpr int kWarps = kThreads / 32;
+    constexpr int smem = kWarps * kDqWarpSmem;
+    const int64_t units = ((p.M + 1) / 2) * p.n_col_tiles;  // (row pair, 512 columns)
+    const int grid = (int)std::min<int64_t>({(units + kWarps - 1) / kWarps, (int64_t)kDequantCtasPerSm * sms,
+                                            (int64_t)kMaxGrid});
     static std::atomic<uint64_t> done{0};
     fp4q_status st = ensure_smem(kern, smem, done);
     if (st != FP4Q_OK) return st;
@@ -349,15 +343,15 @@ fp4q_status launch_dequant_stream(const DequantParams& p, int sms, cudaStream_t 
 }
 
 template <int FMT>
-fp4q_status launch_dequant_h(int had, const DequantParams& p, int grid, int sms, cudaStream_t s) {
+fp4q_status launch_dequant_h(int had, const DequantParams& p, int sms, cudaStream_t s) {
     switch (had) {
         case 0: return launch_dequant_stream<FMT, 0>(p, sms, s);
         case 16: return launch_dequant_stream<FMT, 16>(p, sms, s);
         case 32: return launch_dequant_stream<FMT, 32>(p, sms, s);
-        case 64: return launch_dequant_t<FMT, 64>(p, grid, s);
-        case 128: return launch_dequant_t<FMT, 128>(p, grid, s);
-        case 256: return launch_dequant_t<FMT, 256>(p, grid, s);
-        case 512: return launch_dequant_t<FMT, 512>(p, grid, s);
+        case 64: return launch_dequant_t<FMT, 64>(p, sms, s);
+        case 128: return launch_dequant_t<FMT, 128>(p, sms, s);
+        case 256: return launch_dequant_t<FMT, 256>(p, sms, s);
+        case 512: return launch_dequant_t<FMT, 512>(p, sms, s);
         default: return FP4Q_ERR_INVALID_ARG;
     }
 }
@@ -521,7 +515,7 @@ FP4Q_API fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int6
     // two), so two buffers are taken only where they cost no warp.
     constexpr int kSmemMax = 227 * 1024;
     auto max_warps = [&](int sr) {
-        for (int w = 12; w >= 1; --w)  // at most 384 threads (the kernel's launch bound)
+        for (int w = kArcMaxWarps; w >= 1; --w)  // the kernel's launch bound
             if (arc_layout(K, S, w, sr).total <= kSmemMax) return w;
         return 0;
     };
@@ -584,20 +578,17 @@ FP4Q_API fp4q_status fp4q_dequantize(fp4q_format format, const uint8_t* codes,
     p.M = M;
     p.K = K;
     p.n_col_tiles = (K + kTileCols - 1) / kTileCols;
-    p.n_tiles = ((M + kTileRows - 1) / kTileRows) * p.n_col_tiles;
     p.codes = codes;
     p.scales = scales;
     p.scale_fp32 = scale_fp32;
     p.y = static_cast<uint16_t*>(y);
     p.swizzled = layout == FP4Q_SCALES_SWIZZLED;
     p.had_norm = had_norm(inv_had_size);
-    const int grid =
-        (int)std::min<int64_t>({p.n_tiles, (int64_t)kDequantCtasPerSm * sms, (int64_t)kMaxGrid});
     cudaStream_t s = (cudaStream_t)stream;
     switch (fmt) {
-        case FMT_NVFP4: return launch_dequant_h<FMT_NVFP4>(inv_had_size, p, grid, sms, s);
-        case FMT_MXFP4: return launch_dequant_h<FMT_MXFP4>(inv_had_size, p, grid, sms, s);
-        default: return launch_dequant_h<FMT_DUAL>(inv_had_size, p, grid, sms, s);
+        case FMT_NVFP4: return launch_dequant_h<FMT_NVFP4>(inv_had_size, p, sms, s);
+        case FMT_MXFP4: return launch_dequant_h<FMT_MXFP4>(inv_had_size, p, sms, s);
+        default: return launch_dequant_h<FMT_DUAL>(inv_had_size, p, sms, s);
     }
 }
 

@@ -26,6 +26,11 @@
 
 namespace fp4q {
 
+#ifndef FP4Q_ARC_MAX_WARPS
+#define FP4Q_ARC_MAX_WARPS 14
+#endif
+constexpr int kArcMaxWarps = FP4Q_ARC_MAX_WARPS;  // launch bound: rows in flight per SM
+
 struct ArcParams {
     int64_t M, K, S;
     const int32_t* perm;      // [K]
@@ -67,7 +72,7 @@ __host__ __device__ inline ArcLayout arc_layout(int64_t K, int64_t S, int warps,
 }
 
 template <bool AMAX_ONLY>
-__global__ void __launch_bounds__(384, 1) arc_kernel(const ArcParams p) {
+__global__ void __launch_bounds__(kArcMaxWarps * 32, 1) arc_kernel(const ArcParams p) {
     pdl_wait();
     pdl_trigger();
     extern __shared__ __align__(1024) uint8_t smem_raw[];

@@ -3,26 +3,25 @@
 // (the normalised Sylvester matrix is its own inverse).  This is the receiving
 // side of FP4-compressed activations (FP4Quant abstract).
 //
-// Same tile geometry and thread -> unit map as the quantizer (16 rows x 512
-// columns per tile, one 32-column unit per thread).  Codes and scales are read
-// straight from global memory (0.5-0.6 byte per element); the bf16 output is
-// written with 16-byte stores.  For Hadamard sizes >= 64 the unit first gets
-// H_32 in registers, then the threads of one n-block exchange through a
-// swizzled fp32 scratch, apply H_n2 across the 32-column rows, and store their
-// column slices.
+// A unit is 32 consecutive columns of one row (two NVFP4 blocks, one MXFP4
+// block).  Codes and scales are read straight from global memory (0.5-0.6 byte
+// per element); the bf16 output is written with 16- or 32-byte stores.
+//   n <= 32: dequant_stream_kernel, one unit per thread at a time, several
+//            units' loads in flight, the rotation in registers;
+//   n >= 64: dequant_warp_kernel, a warp per (row pair, 512 columns): H_32 in
+//            registers, an exchange through the warp's own shared memory, then
+//            H_(n/32) across the 32-column sub-rows of each block.
 #pragma once
 
 #include "fp4q_quant.cuh"
 
 namespace fp4q {
 
-constexpr int kTileRows = 16;   // dequantizer tile: 16 rows x 512 columns
-constexpr int kTileCols = 512;
-constexpr int kDqScratchBytes = kTileRows * kTileCols * 4;
+constexpr int kTileCols = 512;  // columns of a dequantizer unit for n >= 64
 
 // In-register butterflies over v[0..N) (unnormalised Walsh-Hadamard).  With
 // PACKED the adds run on pairs of columns with the packed f32x2 add (half the
-// issue slots; the tile dequantizer has FMA-pipe capacity to spare, the
+// issue slots; the warp dequantizer has FMA-pipe capacity to spare, the
 // streaming one has no registers to spare): stride 1 pairs (v[i], v[i+2]) with
 // (v[i+1], v[i+3]); strides >= 2 pair (v[i], v[i+1]) with (v[i+s], v[i+s+1]).
 template <int N, bool PACKED = false>
@@ -75,7 +74,7 @@ struct HadShape {
 
 struct DequantParams {
     int64_t M, K;
-    int64_t n_col_tiles, n_tiles;
+    int64_t n_col_tiles;  // 512-column tiles per row
     const uint8_t* codes;
     const uint8_t* scales;
     const float* scale_fp32;
@@ -85,7 +84,7 @@ struct DequantParams {
 };
 
 // Raw bytes of one 32-column unit: packed codes, its scale byte(s) and the fp32
-// scale, loaded one tile ahead of their use (software pipelining).
+// scale, loaded ahead of their use (software pipelining).
 struct RawUnit {
     uint32_t w[4];
     uint32_t e0, e1;  // scale bytes of the unit's two 16-blocks (MXFP4: e0 only)
@@ -250,181 +249,6 @@ __global__ void __launch_bounds__(kThreads, 3) dequant_stream_kernel(const Dequa
 #endif
 constexpr int kDequantCtasPerSm = FP4Q_DEQUANT_CTAS_PER_SM;
 
-template <int FMT, int HAD>
-__global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_kernel(const DequantParams p) {
-    pdl_wait();
-    pdl_trigger();
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    float* scratch = reinterpret_cast<float*>(smem_raw);
-    const uint32_t tid = threadIdx.x;
-    const uint32_t lane = tid & 31, warp = tid >> 5;
-    const uint32_t r = (lane & 7) + 8 * (warp & 1);
-    const uint32_t j = (lane >> 3) + 4 * (warp >> 1);
-
-    // Unit coordinates of tile t for this thread.
-    auto coords = [&](int64_t t, int64_t& row, int64_t& col, int& nval) {
-        const int64_t rt = t / p.n_col_tiles, ct = t % p.n_col_tiles;
-        row = rt * kTileRows + r;
-        col = ct * kTileCols + 32 * (int64_t)j;
-        nval = (row < p.M && col < p.K) ? (int)min64(32, p.K - col) : 0;
-    };
-    RawUnit cur{};
-    int64_t row, col;
-    int nval;
-    if ((int64_t)blockIdx.x < p.n_tiles) {
-        coords(blockIdx.x, row, col, nval);
-        if (nval) load_raw<FMT>(p, row, col, nval, cur);
-    }
-    for (int64_t t = blockIdx.x; t < p.n_tiles; t += gridDim.x) {
-        coords(t, row, col, nval);
-        const int64_t ct = t % p.n_col_tiles;
-        // issue the next tile's loads before working on this one
-        RawUnit nxt{};
-        if (t + gridDim.x < p.n_tiles) {
-            int64_t row2, col2;
-            int nval2;
-            coords(t + gridDim.x, row2, col2, nval2);
-            if (nval2) load_raw<FMT>(p, row2, col2, nval2, nxt);
-        }
-        bool live = nval > 0;
-        float v[32];
-        if (live) {
-            decode_raw<FMT>(cur, v);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
-        }
-        cur = nxt;
-        uint16_t* yrow = p.y + row * p.K;
-        const bool nval_tile = ct * kTileCols < p.K;  // the tile's columns exist
-
-        if constexpr (HAD <= 32) {
-            if constexpr (HAD == 16) {
-                fwht_reg<16>(v);
-                fwht_reg<16>(v + 16);
-            } else if constexpr (HAD == 32) {
-                fwht_reg<32>(v);
-            }
-            if constexpr (HAD > 0) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] *= p.had_norm;
-            }
-            if (live) {
-                uint32_t o[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) o[i] = bf16x2_pack(v[2 * i], v[2 * i + 1]);
-                uint4* dst = reinterpret_cast<uint4*>(yrow + col);
-                dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-                dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-                if (nval > 16) {
-                    dst[2] = make_uint4(o[8], o[9], o[10], o[11]);
-                    dst[3] = make_uint4(o[12], o[13], o[14], o[15]);
-                }
-            }
-        } else {
-            constexpr int n2 = HadShape<HAD>::n2;
-            constexpr int k1w = HadShape<HAD>::k1w;
-            fwht_reg<32, true>(v);
-            uint8_t* const sc = reinterpret_cast<uint8_t*>(scratch);
-            const bool cross_warp = n2 > 4;
-            if (cross_warp) bar_sync(2, kThreads);
-            else __syncwarp();
-            {
-                uint8_t* rowp = sc + (r * (kTileCols / HAD) + j / n2) * (uint32_t)(n2 * 128) +
-                                (j % n2) * 128;
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch)
-                    *reinterpret_cast<float4*>(rowp + (((ch ^ r) & 7u) << 4)) =
-                        make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
-            }
-            if (cross_warp) bar_sync(2, kThreads);
-            else __syncwarp();
-            // Second half: thread (r2, blk, tau) combines columns k1w*tau .. +k1w
-            // of the n2 sub-rows of block blk of tile row r2.  It is the first
-            // half's thread except for n = 512 (two columns per sub-row), where
-            // 16 lanes take consecutive tau of one row so that a store
-            // instruction writes whole 32-byte sectors (it has crossed the CTA
-            // barrier, so any thread may take any row).
-            uint32_t r2 = r, tau = j % n2, blk = j / n2;
-            if constexpr (k1w == 2) {
-                r2 = (lane >> 4) + 2 * warp;
-                tau = lane & 15;
-                blk = 0;
-            }
-            const uint8_t* sb = sc + (r2 * (kTileCols / HAD) + blk) * (uint32_t)(n2 * 128);
-            if constexpr (k1w == 2) {
-                row = (t / p.n_col_tiles) * kTileRows + r2;
-                yrow = p.y + row * p.K;
-                live = row < p.M && nval_tile;
-            }
-            float a[n2][k1w];
-            const uint32_t k1 = k1w * tau;
-#pragma unroll
-            for (int k2 = 0; k2 < n2; ++k2) {
-                const uint8_t* rowp = sb + k2 * 128;
-                if constexpr (k1w == 2) {
-                    float2 q = *reinterpret_cast<const float2*>(
-                        rowp + ((((k1 >> 2) ^ r2) & 7u) << 4) + (k1 & 3u) * 4u);
-                    a[k2][0] = q.x;
-                    a[k2][1] = q.y;
-                } else {
-#pragma unroll
-                    for (int h = 0; h < k1w / 4; ++h) {
-                        float4 q = *reinterpret_cast<const float4*>(
-                            rowp + (((((k1 >> 2) + h) ^ r2) & 7u) << 4));
-                        a[k2][4 * h] = q.x;
-                        a[k2][4 * h + 1] = q.y;
-                        a[k2][4 * h + 2] = q.z;
-                        a[k2][4 * h + 3] = q.w;
-                    }
-                }
-            }
-            const float2 m1 = make_float2(-1.0f, -1.0f);
-#pragma unroll
-            for (int s = 1; s < n2; s <<= 1) {
-#pragma unroll
-                for (int k2 = 0; k2 < n2; ++k2) {
-                    if ((k2 & s) == 0) {
-#pragma unroll
-                        for (int i = 0; i < k1w; i += 2) {  // k1w is even: packed pairs
-                            const float2 x0 = make_float2(a[k2][i], a[k2][i + 1]);
-                            const float2 x1 = make_float2(a[k2 + s][i], a[k2 + s][i + 1]);
-                            const float2 sm = __fadd2_rn(x0, x1), df = __ffma2_rn(x1, m1, x0);
-                            a[k2][i] = sm.x;
-                            a[k2][i + 1] = sm.y;
-                            a[k2 + s][i] = df.x;
-                            a[k2 + s][i + 1] = df.y;
-                        }
-                    }
-                }
-            }
-            if (live) {
-                const int64_t cb = ct * kTileCols + (int64_t)blk * HAD + k1;
-#pragma unroll
-                for (int k2 = 0; k2 < n2; ++k2) {
-                    uint16_t* dst = yrow + cb + 32 * k2;
-                    if constexpr (k1w == 2) {
-                        *reinterpret_cast<uint32_t*>(dst) =
-                            bf16x2_pack(a[k2][0] * p.had_norm, a[k2][1] * p.had_norm);
-                    } else if constexpr (k1w == 4) {
-                        *reinterpret_cast<uint2*>(dst) =
-                            make_uint2(bf16x2_pack(a[k2][0] * p.had_norm, a[k2][1] * p.had_norm),
-                                       bf16x2_pack(a[k2][2] * p.had_norm, a[k2][3] * p.had_norm));
-                    } else {
-#pragma unroll
-                        for (int h = 0; h < k1w / 8; ++h)
-                            reinterpret_cast<uint4*>(dst)[h] = make_uint4(
-                                bf16x2_pack(a[k2][8 * h + 0] * p.had_norm, a[k2][8 * h + 1] * p.had_norm),
-                                bf16x2_pack(a[k2][8 * h + 2] * p.had_norm, a[k2][8 * h + 3] * p.had_norm),
-                                bf16x2_pack(a[k2][8 * h + 4] * p.had_norm, a[k2][8 * h + 5] * p.had_norm),
-                                bf16x2_pack(a[k2][8 * h + 6] * p.had_norm, a[k2][8 * h + 7] * p.had_norm));
-                    }
-                }
-            }
-        }
-    }
-}
-
 // Hadamard sizes 64..512 without CTA barriers: a warp owns a unit of two rows
 // x 512 columns.  Lane (r2 = lane / 16, l = lane % 16) decodes columns
 // [32 l, 32 l + 32) of row r2 and applies H_32 in registers; the warp then
@@ -439,6 +263,30 @@ constexpr int kDqWarpSmem = 4096;  // per warp: 2 rows x 16 sub-rows x 32 fp32
 // the row writes and for the column reads of every n2.
 __device__ __forceinline__ uint32_t dq_swz(uint32_t l) { return (l & 7u) ^ ((l >> 2) & 1u); }
 
+// Decoded unit times one multiplier per 16-block, m = (E4M3 value * s) * c
+// (MXFP4: 2^(b-127) * c), applied with the packed f32x2 multiply; c is the
+// Hadamard normalisation, moved ahead of the butterflies (a few fp32 ulps from
+// the oracle's order, far inside one bf16 ulp).
+template <int FMT>
+__device__ __forceinline__ void decode_raw_scaled(const RawUnit& u, float c, float* v) {
+    float m0, m1;
+    if constexpr (FMT == FMT_MXFP4) {
+        const uint32_t b = u.e0;
+        m0 = (b ? __uint_as_float(b << 23) : __uint_as_float(0x00400000u)) * c;
+        m1 = m0;
+    } else {
+        m0 = (e4m3_decode(u.e0) * u.s) * c;
+        m1 = (e4m3_decode(u.e1) * u.s) * c;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float m = i < 8 ? m0 : m1;
+        const float2 q = __fmul2_rn(e2m1x2_decode((u.w[i >> 2] >> (8 * (i & 3))) & 0xffu), make_float2(m, m));
+        v[2 * i] = q.x;
+        v[2 * i + 1] = q.y;
+    }
+}
+
 template <int FMT, int HAD>
 __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_warp_kernel(const DequantParams p) {
     pdl_wait();
@@ -446,36 +294,48 @@ __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_warp_kern
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     constexpr int n2 = HadShape<HAD>::n2, k1w = HadShape<HAD>::k1w;
     static_assert(HAD >= 64 && n2 * k1w == 32, "block sizes 64..512");
+    constexpr int kWarps = kThreads / 32;
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint8_t* const ws = smem_raw + warp * kDqWarpSmem;
+    uint8_t* const ws = smem_raw + warp * kDqWarpSmem + (lane >> 4) * 2048u;  // this lane's row
     const uint32_t r2 = lane >> 4, l = lane & 15;
-    const uint32_t m = l, b = m / n2, tau = m % n2, k1 = k1w * tau;
-    const int64_t n_ct = p.n_col_tiles;  // 512-column tiles per row
-    const int64_t n_units = ((p.M + 1) / 2) * n_ct;
-    const int64_t stride = (int64_t)gridDim.x * (kThreads / 32);
-    int64_t u = (int64_t)blockIdx.x * (kThreads / 32) + warp;
-
-    auto valid = [&](int64_t uu, int64_t& row, int64_t& col) {
-        row = (uu / n_ct) * 2 + r2;
-        col = (uu % n_ct) * kTileCols + 32 * (int64_t)l;
-        return row < p.M && col < p.K;  // K % 64 == 0: whole 32-column pieces
+    const uint32_t b = l / n2, tau = l % n2, k1 = k1w * tau;
+    // unit (row pair rp, 512-column tile ct), ct fastest; 32-bit coordinates
+    // (the host keeps rows < 2^31), advanced by the grid stride without division
+    const int32_t n_ct = (int32_t)p.n_col_tiles, n_rp = (int32_t)((p.M + 1) / 2);
+    const int32_t stride = (int32_t)gridDim.x * kWarps;
+    const int32_t drp = stride / n_ct, dct = stride % n_ct;
+    const int32_t u0 = (int32_t)blockIdx.x * kWarps + (int32_t)warp;
+    int32_t rp = u0 / n_ct, ct = u0 % n_ct;
+    auto advance = [&](int32_t& r, int32_t& c) {
+        c += dct;
+        r += drp;
+        if (c >= n_ct) {
+            c -= n_ct;
+            ++r;
+        }
+    };
+    auto in_range = [&](int32_t r, int32_t c) {  // K % 64 == 0: whole 32-column pieces
+        return (int64_t)r * 2 + r2 < p.M && (int64_t)c * kTileCols + 32 * l < p.K;
+    };
+    // phase-B read offset of sub-row sl within the lane's row (swizzled chunk)
+    auto rd_off = [&](uint32_t sl, int h) -> uint32_t {
+        const uint32_t z = dq_swz(sl);
+        if constexpr (k1w == 2) return sl * 128u + (((k1 >> 2) ^ z) << 4) + (k1 & 3u) * 4u;
+        else return sl * 128u + ((((k1 >> 2) + (uint32_t)h) ^ z) << 4);
     };
     RawUnit cur{};
-    {
-        int64_t row, col;
-        if (u < n_units && valid(u, row, col)) load_raw<FMT>(p, row, col, 32, cur);
-    }
-    for (; u < n_units; u += stride) {
-        int64_t row, col;
-        const bool live = valid(u, row, col);
+    if (rp < n_rp && in_range(rp, ct)) load_raw<FMT>(p, (int64_t)rp * 2 + r2, (int64_t)ct * kTileCols + 32 * l, 32, cur);
+    while (rp < n_rp) {
+        const bool live = in_range(rp, ct);
+        const int64_t row = (int64_t)rp * 2 + r2;
+        const int64_t cb = (int64_t)ct * kTileCols + (int64_t)b * HAD + k1;  // phase-B output column
+        int32_t rn = rp, cn = ct;
+        advance(rn, cn);
         RawUnit nxt{};
-        {
-            int64_t row2, col2;
-            if (u + stride < n_units && valid(u + stride, row2, col2)) load_raw<FMT>(p, row2, col2, 32, nxt);
-        }
+        if (rn < n_rp && in_range(rn, cn)) load_raw<FMT>(p, (int64_t)rn * 2 + r2, (int64_t)cn * kTileCols + 32 * l, 32, nxt);
         float v[32];
         if (live) {
-            decode_raw<FMT>(cur, v);
+            decode_raw_scaled<FMT>(cur, p.had_norm, v);
         } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0.0f;
@@ -484,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_warp_kern
         fwht_reg<32, true>(v);
         __syncwarp();  // the previous unit's reads of this warp's scratch are done
         {
-            uint8_t* rowp = ws + r2 * 2048u + l * 128u;
+            uint8_t* rowp = ws + l * 128u;
             const uint32_t z = dq_swz(l);
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch)
@@ -495,17 +355,15 @@ __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_warp_kern
         float a[n2][k1w];
 #pragma unroll
         for (int k2 = 0; k2 < n2; ++k2) {
-            const uint32_t sl = b * n2 + k2;  // sub-row of this block
-            const uint8_t* rowp = ws + r2 * 2048u + sl * 128u;
-            const uint32_t z = dq_swz(sl);
+            const uint32_t sl = b * n2 + (uint32_t)k2;  // sub-row of this block
             if constexpr (k1w == 2) {
-                const float2 q = *reinterpret_cast<const float2*>(rowp + (((k1 >> 2) ^ z) << 4) + (k1 & 3u) * 4u);
+                const float2 q = *reinterpret_cast<const float2*>(ws + rd_off(sl, 0));
                 a[k2][0] = q.x;
                 a[k2][1] = q.y;
             } else {
 #pragma unroll
                 for (int h = 0; h < k1w / 4; ++h) {
-                    const float4 q = *reinterpret_cast<const float4*>(rowp + ((((k1 >> 2) + h) ^ z) << 4));
+                    const float4 q = *reinterpret_cast<const float4*>(ws + rd_off(sl, h));
                     a[k2][4 * h] = q.x;
                     a[k2][4 * h + 1] = q.y;
                     a[k2][4 * h + 2] = q.z;
@@ -532,37 +390,29 @@ __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_warp_kern
                 }
             }
         }
-        // output row of this lane's block: the row of its half-warp, the
-        // block's columns exist when its first column does (K % n == 0)
-        const int64_t cb = (u % n_ct) * kTileCols + (int64_t)b * HAD + k1;
+        // the block's columns exist when its first one does (K % n == 0)
         if (row < p.M && cb < p.K) {
-            uint16_t* yrow = p.y + row * p.K;
-            const float hn = p.had_norm;
+            uint16_t* dst0 = p.y + row * p.K + cb;
 #pragma unroll
             for (int k2 = 0; k2 < n2; ++k2) {
-                uint16_t* dst = yrow + cb + 32 * k2;
+                uint16_t* dst = dst0 + 32 * k2;
                 if constexpr (k1w == 2) {
-                    *reinterpret_cast<uint32_t*>(dst) = bf16x2_pack(a[k2][0] * hn, a[k2][1] * hn);
+                    *reinterpret_cast<uint32_t*>(dst) = bf16x2_pack(a[k2][0], a[k2][1]);
                 } else if constexpr (k1w == 4) {
                     *reinterpret_cast<uint2*>(dst) =
-                        make_uint2(bf16x2_pack(a[k2][0] * hn, a[k2][1] * hn), bf16x2_pack(a[k2][2] * hn, a[k2][3] * hn));
+                        make_uint2(bf16x2_pack(a[k2][0], a[k2][1]), bf16x2_pack(a[k2][2], a[k2][3]));
                 } else {
 #pragma unroll
                     for (int h = 0; h < k1w / 8; ++h)
                         reinterpret_cast<uint4*>(dst)[h] = make_uint4(
-                            bf16x2_pack(a[k2][8 * h + 0] * hn, a[k2][8 * h + 1] * hn),
-                            bf16x2_pack(a[k2][8 * h + 2] * hn, a[k2][8 * h + 3] * hn),
-                            bf16x2_pack(a[k2][8 * h + 4] * hn, a[k2][8 * h + 5] * hn),
-                            bf16x2_pack(a[k2][8 * h + 6] * hn, a[k2][8 * h + 7] * hn));
+                            bf16x2_pack(a[k2][8 * h + 0], a[k2][8 * h + 1]), bf16x2_pack(a[k2][8 * h + 2], a[k2][8 * h + 3]),
+                            bf16x2_pack(a[k2][8 * h + 4], a[k2][8 * h + 5]), bf16x2_pack(a[k2][8 * h + 6], a[k2][8 * h + 7]));
                 }
             }
         }
+        rp = rn;
+        ct = cn;
     }
-}
-
-template <int HAD>
-constexpr int dequant_smem_bytes() {
-    return HAD >= 64 ? kDqScratchBytes : 0;
 }
 
 }  // namespace fp4q

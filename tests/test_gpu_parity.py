@@ -274,13 +274,16 @@ def test_hadamard_static_scale(fq):
 
 
 @pytest.mark.parametrize("n", [16, 32, 64, 128, 256, 512])
-@pytest.mark.parametrize("fmt", ["nvfp4", "dual"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "dual", "mxfp4"])
 def test_dequantize_inverse_hadamard(fq, n, fmt):
     M, K = 33, 1024
     x_bits = workloads.dual_gain(M, K, seed=n + 1)
     if fmt == "nvfp4":
         c, s, sc, _ = oracle.hadamard_quantize(x_bits, n, "nvfp4")
         sct, f = torch.tensor([sc], device="cuda"), fq.FP4Q_NVFP4
+    elif fmt == "mxfp4":
+        c, s, sc, _ = oracle.hadamard_quantize(x_bits, n, "mxfp4")
+        sct, f = None, fq.FP4Q_MXFP4
     else:
         c, s, sc, _ = oracle.hadamard_quantize(x_bits, n, "dual")
         sct, f = torch.from_numpy(sc).cuda(), fq.FP4Q_NVFP4_DUAL
@@ -288,6 +291,25 @@ def test_dequantize_inverse_hadamard(fq, n, fmt):
     y = fq.dequantize(f, torch.from_numpy(c).cuda(), torch.from_numpy(s).cuda(), sct, K, 0, n)
     torch.cuda.synchronize()
     assert_roundtrip_close(bf16_torch_to_bits(y), want, n, name=f"inv-had{n}-{fmt}")
+
+
+@pytest.mark.parametrize("n,fmt", [(512, "dual"), (256, "nvfp4"), (128, "mxfp4"), (64, "dual")])
+def test_dequantize_inverse_hadamard_grid_stride(fq, n, fmt):
+    """Odd row count and more units than resident warps: each warp of the
+    dequantizer walks several (row pair, 512-column) units, the last pair with
+    one live row.  Random code and scale bytes; the oracle dequantizes a sample
+    of rows (rows are independent) that includes the last ones."""
+    M, K = 12001, 4096
+    codes, scales, sc = workloads.random_payload(M, K, fmt, seed=n)
+    f = {"nvfp4": fq.FP4Q_NVFP4, "mxfp4": fq.FP4Q_MXFP4, "dual": fq.FP4Q_NVFP4_DUAL}[fmt]
+    sct = (None if sc is None else
+           torch.tensor([sc], device="cuda") if fmt == "nvfp4" else torch.from_numpy(sc).cuda())
+    y = fq.dequantize(f, torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(), sct, K, 0, n)
+    torch.cuda.synchronize()
+    rows = np.array(sorted(set(range(0, M, 97)) | {M - 2, M - 1}))
+    sc_rows = sc[rows] if fmt == "dual" else sc
+    want = oracle.dequantize_bf16(fmt, codes[rows], scales[rows], sc_rows, inv_had=n)
+    assert_roundtrip_close(bf16_torch_to_bits(y)[rows], want, n, name=f"inv-had{n}-{fmt}-grid")
 
 
 # ----------------------------------------------------------------------------- ARC

@@ -21,6 +21,8 @@ ARCQuant page).  No dataset is involved.
   arc_activations  : N(0,1), 256 outlier channels x30, gamma ~ U(0.5, 1.5),
                      channel order from a separate 512-row calibration draw
   dual_gain        : N(0,1) x per-token gain exp(N(0,1)) (LogNormal(0,1))
+  random_payload   : uniform random code bytes and scale bytes (a dequantizer
+                     input that needs no quantizer run to produce)
 """
 from __future__ import annotations
 
@@ -35,6 +37,7 @@ __all__ = [
     "hadamard_channels",
     "arc_activations",
     "dual_gain",
+    "random_payload",
     "WORKLOADS",
 ]
 
@@ -133,3 +136,22 @@ def dual_gain(M: int = 32768, K: int = 4096, seed: int = 5) -> np.ndarray:
     rng = np.random.default_rng(seed)
     return _chunked_rows(
         M, K, lambda m: rng.standard_normal((m, K)) * np.exp(rng.standard_normal((m, 1))))
+
+
+def random_payload(M: int, K: int, fmt: str, seed: int = 6):
+    """Uniform random bytes in the storage layout of a quantized [M, K] tensor.
+
+    Returns ``(codes [M, K/2] uint8, scales uint8, scale)``: every code byte in
+    0..255 (two E2M1 codes); scale bytes E4M3 in 0x08..0x6f (NVFP4 / dual) or
+    E8M0 in 100..139 (MXFP4); ``scale`` a float32 tensor scale (NVFP4), a
+    [M, K/128] float32 array drawn from U(1e-3, 1) (dual) or None (MXFP4)."""
+    rng = np.random.default_rng(seed)
+    codes = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
+    if fmt == "mxfp4":
+        return codes, rng.integers(100, 140, size=(M, K // 32), dtype=np.uint8), None
+    scales = rng.integers(0x08, 0x70, size=(M, K // 16), dtype=np.uint8)
+    if fmt == "nvfp4":
+        return codes, scales, np.float32(rng.uniform(1e-3, 1.0))
+    if fmt == "dual":
+        return codes, scales, rng.uniform(1e-3, 1.0, size=(M, K // 128)).astype(np.float32)
+    raise ValueError(fmt)
