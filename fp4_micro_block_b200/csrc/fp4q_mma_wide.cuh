@@ -22,11 +22,12 @@
 //   (sync)  the epilogue warps meet (their pass-2 columns were written by
 //           other warpgroups), and the dual format's group maxima of the four
 //           warpgroups meet in shared memory;
-//   pass 2  warpgroup w quantizes output group w % G (columns [32 c, 32 c + 32)
-//           for its G chunks c), so that each lane writes whole 32-byte sectors
-//           of its row, and hands the group's TMEM columns back to the MMA warp
-//           as soon as its warps have read them (the next tile's UMMAs then
-//           overlap the rest of pass 2).
+//   pass 2  two warpgroups per output group, each quantizing two adjacent
+//           32-column chunks (64 consecutive columns, whole 32-byte sectors of
+//           a lane's row); for n = 512 in two rounds, groups 0-1 then 2-3.  A
+//           group's TMEM columns go back to the MMA warp as soon as its two
+//           warpgroups have read them, so the next tile's UMMAs overlap the
+//           rest of pass 2 (n = 512: groups 0 and 1 during the second round).
 #pragma once
 
 #include "fp4q_mma.cuh"
@@ -143,7 +144,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             mbar_init(empty0 + 8 * s, 1);
         }
         for (int b = 0; b < NBUF; ++b) mbar_init(accf0 + 8 * b, 1);
-        for (int k = 0; k < NBUF * G; ++k) mbar_init(relg0 + 8 * k, kWideEpiWarps / G);  // its group's warps
+        for (int k = 0; k < NBUF * G; ++k) mbar_init(relg0 + 8 * k, 8);  // two warpgroups read a group
         for (int k = 0; k < 2; ++k) mbar_init(redb0 + 8 * k, kWideEpiWarps);
         mbar_init(done_bar, 1);
         fence_barrier_init();
@@ -309,8 +310,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0)
+                if (lane == 0) {
                     mbar_arrive(relg0 + 8 * (b * G + (int)(wg % G)));
+                    if constexpr (G == 4) mbar_arrive(relg0 + 8 * (b * G + (int)((wg + 2) % G)));
+                }
                 continue;
             } else {
                 // Pass 2 reads columns that other warpgroups wrote in pass 1: every
@@ -343,24 +346,30 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                         gs[a] = (gm >= 0x1p-90f) ? div_split(-gm, 2688.0f, rcp2688()) : __fdiv_rn(gm, 2688.0f);
                     }
                 }
-                // ---- pass 2: warpgroup wg quantizes output group a = wg % G, chunks
-                // [c0, c0 + G) of its 4 (all of them for n = 512), so that a lane
-                // writes 64 consecutive columns of its row; the group's TMEM
-                // columns go back to the MMA warp once its warps have read them.
-                const int a = (int)(wg % G), c0 = (int)(wg / G) * G;
-                float g = 0.0f;
-                if constexpr (FMT == FMT_DUAL) {
-                    g = gs[0];
-#pragma unroll
-                    for (int q = 1; q < G; ++q) g = a == q ? gs[q] : g;
-                    if (live && c0 == 0) p.scale_fp32[row * (p.K / 128) + ct * G + a] = g;
-                }
-                const ScaleCtx ctx = FMT == FMT_DUAL ? make_ctx(g) : ctx_t;
+                // ---- pass 2: two warpgroups per output group, each quantizing two
+                // adjacent chunks of 32 columns, so that a lane writes 64
+                // consecutive columns (whole 32-byte sectors) of its row.  n = 256:
+                // warpgroup wg takes chunks [2 (wg / 2), +2) of group wg % 2.
+                // n = 512: two rounds, groups {0, 1} then {2, 3}, warpgroup wg
+                // taking chunks [2 (wg % 2), +2) of group 2 h + wg / 2; a group's
+                // TMEM columns go back to the MMA warp as soon as its two
+                // warpgroups have read them, so the next tile's UMMAs for groups
+                // 0 and 1 overlap the second round.
                 const int64_t row_even = row - (lane & 1u);
                 const bool live_even = row_even < p.M, live_odd = row_even + 1 < p.M;
-                const int64_t colg = ct * HAD + a * kMmaTile;  // first column of the group
 #pragma unroll 1
-                for (int c = c0; c < c0 + G; c += 2) {
+                for (int h = 0; h < G / 2; ++h) {
+                    const int a = G == 4 ? 2 * h + (int)(wg / 2) : (int)(wg % 2);
+                    const int c = G == 4 ? 2 * (int)(wg % 2) : 2 * (int)(wg / 2);
+                    float g = 0.0f;
+                    if constexpr (FMT == FMT_DUAL) {
+                        g = gs[0];
+#pragma unroll
+                        for (int q = 1; q < G; ++q) g = a == q ? gs[q] : g;
+                        if (live && c == 0) p.scale_fp32[row * (p.K / 128) + ct * G + a] = g;
+                    }
+                    const ScaleCtx ctx = FMT == FMT_DUAL ? make_ctx(g) : ctx_t;
+                    const int64_t col = ct * HAD + a * kMmaTile + 32 * c;  // first column of the pair
                     uint32_t wa[4], wb[4];
                     float2 n[16];
                     float v[32];
@@ -369,15 +378,12 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                     for (int i = 0; i < 16; ++i) n[i] = make_float2(v[2 * i], v[2 * i + 1]);
                     const uint32_t ea = quant_chunk<FMT>(n, ctx, tab, fold, wa);
                     tmem_ld32(tbuf + a * kMmaTile + 32u * (c + 1), v);
-                    if (c + 2 == c0 + G) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(relg0 + 8 * (b * G + a));
-                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(relg0 + 8 * (b * G + a));
 #pragma unroll
                     for (int i = 0; i < 16; ++i) n[i] = make_float2(v[2 * i], v[2 * i + 1]);
                     const uint32_t eb = quant_chunk<FMT>(n, ctx, tab, fold, wb);
-                    const int64_t col = colg + 32 * c;
                     store_chunk_pair(p.codes + row * kc + col / 2, kc, live_even, live_odd, lane, wa, wb);
                     if (live) {
                         if constexpr (FMT == FMT_MXFP4) {  // two E8M0 bytes, 2-byte aligned
