@@ -20,10 +20,10 @@ namespace fp4q {
 constexpr int kTileCols = 512;  // columns of a dequantizer unit for n >= 64
 
 // In-register butterflies over v[0..N) (unnormalised Walsh-Hadamard).  With
-// PACKED the adds run on pairs of columns with the packed f32x2 add (half the
-// issue slots; the warp dequantizer has FMA-pipe capacity to spare, the
-// streaming one has no registers to spare): stride 1 pairs (v[i], v[i+2]) with
-// (v[i+1], v[i+3]); strides >= 2 pair (v[i], v[i+1]) with (v[i+s], v[i+s+1]).
+// PACKED the strides >= 2 run on the packed f32x2 add, pairing (v[i], v[i+1])
+// with (v[i+s], v[i+s+1]) (half the issue slots; the streaming dequantizer has
+// no registers to spare for it); stride 1 stays scalar, which keeps every
+// pair (v[i], v[i+1]) in its register pair between the stages.
 template <int N, bool PACKED = false>
 __device__ __forceinline__ void fwht_reg(float* v) {
     if constexpr (!PACKED) {
@@ -42,13 +42,10 @@ __device__ __forceinline__ void fwht_reg(float* v) {
     }
     const float2 m1 = make_float2(-1.0f, -1.0f);
 #pragma unroll
-    for (int i = 0; i < N; i += 4) {
-        const float2 a = make_float2(v[i], v[i + 2]), b = make_float2(v[i + 1], v[i + 3]);
-        const float2 s = __fadd2_rn(a, b), d = __ffma2_rn(b, m1, a);
-        v[i] = s.x;
-        v[i + 2] = s.y;
-        v[i + 1] = d.x;
-        v[i + 3] = d.y;
+    for (int i = 0; i < N; i += 2) {  // stride 1 in scalar adds: the pairs stay in place
+        const float a = v[i], b = v[i + 1];
+        v[i] = a + b;
+        v[i + 1] = a - b;
     }
 #pragma unroll
     for (int st = 2; st < N; st <<= 1) {
@@ -298,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_warp_kern
     const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint8_t* const ws = smem_raw + warp * kDqWarpSmem + (lane >> 4) * 2048u;  // this lane's row
     const uint32_t r2 = lane >> 4, l = lane & 15;
-    const uint32_t b = l / n2, tau = l % n2, k1 = k1w * tau;
+    const uint32_t b = n2 == 16 ? 0u : l / n2, tau = l % n2, k1 = k1w * tau;
     // unit (row pair rp, 512-column tile ct), ct fastest; 32-bit coordinates
     // (the host keeps rows < 2^31), advanced by the grid stride without division
     const int32_t n_ct = (int32_t)p.n_col_tiles, n_rp = (int32_t)((p.M + 1) / 2);
@@ -317,9 +314,11 @@ __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_warp_kern
     auto in_range = [&](int32_t r, int32_t c) {  // K % 64 == 0: whole 32-column pieces
         return (int64_t)r * 2 + r2 < p.M && (int64_t)c * kTileCols + 32 * l < p.K;
     };
-    // phase-B read offset of sub-row sl within the lane's row (swizzled chunk)
+    // phase-B read offset of sub-row sl = b n2 + k2 within the lane's row
+    // (swizzled chunk); for n2 >= 8, b n2 is a multiple of 8 and the swizzle
+    // depends on k2 alone, a constant of the unrolled loop
     auto rd_off = [&](uint32_t sl, int h) -> uint32_t {
-        const uint32_t z = dq_swz(sl);
+        const uint32_t z = n2 >= 8 ? dq_swz(sl % n2) : dq_swz(sl);
         if constexpr (k1w == 2) return sl * 128u + (((k1 >> 2) ^ z) << 4) + (k1 & 3u) * 4u;
         else return sl * 128u + ((((k1 >> 2) + (uint32_t)h) ^ z) << 4);
     };

@@ -320,9 +320,10 @@ __device__ __forceinline__ uint32_t mxfp4_unit(const float2* n, float fold, uint
     // codes in element order: v[i] = -n[i].x * 2^(127-b), v[16+i] = -n[i].y * ...
     float v[32];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        v[i] = n[i].x * nm;
-        v[16 + i] = n[i].y * nm;
+    for (int i = 0; i < 16; ++i) {  // packed f32x2 multiply: the same RN products
+        const float2 q = __fmul2_rn(n[i], make_float2(nm, nm));
+        v[i] = q.x;
+        v[16 + i] = q.y;
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) w[i] = e2m1_pack8(v + 8 * i);
