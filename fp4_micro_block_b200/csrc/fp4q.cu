@@ -203,9 +203,9 @@ fp4q_status launch_mma_t(const CUtensorMap& map, const MmaParams& p, int grid, c
     static std::atomic<uint64_t> done{0};
     if constexpr (HAD <= kMmaTile) {
         auto kern = had_mma_kernel<FMT, HAD, AMAX>;
-        fp4q_status st = ensure_smem(kern, kMmaSmemBytes, done);
+        fp4q_status st = ensure_smem(kern, MmaGeo<FMT>::smem, done);
         if (st != FP4Q_OK) return st;
-        return launch(kern, grid, kMmaThreads, kMmaSmemBytes, s, map, p);
+        return launch(kern, grid, MmaGeo<FMT>::threads, MmaGeo<FMT>::smem, s, map, p);
     } else {
         auto kern = had_mma_wide_kernel<FMT, HAD, AMAX>;
         constexpr int smem = Wide<HAD>::smem;

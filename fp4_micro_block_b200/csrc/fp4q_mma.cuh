@@ -13,12 +13,14 @@
 // one of the costs of the format.)
 //
 // CTA roles (one persistent CTA per SM):
-//   warp 0     lane 0 streams X tiles by TMA into a ring of kMmaStages stages;
+//   warps 0, 2 lane 0 of each streams alternate X tiles by TMA into a ring of
+//              kMmaStages stages;
 //   warp 1     allocates TMEM; lane 0 issues 8 UMMAs (K = 16 each) per tile
-//              into one of kEpiGroups fp32 accumulators (128 columns each)
+//              into one of G fp32 accumulators (128 columns each; G = 3,
+//              the dual format 2: MmaGeo)
 //              and commits them to the tile's barriers;
-//   warps 2..  kEpiGroups warpgroups of epilogue: warpgroup g takes the CTA's
-//              tiles j = g (mod kEpiGroups); thread = one row of the tile
+//   warps 3..  G warpgroups of epilogue: warpgroup g takes the CTA's
+//              tiles j = g (mod G); thread = one row of the tile
 //              (TMEM lane), reading 32 columns at a time with tcgen05.ld and
 //              quantizing them in registers (two 16-blocks or one 32-block).
 // Every wait is bounded: a wait that runs out sets g_device_error and the role
@@ -40,11 +42,8 @@ namespace fp4q {
 constexpr int kMmaTile = 128;                         // tile rows = tile columns
 constexpr int kMmaStages = FP4Q_MMA_STAGES;           // X ring depth
 constexpr int kEpiGroups = FP4Q_EPI_GROUPS;           // epilogue warpgroups = accumulators
-constexpr int kMmaThreads = 96 + 128 * kEpiGroups;  // 2 producer warps, the MMA warp, epilogue
 constexpr int kTileBytes = kMmaTile * kMmaTile * 2;   // 32 KiB of bf16
 constexpr int kHalfBytes = kTileBytes / 2;            // one TMA box: 64 columns x 128 rows
-constexpr uint32_t kTmemCols = kEpiGroups * kMmaTile <= 256 ? (kEpiGroups * kMmaTile <= 128 ? 128u : 256u) : 512u;
-static_assert(kEpiGroups * kMmaTile <= 512, "accumulators exceed TMEM");
 
 // UMMA instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major,
 // M = 128, N = 128 (fields: D format [4,6), A format [7,10), B format [10,13),
@@ -132,12 +131,24 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 constexpr int kMmaBOff = 0;
 constexpr int kMmaRingOff = kTileBytes;
 constexpr int kMmaBarOff = kMmaRingOff + kMmaStages * kTileBytes;
-constexpr int kMmaNumBars = 2 * kMmaStages + 2 * kEpiGroups + 1;
-constexpr int kMmaSlotOff = kMmaBarOff + kMmaNumBars * 8;
-constexpr int kMmaTabOff = (kMmaSlotOff + 4 + 15) / 16 * 16;
-constexpr int kMmaRedOff = kMmaTabOff + 128 * 16;
-constexpr int kMmaSmemBytes = 1024 + kMmaRedOff + (kMmaThreads / 32) * 4;
-static_assert(kMmaSmemBytes <= 227 * 1024, "shared memory");
+
+// Epilogue warpgroups (= TMEM accumulators), threads and shared-memory layout
+// per format.  The dual format's two passes over a tile (group maximum, then
+// the quantization) need more registers per thread: it runs two epilogue
+// warpgroups, within the register file without spills, instead of three.
+template <int FMT>
+struct MmaGeo {
+    static constexpr int groups = FMT == FMT_DUAL ? 2 : kEpiGroups;
+    static constexpr int threads = 96 + 128 * groups;  // 2 producer warps, the MMA warp, epilogue
+    static constexpr uint32_t tmem_cols = groups * kMmaTile <= 128 ? 128u : groups * kMmaTile <= 256 ? 256u : 512u;
+    static constexpr int num_bars = 2 * kMmaStages + 2 * groups + 1;
+    static constexpr int slot_off = kMmaBarOff + num_bars * 8;
+    static constexpr int tab_off = (slot_off + 4 + 15) / 16 * 16;
+    static constexpr int red_off = tab_off + 128 * 16;
+    static constexpr int smem = 1024 + red_off + (threads / 32) * 4;
+    static_assert(groups * kMmaTile <= 512, "accumulators exceed TMEM");
+    static_assert(smem <= 227 * 1024, "shared memory");
+};
 
 // Output column held by accumulator column j.  Within each 32-column chunk,
 // accumulator columns 2i and 2i+1 hold output columns i and 16 + i, so that a
@@ -224,19 +235,21 @@ __device__ __forceinline__ void store_chunk_pair(uint8_t* mine, int64_t stride, 
 }
 
 template <int FMT, int HAD, bool AMAX_ONLY>
-__global__ void __launch_bounds__(kMmaThreads, 1)
+__global__ void __launch_bounds__(MmaGeo<FMT>::threads, 1)
     had_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, const MmaParams p) {
+    using Geo = MmaGeo<FMT>;
+    constexpr int kGroups = Geo::groups;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     const uint32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kMmaBarOff);
     const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * kMmaStages;
-    const uint32_t accf0 = empty0 + 8 * kMmaStages, acce0 = accf0 + 8 * kEpiGroups;
-    const uint32_t done_bar = acce0 + 8 * kEpiGroups;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kMmaSlotOff);
-    float4* tab = reinterpret_cast<float4*>(smem + kMmaTabOff);
-    float* red = reinterpret_cast<float*>(smem + kMmaRedOff);
+    const uint32_t accf0 = empty0 + 8 * kMmaStages, acce0 = accf0 + 8 * kGroups;
+    const uint32_t done_bar = acce0 + 8 * kGroups;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Geo::slot_off);
+    float4* tab = reinterpret_cast<float4*>(smem + Geo::tab_off);
+    float* red = reinterpret_cast<float*>(smem + Geo::red_off);
     constexpr bool kOddLog = HAD == 32 || HAD == 128;  // RN(1/sqrt(2)) left for the epilogue
 
     if (tid == 0) {
@@ -245,7 +258,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, 1);
         }
-        for (int g = 0; g < kEpiGroups; ++g) {
+        for (int g = 0; g < kGroups; ++g) {
             mbar_init(accf0 + 8 * g, 1);
             mbar_init(acce0 + 8 * g, 4);  // one arrival per epilogue warp
         }
@@ -253,7 +266,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_alloc(smem_u32(tmem_slot), Geo::tmem_cols);
         tmem_relinquish();
     }
     build_hadamard_b<HAD>(smem + kMmaBOff);
@@ -312,10 +325,10 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         if (lane == 0) {
             const uint32_t b_addr = smem_u32(smem + kMmaBOff);
             for (int64_t j = 0; j < n_my; ++j) {
-                const int s = (int)(j % kMmaStages), a = (int)(j % kEpiGroups);
+                const int s = (int)(j % kMmaStages), a = (int)(j % kGroups);
                 bool ok = mbar_wait(full0 + 8 * s, (uint32_t)((j / kMmaStages) & 1));
-                if (ok && j >= kEpiGroups)
-                    ok = mbar_wait(acce0 + 8 * a, (uint32_t)((j / kEpiGroups - 1) & 1));
+                if (ok && j >= kGroups)
+                    ok = mbar_wait(acce0 + 8 * a, (uint32_t)((j / kGroups - 1) & 1));
                 if (!ok) {
                     atomicOr(&g_device_error, kErrWaitTimeout);
                     break;
@@ -345,8 +358,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         const float fold = kOddLog ? __uint_as_float(0x3f3504f3u) : 1.0f;
         const int64_t kc = p.K / 2;
 #pragma unroll 1
-        for (int64_t j = g; j < n_my; j += kEpiGroups) {
-            const bool ok = mbar_wait(accf0 + 8 * g, (uint32_t)((j / kEpiGroups) & 1));
+        for (int64_t j = g; j < n_my; j += kGroups) {
+            const bool ok = mbar_wait(accf0 + 8 * g, (uint32_t)((j / kGroups) & 1));
             if (!__all_sync(0xffffffffu, ok)) {
                 if (lane == 0) atomicOr(&g_device_error, kErrWaitTimeout);
                 break;
@@ -454,13 +467,13 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     if constexpr (AMAX_ONLY) {
         if (tid == 0) {
             float m = 0.0f;
-            for (int w = 0; w < kMmaThreads / 32; ++w) m = fmaxf(m, red[w]);
+            for (int w = 0; w < Geo::threads / 32; ++w) m = fmaxf(m, red[w]);
             p.partials[blockIdx.x] = m;
         }
     }
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc(tmem_base, Geo::tmem_cols);
     }
 }
 
