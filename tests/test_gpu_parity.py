@@ -312,6 +312,32 @@ def test_dequantize_inverse_hadamard_grid_stride(fq, n, fmt):
     assert_roundtrip_close(bf16_torch_to_bits(y)[rows], want, n, name=f"inv-had{n}-{fmt}-grid")
 
 
+@pytest.mark.parametrize("layout", [0, 1])
+def test_empty_inputs(fq, layout):
+    """M = 0 through every entry point: no launch, no error, empty outputs."""
+    K = 1024
+    x = torch.empty((0, K), dtype=torch.bfloat16, device="cuda")
+    c, s, sf = fq.quantize_nvfp4(x, layout=layout)
+    assert c.shape == (0, K // 2) and float(sf.item()) == 0.0
+    c, s, sf = fq.quantize_nvfp4(x, tensor_scale=torch.tensor([0.5], device="cuda"), layout=layout)
+    assert float(sf.item()) == 0.5
+    c, s = fq.quantize_mxfp4(x, layout=layout)
+    assert c.shape == (0, K // 2)
+    for n in (16, 128, 512):
+        for f in (fq.FP4Q_NVFP4, fq.FP4Q_MXFP4, fq.FP4Q_NVFP4_DUAL):
+            c, s, g = fq.hadamard_quantize(x, n, f, layout=layout)
+            y = fq.dequantize(f, c, s, g if f != fq.FP4Q_NVFP4 else torch.ones(1, device="cuda"), K,
+                              layout, n)
+            assert y.shape == (0, K)
+    gamma = torch.ones(K, dtype=torch.bfloat16, device="cuda")
+    perm = torch.arange(K, dtype=torch.int32, device="cuda")
+    outl = torch.arange(64, dtype=torch.int32, device="cuda")
+    c, s, sf = fq.arc_quantize(x, gamma, perm, outl, layout=layout)
+    assert c.shape == (0, (K + 64) // 2)
+    torch.cuda.synchronize()
+    assert fq.fp4q_device_error() == 0
+
+
 # ----------------------------------------------------------------------------- ARC
 
 def arc_case(fq, M, K, S, seed, static=False, layout=0):
