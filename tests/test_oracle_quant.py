@@ -327,3 +327,22 @@ def test_swizzle_tile_structure():
     assert oracle.swizzle_offset(127, 3, n) == 511
     assert oracle.swizzle_offset(0, 4, n) == 512
     assert oracle.swizzle_offset(128, 0, n) == 512 * 4
+
+
+def test_swizzle_matches_the_block_scaled_gemm_library_layout():
+    """The 128x4 tiled scale layout against vLLM's helper that lays out NVFP4
+    block scales for the CUTLASS / FlashInfer block-scaled GEMMs (plain torch
+    reshapes; its final device copy is bypassed on this CPU-only host)."""
+    from unittest import mock
+
+    torch = pytest.importorskip("torch")
+    try:
+        from vllm.model_executor.layers.quantization.utils.nvfp4_utils import swizzle_blockscale
+    except Exception as e:  # not importable here
+        pytest.skip(f"vllm helper unavailable: {type(e).__name__}")
+    with mock.patch.object(torch.Tensor, "cuda", lambda self, *a, **k: self):
+        for M, n in [(1, 1), (128, 4), (130, 9), (300, 64), (256, 272)]:
+            lin = np.random.default_rng(M + n).integers(1, 127, (M, n), dtype=np.uint8)
+            ref = swizzle_blockscale(torch.from_numpy(lin).view(torch.float8_e4m3fn))
+            want = ref.contiguous().view(torch.uint8).numpy().reshape(-1)
+            assert np.array_equal(oracle.swizzle_scales(lin), want), (M, n)
