@@ -382,20 +382,35 @@ static __device__ __align__(256) float g_noalloc_partials[kNoAllocPartials];
 namespace {
 std::atomic<float*> g_noalloc_ptr[kMaxDevices];
 
-// Device address of the scratch on the current device, looked up once per device.
-fp4q_status noalloc_scratch(float** out) {
+// Device address of the scratch on the current device.  Outside stream capture
+// it is looked up on every call (so a context re-created after
+// cudaDeviceReset gets its own address) and cached; while `stream` is
+// capturing, the cached address of the last uncaptured call is used.
+fp4q_status noalloc_scratch(cudaStream_t stream, float** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FP4Q_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return FP4Q_ERR_UNSUPPORTED;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return FP4Q_ERR_CUDA;
     float* ptr = g_noalloc_ptr[dev].load(std::memory_order_acquire);
-    if (!ptr) {
+    if (cap == cudaStreamCaptureStatusNone) {
         void* a = nullptr;
         if (cudaGetSymbolAddress(&a, g_noalloc_partials) != cudaSuccess || !a) return FP4Q_ERR_CUDA;
         ptr = static_cast<float*>(a);
         g_noalloc_ptr[dev].store(ptr, std::memory_order_release);
     }
+    if (!ptr) return FP4Q_ERR_CUDA;  // first call made under capture: no address yet
     *out = ptr;
     return FP4Q_OK;
+}
+
+// CTAs of the amax pre-pass that fp4q_quantize_nvfp4 launches in DYNAMIC mode
+// (one partial maximum each): the register quantizer's grid for NVFP4 without
+// rotation, min(tiles, CTAs per SM x SMs, kMaxGrid).
+int64_t nvfp4_prepass_grid(int64_t M, int64_t K, int sms) {
+    using G = QGeo<FMT_NVFP4, 0>;
+    const int64_t tiles = (M + kQBoxRows - 1) / kQBoxRows * ((K + G::tc - 1) / G::tc);
+    return std::min<int64_t>({tiles, (int64_t)kQCtas * sms, (int64_t)kMaxGrid});
 }
 }  // namespace
 
@@ -430,14 +445,13 @@ FP4Q_API fp4q_status fp4q_quantize_nvfp4_noalloc(const void* x, int64_t M, int64
     fp4q_status st = check_x(x, M, K, ldx);
     if (st != FP4Q_OK) return st;
     if (K % 16 != 0) return FP4Q_ERR_INVALID_ARG;
+    if (layout != FP4Q_SCALES_LINEAR && layout != FP4Q_SCALES_SWIZZLED) return FP4Q_ERR_INVALID_ARG;
     if (M == 0) return FP4Q_OK;
-    // One partial maximum per pre-pass CTA: the pre-pass runs one CTA per SM
-    // and never more than kMaxGrid, so this only trips if that cap is ever raised.
     int sms = 0;
     if ((st = sm_count(&sms)) != FP4Q_OK) return st;
-    if (std::min(sms, kMaxGrid) > kNoAllocPartials) return FP4Q_ERR_UNSUPPORTED;
+    if (nvfp4_prepass_grid(M, K, sms) > kNoAllocPartials) return FP4Q_ERR_UNSUPPORTED;
     float* scratch = nullptr;
-    if ((st = noalloc_scratch(&scratch)) != FP4Q_OK) return st;
+    if ((st = noalloc_scratch((cudaStream_t)stream, &scratch)) != FP4Q_OK) return st;
     return quantize_common(x, M, K, ldx, 0, FMT_NVFP4, codes, scales, tensor_scale,
                            FP4Q_TSCALE_DYNAMIC, layout, scratch,
                            (size_t)kNoAllocPartials * sizeof(float), (cudaStream_t)stream);

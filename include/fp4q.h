@@ -128,12 +128,17 @@ fp4q_status fp4q_quantize_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx
  * allocating routine.  (Not a method of the pages: they have no counterpart.)
  *   Arguments and results are those of fp4q_quantize_nvfp4 with
  *   mode = FP4Q_TSCALE_DYNAMIC: *tensor_scale is written.
- *   Limit: at most 4096 partial maxima; the pre-pass grid never exceeds 4096
- *   CTAs, so every M and K accepted by fp4q_quantize_nvfp4 fits, and a grid
- *   above the limit would return FP4Q_ERR_UNSUPPORTED.
- *   Set-up: the first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   Limit: at most 4096 partial maxima, one per CTA of the amax pre-pass,
+ *   whose grid is min(row tiles x column tiles, CTAs per SM x SMs, 4096); so
+ *   every M and K accepted by fp4q_quantize_nvfp4 fits, and a grid above the
+ *   limit would return FP4Q_ERR_UNSUPPORTED before anything is launched.
+ *   Set-up: a call looks up the array's device address (cudaGetSymbolAddress)
+ *   on the current device whenever `stream` is not capturing, and caches it;
+ *   a call on a capturing stream uses the address cached by the last
+ *   uncaptured call on that device.  So make the first call on a device
+ *   before any stream capture, and, after cudaDeviceReset (which re-creates
+ *   the context and so the array), make one uncaptured call before capturing
+ *   again; a first call under capture returns FP4Q_ERR_CUDA.
  *   Sharing: every call on a device uses the same array, which keeps the last
  *   call's contents.  Nothing in it needs clearing (each call's pre-pass writes
  *   every entry its quantizer reads), but calls that overlap on the GPU (for

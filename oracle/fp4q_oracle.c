@@ -27,7 +27,7 @@
  *     (ARCQuant, "Methodologie" items 1, 2, 3 and 5).
  *
  * Numeric rules (where the pages only name the formats, these are the plain
- * readings; every one is listed in the design doc):
+ * readings of them, each taken where the pages leave the step open):
  *   E2M1   : magnitudes {0,.5,1,1.5,2,3,4,6}; nearest value, ties to the even
  *            code (mantissa bit 0), |v| > 6 saturates to 6, sign always kept
  *            (a negative value that rounds to zero is code 0x8).

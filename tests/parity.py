@@ -75,22 +75,18 @@ def assert_bitexact(name: str, got: np.ndarray, want: np.ndarray):
                              f"got {got[idx]!r} want {want[idx]!r}")
 
 
-def assert_tolerant(fmt: str, K: int, gpu, orc, y_orc: np.ndarray, *, frac: float = 1e-4,
-                    name: str = ""):
-    """gpu/orc = (codes, scales_linear, scale_fp32).  y_orc: oracle's unquantized fp32."""
+def tolerant_counts(fmt: str, K: int, gpu, orc, y_orc: np.ndarray, name: str = "") -> dict:
+    """Element-wise part of the tolerance rule; returns the counts that the
+    fraction limits apply to.  gpu/orc = (codes, scales_linear, scale_fp32);
+    y_orc: the oracle's unquantized fp32 values."""
     cg, sg, fg = gpu
     co, so, fo = orc
     dg = block_scale(fmt, sg, fg, K)
     do = block_scale(fmt, so, fo, K)
     vg = code_values(cg) * dg
     vo = code_values(co) * do
-    n = vg.size
-    allow = max(1, math.ceil(frac * n))
     scale_diff = np.repeat(sg != so, 16 if fmt != "mxfp4" else 32, axis=1)[:, :K]
-    n_blocks = sg.size
     n_blocks_diff = int((sg != so).sum())
-    assert n_blocks_diff <= max(1, math.ceil(frac * n_blocks)), (
-        f"{name}: {n_blocks_diff} of {n_blocks} scale bytes differ")
     if n_blocks_diff:
         diff_bytes = np.abs(sg.astype(np.int64) - so.astype(np.int64))[sg != so]
         assert np.all(diff_bytes <= 1), f"{name}: scale bytes differ by more than one step"
@@ -98,7 +94,6 @@ def assert_tolerant(fmt: str, K: int, gpu, orc, y_orc: np.ndarray, *, frac: floa
     # elements of same-scale blocks that disagree: must be one grid step apart
     bad = ~close & ~scale_diff
     nbad = int(bad.sum())
-    assert nbad <= allow, f"{name}: {nbad} of {n} codes differ (allowed {allow})"
     if nbad:
         ug = oracle.unpack_codes(cg)[bad]
         uo = oracle.unpack_codes(co)[bad]
@@ -114,33 +109,115 @@ def assert_tolerant(fmt: str, K: int, gpu, orc, y_orc: np.ndarray, *, frac: floa
         err = np.abs(vg[scale_diff] - y)
         bound = np.where(v > 6, (v - 6 + 1e-3) * dg[scale_diff], (step / 2 + 1e-3) * dg[scale_diff])
         assert np.all(err <= bound * (1 + 1e-6)), f"{name}: error bound violated in rescaled blocks"
-    return {"codes_off": nbad, "blocks_rescaled": n_blocks_diff, "n": n}
+    return {"codes_off": nbad, "blocks_rescaled": n_blocks_diff, "n": int(vg.size),
+            "n_blocks": int(sg.size)}
 
 
-def assert_roundtrip_close(got_bits: np.ndarray, want_bits: np.ndarray, n: int, name: str = "",
-                           max_frac: float = 3e-2):
-    """bf16 outputs of an inverse-Hadamard dequantizer against the oracle's.
+def check_fractions(c: dict, frac: float = 1e-4, name: str = "") -> dict:
+    """The fraction limits of the tolerance rule on (summed) counts."""
+    allow = max(1, math.ceil(frac * c["n"]))
+    assert c["blocks_rescaled"] <= max(1, math.ceil(frac * c["n_blocks"])), (
+        f"{name}: {c['blocks_rescaled']} of {c['n_blocks']} scale bytes differ")
+    assert c["codes_off"] <= allow, f"{name}: {c['codes_off']} of {c['n']} codes differ (allowed {allow})"
+    return c
 
-    The GPU rotates in fp32 butterflies, the oracle in binary64 rounded once;
-    the difference before the final bf16 rounding is a few fp32 ulps of the
-    Hadamard block's magnitude.  So each element may differ by one bf16 ulp of
-    itself (a rounding flip) plus 2^-18 of the block's largest magnitude (a
-    cancelled, near-zero element), and at most `max_frac` of them may differ.
-    The dequantized inputs carry only a few significant bits, so binary64 sums
-    are often exact where fp32 butterflies are not, and single-ulp bf16 flips
-    are far more frequent than for random data: about 1.3% of the outputs for
-    n = 16 when the fp32 butterflies are replayed on the host in numpy.  The
-    element-wise one-ulp bound is the check that catches a wrong sign, index
-    or scale."""
+
+def assert_tolerant(fmt: str, K: int, gpu, orc, y_orc: np.ndarray, *, frac: float = 1e-4,
+                    name: str = ""):
+    """gpu/orc = (codes, scales_linear, scale_fp32).  y_orc: oracle's unquantized fp32."""
+    return check_fractions(tolerant_counts(fmt, K, gpu, orc, y_orc, name), frac, name)
+
+
+def add_counts(a: dict | None, b: dict) -> dict:
+    return dict(b) if a is None else {k: a[k] + b[k] for k in a}
+
+
+def _bf16_boundary_distance(w: np.ndarray) -> np.ndarray:
+    """Distance (float64) from each fp32 value to the nearest bf16 rounding
+    boundary: the midpoints between |w|'s two bf16 neighbours and between the
+    lower neighbour and the bf16 value below it."""
+    a = np.abs(np.asarray(w, np.float32))
+    u = a.view(np.uint32)
+    lo_b = u & np.uint32(0xFFFF0000)
+    lo = lo_b.view(np.float32).astype(np.float64)
+    hi = (lo_b + np.uint32(0x10000)).view(np.float32).astype(np.float64)
+    below = np.where(lo_b > 0, lo_b - np.uint32(0x10000), np.uint32(0)).view(np.float32).astype(np.float64)
+    below = np.where(lo_b > 0, below, -lo)
+    a64 = a.astype(np.float64)
+    return np.minimum(np.abs((lo + hi) / 2 - a64), a64 - (below + lo) / 2)
+
+
+def assert_roundtrip(got_bits: np.ndarray, want_f32: np.ndarray, n: int, name: str = "") -> dict:
+    """bf16 output of an inverse-Hadamard dequantizer against the oracle.
+
+    `want_f32` is the oracle's value w: the binary64 product H_n * dq rounded
+    once to fp32.  The kernels compute the same product in fp32 (one rounding
+    of the folded multiplier at decode, then log2(n) butterfly stages).  Each
+    rounding adds an error of at most 2^-24 of the value it rounds; an
+    unnormalised butterfly stage multiplies the l2 norm of an error vector by
+    sqrt(2), so the errors of all stages, carried to the output, stay below
+    (log2(n) + 6) * 2^-24 * ||w_block||_2 in every element (3 decode roundings
+    and a margin of 3).  With the 2^-24 |w| of the oracle's own fp32 rounding
+    this is the window delta.  Consequences checked here:
+      * an element whose w lies farther than delta from every bf16 rounding
+        boundary is BIT-EXACT (both sides round the same value the same way);
+      * inside the window the two results may be the two bf16 neighbours of
+        the boundary: |got - w| <= one bf16 ulp + delta.
+    The dequantized inputs carry few significant bits, so many outputs are
+    exact bf16 midpoints (ties the oracle rounds to even, the kernel sees a
+    few fp32 ulps to one side): this window holds about 1-3 % of the elements,
+    and it is the only place a difference is allowed."""
     got = oracle.bf16_to_f32(got_bits).astype(np.float64)
-    want = oracle.bf16_to_f32(want_bits).astype(np.float64)
-    M, K = want.shape
-    blk = np.abs(want).reshape(M, K // n, n).max(axis=2)
-    blk = np.repeat(blk, n, axis=1)
-    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(want), np.abs(got)) + 1e-300)) - 7)
-    diff = np.abs(got - want)
-    bound = ulp + 2.0 ** -18 * blk
-    bad = diff > bound
-    assert not bad.any(), (f"{name}: {int(bad.sum())} elements beyond one bf16 ulp; first "
-                           f"{np.argwhere(bad)[0]}: got {got[bad][0]} want {want[bad][0]}")
-    assert (diff > 0).mean() <= max_frac, f"{name}: {(diff > 0).mean():.2e} of elements differ"
+    w = np.asarray(want_f32, np.float32)
+    want_bits = oracle.f32_to_bf16(w)
+    M, K = w.shape
+    w64 = w.astype(np.float64)
+    L = int(round(math.log2(n)))
+    blk = np.sqrt(np.square(w64).reshape(M, K // n, n).sum(axis=2))
+    delta = (L + 6) * 2.0 ** -24 * np.repeat(blk, n, axis=1) + 2.0 ** -24 * np.abs(w64)
+    window = _bf16_boundary_distance(w) <= delta
+    g_bits = np.asarray(got_bits, np.uint16)
+    outside_bad = (g_bits != want_bits) & ~window
+    assert not outside_bad.any(), (
+        f"{name}: {int(outside_bad.sum())} elements outside the rounding window differ; first "
+        f"{np.argwhere(outside_bad)[0]}: got {got[outside_bad][0]} want "
+        f"{oracle.bf16_to_f32(want_bits)[outside_bad][0]}")
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(w64), np.abs(got)) + 1e-300)) - 7)
+    inside_bad = window & (np.abs(got - w64) > ulp + delta)
+    assert not inside_bad.any(), (f"{name}: {int(inside_bad.sum())} window elements beyond one "
+                                  f"bf16 ulp + delta")
+    return {"window": int(window.sum()), "differ": int((g_bits != want_bits).sum()), "n": w.size}
+
+
+def block_l2_identity(x_bits, xhat_bits, dq_y, y_orc, w_orc, n: int, name: str = ""):
+    """Per n-block l2 identity of the round trip (orthonormal H):
+    ||x^ - x||_2 = ||y^ - y||_2 with x the bf16 input, y = H x its rotation
+    (oracle, fp32), y^ the dequantized codes and x^ = H y^.
+      * w_orc = oracle's H y^ (fp32): equal to ||y^ - y|| within 1e-5 relative
+        (plus the fp32 roundings of y and w, 2^-23 ||x_block||);
+      * the kernel's bf16 x^: within the a-priori bound of its bf16 rounding
+        and fp32 error, ||1/2 ulp_bf16(w) + delta||_2 of the block, which does
+        not depend on the kernel's output."""
+    x = oracle.bf16_to_f32(x_bits).astype(np.float64)
+    M, K = x.shape
+    nb = K // n
+    blocks = lambda a: np.asarray(a, np.float64).reshape(M, nb, n)
+    e_y = np.sqrt(np.square(blocks(dq_y) - blocks(y_orc)).sum(axis=2))
+    e_w = np.sqrt(np.square(blocks(w_orc) - blocks(x)).sum(axis=2))
+    nx = np.sqrt(np.square(blocks(x)).sum(axis=2))
+    tol_w = 1e-5 * e_y + 2.0 ** -23 * nx
+    assert np.all(np.abs(e_w - e_y) <= tol_w), (
+        f"{name}: oracle inverse breaks the l2 identity, worst "
+        f"{np.max(np.abs(e_w - e_y) - tol_w)}")
+    xh = oracle.bf16_to_f32(xhat_bits).astype(np.float64)
+    e_g = np.sqrt(np.square(blocks(xh) - blocks(x)).sum(axis=2))
+    w64 = blocks(w_orc)
+    L = int(round(math.log2(n)))
+    wn = np.sqrt(np.square(w64).sum(axis=2))
+    half_ulp = np.exp2(np.floor(np.log2(np.abs(w64) + 1e-300)) - 8)
+    per = half_ulp + (L + 6) * 2.0 ** -24 * wn[..., None] + 2.0 ** -24 * np.abs(w64)
+    bound = np.sqrt(np.square(per).sum(axis=2)) + tol_w
+    assert np.all(np.abs(e_g - e_y) <= bound), (
+        f"{name}: kernel round trip breaks the l2 identity, worst excess "
+        f"{np.max(np.abs(e_g - e_y) - bound)}")
+    return {"rel_err_median": float(np.median(e_y / np.maximum(nx, 1e-300)))}

@@ -288,9 +288,14 @@ def test_arc_residual_layout_and_linearity():
     prim, res = dq[:, :K], dq[:, K:]
     yo = y.astype(np.float64)[:, outl]
     r_true = yo - prim[:, outl]
-    # residual codes approximate the primary error of the outlier channels
+    # residual codes approximate the primary error of the outlier channels to
+    # round-to-nearest accuracy: half a grid step times the residual block's
+    # scale d (saturated elements: (|v| - 6) d), plus the binary32 rounding of
+    # the residual itself (2^-24 |r|)
     d_res = np.repeat(lib_decode_e4m3(scales[:, K // 16:]), 16, axis=1) * float(s_t)
-    assert np.all(np.abs(r_true - res) <= d_res * 0.5 * 2 + 1e-12)
+    v = np.abs(r_true) / d_res
+    bound = np.where(v > 6, v - 6, grid_step(v) / 2) * d_res
+    assert np.all(np.abs(r_true - res) <= bound * (1 + 1e-6) + 2.0 ** -24 * np.abs(r_true))
     # two-stage error is below the primary error on the outliers (on aggregate)
     assert np.linalg.norm(yo - prim[:, outl] - res) < 0.5 * np.linalg.norm(yo - prim[:, outl])
     # linearity of the augmented GEMM: [Q(x) | Q(r)] @ [W ; W_S] equals (Q(x) + Q(r) on S) @ W
@@ -301,6 +306,47 @@ def test_arc_residual_layout_and_linearity():
     corrected[:, outl] += res
     np.testing.assert_allclose(dq @ W_aug, corrected @ W, rtol=1e-12, atol=1e-12)
 
+
+
+def test_arc_residual_half_by_brute_force():
+    """The residual columns are the NVFP4 quantization, with the primary's s_t,
+    of r = fl32(y - dq) on the outlier positions (ARCQuant, Methodologie item 2:
+    residual = original - primary), found here by exhaustive search with exact
+    rationals: the scale byte nearest (ties even) to (amax_r / 6) / s_t, then
+    each code nearest (ties to the even code, sign kept) to fl32(r / d)."""
+    M, K, S = 6, 128, 32
+    x, gamma, perm, outl = workloads.arc_activations(M, K, seed=35, S=S, calib_rows=64)
+    codes, scales, s_t, y = oracle.arc(x, gamma, perm, outl)
+    s_t = np.float32(s_t)
+    prod = (lib_decode_codes(codes[:, : K // 2]) *
+            np.repeat(lib_decode_e4m3(scales[:, : K // 16]), 16, axis=1)).astype(np.float32)
+    dq = prod * s_t  # binary32 product (the first one is exact)
+    r = (y[:, outl] - dq[:, outl]).astype(np.float32)
+    e4_vals = [Fraction(float(v)) for v in lib_decode_e4m3(np.arange(127))]
+    grid = {c: Fraction(float(v))
+            for c, v in enumerate(np.arange(16, dtype=np.uint8).view(F4).astype(np.float64))}
+    u = oracle.unpack_codes(codes[:, K // 2:])
+    for row in range(M):
+        for b in range(S // 16):
+            blk = r[row, 16 * b:16 * b + 16]
+            ratio = (np.float32(np.abs(blk).max()) / np.float32(6.0)) / s_t
+            ds = [abs(Fraction(float(ratio)) - v) for v in e4_vals]
+            best = min(ds)
+            want = [i for i, dv in enumerate(ds) if dv == best]
+            want = [i for i in want if i % 2 == 0] or want
+            assert int(scales[row, K // 16 + b]) == want[0]
+            d = np.float32(lib_decode_e4m3(np.uint8(want[0])) * s_t)
+            for k in range(16):
+                q32 = np.float32(blk[k]) / d if d > 0 else np.float32(0)
+                q = Fraction(float(q32))
+                neg = bool(np.signbit(q32))
+                cands = sorted((abs(q - grid[c]), c) for c in range(16) if bool(c & 8) == neg)
+                best_c = [c for dv, c in cands if dv == cands[0][0]]
+                best_c = [c for c in best_c if c % 2 == 0] or best_c
+                if d == 0:
+                    assert u[row, 16 * b + k] == 0
+                else:
+                    assert u[row, 16 * b + k] == best_c[0], (row, b, k)
 
 # ----------------------------------------------------------------------------- swizzle
 

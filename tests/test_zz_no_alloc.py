@@ -80,3 +80,8 @@ def test_no_alloc_rejects_bad_arguments_without_launching(fq):
                                          None) == fq.FP4Q_ERR_ALIGNMENT
     assert L.fp4q_quantize_nvfp4_noalloc(0x10000, 0, 64, 64, None, None, None, 0,
                                          None) == fq.FP4Q_OK
+    # an invalid layout is rejected before the M == 0 no-op, as in fp4q_quantize_nvfp4
+    assert L.fp4q_quantize_nvfp4_noalloc(0x10000, 0, 64, 64, None, None, None, 7,
+                                         None) == fq.FP4Q_ERR_INVALID_ARG
+    assert L.fp4q_quantize_nvfp4(0x10000, 0, 64, 64, None, None, None, fq.FP4Q_TSCALE_DYNAMIC, 7,
+                                 None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
