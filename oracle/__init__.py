@@ -53,6 +53,7 @@ def lib() -> C.CDLL:
             "orc_hadamard": (None, [p, i64, i64, i64, C.c_int, p]),
             "orc_rmsnorm_permute": (None, [p, i64, i64, i64, p, p, f64, p]),
             "orc_arc_quantize": (None, [p, i64, i64, i64, p, f32, p, p]),
+            "orc_arc_quantize_mxfp4": (None, [p, i64, i64, i64, p, p, p]),
             "orc_e2m1_encode_array": (None, [p, i64, p]),
             "orc_e4m3_encode_array": (None, [p, i64, p]),
             "orc_e4m3_decode_array": (None, [p, i64, p]),
@@ -257,16 +258,25 @@ def rmsnorm_permute(x: np.ndarray, gamma: np.ndarray, perm, eps: float) -> np.nd
     return y
 
 
-def arc_quantize(y: np.ndarray, outliers, s_t: float):
+def arc_quantize(y: np.ndarray, outliers, s_t: float | None, fmt: str = "nvfp4"):
+    """Primary + residual quantization of the prepared matrix y; NVFP4 (block
+    16, tensor scale s_t) or MXFP4 (block 32, s_t unused)."""
     y = _f32(y)
     M, K = y.shape
     o = np.ascontiguousarray(outliers, np.int32)
     S = o.size
-    assert K % 16 == 0 and S % 16 == 0
+    B = 16 if fmt == "nvfp4" else 32
+    assert K % B == 0 and S % B == 0
     codes = np.empty((M, (K + S) // 2), np.uint8)
-    scales = np.empty((M, (K + S) // 16), np.uint8)
-    lib().orc_arc_quantize(_ptr(y), M, K, S, _ptr(o) if S else None, float(s_t), _ptr(codes),
-                           _ptr(scales))
+    scales = np.empty((M, (K + S) // B), np.uint8)
+    if fmt == "nvfp4":
+        lib().orc_arc_quantize(_ptr(y), M, K, S, _ptr(o) if S else None, float(s_t), _ptr(codes),
+                               _ptr(scales))
+    elif fmt == "mxfp4":
+        lib().orc_arc_quantize_mxfp4(_ptr(y), M, K, S, _ptr(o) if S else None, _ptr(codes),
+                                     _ptr(scales))
+    else:
+        raise ValueError(fmt)
     return codes, scales
 
 
@@ -309,8 +319,14 @@ def arc_prepare(x_bits, gamma_bits, perm, eps: float = 1e-6) -> np.ndarray:
     return rmsnorm_permute(bf16_to_f32(x_bits), bf16_to_f32(gamma_bits), perm, eps)
 
 
-def arc(x_bits, gamma_bits, perm, outliers, eps: float = 1e-6, s_t: float | None = None):
+def arc(x_bits, gamma_bits, perm, outliers, eps: float = 1e-6, s_t: float | None = None,
+        fmt: str = "nvfp4"):
+    """ARCQuant path: reorder + RMSNorm, primary + residual quantization.
+    Returns (codes, scales, s_t (NVFP4) or None (MXFP4), y)."""
     y = arc_prepare(x_bits, gamma_bits, perm, eps)
+    if fmt == "mxfp4":
+        c, s = arc_quantize(y, outliers, None, "mxfp4")
+        return c, s, None, y
     if s_t is None:
         s_t = tensor_scale(amax(y))
     c, s = arc_quantize(y, outliers, s_t)

@@ -434,6 +434,36 @@ ORC_EXPORT void orc_arc_quantize(const float* y, int64_t M, int64_t K, int64_t S
 /* Array forms of the scalar encoders (for the Python binding)                */
 /* ------------------------------------------------------------------------ */
 
+/* ARCQuant two-stage path in MXFP4 (ARCQuant summary, "Generalisabilite": the
+ * residual scheme carries over to MXFP4; MR-GPTQ abstract: MXFP4's 32-element
+ * blocks with a power-of-two scale).  Primary: MXFP4 of every row of y.
+ * Residual of outlier position p: r = y[p] - E2M1val(code) * 2^(b - 127), b the
+ * primary scale byte of p's block (the product is exact; the difference is one
+ * binary32 rounding).  The S residuals are quantized in 32-blocks with their
+ * own E8M0 scales and appended along K: codes [M, (K+S)/2], scales
+ * [M, (K+S)/32]. */
+ORC_EXPORT void orc_arc_quantize_mxfp4(const float* y, int64_t M, int64_t K, int64_t S,
+                                       const int32_t* outliers, uint8_t* codes,
+                                       uint8_t* scales) {
+    int64_t KS = K + S;
+    float* res = (float*)malloc(sizeof(float) * (size_t)(S > 0 ? S : 1));
+    for (int64_t r = 0; r < M; ++r) {
+        const float* yr = y + r * K;
+        uint8_t* cr = codes + r * (KS / 2);
+        uint8_t* sr = scales + r * (KS / 32);
+        orc_mxfp4_quantize(yr, 1, K, K, cr, sr);
+        for (int64_t j = 0; j < S; ++j) {
+            int64_t p = outliers[j];
+            uint8_t byte = cr[p / 2];
+            uint8_t c = (p & 1) ? (byte >> 4) : (byte & 15);
+            float dq = orc_e2m1_decode(c) * orc_e8m0_decode(sr[p / 32]);
+            res[j] = yr[p] - dq;
+        }
+        if (S > 0) orc_mxfp4_quantize(res, 1, S, S, cr + K / 2, sr + K / 32);
+    }
+    free(res);
+}
+
 ORC_EXPORT void orc_e2m1_encode_array(const float* v, int64_t n, uint8_t* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = orc_e2m1_encode(v[i]);
 }

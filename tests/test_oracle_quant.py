@@ -348,6 +348,74 @@ def test_arc_residual_half_by_brute_force():
                 else:
                     assert u[row, 16 * b + k] == best_c[0], (row, b, k)
 
+
+def _floor_log2_exact(a: float) -> int:
+    """floor(log2 a) for a > 0 by exact rational comparison."""
+    fa = Fraction(a)
+    e = 0
+    while Fraction(2) ** e > fa:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= fa:
+        e += 1
+    return e
+
+
+def test_arc_mxfp4_two_stage_by_brute_force():
+    """MXFP4 variant of the two-stage path (ARCQuant summary, Generalisabilite:
+    the scheme carries over to MXFP4; MR-GPTQ abstract: 32-element blocks with a
+    power-of-two scale).  Primary half: MXFP4 of y.  Residual half: MXFP4 of
+    r = fl32(y - dq) on the outlier positions, dq = E2M1val * 2^(b-127) decoded
+    with ml_dtypes; the residual scale byte is floor(log2 amax_r) - 2 + 127 by
+    exact rational search, each code the nearest grid value (ties to the even
+    code, sign kept) of r * 2^(127-b), which is exact."""
+    M, K, S = 6, 256, 64
+    x, gamma, perm, outl = workloads.arc_activations(M, K, seed=36, S=S, calib_rows=64)
+    codes, scales, s_t, y = oracle.arc(x, gamma, perm, outl, fmt="mxfp4")
+    assert s_t is None and codes.shape == (M, (K + S) // 2) and scales.shape == (M, (K + S) // 32)
+    c1, s1 = oracle.mxfp4_quantize(y)
+    np.testing.assert_array_equal(codes[:, : K // 2], c1)
+    np.testing.assert_array_equal(scales[:, : K // 32], s1)
+    dq = lib_decode_codes(codes[:, : K // 2]) * np.exp2(
+        np.repeat(scales[:, : K // 32].astype(np.float64), 32, axis=1) - 127)
+    assert np.array_equal(dq.astype(np.float32).astype(np.float64), dq)  # exact in binary32
+    r = (y[:, outl] - dq[:, outl].astype(np.float32)).astype(np.float32)
+    grid = {c: Fraction(float(v))
+            for c, v in enumerate(np.arange(16, dtype=np.uint8).view(F4).astype(np.float64))}
+    u = oracle.unpack_codes(codes[:, K // 2:])
+    for row in range(M):
+        for b in range(S // 32):
+            blk = r[row, 32 * b:32 * b + 32]
+            am = float(np.abs(blk).max())
+            want_b = 0 if am == 0 else min(254, max(0, _floor_log2_exact(am) - 2 + 127))
+            assert int(scales[row, K // 32 + b]) == want_b
+            for k in range(32):
+                if am == 0:
+                    assert u[row, 32 * b + k] == 0
+                    continue
+                v = Fraction(float(blk[k])) * Fraction(2) ** (127 - want_b)
+                neg = bool(np.signbit(blk[k]))
+                cands = sorted((abs(abs(v) - grid[c & 7]), c) for c in range(16)
+                               if bool(c & 8) == neg)
+                best = [c for dv, c in cands if dv == cands[0][0]]
+                best = [c for c in best if c % 2 == 0] or best
+                assert u[row, 32 * b + k] == best[0], (row, b, k)
+    # error bound of the residual stage, and the two stages beat one on the outliers
+    res = lib_decode_codes(codes[:, K // 2:]) * np.exp2(
+        np.repeat(scales[:, K // 32:].astype(np.float64), 32, axis=1) - 127)
+    d = np.exp2(np.repeat(scales[:, K // 32:].astype(np.float64), 32, axis=1) - 127)
+    v = np.abs(r.astype(np.float64)) / d
+    bound = np.where(v > 6, v - 6, grid_step(v) / 2) * d
+    assert np.all(np.abs(r - res) <= bound * (1 + 1e-9))
+    yo = y.astype(np.float64)[:, outl]
+    assert np.linalg.norm(yo - dq[:, outl] - res) < 0.5 * np.linalg.norm(yo - dq[:, outl])
+    # linearity of the augmented GEMM with the MXFP4 operand
+    W = np.random.default_rng(37).standard_normal((K, 5))
+    full = np.concatenate([dq, res], axis=1)
+    corrected = dq.copy()
+    corrected[:, outl] += res
+    np.testing.assert_allclose(full @ np.concatenate([W, W[outl]], axis=0), corrected @ W,
+                               rtol=1e-12, atol=1e-12)
+
 # ----------------------------------------------------------------------------- swizzle
 
 def test_swizzle_is_a_bijection_with_zero_padding():
