@@ -2,27 +2,34 @@
 """Throughput of the micro-block FP4 quantizer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME]
+                    [--workload NAME] [--units U]
 
-One step = one pass of the path over one batch.  The default workload is the
-MXFP4 round trip on a bf16 4096 x 4096 matrix of 0.5*Student-t(3) activations:
-quantize (block 32, E8M0 scale, E2M1 codes) then dequantize back to bf16.
-Other workloads (``--workload``) time the remaining paths at their full sizes.
+The default workload is the largest one: the dual-scale round trip on a bf16
+32768 x 4096 tensor (N(0,1) x LogNormal(0,1) per-token gain): block-Hadamard
+rotation of size 512, per-128 FP32 group scale + per-16 E4M3 micro-scale,
+E2M1 codes packed, then dequantize + inverse FWHT-512 back to bf16.  Other
+workloads (``--workload``) time the remaining paths at their full sizes.
 
-Metric: input GB/s = bf16 input bytes per step x steps / device time of the
-K timed steps (CUDA events, max over ranks); inputs resident in HBM.  Inputs
-and outputs rotate over enough buffer sets to exceed 4x the L2 cache, so no
-step reads data a previous step left in L2.  Under torchrun every rank
-quantizes its own batch (weak scaling; the path has no exchange step).
+One step = U batches of the workload, each a full-size tensor, in phases: the
+first kernel of the path over all U batches back to back, then the next kernel
+over all U batches.  CUDA events at the phase boundaries give each kernel's
+duration as a back-to-back loop of that kernel alone, inside the timed region;
+U is sized so that one step is a few milliseconds.  The batches rotate over R
+resident buffer sets whose total exceeds 4x the L2 cache, so no launch reads
+data an earlier launch left in L2.
+
+Metric: input GB/s = bf16 input bytes x U x steps / device time of the K timed
+steps (CUDA events, max over ranks), inputs resident in HBM.  Under torchrun
+every rank quantizes its own batches (weak scaling; the path has no exchange
+step).
 
 The JSON line adds: the roofline of the dominant kernel (algorithmic bytes per
-launch / its duration in the timed loop: the step time times its share of the
-CUDA-event-bracketed launch times, taken on every 8th timed step,
-against the measured HBM copy bandwidth), an end-to-end figure through the
-public API with host buffers (pinned host -> device copy of the input, both
-calls, device -> host copy of the outputs, all inside the timed region), the
-SM clocks sampled during the timed region, and the CPU oracle timed on the
-host as a baseline (rank 0, N = 1).
+launch / its mean back-to-back duration in the timed steps, against the
+measured HBM copy bandwidth), every kernel's mean duration, an end-to-end
+figure through the public API with host buffers (pinned host -> device copy of
+one batch, the path, device -> host copy of its outputs, all inside the timed
+region), the SM clocks sampled during the timed region, and the CPU oracle
+timed on the host as a baseline (rank 0, N = 1).
 """
 from __future__ import annotations
 
@@ -46,15 +53,25 @@ import workloads  # noqa: E402
 MIB = 1 << 20
 L2_BYTES = 126 * 10**6
 METRIC = "input GB/s quantized to NVFP4/MXFP4 on 1 B200; % of HBM roofline"
-EV_EVERY = 8  # timed steps between two steps whose kernels are bracketed by events
+STEP_BYTES = 24e9  # algorithmic bytes per step (about 4 ms at the HBM roofline)
+WARM_S = 0.3  # minimum warm-up time (s)
 
 
 # ----------------------------------------------------------------------------- workloads
 
-def make_workload(name: str):
+def make_workload(name: str, rows: int = 0):
+    """The workload `name` (at its full size, or with `rows` rows when given)."""
+    wl = _make_workload(name)
+    if rows and rows != wl["M"]:
+        wl = _make_workload(name, rows)
+        wl["desc"] += f" [{rows} rows]"
+    return wl
+
+
+def _make_workload(name: str, rows: int = 0):
     """Returns dict(desc, M, K, inputs(np), bytes_in, kernels=[(label, alg_bytes)], ...)."""
     if name == "mxfp4":
-        M, K = 4096, 4096
+        M, K = rows or 4096, 4096
         return dict(name=name, M=M, K=K, fmt="MXFP4", had=0,
                     desc="mxfp4_4096x4096 quantize + dequantize round trip "
                          "(bf16 0.5*Student-t(3), block 32, E8M0)",
@@ -62,7 +79,7 @@ def make_workload(name: str):
                     kernels=[("quantize", M * K * 2 + M * K // 2 + M * K // 32),
                              ("dequantize", M * K // 2 + M * K // 32 + M * K * 2)])
     if name == "nvfp4":
-        M, K = 256, 1024
+        M, K = rows or 256, 1024
         return dict(name=name, M=M, K=K, fmt="NVFP4", had=0,
                     desc="nvfp4_256x1024 quantize, dynamic tensor scale (N(0,1), 1% x20)",
                     x=lambda: workloads.nvfp4_outliers(M, K, seed=1),
@@ -70,20 +87,26 @@ def make_workload(name: str):
                     launches=2)
     if name.startswith("hadamard"):
         n = int(name[len("hadamard"):] or 128)
-        M, K = 8192, 4096
+        M, K = rows or 8192, 4096
         return dict(name=name, M=M, K=K, fmt="NVFP4", had=n,
                     desc=f"hadamard{n}+nvfp4_8192x4096 quantize, static tensor scale "
                          "(N(0,1), 64 channels x50)",
                     x=lambda: workloads.hadamard_channels(M, K, seed=3),
                     kernels=[("quantize", M * K * 2 + M * K // 2 + M * K // 16)])
     if name == "arc":
-        M, K, S = 8192, 4096, 256
+        M, K, S = rows or 8192, 4096, 256
         return dict(name=name, M=M, K=K, S=S, fmt="NVFP4", had=0,
                     desc="arc_8192x4096 reorder+RMSNorm+NVFP4+residual(S=256), static tensor scale",
                     x=lambda: workloads.arc_activations(M, K, seed=4, S=S),
                     kernels=[("arc", M * K * 2 + M * (K + S) // 2 + M * (K + S) // 16)])
+    if name == "arc_mxfp4":
+        M, K, S = rows or 8192, 4096, 256
+        return dict(name=name, M=M, K=K, S=S, fmt="MXFP4", had=0,
+                    desc="arc_mxfp4_8192x4096 reorder+RMSNorm+MXFP4+residual(S=256)",
+                    x=lambda: workloads.arc_activations(M, K, seed=4, S=S),
+                    kernels=[("arc", M * K * 2 + M * (K + S) // 2 + M * (K + S) // 32)])
     if name == "dual":
-        M, K = 32768, 4096
+        M, K = rows or 32768, 4096
         return dict(name=name, M=M, K=K, fmt="DUAL", had=512,
                     desc="dual_fwht512_32768x4096 quantize + dequantize/inverse-FWHT round trip "
                          "(N(0,1) x LogNormal(0,1) per-token gain)",
@@ -168,19 +191,43 @@ def peaks():
         return 6650.0, "fallback"
 
 
-def kernel_source_sha() -> str:
+def peaks_tensor():
+    """Dense bf16 tensor TFLOP/s (burst figure) from MEASURED_PEAKS.json, else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]) * 1e12, "measured"
+    except (OSError, KeyError, ValueError):
+        return 1590e12, "fallback"
+
+
+# Source files each timed kernel is compiled from (the entry points' host code
+# in fp4q.cu excluded): a committed ncu figure is used only while they are unchanged.
+_COMMON = ["fp4q_device.cuh", "fp4q_unit.cuh", "fp4q_quant.cuh"]
+KERNEL_SOURCES = {
+    ("dual", "quantize"): _COMMON + ["fp4q_mma.cuh", "fp4q_mma_wide.cuh"],
+    ("dual", "dequantize"): _COMMON + ["fp4q_dequant.cuh"],
+    ("mxfp4", "quantize"): _COMMON,
+    ("mxfp4", "dequantize"): _COMMON + ["fp4q_dequant.cuh"],
+    ("arc", "arc"): _COMMON + ["fp4q_arc.cuh"],
+    ("arc_mxfp4", "arc"): _COMMON + ["fp4q_arc.cuh"],
+}
+
+
+def kernel_source_sha(files=None) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "fp4_micro_block_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(fn.encode() + f.read())
+    names = sorted(files) if files else sorted(fn for fn in os.listdir(csrc) if fn.endswith((".cu", ".cuh")))
+    for fn in names:
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def ncu_traffic(workload: str, kernel_label: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
+    the current sources of that kernel (else None)."""
     path = os.path.join(ROOT, "profiles", f"traffic_{workload}_{kernel_label}.txt")
     try:
         txt = open(path).read()
@@ -188,7 +235,7 @@ def ncu_traffic(workload: str, kernel_label: str):
         return None
     sha = re.search(r"source_sha:\s*(\w+)", txt)
     val = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
-    if not sha or not val or sha.group(1) != kernel_source_sha():
+    if not sha or not val or sha.group(1) != kernel_source_sha(KERNEL_SOURCES.get((workload, kernel_label))):
         return None
     return float(val.group(1))
 
@@ -201,11 +248,11 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wl = make_workload(args.workload)
+    wl = make_workload(args.workload, args.rows)
     M, K = wl["M"], wl["K"]
     raw = wl["x"]()
     gamma_t = perm_t = outl_t = None
-    if wl["name"] == "arc":
+    if wl["name"].startswith("arc"):
         x_np, gamma, perm, outl = raw
         gamma_t = torch.from_numpy(gamma.view(np.int16)).view(torch.bfloat16).to(dev)
         perm_t = torch.from_numpy(perm).to(dev)
@@ -219,10 +266,14 @@ def run_ours(args, rank, world, local_rank):
     KS = K + S
     fmt = {"MXFP4": fq.FP4Q_MXFP4, "NVFP4": fq.FP4Q_NVFP4, "DUAL": fq.FP4Q_NVFP4_DUAL}[wl["fmt"]]
     B = 32 if fmt == fq.FP4Q_MXFP4 else 16
-    set_bytes = in_bytes + M * KS // 2 + M * KS // B + (M * K * 2 if len(wl["kernels"]) > 1 and
-                                                          wl["kernels"][-1][0] == "dequantize" else 0)
-    R = max(2, int(np.ceil(4 * L2_BYTES / set_bytes)))
-    R = min(R, 64)
+    labels = [k for k, _ in wl["kernels"]]
+    alg = dict(wl["kernels"])
+    has_dq = labels[-1] == "dequantize"
+    set_bytes = in_bytes + M * KS // 2 + M * KS // B + (M * K * 2 if has_dq else 0)
+    R = min(64, max(2, int(np.ceil(4 * L2_BYTES / set_bytes))))
+    # batches per step: about STEP_BYTES of algorithmic traffic, so that a step
+    # lasts a few milliseconds whatever the workload
+    U = args.units or min(2048, max(R, int(np.ceil(STEP_BYTES / sum(alg.values())))))
     xs, outs = [], []
     for i in range(R):
         xi = x_host.to(dev)
@@ -234,7 +285,7 @@ def run_ours(args, rank, world, local_rank):
             sf = torch.empty((M, K // 128), dtype=torch.float32, device=dev)
         else:
             sf = None
-        y = torch.empty((M, K), dtype=torch.bfloat16, device=dev) if wl["kernels"][-1][0] == "dequantize" else None
+        y = torch.empty((M, K), dtype=torch.bfloat16, device=dev) if has_dq else None
         xs.append(xi)
         outs.append((codes, scales, sf, y))
     ws = fq.workspace(dev)
@@ -243,11 +294,11 @@ def run_ours(args, rank, world, local_rank):
     L = fq.lib()
 
     # static tensor scale for the Hadamard / ARC workloads: the dynamic value of a first call
-    if wl["name"].startswith("hadamard") or wl["name"] == "arc":
+    if wl["name"].startswith("hadamard") or wl["name"] == "arc":  # NVFP4 tensor scale
         for i in range(R):
             codes, scales, sf, _ = outs[i]
-            if wl["name"] == "arc":
-                fq.fp4q_arc_quantize(xs[i], gamma_t, 1e-6, perm_t, outl_t, codes, scales, sf,
+            if wl["name"].startswith("arc"):
+                fq.fp4q_arc_quantize(xs[i], gamma_t, 1e-6, perm_t, outl_t, fmt, codes, scales, sf,
                                      fq.FP4Q_TSCALE_DYNAMIC, 0, ws)
             else:
                 fq.fp4q_hadamard_quantize(xs[i], wl["had"], fmt, codes, scales, sf,
@@ -255,7 +306,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
 
     p = lambda t: None if t is None else t.data_ptr()
-    calls = []  # per set: list of zero-arg callables, one per kernel label
+    calls = []  # per buffer set: one zero-arg callable per kernel label
     for i in range(R):
         codes, scales, sf, y = outs[i]
         xp, cp, sp, fp, yp = p(xs[i]), p(codes), p(scales), p(sf), p(y)
@@ -270,45 +321,53 @@ def run_ours(args, rank, world, local_rank):
         elif wl["name"].startswith("hadamard"):
             calls.append([lambda xp=xp, cp=cp, sp=sp, fp=fp: L.fp4q_hadamard_quantize(
                 xp, M, K, K, wl["had"], fmt, cp, sp, fp, fq.FP4Q_TSCALE_STATIC, 0, None, 0, sh)])
-        elif wl["name"] == "arc":
+        elif wl["name"].startswith("arc"):
             calls.append([lambda xp=xp, cp=cp, sp=sp, fp=fp: L.fp4q_arc_quantize(
-                xp, M, K, K, gamma_t.data_ptr(), 1e-6, perm_t.data_ptr(), outl_t.data_ptr(), S, cp, sp,
+                xp, M, K, K, gamma_t.data_ptr(), 1e-6, perm_t.data_ptr(), outl_t.data_ptr(), S, fmt, cp, sp,
                 fp, fq.FP4Q_TSCALE_STATIC, 0, None, 0, sh)])
         elif wl["name"] == "dual":
             calls.append([lambda xp=xp, cp=cp, sp=sp, fp=fp: L.fp4q_hadamard_quantize(
                 xp, M, K, K, 512, fmt, cp, sp, fp, 0, 0, None, 0, sh),
                 lambda cp=cp, sp=sp, fp=fp, yp=yp: L.fp4q_dequantize(fmt, cp, sp, fp, M, K, 0, 512, yp, sh)])
-    labels = [k for k, _ in wl["kernels"]]
-    # launches of our kernels per step (the NVFP4 dynamic mode runs an amax pre-pass
-    # and the quantizer inside one entry point)
-    launches_per_step = wl.get("launches", len(wl["kernels"]))
+    # launches of our kernels per batch (the NVFP4 dynamic mode runs an amax
+    # pre-pass and the quantizer inside one entry point)
+    launches_per_batch = wl.get("launches", len(wl["kernels"]))
+    n_lab = len(labels)
 
-    def step(k, evs=None):
-        cs = calls[k % R]
-        for j, c in enumerate(cs):
+    def step(evs=None):
+        """U batches, one phase per kernel label; evs[j] is recorded before phase j."""
+        for j in range(n_lab):
             if evs is not None:
                 evs[j].record(stream)
-            st = c()
-            if st != 0:
-                raise RuntimeError(f"{labels[j]}: {fq.status_string(st)}")
+            for u in range(U):
+                st = calls[u % R][j]()
+                if st != 0:
+                    raise RuntimeError(f"{labels[j]}: {fq.status_string(st)}")
         if evs is not None:
-            evs[len(cs)].record(stream)
+            evs[n_lab].record(stream)
 
     dist = world > 1
     if dist:
         import torch.distributed as tdist
 
-    for k in range(args.warmup):
-        step(k)
+    # warm-up: W steps, continued until WARM_S seconds have passed (clocks and
+    # caches settled); the same count on every rank
+    t0 = time.perf_counter()
+    n_warm = 0
+    while n_warm < args.warmup or time.perf_counter() - t0 < WARM_S:
+        step()
+        torch.cuda.synchronize()
+        n_warm += 1
+    if dist:
+        t = torch.tensor([n_warm], device=dev, dtype=torch.int64)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        for _ in range(int(t.item()) - n_warm):
+            step()
+        n_warm = int(t.item())
     torch.cuda.synchronize()
     assert fq.fp4q_device_error() == 0
 
-    # Per-kernel CUDA events on every EV_EVERY-th timed step only: an event
-    # recorded between two kernels ends the overlap of programmatic dependent
-    # launch there, so bracketing every launch would slow the timed steps down.
-    n_lab = len(labels)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_lab + 1)] if k % EV_EVERY == 0 else None
-           for k in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_lab + 1)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
@@ -321,7 +380,7 @@ def run_ours(args, rank, world, local_rank):
     w0 = sampler.mark()
     t_start.record(stream)
     for k in range(args.steps):
-        step(k, evs[k])
+        step(evs[k])
     t_end.record(stream)
     torch.cuda.synchronize()
     w1 = sampler.mark()
@@ -331,68 +390,63 @@ def run_ours(args, rank, world, local_rank):
     assert fq.fp4q_device_error() == 0
 
     total_ms = t_start.elapsed_time(t_end)
-    per_kernel = {lab: [] for lab in labels}
-    for k in range(args.steps):
-        if evs[k] is None:
-            continue
-        for j, lab in enumerate(labels):
-            per_kernel[lab].append(evs[k][j].elapsed_time(evs[k][j + 1]))
+    phase_ms = np.array([[evs[k][j].elapsed_time(evs[k][j + 1]) for j in range(n_lab)]
+                         for k in range(args.steps)])
     if dist:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        t = torch.tensor([total_ms] + phase_ms.sum(axis=0).tolist(), device=dev, dtype=torch.float64)
         tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        total_ms = float(t.item())
-
-    # dominant kernel: largest total time.  Its duration inside the timed loop is
-    # the step time times its share of the event-bracketed launch times: a
-    # bracketed launch also includes the dispatch latency that programmatic
-    # dependent launch hides between consecutive kernels of the timed loop.
-    alg = dict(wl["kernels"])
-    dom = max(labels, key=lambda l: sum(per_kernel[l]))
-    bracketed = {l: float(np.mean(per_kernel[l])) for l in labels}
-    share = bracketed[dom] / sum(bracketed.values())
-    dom_ms = total_ms / args.steps * share
-    achieved = alg[dom] / (dom_ms * 1e-3) / 1e9
+        total_ms = float(t[0].item())
+        phase_tot = t[1:].cpu().numpy()
+    else:
+        phase_tot = phase_ms.sum(axis=0)
+    # mean duration of one launch of each kernel in its back-to-back phase
+    launch_us = {lab: float(phase_tot[j] / (args.steps * U) * 1e3) for j, lab in enumerate(labels)}
+    dom = max(labels, key=lambda l: launch_us[l])
+    achieved = alg[dom] / (launch_us[dom] * 1e-6) / 1e9
     peak, peak_src = peaks()
-    value = in_bytes * args.steps * world / (total_ms * 1e-3) / 1e9
+    value = in_bytes * U * args.steps * world / (total_ms * 1e-3) / 1e9
 
     # ---------------------------------------------------------------- end to end
-    e2e = None
-    if True:  # every rank copies its own batch (weak scaling)
-        n_e2e = max(3, min(args.steps, 20))
-        x_pin = x_host.pin_memory()
-        codes, scales, sf, y = outs[0]
-        h_codes = torch.empty(codes.shape, dtype=codes.dtype).pin_memory()
-        h_scales = torch.empty(scales.shape, dtype=scales.dtype).pin_memory()
-        h_sf = torch.empty(sf.shape, dtype=sf.dtype).pin_memory() if sf is not None else None
-        h_y = torch.empty(y.shape, dtype=y.dtype).pin_memory() if y is not None else None
-        d2h = codes.numel() + scales.numel() + (sf.numel() * 4 if sf is not None else 0) + \
-            (y.numel() * 2 if y is not None else 0)
+    n_e2e = max(3, min(args.steps, 20))
+    x_pin = x_host.pin_memory()
+    codes, scales, sf, y = outs[0]
+    h_codes = torch.empty(codes.shape, dtype=codes.dtype).pin_memory()
+    h_scales = torch.empty(scales.shape, dtype=scales.dtype).pin_memory()
+    h_sf = torch.empty(sf.shape, dtype=sf.dtype).pin_memory() if sf is not None else None
+    h_y = torch.empty(y.shape, dtype=y.dtype).pin_memory() if y is not None else None
+    d2h = codes.numel() + scales.numel() + (sf.numel() * 4 if sf is not None else 0) + \
+        (y.numel() * 2 if y is not None else 0)
 
-        def e2e_step():
-            xs[0].copy_(x_pin, non_blocking=True)
-            step(0)
-            h_codes.copy_(codes, non_blocking=True)
-            h_scales.copy_(scales, non_blocking=True)
-            if h_sf is not None:
-                h_sf.copy_(sf, non_blocking=True)
-            if h_y is not None:
-                h_y.copy_(y, non_blocking=True)
+    def e2e_step():
+        xs[0].copy_(x_pin, non_blocking=True)
+        for j in range(n_lab):
+            st = calls[0][j]()
+            if st != 0:
+                raise RuntimeError(f"{labels[j]}: {fq.status_string(st)}")
+        h_codes.copy_(codes, non_blocking=True)
+        h_scales.copy_(scales, non_blocking=True)
+        if h_sf is not None:
+            h_sf.copy_(sf, non_blocking=True)
+        if h_y is not None:
+            h_y.copy_(y, non_blocking=True)
 
+    e2e_step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n_e2e):
         e2e_step()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = a.elapsed_time(b)
-        if dist:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": round(in_bytes * n_e2e * world / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
-               "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": int(d2h), "steps": n_e2e}
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b)
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": round(in_bytes * n_e2e * world / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+           "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": int(d2h), "steps": n_e2e,
+           "step": "one batch: host->device copy, the path through the C ABI, device->host copy"}
+    assert fq.fp4q_device_error() == 0
 
     # ---------------------------------------------------------------- CPU oracle baseline
     cpu = None
@@ -414,28 +468,129 @@ def run_ours(args, rank, world, local_rank):
         "dtype": "f32",
         "data": "synthetic",
         "config": {"workload": wl["desc"], "M": M, "K": K, "format": wl["fmt"],
-                   "hadamard": wl["had"], "per_rank_batch": f"{M}x{K} bf16",
-                   "global_batch": f"{world}x{M}x{K}",
-                   "l2": f"inputs/outputs rotate over {R} buffer sets "
+                   "hadamard": wl["had"], "batches_per_step": U,
+                   "per_rank_batch": f"{U}x{M}x{K} bf16 per step",
+                   "global_batch": f"{world}x{U}x{M}x{K}",
+                   "l2": f"inputs larger than L2; batches rotate over {R} buffer sets "
                          f"({R * set_bytes / MIB:.0f} MiB > 4x126 MB L2)",
                    "parallelism": f"dp{world}"},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
                      "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": traffic, "peak_source": peak_src,
-                     "alg_bytes_per_launch": alg[dom], "mean_launch_us": round(dom_ms * 1e3, 3),
-                     "step_share": round(share, 4),
-                     "bracketed_launch_us": round(bracketed[dom] * 1e3, 3),
-                     "bracketed_steps": len(per_kernel[dom]),
+                     "alg_bytes_per_launch": alg[dom], "mean_launch_us": round(launch_us[dom], 3),
+                     "timing": f"CUDA events around the {U} back-to-back launches of each phase, "
+                               f"every timed step",
                      "frac_of_nominal_8000": round(achieved / 8000.0, 4)},
-        "kernels_us": {lab: round(total_ms / args.steps * bracketed[lab] / sum(bracketed.values()) * 1e3, 3)
-                       for lab in labels},
+        "kernels_us": {lab: round(launch_us[lab], 3) for lab in labels},
+        "kernels_frac": {lab: round(alg[lab] / (launch_us[lab] * 1e-6) / 1e9 / peak, 4) for lab in labels},
         "e2e": e2e,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": launches_per_batch * U * args.steps,
+        "warmup_steps_run": n_warm,
         "clocks": clocks,
         "cpu_baseline": cpu,
         "impl": "ours",
     }
     return line
+
+
+def run_arc_gemm(args, local_rank):
+    """ARCQuant's cost on the consumer side: the fused ARC quantizer plus the
+    block-scaled NVFP4 GEMM over K + S, against the same fused kernel without
+    residual channels (S = 0) plus the GEMM over K.  Activations: the ARC
+    workload (bf16 8192 x 4096, 256 outlier channels); weights: bf16
+    N(0,1) 4096 x 4096 in the activations' channel order, quantized NVFP4 once
+    outside the timed region ([W | W_S] for K + S).  Each kernel is timed as a
+    back-to-back phase of U launches inside every step (CUDA events)."""
+    import torch
+    import fp4_micro_block_b200 as fq
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    M, K, S, N = 8192, 4096, 256, 4096
+    x_np, gamma, perm, outl = workloads.arc_activations(M, K, seed=4, S=S)
+    rng = np.random.default_rng(7)
+    w = workloads.to_bf16_bits(rng.standard_normal((N, K)))[:, perm]
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    g_t, p_t, o_t = bf(gamma), torch.from_numpy(perm).to(dev), torch.from_numpy(outl).to(dev)
+    SW = fq.FP4Q_SCALES_SWIZZLED
+    wb_aug = fq.quantize_nvfp4(bf(np.concatenate([w, w[:, outl]], axis=1)), None, SW)
+    wb_k = fq.quantize_nvfp4(bf(w), None, SW)
+    R = 4  # input sets: 4 x 64 MiB of activations > 2 x L2
+    xs = [bf(x_np) for _ in range(R)]
+    st = fq.arc_quantize(xs[0], g_t, p_t, o_t, 1e-6, None, SW)[2]  # calibrated s_t stand-in
+    outs_aug = [fq.alloc_outputs(M, K + S, fq.FP4Q_NVFP4, SW, dev) for _ in range(R)]
+    outs_k = [fq.alloc_outputs(M, K, fq.FP4Q_NVFP4, SW, dev) for _ in range(R)]
+    for o in outs_aug + outs_k:
+        o[2].copy_(st)
+    d = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    L, sh = fq.lib(), torch.cuda.current_stream(dev).cuda_stream
+    pp = lambda t: t.data_ptr()
+
+    def arc(i, with_res):
+        c, s_, sf = (outs_aug if with_res else outs_k)[i]
+        return L.fp4q_arc_quantize(pp(xs[i]), M, K, K, pp(g_t), 1e-6, pp(p_t), pp(o_t) if with_res else None,
+                                   S if with_res else 0, fq.FP4Q_NVFP4, pp(c), pp(s_), pp(sf),
+                                   fq.FP4Q_TSCALE_STATIC, SW, None, 0, sh)
+
+    def gemm(i, with_res):
+        c, s_, sf = (outs_aug if with_res else outs_k)[i]
+        wc, ws, wt = wb_aug if with_res else wb_k
+        return L.fp4q_gemm_nvfp4(pp(c), pp(s_), pp(sf), pp(wc), pp(ws), pp(wt), M, N, K + S if with_res else K,
+                                 pp(d), 1, sh)
+
+    labels = ["arc_S256", "gemm_K4352", "arc_S0", "gemm_K4096"]
+    fns = [lambda i: arc(i, True), lambda i: gemm(i, True), lambda i: arc(i, False), lambda i: gemm(i, False)]
+    U = args.units or 16
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        for j, f in enumerate(fns):
+            if evs is not None:
+                evs[j].record(stream)
+            for u in range(U):
+                st_ = f(u % R)
+                if st_ != 0:
+                    raise RuntimeError(f"{labels[j]}: {fq.status_string(st_)}")
+        if evs is not None:
+            evs[len(fns)].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert fq.fp4q_device_error() == 0
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    torch.cuda.synchronize()
+    w0 = sampler.mark()
+    for k in range(args.steps):
+        step(evs[k])
+    torch.cuda.synchronize()
+    clocks = sampler.stop(w0, sampler.mark())
+    assert fq.fp4q_device_error() == 0
+    us = {lab: float(np.sum([evs[k][j].elapsed_time(evs[k][j + 1]) for k in range(args.steps)])
+                     / (args.steps * U) * 1e3) for j, lab in enumerate(labels)}
+    flops = {"gemm_K4352": 2.0 * M * N * (K + S), "gemm_K4096": 2.0 * M * N * K}
+    bf16_peak, src = peaks_tensor()
+    fp4_peak = 4.0 * bf16_peak  # dense FP4 : bf16 tensor rate, 9 : 2.25 PFLOP/s nominal
+    tf = {k: flops[k] / (us[k] * 1e-6) / 1e12 for k in flops}
+    overhead = (us["arc_S256"] + us["gemm_K4352"]) / (us["arc_S0"] + us["gemm_K4096"]) - 1.0
+    return {
+        "metric": "ARC residual overhead: (fused ARC quantize + NVFP4 GEMM over K+S) / (same with S=0, GEMM over K) - 1",
+        "value": round(overhead, 4), "unit": "fraction", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "higher_is_better": False, "data": "synthetic", "impl": "ours",
+        "config": {"workload": "arc_gemm: activations 8192x4096 (256 outlier channels x30), "
+                               "weights 4096x4096, NVFP4, tiled scales, bf16 output",
+                   "batches_per_step": U, "input_sets": R},
+        "kernels_us": {k: round(v, 3) for k, v in us.items()},
+        "gemm_tflops": {k: round(v, 1) for k, v in tf.items()},
+        "roofline": {"bound": "tensor", "kernel": "gemm_K4352", "achieved": round(tf["gemm_K4352"], 1),
+                     "peak": round(fp4_peak / 1e12, 1), "unit": "TFLOP/s",
+                     "frac": round(tf["gemm_K4352"] * 1e12 / fp4_peak, 4),
+                     "peak_source": f"{src} bf16 x 4 (nominal dense FP4 : bf16 ratio)"},
+        "pages_overhead": "about 4.9% of total latency (ARCQuant, Resultats Experimentaux, Efficacite)",
+        "clocks": clocks,
+    }
 
 
 def cpu_baseline(wl, x_np, raw, budget_s: float = 20.0):
@@ -454,9 +609,9 @@ def cpu_baseline(wl, x_np, raw, budget_s: float = 20.0):
             oracle.quantize_nvfp4(xb)
         elif name.startswith("hadamard"):
             oracle.hadamard_quantize(xb, wl["had"], "nvfp4", s_t=0.01)
-        elif name == "arc":
+        elif name.startswith("arc"):
             _, gamma, perm, outl = raw
-            oracle.arc(xb, gamma, perm, outl, s_t=0.01)
+            oracle.arc(xb, gamma, perm, outl, s_t=0.01, fmt=wl["fmt"].lower())
         elif name == "dual":
             c, s, g, _ = oracle.hadamard_quantize(xb, 512, "dual")
             oracle.dequantize_bf16("dual", c, s, g, inv_had=512)
@@ -473,14 +628,29 @@ def cpu_baseline(wl, x_np, raw, budget_s: float = 20.0):
     dt = time.perf_counter() - t
     return {"value": round(n * K * 2 / dt / 1e9, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": f"first {n} of {M} rows ({n * K} elements), {dt:.1f} s",
-            "seconds": round(dt, 2)}
+            "seconds": round(dt, 2), **host_info()}
+
+
+def host_info() -> dict:
+    """The host the oracle ran on: its logical CPU count and model name.  The
+    oracle is single-threaded scalar C, so it used one of them."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cores": os.cpu_count(), "cpu_model": model, "threads_used": 1}
 
 
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args, rank, world):
     """The oracle (plain C, one core) timed as this metric's reference arm."""
-    wl = make_workload(args.workload)
+    wl = make_workload(args.workload, args.rows)
     raw = wl["x"]()
     x_np = raw[0] if isinstance(raw, tuple) else raw
     import oracle
@@ -502,9 +672,9 @@ def run_reference(args, rank, world):
             oracle.quantize_nvfp4(xb)
         elif wl["name"].startswith("hadamard"):
             oracle.hadamard_quantize(xb, wl["had"], "nvfp4", s_t=0.01)
-        elif wl["name"] == "arc":
+        elif wl["name"].startswith("arc"):
             _, gamma, perm, outl = raw
-            oracle.arc(xb, gamma, perm, outl, s_t=0.01)
+            oracle.arc(xb, gamma, perm, outl, s_t=0.01, fmt=wl["fmt"].lower())
         else:
             c, s, g, _ = oracle.hadamard_quantize(xb, 512, "dual")
             oracle.dequantize_bf16("dual", c, s, g, inv_had=512)
@@ -524,7 +694,7 @@ def run_reference(args, rank, world):
                    "hadamard": wl["had"], "parallelism": f"dp{world}"},
         "impl": "reference",
         "cpu_baseline": {"value": round(v, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"first {n} of {M} rows per step"},
+                         "sample": f"first {n} of {M} rows per step", **host_info()},
         "e2e": {"value": round(v, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -535,11 +705,15 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mxfp4",
-                    help="mxfp4 (default) | nvfp4 | hadamard128 | hadamard16 | hadamard32 | arc | dual")
+    ap.add_argument("--workload", default="dual",
+                    help="dual (default) | mxfp4 | nvfp4 | hadamard128 | hadamard16 | hadamard32 | arc | arc_mxfp4 | arc_gemm")
+    ap.add_argument("--rows", type=int, default=0,
+                    help="override the workload's row count (small cases for profiler captures)")
+    ap.add_argument("--units", type=int, default=0,
+                    help="batches per step (default: about 24 GB of algorithmic traffic per step)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     args = ap.parse_args()
@@ -563,6 +737,10 @@ def main():
         torch.cuda.set_device(local_rank)
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                  device_id=torch.device("cuda", local_rank))
+    if args.workload == "arc_gemm":
+        if rank == 0:
+            print(json.dumps(run_arc_gemm(args, local_rank)), flush=True)
+        return
     try:
         line = run_ours(args, rank, world, local_rank)
     finally:

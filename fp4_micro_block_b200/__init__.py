@@ -19,7 +19,9 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libfp4q.so")
+# FP4Q_LIBRARY selects another build of the library (a variant made with
+# `python -m fp4_micro_block_b200.build --define ... --out ...`).
+LIB_PATH = os.environ.get("FP4Q_LIBRARY") or os.path.join(_HERE, "libfp4q.so")
 
 # enum values of include/fp4q.h
 FP4Q_OK, FP4Q_ERR_INVALID_ARG, FP4Q_ERR_UNSUPPORTED, FP4Q_ERR_ALIGNMENT, FP4Q_ERR_CUDA, \
@@ -32,7 +34,7 @@ FP4Q_WORKSPACE_BYTES = 16384
 EXPORTED = [
     "fp4q_quantize_nvfp4", "fp4q_quantize_nvfp4_noalloc", "fp4q_quantize_mxfp4", "fp4q_hadamard_quantize", "fp4q_arc_quantize",
     "fp4q_dequantize", "fp4q_workspace_bytes", "fp4q_scales_bytes", "fp4q_status_string",
-    "fp4q_device_error", "fp4q_selftest_div",
+    "fp4q_device_error", "fp4q_selftest_div", "fp4q_gemm_nvfp4",
 ]
 
 
@@ -45,20 +47,25 @@ class Fp4qError(RuntimeError):
 def _load() -> C.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with `python -m fp4_micro_block_b200.build`")
-    L = C.CDLL(LIB_PATH)
+    return declare(C.CDLL(LIB_PATH))
+
+
+def declare(L: C.CDLL) -> C.CDLL:
+    """Sets the argument and result types of the C entry points on a loaded library."""
     p, i64, f32, i32, sz = C.c_void_p, C.c_int64, C.c_float, C.c_int, C.c_size_t
     sigs = {
         "fp4q_quantize_nvfp4": (i32, [p, i64, i64, i64, p, p, p, i32, i32, p, sz, p]),
         "fp4q_quantize_nvfp4_noalloc": (i32, [p, i64, i64, i64, p, p, p, i32, p]),
         "fp4q_quantize_mxfp4": (i32, [p, i64, i64, i64, p, p, i32, p]),
         "fp4q_hadamard_quantize": (i32, [p, i64, i64, i64, i32, i32, p, p, p, i32, i32, p, sz, p]),
-        "fp4q_arc_quantize": (i32, [p, i64, i64, i64, p, f32, p, p, i64, p, p, p, i32, i32, p, sz, p]),
+        "fp4q_arc_quantize": (i32, [p, i64, i64, i64, p, f32, p, p, i64, i32, p, p, p, i32, i32, p, sz, p]),
         "fp4q_dequantize": (i32, [i32, p, p, p, i64, i64, i32, i32, p, p]),
         "fp4q_workspace_bytes": (sz, [i64, i64]),
         "fp4q_scales_bytes": (i64, [i64, i64, i32]),
         "fp4q_status_string": (C.c_char_p, [i32]),
         "fp4q_device_error": (i32, []),
         "fp4q_selftest_div": (i32, [p, p, i64, p, p, p]),
+        "fp4q_gemm_nvfp4": (i32, [p, p, p, p, p, p, i64, i64, i64, p, i32, p]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -161,14 +168,14 @@ def fp4q_hadamard_quantize(x, had_size, fmt, codes, scales, scale_fp32,
                   "fp4q_hadamard_quantize")
 
 
-def fp4q_arc_quantize(x, gamma, eps, perm, outliers, codes, scales, tensor_scale,
+def fp4q_arc_quantize(x, gamma, eps, perm, outliers, fmt, codes, scales, tensor_scale,
                       mode=FP4Q_TSCALE_DYNAMIC, layout=FP4Q_SCALES_LINEAR, workspace=None,
                       stream=None):
     M, K = x.shape
     S = 0 if outliers is None else outliers.numel()
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     return _check(_lib.fp4q_arc_quantize(_ptr(x), M, K, _ld(x), _ptr(gamma), float(eps), _ptr(perm),
-                                         _ptr(outliers), S, _ptr(codes), _ptr(scales),
+                                         _ptr(outliers), S, int(fmt), _ptr(codes), _ptr(scales),
                                          _ptr(tensor_scale), mode, layout, _ptr(workspace),
                                          ws_bytes, _stream(stream)), "fp4q_arc_quantize")
 
@@ -178,6 +185,18 @@ def fp4q_dequantize(fmt, codes, scales, scale_fp32, M, K, y, layout=FP4Q_SCALES_
     return _check(_lib.fp4q_dequantize(int(fmt), _ptr(codes), _ptr(scales), _ptr(scale_fp32), M, K,
                                        layout, int(inv_had_size), _ptr(y), _stream(stream)),
                   "fp4q_dequantize")
+
+
+def fp4q_gemm_nvfp4(a_codes, a_scales, a_scale, b_codes, b_scales, b_scale, K, d, stream=None):
+    """d [M, N] (float32 or bfloat16) = a_scale b_scale (A B^T) of two NVFP4
+    tensors in the quantizers' output form (SWIZZLED scale buffers)."""
+    M, N = d.shape
+    if d.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("d must be float32 or bfloat16")
+    return _check(_lib.fp4q_gemm_nvfp4(_ptr(a_codes), _ptr(a_scales), _ptr(a_scale), _ptr(b_codes),
+                                       _ptr(b_scales), _ptr(b_scale), M, N, K, _ptr(d),
+                                       int(d.dtype == torch.bfloat16), _stream(stream)),
+                  "fp4q_gemm_nvfp4")
 
 
 def fp4q_device_error() -> int:
@@ -253,16 +272,18 @@ def hadamard_quantize(x, had_size, fmt=FP4Q_NVFP4, tensor_scale=None, layout=FP4
 
 
 def arc_quantize(x, gamma, perm, outliers, eps=1e-6, tensor_scale=None,
-                 layout=FP4Q_SCALES_LINEAR, ws=None):
+                 layout=FP4Q_SCALES_LINEAR, ws=None, fmt=FP4Q_NVFP4):
+    """ARCQuant path; returns (codes, scales, tensor scale (NVFP4) or None (MXFP4))."""
     M, K = x.shape
     S = 0 if outliers is None else outliers.numel()
-    codes, scales, sf = alloc_outputs(M, K + S, FP4Q_NVFP4, layout, x.device)
+    codes, scales, sf = alloc_outputs(M, K + S, fmt, layout, x.device)
     mode = FP4Q_TSCALE_DYNAMIC
-    if tensor_scale is not None:
-        sf.copy_(tensor_scale.reshape(1))
-        mode = FP4Q_TSCALE_STATIC
-    ws = workspace(x.device) if (ws is None and mode == FP4Q_TSCALE_DYNAMIC) else ws
-    fp4q_arc_quantize(x, gamma, eps, perm, outliers, codes, scales, sf, mode, layout, ws)
+    if fmt == FP4Q_NVFP4:
+        if tensor_scale is not None:
+            sf.copy_(tensor_scale.reshape(1))
+            mode = FP4Q_TSCALE_STATIC
+        ws = workspace(x.device) if (ws is None and mode == FP4Q_TSCALE_DYNAMIC) else ws
+    fp4q_arc_quantize(x, gamma, eps, perm, outliers, fmt, codes, scales, sf, mode, layout, ws)
     return codes, scales, sf
 
 
@@ -271,3 +292,10 @@ def dequantize(fmt, codes, scales, scale_fp32, K, layout=FP4Q_SCALES_LINEAR, inv
     y = torch.empty((M, K), dtype=torch.bfloat16, device=codes.device)
     fp4q_dequantize(fmt, codes, scales, scale_fp32, M, K, y, layout, inv_had_size)
     return y
+
+
+def gemm_nvfp4(a_codes, a_scales, a_scale, b_codes, b_scales, b_scale, K, out_dtype=torch.float32):
+    """Allocates D [M, N] and calls fp4q_gemm_nvfp4."""
+    d = torch.empty((a_codes.shape[0], b_codes.shape[0]), dtype=out_dtype, device=a_codes.device)
+    fp4q_gemm_nvfp4(a_codes, a_scales, a_scale, b_codes, b_scales, b_scale, K, d)
+    return d

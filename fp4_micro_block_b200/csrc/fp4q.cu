@@ -9,21 +9,19 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <type_traits>
 #include <utility>
 
 #include "../../include/fp4q.h"
 #include "fp4q_arc.cuh"
 #include "fp4q_dequant.cuh"
 #include "fp4q_device.cuh"
+#include "fp4q_gemm.cuh"
 #include "fp4q_mma.cuh"
 #include "fp4q_mma_wide.cuh"
 #include "fp4q_quant.cuh"
 
 #define FP4Q_API extern "C" __attribute__((visibility("default")))
-
-#ifndef FP4Q_ARC_STAGES
-#define FP4Q_ARC_STAGES 2  // row buffers per ARC warp, where they cost no warp
-#endif
 
 namespace {
 
@@ -87,6 +85,29 @@ fp4q_status make_x_map(CUtensorMap* map, const void* x, int64_t M, int64_t K, in
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FP4Q_OK : FP4Q_ERR_CUDA;
+}
+
+#ifdef FP4Q_TEST_HOOKS
+// Test build only: index of a tile that CTA 0 of the next register-path
+// quantizer launch does not issue (-1: none); consumed by that launch.
+std::atomic<int64_t> g_test_skip_tile{-1};
+#endif
+
+// uint8 [rows, row_bytes] (packed E2M1 codes), boxes of 128 bytes x box_rows
+// rows with the 128-byte swizzle, zero fill outside the matrix.
+fp4q_status make_codes_map(CUtensorMap* map, const void* codes, int64_t rows, int64_t row_bytes,
+                           uint32_t box_rows) {
+    EncodeTiledFn enc;
+    fp4q_status st = encode_fn(&enc);
+    if (st != FP4Q_OK) return st;
+    cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {128u, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FP4Q_OK : FP4Q_ERR_CUDA;
 }
@@ -196,7 +217,10 @@ float had_norm(int n) { return n > 0 ? (float)(1.0 / std::sqrt((double)n)) : 1.0
 // kernels (sizes 16..128: one UMMA tile per block group; 256, 512: H_128 on
 // the tensor cores and the cross-group butterfly in the epilogue); other
 // shapes use the register-FWHT warp pipelines.
-bool use_mma(int had, int64_t K) { return had >= 16 && K % kMmaTile == 0; }
+#ifndef FP4Q_REGISTER_FWHT_MAX
+#define FP4Q_REGISTER_FWHT_MAX 0  // rotations up to this size take the register path on every K
+#endif
+bool use_mma(int had, int64_t K) { return had > FP4Q_REGISTER_FWHT_MAX && had >= 16 && K % kMmaTile == 0; }
 
 template <int FMT, int HAD, bool AMAX>
 fp4q_status launch_mma_t(const CUtensorMap& map, const MmaParams& p, int grid, cudaStream_t s) {
@@ -272,6 +296,9 @@ fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, in
     p.swizzled = layout == FP4Q_SCALES_SWIZZLED;
     p.dynamic = dynamic;
     p.had_norm = had_norm(had);
+#ifdef FP4Q_TEST_HOOKS
+    p.skip_tile = g_test_skip_tile.exchange(-1);
+#endif
 
     if (p.swizzled) {  // padding rows/columns of the tiled layout read as zero
         const int64_t ncols = K / B;
@@ -355,6 +382,14 @@ fp4q_status launch_dequant_h(int had, const DequantParams& p, int sms, cudaStrea
         default: return FP4Q_ERR_INVALID_ARG;
     }
 }
+
+// ---------------------------------------------------------------- ARC launch
+// One ARC kernel instantiation and its shared-memory size.
+template <int FMT, bool AMAX_ONLY>
+struct ArcKern {
+    static constexpr void (*fn)(const ArcParams) = arc_kernel<FMT, AMAX_ONLY>;
+    static int total(int64_t K, int64_t S, int warps) { return arc_layout<AMAX_ONLY>(K, S, warps).total; }
+};
 
 // ---------------------------------------------------------------- self-test kernel
 __global__ void selftest_div_kernel(const float* x, const float* d, int64_t n, float* qf,
@@ -483,25 +518,28 @@ FP4Q_API fp4q_status fp4q_hadamard_quantize(const void* x, int64_t M, int64_t K,
 
 FP4Q_API fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int64_t ldx,
                                        const void* gamma, float eps, const int32_t* perm,
-                                       const int32_t* outliers, int64_t S, uint8_t* codes,
-                                       uint8_t* scales, float* tensor_scale,
+                                       const int32_t* outliers, int64_t S, fp4q_format format,
+                                       uint8_t* codes, uint8_t* scales, float* tensor_scale,
                                        fp4q_tscale_mode mode, fp4q_scale_layout layout,
                                        void* workspace, size_t workspace_bytes,
                                        fp4q_stream_t stream) {
     fp4q_status st = check_x(x, M, K, ldx);
     if (st != FP4Q_OK) return st;
-    if (K % 16 != 0 || S < 0 || S % 16 != 0 || S > K) return FP4Q_ERR_INVALID_ARG;
+    if (format != FP4Q_NVFP4 && format != FP4Q_MXFP4) return FP4Q_ERR_INVALID_ARG;
+    const bool mx = format == FP4Q_MXFP4;
+    const int B = mx ? 32 : 16;
+    if (K % B != 0 || S < 0 || S % B != 0 || S > K) return FP4Q_ERR_INVALID_ARG;
     if (K > 16384) return FP4Q_ERR_UNSUPPORTED;
     if (!(eps >= 0.0f) || !std::isfinite(eps)) return FP4Q_ERR_INVALID_ARG;
-    if (mode != FP4Q_TSCALE_DYNAMIC && mode != FP4Q_TSCALE_STATIC) return FP4Q_ERR_INVALID_ARG;
+    if (!mx && mode != FP4Q_TSCALE_DYNAMIC && mode != FP4Q_TSCALE_STATIC) return FP4Q_ERR_INVALID_ARG;
     if (layout != FP4Q_SCALES_LINEAR && layout != FP4Q_SCALES_SWIZZLED) return FP4Q_ERR_INVALID_ARG;
     if (M == 0) return FP4Q_OK;
     if ((st = check_out(codes, scales)) != FP4Q_OK) return st;
-    if (!gamma || !perm || !tensor_scale || (S > 0 && !outliers)) return FP4Q_ERR_INVALID_ARG;
-    if (!aligned(gamma, 2) || !aligned(perm, 4) || !aligned(tensor_scale, 4) ||
+    if (!gamma || !perm || (!mx && !tensor_scale) || (S > 0 && !outliers)) return FP4Q_ERR_INVALID_ARG;
+    if (!aligned(gamma, 2) || !aligned(perm, 4) || (!mx && !aligned(tensor_scale, 4)) ||
         (S > 0 && !aligned(outliers, 4)))
         return FP4Q_ERR_ALIGNMENT;
-    const bool dynamic = mode == FP4Q_TSCALE_DYNAMIC;
+    const bool dynamic = !mx && mode == FP4Q_TSCALE_DYNAMIC;
     if (dynamic && (!workspace || workspace_bytes < FP4Q_WORKSPACE_BYTES)) return FP4Q_ERR_INVALID_ARG;
     if (dynamic && !aligned(workspace, 4)) return FP4Q_ERR_ALIGNMENT;
 
@@ -523,43 +561,42 @@ FP4Q_API fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int6
     p.partials = static_cast<float*>(workspace);
     p.swizzled = layout == FP4Q_SCALES_SWIZZLED;
     p.dynamic = dynamic;
-    // Warps per CTA (one row each) and row buffers per warp.  The kernel is
-    // bound by issue latency, not by the row copies: more warps beat a second
-    // buffer (K = 4096: 12 warps with one buffer run 8% faster than 11 with
-    // two), so two buffers are taken only where they cost no warp.
+    // Warps per CTA (a row pair each): as many as the shared memory holds, up
+    // to the kernel's launch bound.
     constexpr int kSmemMax = 227 * 1024;
-    auto max_warps = [&](int sr) {
-        for (int w = kArcMaxWarps; w >= 1; --w)  // the kernel's launch bound
-            if (arc_layout(K, S, w, sr).total <= kSmemMax) return w;
+    auto warps_for = [&](auto amax_only) -> int {
+        constexpr bool A = decltype(amax_only)::value;
+        for (int w = arc_max_warps<A>(); w >= 1; --w)
+            if (arc_layout<A>(K, S, w).total <= kSmemMax) return w;
         return 0;
     };
-    int SR = FP4Q_ARC_STAGES, W = max_warps(SR);
-    if (SR > 1 && max_warps(1) > W) {
-        SR = 1;
-        W = max_warps(1);
-    }
-    if (W == 0) return FP4Q_ERR_UNSUPPORTED;
-    p.warps = W;
-    p.stages = SR;
-    const int threads = 32 * W;
-    const int smem = arc_layout(K, S, W, SR).total;
-    const int grid = (int)std::min<int64_t>({(M + W - 1) / W, (int64_t)sms, (int64_t)kMaxGrid});
-    p.n_partials = grid;
+    const int W = warps_for(std::false_type{});
+    const int Wa = dynamic ? warps_for(std::true_type{}) : 1;
+    if (W == 0 || Wa == 0) return FP4Q_ERR_UNSUPPORTED;
+    const int64_t pairs = (M + 1) / 2;
     if (p.swizzled) {
-        const int64_t ncols = (K + S) / 16;
+        const int64_t ncols = (K + S) / B;
         const int64_t bytes = fp4q_scales_bytes(M, ncols, FP4Q_SCALES_SWIZZLED);
         if (bytes != M * ncols && cudaMemsetAsync(scales, 0, (size_t)bytes, (cudaStream_t)stream) != cudaSuccess)
             return FP4Q_ERR_CUDA;
     }
     // The shared-memory size depends on K and S, so the attribute is set on every call.
-    auto run = [&](auto kern) -> fp4q_status {
+    auto run = [&](auto kern, int warps) -> fp4q_status {
+        const int grid = (int)std::min<int64_t>({(pairs + warps - 1) / warps, (int64_t)sms, (int64_t)kMaxGrid});
+        p.warps = warps;
+        const int smem = decltype(kern)::total(K, S, warps);
         if (smem > 48 * 1024 &&
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            cudaFuncSetAttribute(kern.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return FP4Q_ERR_CUDA;
-        return launch(kern, grid, threads, smem, (cudaStream_t)stream, p);
+        return launch(kern.fn, grid, 32 * warps, smem, (cudaStream_t)stream, p);
     };
-    if (dynamic && (st = run(arc_kernel<true>)) != FP4Q_OK) return st;
-    return run(arc_kernel<false>);
+    if (dynamic) {
+        const int grid_a = (int)std::min<int64_t>({(pairs + Wa - 1) / Wa, (int64_t)sms, (int64_t)kMaxGrid});
+        if ((st = run(ArcKern<FMT_NVFP4, true>{}, Wa)) != FP4Q_OK) return st;
+        p.n_partials = grid_a;
+    }
+    if (mx) return run(ArcKern<FMT_MXFP4, false>{}, W);
+    return run(ArcKern<FMT_NVFP4, false>{}, W);
 }
 
 FP4Q_API fp4q_status fp4q_dequantize(fp4q_format format, const uint8_t* codes,
@@ -606,6 +643,47 @@ FP4Q_API fp4q_status fp4q_dequantize(fp4q_format format, const uint8_t* codes,
     }
 }
 
+FP4Q_API fp4q_status fp4q_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales,
+                                     const float* a_scale, const uint8_t* b_codes,
+                                     const uint8_t* b_scales, const float* b_scale, int64_t M,
+                                     int64_t N, int64_t K, void* d, int d_bf16, fp4q_stream_t stream) {
+    if (M < 0 || N <= 0 || K <= 0) return FP4Q_ERR_INVALID_ARG;
+    if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim) return FP4Q_ERR_UNSUPPORTED;
+    if (K % kGemmBK != 0 || N % kGemmBN != 0) return FP4Q_ERR_UNSUPPORTED;
+    if (d_bf16 != 0 && d_bf16 != 1) return FP4Q_ERR_INVALID_ARG;
+    if (M == 0) return FP4Q_OK;
+    if (!a_codes || !a_scales || !a_scale || !b_codes || !b_scales || !b_scale || !d)
+        return FP4Q_ERR_INVALID_ARG;
+    if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(a_scales, 16) || !aligned(b_scales, 16) ||
+        !aligned(a_scale, 4) || !aligned(b_scale, 4) || !aligned(d, 16))
+        return FP4Q_ERR_ALIGNMENT;
+    int sms = 0;
+    fp4q_status st;
+    if ((st = sm_count(&sms)) != FP4Q_OK) return st;
+    CUtensorMap map_a, map_b;
+    std::memset(&map_a, 0, sizeof(map_a));
+    std::memset(&map_b, 0, sizeof(map_b));
+    if ((st = make_codes_map(&map_a, a_codes, M, K / 2, kGemmBM)) != FP4Q_OK) return st;
+    if ((st = make_codes_map(&map_b, b_codes, N, K / 2, kGemmBN)) != FP4Q_OK) return st;
+    GemmParams p{};
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.a_sf = a_scales;
+    p.b_sf = b_scales;
+    p.a_scale = a_scale;
+    p.b_scale = b_scale;
+    p.d = d;
+    p.out_bf16 = d_bf16;
+    p.n_mt = (M + kGemmBM - 1) / kGemmBM;
+    p.n_tiles = p.n_mt * (N / kGemmBN);
+    p.sf_nc = K / 64;
+    static std::atomic<uint64_t> done{0};
+    if ((st = ensure_smem(gemm_nvfp4_kernel, kGemmSmem, done)) != FP4Q_OK) return st;
+    const int grid = (int)std::min<int64_t>({p.n_tiles, (int64_t)sms, (int64_t)kMaxGrid});
+    return launch(gemm_nvfp4_kernel, grid, kGemmThreads, kGemmSmem, (cudaStream_t)stream, map_a, map_b, p);
+}
+
 FP4Q_API const char* fp4q_status_string(fp4q_status status) {
     switch (status) {
         case FP4Q_OK: return "FP4Q_OK";
@@ -635,3 +713,10 @@ FP4Q_API fp4q_status fp4q_selftest_div(const float* x, const float* d, int64_t n
     selftest_div_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(x, d, n, q_fast, q_ieee);
     return launch_status();
 }
+
+#ifdef FP4Q_TEST_HOOKS
+// Test build only (not declared in include/fp4q.h): makes CTA 0 of the next
+// register-path quantizer launch skip issuing its tile number j, so that the
+// consumers' bounded wait for it runs out and the kernel takes its timeout path.
+FP4Q_API void fp4q_test_skip_tile(int64_t j) { g_test_skip_tile.store(j); }
+#endif

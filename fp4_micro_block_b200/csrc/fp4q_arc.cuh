@@ -1,25 +1,41 @@
 // fp4q_arc.cuh -- ARCQuant fused kernel for sm_100a: channel reorder + RMSNorm
-// + primary NVFP4 quantization + NVFP4 quantization of the residual of the
-// outlier channels, written as one [primary K | residual S] GEMM operand
-// (ARCQuant summary, "Methodologie" items 1-5).
+// + primary quantization + quantization of the residual of the outlier
+// channels, written as one [primary K | residual S] GEMM operand (ARCQuant
+// summary, "Methodologie" items 1-5), in NVFP4 or MXFP4 ("Generalisabilite":
+// the scheme carries over to MXFP4).
 //
-// One warp per row: a row never needs more than its own warp, so there is no
-// CTA-wide barrier on the path.  Each warp streams its rows through a private
-// ring of row buffers filled by 1-D bulk copies (lane 0 refills a buffer once
-// the warp's stores of that row, which consume every value read from it, have
-// issued).  Per row:
-//   1. sum of squares over the row in natural order (16-byte loads, shuffle
-//      reduction) -> rs = 1 / sqrt(mean + eps);
-//   2. lane l owns output blocks b = l, l + 32, ... (reordered positions
-//      16b..16b+15); for each pair of them it gathers x[perm[p]] from the row
-//      buffer, applies rs and gamma[perm[p]] and quantizes the two blocks as
-//      one unit (32 consecutive blocks per store instruction);
-//   3. at the outlier positions (a per-block bit mask) it forms the residual
-//      y - (E2M1val * E4M3val) * s_t into a per-warp buffer indexed by outlier
-//      slot; after a warp barrier, lanes quantize the S/16 residual blocks.
-// The CTA keeps perm and gamma as one 32-bit word per position (channel index
-// | bf16 gamma of that channel), the outlier bit mask per block and the slot of
-// every outlier position, built once per CTA.
+// One warp owns a PAIR of rows at a time: there is no CTA-wide barrier on the
+// path.  Each warp streams its row pairs through its own 4K-byte buffer, filled
+// by two 1-D bulk copies (row 0 in the first half, row 1 in the second).  Per
+// pair:
+//   1. natural order (conflict-free 16-byte reads of both rows): the sum of
+//      squares of each row, and one 32-bit word per channel holding the bf16 of
+//      row 0 (low half) and of row 1 (high half), written IN PLACE: lane l
+//      reads channels 8j..8j+7 of both rows (16 bytes at 16 j of each half)
+//      and writes their 8 words back to the same 32 bytes, channels 8j..8j+3
+//      into the first half and 8j+4..8j+7 into the second, so the word of
+//      channel c sits at 16 (c >> 3) + 4 (c & 3) + ((c >> 2) & 1) * 2K;
+//   2. reordered order: lane l owns the output blocks b = l, l + 32, ... (two
+//      at a time); one shared-memory load per position gathers that position's
+//      channel for both rows, a packed multiply applies -gamma of the channel,
+//      and the two rows' blocks are quantized side by side (NVFP4: one unit of
+//      two 16-blocks; MXFP4: one 32-block unit per row).  The RMS factor rs of
+//      each row is not applied per element: it scales the block maximum and
+//      the quotient multiplier of its row (the "fold" of the unit quantizers),
+//      so y = z * rs with z = x * gamma;
+//   3. at the outlier positions (a bit mask per 16-block) the residual
+//      y - dequant(primary) goes to a per-warp buffer in position order; after
+//      a warp barrier the lanes quantize the residual blocks (residual column j
+//      reads the slot of outlier j); then the buffer takes the next pair.
+// A warp waits for each pair's copies; the other warps of the SM (up to 12,
+// one buffer each) hide that latency.
+// Per CTA (built once): for every position q a 32-bit word (byte offset of the
+// word of channel perm[q] | bf16 gamma of that channel << 16), laid out so that
+// the 16-byte loads of 32 lanes (blocks b = lane + 32 i) are consecutive; per
+// 16-position group the outlier bit mask and the number of outlier positions
+// before the group; the slot of every residual column; the NVFP4 scale table
+// (d, RN(1/d)).  The amax pre-pass of the dynamic tensor scale streams the
+// rows in natural order through two buffers per warp.
 #pragma once
 
 #include "fp4q_quant.cuh"
@@ -27,9 +43,14 @@
 namespace fp4q {
 
 #ifndef FP4Q_ARC_MAX_WARPS
-#define FP4Q_ARC_MAX_WARPS 14
+#define FP4Q_ARC_MAX_WARPS 12
 #endif
-constexpr int kArcMaxWarps = FP4Q_ARC_MAX_WARPS;  // launch bound: rows in flight per SM
+// Launch bounds (warps per CTA, one CTA per SM): the quantizer keeps two
+// blocks of both rows in registers; the amax pre-pass is a light streaming loop.
+constexpr int kArcMaxWarps = FP4Q_ARC_MAX_WARPS;
+constexpr int kArcAmaxMaxWarps = 16;
+template <bool AMAX_ONLY>
+constexpr int arc_max_warps() { return AMAX_ONLY ? kArcAmaxMaxWarps : kArcMaxWarps; }
 
 struct ArcParams {
     int64_t M, K, S;
@@ -40,253 +61,486 @@ struct ArcParams {
     int64_t ldx_bytes;
     float eps;
     uint8_t* codes;           // [M, (K+S)/2]
-    uint8_t* scales;          // [M, (K+S)/16] or swizzled
-    float* tensor_scale;
+    uint8_t* scales;          // [M, (K+S)/B] or swizzled
+    float* tensor_scale;      // NVFP4 only
     float* partials;
     int n_partials;
     int swizzled;
     int dynamic;
-    int warps;                // warps per CTA (one row each at a time)
-    int stages;               // row buffers per warp
+    int warps;                // warps per CTA (one row pair each at a time)
 };
 
-// Shared-memory layout (byte offsets), all 16-byte aligned.
+// Shared-memory layout (byte offsets).  CTA part: tab (u32 [K]), om (u32 per
+// 16-position group), rslot (u16 [S]), red (f32 [32]), stab (float2 [128]);
+// then per warp: the pair buffer (2 rows of bf16, then the interleaved words;
+// the pre-pass: two stages of 2 rows), residuals (f32 [2][S]), mbarriers.
 struct ArcLayout {
-    int ring, pg, omask, oidx, rslot, res, bars, red, tab, total;
+    int tab, om, rslot, red, stab, warp0, warp_bytes, land, res, bar, total;
 };
 
-__host__ __device__ inline ArcLayout arc_layout(int64_t K, int64_t S, int warps, int stages) {
+__host__ __device__ inline int arc_al(int64_t v) { return (int)((v + 127) / 128 * 128); }
+
+template <bool AMAX_ONLY>
+__host__ __device__ inline ArcLayout arc_layout(int64_t K, int64_t S, int warps) {
     ArcLayout l;
-    const int row_bytes = (int)K * 2;
-    l.ring = 0;
-    l.pg = l.ring + warps * stages * row_bytes;                 // u32 [K]
-    l.omask = l.pg + (int)K * 4;                                // u32 [K/16]
-    l.oidx = l.omask + (int)((K / 16 * 4 + 15) / 16 * 16);      // i16 [K]
-    l.rslot = l.oidx + (int)((K * 2 + 15) / 16 * 16);           // i16 [S]
-    l.res = l.rslot + (int)((S * 2 + 15) / 16 * 16);            // f32 [warps][S]
-    l.bars = l.res + (int)((warps * S * 4 + 15) / 16 * 16);     // u64 [warps][stages]
-    l.red = l.bars + (warps * stages * 8 + 15) / 16 * 16;       // f32 [32]
-    l.tab = l.red + 128;                                        // float4 [128]
-    l.total = l.tab + 128 * 16 + 128;                           // + alignment slack
+    int off = 0;
+    l.tab = off;
+    off += AMAX_ONLY ? 0 : arc_al(K * 4);
+    l.om = off;
+    off += AMAX_ONLY ? 0 : arc_al((K / 16) * 4);
+    l.rslot = off;
+    off += AMAX_ONLY ? 0 : arc_al(S * 2);
+    l.red = off;
+    off += 128;
+    l.stab = off;
+    off += AMAX_ONLY ? 0 : 128 * 8;
+    l.warp0 = off;
+    const int stages = AMAX_ONLY ? 2 : 1;
+    int w = 0;
+    l.land = w;
+    w += arc_al(stages * 2 * K * 2);
+    l.res = w;
+    w += AMAX_ONLY ? 0 : arc_al(2 * S * 4);
+    l.bar = w;
+    w += 128;
+    l.warp_bytes = w;
+    l.total = off + warps * w + 128;  // + alignment slack of the dynamic buffer
     return l;
 }
 
-template <bool AMAX_ONLY>
-__global__ void __launch_bounds__(kArcMaxWarps * 32, 1) arc_kernel(const ArcParams p) {
+// Byte offset of the interleaved word of channel c in a pair buffer of K channels.
+__host__ __device__ inline uint32_t arc_word_off(uint32_t c, uint32_t K) {
+    return 16u * (c >> 3) + 4u * (c & 3u) + ((c >> 2) & 1u) * 2u * K;
+}
+
+// Packed f32x2 arithmetic (sm_100a).
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+// NVFP4 rule for the two blocks of a unit (component x: row 0, y: row 1) with a
+// fold per component: the unit holds -z and v = z * fold.  Scale bytes from
+// RN(RN(amax(v) * RN(1/6)) * RN(1/s)) and quotients z * RN(RN(1/d) * fold), as
+// in nvfp4_unit's table path.  stab[e] = (d, RN(1/d)) for the tensor scale s.
+__device__ __forceinline__ uint32_t arc_nvfp4_unit(const float2* n, float2 am, const ScaleCtx& c,
+                                                   const float2* stab, float2 fold, uint32_t (&w)[4]) {
+    am.x *= fold.x;
+    am.y *= fold.y;
+    const uint32_t b0 = __float_as_uint(am.x), b1 = __float_as_uint(am.y);
+    const uint32_t tiny = __float_as_uint(0x1p-90f);
+    const bool in_range = c.fast && (b0 - 1u) >= tiny - 1u && (b1 - 1u) >= tiny - 1u &&
+                          fmaxf(am.x, am.y) <= c.am_max;
+    if (!in_range) {
+        const uint32_t e0 = nvfp4_block_ieee<false>(n, am.x, c.s, fold.x, w[0], w[1]);
+        const uint32_t e1 = nvfp4_block_ieee<true>(n, am.y, c.s, fold.y, w[2], w[3]);
+        return e0 | (e1 << 8);
+    }
+    const float k6 = __uint_as_float(0x3e2aaaabu);  // RN(1/6)
+    const uint32_t e2 = e4m3x2_encode(make_float2((am.x * k6) * c.rs.rn, (am.y * k6) * c.rs.rn));
+    const float2 t0 = stab[e2 & 0xffu], t1 = stab[e2 >> 8];
+    const float2 m = make_float2(-(t0.y * fold.x), -(t1.y * fold.y));  // n holds -z
+    float q0[16], q1[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float2 q = fmul2(n[i], m);
+        q0[i] = q.x;
+        q1[i] = q.y;
+    }
+    w[0] = e2m1_pack8(q0);
+    w[1] = e2m1_pack8(q0 + 8);
+    w[2] = e2m1_pack8(q1);
+    w[3] = e2m1_pack8(q1 + 8);
+    if (t0.x == 0.0f) w[0] = w[1] = 0u;  // zero block scale: all codes +0
+    if (t1.x == 0.0f) w[2] = w[3] = 0u;
+    return e2;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    return __byte_perm(a, b, sel);
+}
+
+// Store one scale byte of (row, col).
+__device__ __forceinline__ void put_scale(const ArcParams& p, int64_t row, int64_t col, int64_t nsc,
+                                          int64_t nC, uint32_t byte) {
+    if (p.swizzled) p.scales[swizzle_offset(row, col, nC)] = (uint8_t)byte;
+    else p.scales[row * nsc + col] = (uint8_t)byte;
+}
+
+template <int FMT, bool AMAX_ONLY>
+__global__ void __launch_bounds__(arc_max_warps<AMAX_ONLY>() * 32, 1) arc_kernel(const ArcParams p) {
+    static_assert(FMT == FMT_NVFP4 || (FMT == FMT_MXFP4 && !AMAX_ONLY), "formats of the ARC path");
+    constexpr int B = FMT == FMT_MXFP4 ? 32 : 16;  // block size
+    constexpr int Q = B / 4;                       // 16-byte table quads per block
+    constexpr int SR = AMAX_ONLY ? 2 : 1;          // landing stages per warp
     pdl_wait();
     pdl_trigger();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                                ~uintptr_t(127));
-    const int K = (int)p.K, S = (int)p.S, nb = K / 16, W = p.warps, SR = p.stages;
-    const ArcLayout L = arc_layout(p.K, p.S, W, SR);
+    const int K = (int)p.K, S = (int)p.S, nbB = K / B, ng = K / 16, W = p.warps;
+    const ArcLayout L = arc_layout<AMAX_ONLY>(p.K, p.S, W);
     const uint32_t row_bytes = (uint32_t)K * 2u;
-    uint32_t* pg = reinterpret_cast<uint32_t*>(smem + L.pg);
-    uint32_t* omask = reinterpret_cast<uint32_t*>(smem + L.omask);
-    int16_t* oidx = reinterpret_cast<int16_t*>(smem + L.oidx);
-    int16_t* rslot = reinterpret_cast<int16_t*>(smem + L.rslot);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+    uint32_t* tab = reinterpret_cast<uint32_t*>(smem + L.tab);
+    uint32_t* om = reinterpret_cast<uint32_t*>(smem + L.om);
+    uint16_t* rslot = reinterpret_cast<uint16_t*>(smem + L.rslot);
     float* red = reinterpret_cast<float*>(smem + L.red);
-    float4* tab = reinterpret_cast<float4*>(smem + L.tab);
+    float2* stab = reinterpret_cast<float2*>(smem + L.stab);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nthreads = blockDim.x;
 
-    // ---- per-CTA tables
-    bool bad_index = false;
-    // pg: word of position q = 16b + 4k4 + t at index 4 (k4 nb + b) + t, so that
-    // the 16-byte loads of 32 lanes (blocks b = lane + 32i) are consecutive
-    for (int q = tid; q < K; q += nthreads) {
-        int c = p.perm[q];
-        if ((unsigned)c >= (unsigned)K) {  // not a channel: clamp, flag
-            bad_index = true;
-            c = 0;
-        }
-        const int b = q >> 4, k4 = (q >> 2) & 3, t = q & 3;
-        pg[4 * (k4 * nb + b) + t] = (uint32_t)c | ((uint32_t)p.gamma[c] << 16);
-        oidx[q] = -1;
+    // ---- this warp's buffer and barriers; its first pairs' copies overlap the
+    // building of the CTA tables below
+    uint8_t* const wb = smem + L.warp0 + (size_t)warp * L.warp_bytes;
+    uint64_t* const bars = reinterpret_cast<uint64_t*>(wb + L.bar);
+    const int64_t P = (p.M + 1) / 2;  // row pairs
+    const int64_t gw = (int64_t)blockIdx.x * W + warp, nw = (int64_t)gridDim.x * W;
+    const int64_t n_my = P > gw ? (P - 1 - gw) / nw + 1 : 0;
+    uint8_t* const land = wb + L.land;
+    auto issue = [&](int64_t i) {  // lane 0: pair i of this warp into stage i % SR
+        const int64_t r0 = 2 * (gw + i * nw);
+        const bool two = r0 + 1 < p.M;
+        const uint32_t bar = smem_u32(&bars[i % SR]);
+        uint8_t* dst = land + (i % SR) * 2 * row_bytes;
+        // the buffer was last written through the generic proxy (interleaved
+        // words): order those writes before the asynchronous copies
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(bar, two ? 2 * row_bytes : row_bytes);
+        bulk_load_1d(smem_u32(dst), p.x + r0 * p.ldx_bytes, row_bytes, bar);
+        if (two) bulk_load_1d(smem_u32(dst + row_bytes), p.x + (r0 + 1) * p.ldx_bytes, row_bytes, bar);
+    };
+    if (lane == 0) {
+        for (int k = 0; k < SR; ++k) mbar_init(smem_u32(&bars[k]), 1);
+        fence_barrier_init();
+        for (int64_t i = 0; i < min64(SR, n_my); ++i) issue(i);
     }
-    for (int b = tid; b < nb; b += nthreads) omask[b] = 0u;
-    if (tid < W * SR) mbar_init(smem_u32(&bars[tid]), 1);
-    __syncthreads();
-    for (int i = tid; i < S; i += nthreads) {  // slot of every outlier position
-        int q = p.outliers[i];
-        if ((unsigned)q >= (unsigned)K) {
-            bad_index = true;
-            q = 0;
-        }
-        oidx[q] = (int16_t)i;  // a position listed twice keeps one slot
-        atomicOr(&omask[q >> 4], 1u << (q & 15));
-    }
-    __syncthreads();
-    for (int i = tid; i < S; i += nthreads) {  // slot read by residual element i
-        const unsigned q = (unsigned)p.outliers[i];
-        rslot[i] = oidx[q < (unsigned)K ? q : 0u];
-    }
-    if (bad_index) atomicOr(&g_device_error, kErrBadIndex);
-    if (tid == 0) fence_barrier_init();
+    __syncwarp();
 
+    // ---- per-CTA tables
     float s_t = 0.0f;
     if constexpr (!AMAX_ONLY) {
-        if (p.dynamic) {
-            s_t = tensor_scale_from_partials(p.partials, p.n_partials, red);
-            if (blockIdx.x == 0 && tid == 0) *p.tensor_scale = s_t;
-        } else {
-            s_t = *p.tensor_scale;
+        bool bad_index = false;
+        // word of position q = B b + 4 k + t at index 4 (k nbB + b) + t; four
+        // positions per thread at a time, so that their loads overlap
+        for (int q0 = tid; q0 < K; q0 += 4 * nthreads) {
+            int c[4];
+            uint32_t g[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int q = q0 + u * nthreads;
+                c[u] = q < K ? __ldg(p.perm + q) : 0;
+                if ((unsigned)c[u] >= (unsigned)K) {  // not a channel: clamp, flag
+                    bad_index = true;
+                    c[u] = 0;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) g[u] = __ldg(p.gamma + c[u]);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int q = q0 + u * nthreads;
+                if (q >= K) continue;
+                const int b = q / B, k = (q % B) >> 2, t = q & 3;
+                tab[4 * (k * nbB + b) + t] = arc_word_off((uint32_t)c[u], (uint32_t)K) | (g[u] << 16);
+            }
         }
-        build_table(tab, s_t);
+        for (int g = tid; g < ng; g += nthreads) om[g] = 0u;
+        __syncthreads();
+        for (int i = tid; i < S; i += nthreads) {  // outlier bit of every listed position
+            int q = p.outliers[i];
+            if ((unsigned)q >= (unsigned)K) {
+                bad_index = true;
+                q = 0;
+            }
+            atomicOr(&om[q >> 4], 1u << (q & 15));
+        }
+        __syncthreads();
+        if (warp == 0) {  // outlier positions before each group: warp-wide exclusive scan
+            const int per = (ng + 31) / 32, g0 = lane * per;
+            int cnt = 0;
+            for (int g = g0; g < min(ng, g0 + per); ++g) cnt += __popc(om[g] & 0xffffu);
+            int inc = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += v;
+            }
+            int run = inc - cnt;
+            for (int g = g0; g < min(ng, g0 + per); ++g) {
+                const uint32_t m = om[g] & 0xffffu;
+                om[g] = m | ((uint32_t)run << 16);
+                run += __popc(m);
+            }
+        }
+        __syncthreads();
+        for (int i = tid; i < S; i += nthreads) {  // slot (position rank) of residual column i
+            const unsigned q0 = (unsigned)p.outliers[i], q = q0 < (unsigned)K ? q0 : 0u;
+            const uint32_t w = om[q >> 4];
+            rslot[i] = (uint16_t)((w >> 16) + __popc(w & ((1u << (q & 15)) - 1u)));
+        }
+        if (bad_index) atomicOr(&g_device_error, kErrBadIndex);
+        if constexpr (FMT == FMT_NVFP4) {
+            if (p.dynamic) {
+                s_t = tensor_scale_from_partials(p.partials, p.n_partials, red);
+                if (blockIdx.x == 0 && tid == 0) *p.tensor_scale = s_t;
+            } else {
+                s_t = *p.tensor_scale;
+            }
+            for (int e = tid; e < 128; e += nthreads) {
+                const float d = (e < 127) ? e4m3_decode((uint32_t)e) * s_t : 0.0f;
+                const bool ok = d >= 0x1p-100f && d <= 0x1p100f;
+                stab[e] = make_float2(d, ok ? __frcp_rn(d) : 0.0f);
+            }
+        }
     }
     __syncthreads();
 
     const ScaleCtx ctx = make_ctx(s_t);
-    const int64_t KS = p.K + p.S, kcs = KS / 2, nsc = KS / 16, nC = (nsc + 3) / 4;
-    const int64_t gw = (int64_t)blockIdx.x * W + warp, nw = (int64_t)gridDim.x * W;
-    const int64_t n_my = p.M > gw ? (p.M - 1 - gw) / nw + 1 : 0;
-    uint8_t* ring = smem + L.ring + (size_t)warp * SR * row_bytes;
-    uint64_t* wbars = bars + warp * SR;
-    float* res = reinterpret_cast<float*>(smem + L.res) + warp * S;
+    const int64_t KS = p.K + p.S, kcs = KS / 2, nsc = KS / B, nC = (nsc + 3) / 4;
+    float* const res = reinterpret_cast<float*>(wb + L.res);
     float my_amax = 0.0f;
 
-    auto issue = [&](int64_t i) {  // lane 0: row i of this warp into buffer i % SR
-        const int64_t row = gw + i * nw;
-        const uint32_t bar = smem_u32(&wbars[i % SR]);
-        mbar_arrive_expect_tx(bar, row_bytes);
-        bulk_load_1d(smem_u32(ring + (i % SR) * row_bytes), p.x + row * p.ldx_bytes, row_bytes, bar);
-    };
-    if (lane == 0)
-        for (int64_t i = 0; i < min64(SR, n_my); ++i) issue(i);
-
     for (int64_t i = 0; i < n_my; ++i) {
-        const bool ok = mbar_wait(smem_u32(&wbars[i % SR]), (uint32_t)((i / SR) & 1));
+        const bool ok = mbar_wait(smem_u32(&bars[i % SR]), (uint32_t)((i / SR) & 1));
         if (!__all_sync(0xffffffffu, ok)) {
             if (lane == 0) {
                 atomicOr(&g_device_error, kErrWaitTimeout);
                 for (int64_t k = i; k < min64(n_my, i + SR); ++k)
-                    (void)mbar_wait(smem_u32(&wbars[k % SR]), (uint32_t)((k / SR) & 1));
+                    (void)mbar_wait(smem_u32(&bars[k % SR]), (uint32_t)((k / SR) & 1));
             }
             break;
         }
-        const int64_t row = gw + i * nw;
-        const uint8_t* xr = ring + (i % SR) * row_bytes;
-        const uint16_t* xs = reinterpret_cast<const uint16_t*>(xr);
+        const int64_t r0 = 2 * (gw + i * nw);
+        const bool two = r0 + 1 < p.M;
+        uint8_t* const l0 = land + (i % SR) * 2 * row_bytes;
+        uint8_t* const l1 = l0 + row_bytes;
 
-        // 1. sum of squares (natural order) and the row's RMS factor
-        float ss = 0.0f;
-        for (int k = 8 * lane; k < K; k += 256) {
-            const uint4 q = *reinterpret_cast<const uint4*>(xr + 2 * k);
-            float a;
-            a = bf16lo(q.x); ss = fmaf(a, a, ss);
-            a = bf16hi(q.x); ss = fmaf(a, a, ss);
-            a = bf16lo(q.y); ss = fmaf(a, a, ss);
-            a = bf16hi(q.y); ss = fmaf(a, a, ss);
-            a = bf16lo(q.z); ss = fmaf(a, a, ss);
-            a = bf16hi(q.z); ss = fmaf(a, a, ss);
-            a = bf16lo(q.w); ss = fmaf(a, a, ss);
-            a = bf16hi(q.w); ss = fmaf(a, a, ss);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        const float rs = __frcp_rn(__fsqrt_rn(__fdiv_rn(ss, (float)K) + p.eps));
-
-        // 2. reorder + normalise + quantize, two blocks (b, b + 32) per unit;
-        // y is kept negated (unit pairs), -y = (x * rs) * (-gamma).
-        auto gather = [&](int b, float* ny) {
-            if (b >= nb) {
-#pragma unroll
-                for (int k = 0; k < 16; ++k) ny[k] = 0.0f;
-                return;
+        float2 ss = make_float2(0.0f, 0.0f), sq = make_float2(0.0f, 0.0f);
+        if constexpr (AMAX_ONLY) {
+            // natural order: sums of squares and max |x gamma| of both rows
+            float2 zmax = make_float2(0.0f, 0.0f);
+            for (int c = 4 * lane; c < K; c += 128) {
+                const uint2 a = *reinterpret_cast<const uint2*>(l0 + 2 * c);
+                const uint2 b = two ? *reinterpret_cast<const uint2*>(l1 + 2 * c) : make_uint2(0u, 0u);
+                const float2 v0 = make_float2(bf16lo(a.x), bf16lo(b.x)), v1 = make_float2(bf16hi(a.x), bf16hi(b.x));
+                const float2 v2 = make_float2(bf16lo(a.y), bf16lo(b.y)), v3 = make_float2(bf16hi(a.y), bf16hi(b.y));
+                ss = ffma2(v0, v0, ss);
+                sq = ffma2(v1, v1, sq);
+                ss = ffma2(v2, v2, ss);
+                sq = ffma2(v3, v3, sq);
+                // gamma in natural order (2-byte aligned: 16-bit loads)
+                const float g0 = bf16lo(__ldg(p.gamma + c)), g1 = bf16lo(__ldg(p.gamma + c + 1));
+                const float g2 = bf16lo(__ldg(p.gamma + c + 2)), g3 = bf16lo(__ldg(p.gamma + c + 3));
+                const float2 z0 = fmul2(v0, dup2(g0)), z1 = fmul2(v1, dup2(g1));
+                const float2 z2 = fmul2(v2, dup2(g2)), z3 = fmul2(v3, dup2(g3));
+                zmax.x = fmaxf(zmax.x, max3(fabsf(z0.x), fabsf(z1.x), fmaxf(fabsf(z2.x), fabsf(z3.x))));
+                zmax.y = fmaxf(zmax.y, max3(fabsf(z0.y), fabsf(z1.y), fmaxf(fabsf(z2.y), fabsf(z3.y))));
             }
+            ss = make_float2(ss.x + sq.x, ss.y + sq.y);
 #pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-                const uint4 w4 = *reinterpret_cast<const uint4*>(pg + 4 * (k4 * nb + b));
-                const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+            for (int o = 16; o > 0; o >>= 1) {
+                ss.x += __shfl_xor_sync(0xffffffffu, ss.x, o);
+                ss.y += __shfl_xor_sync(0xffffffffu, ss.y, o);
+                zmax.x = fmaxf(zmax.x, __shfl_xor_sync(0xffffffffu, zmax.x, o));
+                zmax.y = fmaxf(zmax.y, __shfl_xor_sync(0xffffffffu, zmax.y, o));
+            }
+            const float rK = (float)K;
+            const float2 rs = make_float2(__frcp_rn(__fsqrt_rn(__fdiv_rn(ss.x, rK) + p.eps)),
+                                          __frcp_rn(__fsqrt_rn(__fdiv_rn(ss.y, rK) + p.eps)));
+            // every value read from the stage is consumed above: refill it
+            __syncwarp();
+            if (lane == 0 && i + SR < n_my) issue(i + SR);
+            my_amax = fmaxf(my_amax, zmax.x * rs.x);
+            if (two) my_amax = fmaxf(my_amax, zmax.y * rs.y);
+        } else {
+            // 1. natural order, in place: sums of squares and the interleaved words
+#pragma unroll 2
+            for (int j = lane; 8 * j < K; j += 32) {
+                const uint4 a = *reinterpret_cast<const uint4*>(l0 + 16 * j);
+                const uint4 b = two ? *reinterpret_cast<const uint4*>(l1 + 16 * j) : make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const float xv = bf16lo(xs[wv[t] & 0xffffu]);
-                    const float g = __uint_as_float(wv[t] & 0xffff0000u);
-                    ny[4 * k4 + t] = (xv * rs) * -g;
+                for (int q = 0; q < 4; ++q) {
+                    const float2 lo = make_float2(bf16lo(av[q]), bf16lo(bv[q]));
+                    const float2 hi = make_float2(bf16hi(av[q]), bf16hi(bv[q]));
+                    ss = ffma2(lo, lo, ss);
+                    sq = ffma2(hi, hi, sq);
+                }
+                *reinterpret_cast<uint4*>(l0 + 16 * j) =
+                    make_uint4(prmt(a.x, b.x, 0x5410u), prmt(a.x, b.x, 0x7632u), prmt(a.y, b.y, 0x5410u),
+                               prmt(a.y, b.y, 0x7632u));
+                *reinterpret_cast<uint4*>(l1 + 16 * j) =
+                    make_uint4(prmt(a.z, b.z, 0x5410u), prmt(a.z, b.z, 0x7632u), prmt(a.w, b.w, 0x5410u),
+                               prmt(a.w, b.w, 0x7632u));
+            }
+            ss = make_float2(ss.x + sq.x, ss.y + sq.y);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                ss.x += __shfl_xor_sync(0xffffffffu, ss.x, o);
+                ss.y += __shfl_xor_sync(0xffffffffu, ss.y, o);
+            }
+            const float rK = (float)K;
+            const float2 rs = make_float2(__frcp_rn(__fsqrt_rn(__fdiv_rn(ss.x, rK) + p.eps)),
+                                          __frcp_rn(__fsqrt_rn(__fdiv_rn(ss.y, rK) + p.eps)));
+            __syncwarp();  // every lane's interleaved words are written
+
+            // 2. reordered positions: gather both rows, quantize, store
+            const int64_t r1 = r0 + 1;
+            uint8_t* cp0 = p.codes + r0 * kcs;
+            uint8_t* cp1 = p.codes + r1 * kcs;
+            // (-z row 0, -z row 1) of the B positions of block b
+            auto gather = [&](int b, float2* v) {
+#pragma unroll
+                for (int k = 0; k < Q; ++k) {
+                    const uint4 tw = *reinterpret_cast<const uint4*>(tab + 4 * (k * nbB + b));
+                    const uint32_t wv[4] = {tw.x, tw.y, tw.z, tw.w};
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const uint32_t xw = *reinterpret_cast<const uint32_t*>(l0 + (wv[t] & 0xffffu));
+                        const float ng_ = -__uint_as_float(wv[t] & 0xffff0000u);
+                        v[4 * k + t] = fmul2(make_float2(bf16lo(xw), bf16hi(xw)), dup2(ng_));
+                    }
+                }
+            };
+            // quantize + store block b of both rows, and its outlier residuals
+            auto emit = [&](int b, const float2* v) {
+                if constexpr (FMT == FMT_NVFP4) {
+                    uint32_t w[4];
+                    const uint32_t e2 = arc_nvfp4_unit(v, amax_pair(v), ctx, stab, rs, w);
+                    *reinterpret_cast<uint2*>(cp0 + 8 * b) = make_uint2(w[0], w[1]);
+                    put_scale(p, r0, b, nsc, nC, e2 & 0xffu);
+                    if (two) {
+                        *reinterpret_cast<uint2*>(cp1 + 8 * b) = make_uint2(w[2], w[3]);
+                        put_scale(p, r1, b, nsc, nC, e2 >> 8);
+                    }
+                    // 3. residuals of the outlier positions of the block
+                    const uint32_t o = om[b];
+                    if (o & 0xffffu) {
+                        const float es0 = e4m3_decode(e2 & 0xffu), es1 = e4m3_decode(e2 >> 8);
+#pragma unroll
+                        for (int k = 0; k < 16; k += 2) {
+                            const uint32_t m2 = (o >> k) & 3u;
+                            if (m2 == 0u) continue;
+                            const uint32_t sh = 4 * (k & 7);
+                            const float2 c0 = e2m1x2_decode((w[k >> 3] >> sh) & 0xffu);      // row 0, k, k+1
+                            const float2 c1 = e2m1x2_decode((w[2 + (k >> 3)] >> sh) & 0xffu);  // row 1
+                            const int base = (int)(o >> 16) + __popc(o & ((1u << k) - 1u));
+                            // residual y - (E2M1 value * E4M3 value) * s_t, y = z * rs
+                            if (m2 & 1u) {
+                                res[base] = -v[k].x * rs.x - (c0.x * es0) * s_t;
+                                res[S + base] = -v[k].y * rs.y - (c1.x * es1) * s_t;
+                            }
+                            if (m2 & 2u) {
+                                const int s1 = base + (int)(m2 & 1u);
+                                res[s1] = -v[k + 1].x * rs.x - (c0.y * es0) * s_t;
+                                res[S + s1] = -v[k + 1].y * rs.y - (c1.y * es1) * s_t;
+                            }
+                        }
+                    }
+                } else {  // MXFP4: one 32-block unit per row
+                    float2 u0[16], u1[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        u0[k] = make_float2(v[k].x, v[16 + k].x);
+                        u1[k] = make_float2(v[k].y, v[16 + k].y);
+                    }
+                    uint32_t w0[4], w1[4];
+                    const uint32_t e0 = mxfp4_unit(u0, rs.x, w0);
+                    const uint32_t e1 = mxfp4_unit(u1, rs.y, w1);
+                    *reinterpret_cast<uint4*>(cp0 + 16 * b) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+                    put_scale(p, r0, b, nsc, nC, e0);
+                    if (two) {
+                        *reinterpret_cast<uint4*>(cp1 + 16 * b) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+                        put_scale(p, r1, b, nsc, nC, e1);
+                    }
+                    const uint32_t oa = om[2 * b], ob = om[2 * b + 1];
+                    if ((oa | ob) & 0xffffu) {
+                        const float es0 = e0 ? __uint_as_float(e0 << 23) : __uint_as_float(0x00400000u);
+                        const float es1 = e1 ? __uint_as_float(e1 << 23) : __uint_as_float(0x00400000u);
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t o = h ? ob : oa;
+#pragma unroll
+                            for (int k = 0; k < 16; k += 2) {
+                                const uint32_t m2 = (o >> k) & 3u;
+                                if (m2 == 0u) continue;
+                                const int kk = 16 * h + k;  // position within the block
+                                const uint32_t sh = 4 * (kk & 7);
+                                const float2 c0 = e2m1x2_decode((w0[kk >> 3] >> sh) & 0xffu);
+                                const float2 c1 = e2m1x2_decode((w1[kk >> 3] >> sh) & 0xffu);
+                                const int base = (int)(o >> 16) + __popc(o & ((1u << k) - 1u));
+                                if (m2 & 1u) {
+                                    res[base] = -v[kk].x * rs.x - c0.x * es0;
+                                    res[S + base] = -v[kk].y * rs.y - c1.x * es1;
+                                }
+                                if (m2 & 2u) {
+                                    const int s1 = base + (int)(m2 & 1u);
+                                    res[s1] = -v[kk + 1].x * rs.x - c0.y * es0;
+                                    res[S + s1] = -v[kk + 1].y * rs.y - c1.y * es1;
+                                }
+                            }
+                        }
+                    }
+                }
+            };
+            if constexpr (FMT == FMT_NVFP4) {
+                // two blocks per step (their gathers in flight together)
+                for (int b = lane; b < nbB; b += 64) {
+                    float2 va[B], vb[B];
+                    const bool second = b + 32 < nbB;
+                    gather(b, va);
+                    if (second) gather(b + 32, vb);
+                    emit(b, va);
+                    if (second) emit(b + 32, vb);
+                }
+            } else {  // a 32-block already has 32 gathers in flight
+                for (int b = lane; b < nbB; b += 32) {
+                    float2 va[B];
+                    gather(b, va);
+                    emit(b, va);
                 }
             }
-        };
-        for (int b0 = lane; b0 < nb; b0 += 64) {
-            const int b1 = b0 + 32;
-            float2 n[16];
-            {
-                float y0[16], y1[16];
-                gather(b0, y0);
-                gather(b1, y1);
+            __syncwarp();
+            // residual blocks: slots of columns B j .. B j + B - 1 -> columns K + B j
+            for (int j = lane; B * j < S; j += 32) {
+                const int64_t col = nbB + j;
+                if constexpr (FMT == FMT_NVFP4) {
+                    float2 n[16];
 #pragma unroll
-                for (int k = 0; k < 16; ++k) n[k] = make_float2(y0[k], y1[k]);
-            }
-            const float2 am = amax_pair(n);
-            if constexpr (AMAX_ONLY) {
-                my_amax = fmaxf(my_amax, b1 < nb ? fmaxf(am.x, am.y) : am.x);
-                pin(my_amax);
-                continue;
-            } else {
-                uint32_t w[4];
-                const uint32_t e2 = nvfp4_unit<true, false>(n, am, ctx, tab, 1.0f, w);
-                uint8_t* cp = p.codes + row * kcs;
-                *reinterpret_cast<uint2*>(cp + 8 * b0) = make_uint2(w[0], w[1]);
-                if (b1 < nb) *reinterpret_cast<uint2*>(cp + 8 * b1) = make_uint2(w[2], w[3]);
-                if (p.swizzled) {
-                    p.scales[swizzle_offset(row, b0, nC)] = (uint8_t)(e2 & 0xffu);
-                    if (b1 < nb) p.scales[swizzle_offset(row, b1, nC)] = (uint8_t)(e2 >> 8);
+                    for (int k = 0; k < 16; ++k) {
+                        const int sl = rslot[16 * j + k];
+                        n[k] = make_float2(-res[sl], -res[S + sl]);
+                    }
+                    uint32_t w[4];
+                    const uint32_t e2 = arc_nvfp4_unit(n, amax_pair(n), ctx, stab, make_float2(1.0f, 1.0f), w);
+                    *reinterpret_cast<uint2*>(cp0 + p.K / 2 + 8 * j) = make_uint2(w[0], w[1]);
+                    put_scale(p, r0, col, nsc, nC, e2 & 0xffu);
+                    if (two) {
+                        *reinterpret_cast<uint2*>(cp1 + p.K / 2 + 8 * j) = make_uint2(w[2], w[3]);
+                        put_scale(p, r1, col, nsc, nC, e2 >> 8);
+                    }
                 } else {
-                    p.scales[row * nsc + b0] = (uint8_t)(e2 & 0xffu);
-                    if (b1 < nb) p.scales[row * nsc + b1] = (uint8_t)(e2 >> 8);
-                }
-                // 3. residuals of the outlier positions of the two blocks
+                    float2 u0[16], u1[16];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int b = h ? b1 : b0;
-                    if (b >= nb) continue;
-                    const uint32_t m = omask[b];
-                    if (m == 0u) continue;
-                    const float es = e4m3_decode(h ? (e2 >> 8) : (e2 & 0xffu));
-#pragma unroll
-                    for (int k = 0; k < 16; k += 2) {
-                        // two codes (one byte), E2M1 values, dequantized primary
-                        const uint32_t byte = (w[2 * h + (k >> 3)] >> (4 * (k & 7))) & 0xffu;
-                        const float2 cv = e2m1x2_decode(byte);
-                        const float y0 = -(h ? n[k].y : n[k].x), y1 = -(h ? n[k + 1].y : n[k + 1].x);
-                        if (m & (1u << k)) res[max(0, (int)oidx[16 * b + k])] = y0 - (cv.x * es) * s_t;
-                        if (m & (2u << k)) res[max(0, (int)oidx[16 * b + k + 1])] = y1 - (cv.y * es) * s_t;
+                    for (int k = 0; k < 16; ++k) {
+                        const int sa = rslot[32 * j + k], sb = rslot[32 * j + 16 + k];
+                        u0[k] = make_float2(-res[sa], -res[sb]);
+                        u1[k] = make_float2(-res[S + sa], -res[S + sb]);
+                    }
+                    uint32_t w0[4], w1[4];
+                    const uint32_t e0 = mxfp4_unit(u0, 1.0f, w0);
+                    const uint32_t e1 = mxfp4_unit(u1, 1.0f, w1);
+                    *reinterpret_cast<uint4*>(cp0 + p.K / 2 + 16 * j) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+                    put_scale(p, r0, col, nsc, nC, e0);
+                    if (two) {
+                        *reinterpret_cast<uint4*>(cp1 + p.K / 2 + 16 * j) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+                        put_scale(p, r1, col, nsc, nC, e1);
                     }
                 }
             }
-        }
-        if constexpr (!AMAX_ONLY) {
+            // Every value read from the buffer (the gathers) and from the
+            // residual slots has been consumed by the stores above: the buffer
+            // takes the next pair.
             __syncwarp();
-            // residual blocks: slots 16j..16j+15 -> columns K + 16j
-            for (int j0 = lane; 16 * j0 < S; j0 += 64) {
-                const int j1 = j0 + 32;
-                const bool has1 = 16 * j1 < S;
-                float2 n[16];
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const float r0 = res[rslot[16 * j0 + k]];
-                    const float r1 = has1 ? res[rslot[16 * j1 + k]] : 0.0f;
-                    n[k] = make_float2(-r0, -r1);
-                }
-                uint32_t w[4];
-                const uint32_t e2 = nvfp4_unit<true, false>(n, amax_pair(n), ctx, tab, 1.0f, w);
-                uint8_t* cp = p.codes + row * kcs + p.K / 2;
-                *reinterpret_cast<uint2*>(cp + 8 * j0) = make_uint2(w[0], w[1]);
-                if (has1) *reinterpret_cast<uint2*>(cp + 8 * j1) = make_uint2(w[2], w[3]);
-                const int64_t c0 = nb + j0, c1 = nb + j1;
-                if (p.swizzled) {
-                    p.scales[swizzle_offset(row, c0, nC)] = (uint8_t)(e2 & 0xffu);
-                    if (has1) p.scales[swizzle_offset(row, c1, nC)] = (uint8_t)(e2 >> 8);
-                } else {
-                    p.scales[row * nsc + c0] = (uint8_t)(e2 & 0xffu);
-                    if (has1) p.scales[row * nsc + c1] = (uint8_t)(e2 >> 8);
-                }
-            }
+            if (lane == 0 && i + SR < n_my) issue(i + SR);
         }
-        // Every value read from the row buffer is consumed by the stores (or
-        // the maximum) above, which issue before the refill below; the residual
-        // buffer is rewritten for the next row only after this warp barrier.
-        __syncwarp();
-        if (lane == 0 && i + SR < n_my) issue(i + SR);
     }
 
     if constexpr (AMAX_ONLY) {

@@ -25,7 +25,13 @@ constexpr unsigned int kErrWaitTimeout = 1u;
 constexpr unsigned int kErrBadIndex = 2u;  // a channel / outlier index outside [0, K)
 // Upper bound of try_wait polls before a wait gives up (each poll may suspend
 // the thread for a short, hardware-chosen time).  Far above any real latency.
+// The test build (FP4Q_TEST_HOOKS) cuts it short so that a test can make a
+// wait run out quickly.
+#ifdef FP4Q_TEST_HOOKS
+constexpr uint32_t kWaitPolls = 1u << 14;
+#else
 constexpr uint32_t kWaitPolls = 1u << 22;
+#endif
 
 // ------------------------------------------------------------------------------
 // Format conversions

@@ -55,6 +55,9 @@ struct QuantParams {
     int swizzled;               // scale layout
     int dynamic;                // NVFP4: 1 = tensor scale from partials, 0 = read *scale_fp32
     float had_norm;             // RN(1/sqrt(n)), 1 without rotation
+#ifdef FP4Q_TEST_HOOKS
+    int64_t skip_tile;          // test build: CTA 0 never issues its tile of this index
+#endif
 };
 
 template <int FMT, int HAD>
@@ -173,6 +176,10 @@ __global__ void __launch_bounds__(QGeo<FMT, HAD>::threads, kQCtas)
                     break;
                 }
                 const int64_t t = blockIdx.x + j * gridDim.x;
+#ifdef FP4Q_TEST_HOOKS
+                // a tile that never arrives: its consumers' wait runs out
+                if (blockIdx.x == 0 && j == p.skip_tile) continue;
+#endif
                 const int32_t x0 = (int32_t)((t % p.n_cs) * G::tc), y0 = (int32_t)((t / p.n_cs) * kQBoxRows);
                 const uint32_t dst = smem_u32(smem + s * G::stage_bytes);
                 mbar_arrive_expect_tx(full0 + 8 * s, G::stage_bytes);

@@ -178,14 +178,17 @@ fp4q_status fp4q_hadamard_quantize(const void* x, int64_t M, int64_t K, int64_t 
                                    void* workspace, size_t workspace_bytes,
                                    fp4q_stream_t stream);
 
-/* fp4q_arc_quantize -- ARCQuant fused reorder + RMSNorm + primary NVFP4 +
- * residual NVFP4 of the outlier channels.
+/* fp4q_arc_quantize -- ARCQuant fused reorder + RMSNorm + primary quantization
+ * + residual quantization of the outlier channels, in NVFP4 or MXFP4.
  *   For each row: y[p] = x[perm[p]] / sqrt(mean_k x[k]^2 + eps) * gamma[perm[p]]
- *   (p = 0..K-1), primary = NVFP4(y) with tensor scale s_t; for j < S, the
- *   residual res[j] = y[outliers[j]] - dq(outliers[j]) with
- *   dq = (E2M1 value * E4M3 value) * s_t, quantized NVFP4 with the same s_t.
+ *   (p = 0..K-1), primary = Q(y); for j < S, the residual
+ *   res[j] = y[outliers[j]] - dq(outliers[j]), quantized in the same format.
+ *     FP4Q_NVFP4: blocks of 16, E4M3 scales, one tensor scale s_t for both
+ *       halves; dq = (E2M1 value * E4M3 value) * s_t.
+ *     FP4Q_MXFP4: blocks of 32, E8M0 scales; dq = E2M1 value * 2^(b - 127).
+ *       tensor_scale, mode and workspace are unused (may be NULL / 0).
  *   Output row = [primary K columns | residual S columns]:
- *   codes uint8 [M, (K+S)/2], scales [M, (K+S)/16] (or swizzled).
+ *   codes uint8 [M, (K+S)/2], scales [M, (K+S)/B] (or swizzled).
  *   gamma     bf16 [K], indexed by ORIGINAL channel.
  *   perm      int32 [K], perm[p] = original channel placed at position p
  *             (a permutation of 0..K-1; entries outside [0, K) are replaced
@@ -194,16 +197,19 @@ fp4q_status fp4q_hadamard_quantize(const void* x, int64_t M, int64_t K, int64_t 
  *             out-of-range handling as perm); the
  *             calibrated choice is 0..S-1 (channels sorted by descending
  *             calibration absmax).  May be NULL when S == 0.
- *   tensor_scale / mode / workspace as for fp4q_quantize_nvfp4; DYNAMIC uses the
- *   amax of y.
- * Requires K % 16 == 0, S % 16 == 0, 0 <= S <= K, K <= 16384, eps >= 0.
+ *   tensor_scale / mode / workspace as for fp4q_quantize_nvfp4 (NVFP4 only);
+ *   DYNAMIC uses the amax of y.
+ * Requires K % B == 0, S % B == 0, 0 <= S <= K, K <= 16384, eps >= 0, and that
+ * one warp's buffers fit in shared memory (12 K + 8 S bytes plus the CTA's
+ * 4 K + S/8 + 1.3 KiB, within 227 KiB), else FP4Q_ERR_UNSUPPORTED.
  * Defined by: ARCQuant summary, "Methodologie" items 1 (reorder by absolute
  * maximum, subset S), 2 (two-stage quantization), 3 (residual channels
  * concatenated along K) and 5 (one fused kernel: reorder, RMSNorm, primary and
- * residual quantization, GEMM-ready channel layout). */
+ * residual quantization, GEMM-ready channel layout); "Generalisabilite" (the
+ * scheme extends to MXFP4). */
 fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int64_t ldx,
                               const void* gamma, float eps, const int32_t* perm,
-                              const int32_t* outliers, int64_t S,
+                              const int32_t* outliers, int64_t S, fp4q_format format,
                               uint8_t* codes, uint8_t* scales, float* tensor_scale,
                               fp4q_tscale_mode mode, fp4q_scale_layout layout,
                               void* workspace, size_t workspace_bytes,
@@ -225,6 +231,28 @@ fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int64_t ldx,
 fp4q_status fp4q_dequantize(fp4q_format format, const uint8_t* codes, const uint8_t* scales,
                             const float* scale_fp32, int64_t M, int64_t K,
                             fp4q_scale_layout layout, int inv_had_size, void* y,
+                            fp4q_stream_t stream);
+
+/* fp4q_gemm_nvfp4 -- the consumer of NVFP4 activations: a block-scaled GEMM on
+ * the tensor cores,
+ *   D[m, n] = a_scale * b_scale *
+ *             sum_k (E2M1(A[m,k]) * E4M3(SA[m,k/16])) * (E2M1(B[n,k]) * E4M3(SB[n,k/16]))
+ * with the products accumulated in FP32.
+ *   a_codes   uint8 [M, K/2], a_scales the SWIZZLED scale buffer of A (as
+ *             fp4q_quantize_nvfp4 / fp4q_arc_quantize write it), a_scale 1 float.
+ *   b_codes   uint8 [N, K/2], b_scales SWIZZLED, b_scale 1 float (the weights,
+ *             quantized the same way).
+ *   d         [M, N] row-major, FP32 (d_bf16 = 0) or bf16 rounded to nearest
+ *             even (d_bf16 = 1).   (written)
+ * Requires K % 256 == 0 and N % 256 == 0 (else FP4Q_ERR_UNSUPPORTED); any M;
+ * 16-byte aligned codes, scales and d.  The ARCQuant operand is consumed with
+ * K + S in place of K against weights [W | W_S].
+ * Defined by: ARCQuant summary, "Methodologie" items 3-4 (one GEMM over the
+ * augmented reduction dimension K + S, the residual channels concatenated
+ * along K) and MR-GPTQ abstract (kernels consuming NVFP4 activations on B200). */
+fp4q_status fp4q_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_scale,
+                            const uint8_t* b_codes, const uint8_t* b_scales, const float* b_scale,
+                            int64_t M, int64_t N, int64_t K, void* d, int d_bf16,
                             fp4q_stream_t stream);
 
 /* Human-readable name of a status code (static string, never NULL). */

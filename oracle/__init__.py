@@ -350,3 +350,25 @@ def dequantize(fmt: str, codes, scales, scale=None, inv_had: int = 0) -> np.ndar
 
 def dequantize_bf16(fmt: str, codes, scales, scale=None, inv_had: int = 0) -> np.ndarray:
     return f32_to_bf16(dequantize(fmt, codes, scales, scale, inv_had))
+
+
+# --------------------------------------------------------------------------- consumer GEMM
+
+def nvfp4_block_values(codes, scales) -> np.ndarray:
+    """E2M1 value * E4M3 block-scale value of every element (float64, exact)."""
+    codes = np.ascontiguousarray(codes, np.uint8)
+    K = codes.shape[1] * 2
+    v = e2m1_decode(unpack_codes(codes)).astype(np.float64)
+    return v * np.repeat(e4m3_decode(scales).astype(np.float64), 16, axis=1)[:, :K]
+
+
+def nvfp4_gemm(a_codes, a_scales, s_a, b_codes, b_scales, s_b):
+    """The block-scaled NVFP4 GEMM a consumer runs on the quantized operands
+    (ARCQuant summary, Methodologie items 3-4: one GEMM over the augmented K):
+    D = s_a s_b (A B^T) with A, B the E2M1 * E4M3 values, in float64 (each
+    product is exact; the float64 sum errs by at most 2^-53 of the sum of the
+    magnitudes).  Returns (D, the same product of the magnitudes |A| |B|^T)."""
+    A = nvfp4_block_values(a_codes, a_scales)
+    B = nvfp4_block_values(b_codes, b_scales)
+    s = float(s_a) * float(s_b)
+    return (A @ B.T) * s, (np.abs(A) @ np.abs(B).T) * s

@@ -132,6 +132,37 @@ def add_counts(a: dict | None, b: dict) -> dict:
     return dict(b) if a is None else {k: a[k] + b[k] for k in a}
 
 
+def arc_counts(fmt: str, K: int, outl, gpu, orc_primary, y_orc: np.ndarray, name: str = "") -> dict:
+    """Tolerance counts of an ARCQuant output row block [primary K | residual S].
+
+    The primary columns are compared with the oracle's quantization of y.  The
+    residual columns are compared with the oracle's quantization of the
+    residual of the kernel's OWN primary codes, r = y - dq(primary), since the
+    residual is defined against the primary value actually produced (ARCQuant
+    summary, Methodologie item 2); a primary code one step off (allowed by the
+    rule) would otherwise shift its residual by a whole primary step.
+    gpu = (codes [M, (K+S)/2], linear scales [M, (K+S)/B], s_t or None);
+    orc_primary = (codes [M, K/2], scales [M, K/B], s_t or None)."""
+    cg, sg, fg = gpu
+    co, so, fo = orc_primary
+    B = 32 if fmt == "mxfp4" else 16
+    c = tolerant_counts(fmt, K, (cg[:, :K // 2], sg[:, :K // B], fg), (co, so, fo), y_orc, name)
+    S = len(outl)
+    if S == 0:
+        return c
+    if fmt == "mxfp4":
+        dq = oracle.mxfp4_dequantize(cg[:, :K // 2], sg[:, :K // B])
+    else:
+        dq = oracle.nvfp4_dequantize(cg[:, :K // 2], sg[:, :K // B], float(np.asarray(fg).reshape(-1)[0]))
+    r = (np.asarray(y_orc, np.float32)[:, outl] - dq[:, outl]).astype(np.float32)
+    if fmt == "mxfp4":
+        cr, sr = oracle.mxfp4_quantize(r)
+    else:
+        cr, sr = oracle.nvfp4_quantize(r, fo)
+    c2 = tolerant_counts(fmt, S, (cg[:, K // 2:], sg[:, K // B:], fg), (cr, sr, fo), r, name + "-residual")
+    return add_counts(c, c2)
+
+
 def _bf16_boundary_distance(w: np.ndarray) -> np.ndarray:
     """Distance (float64) from each fp32 value to the nearest bf16 rounding
     boundary: the midpoints between |w|'s two bf16 neighbours and between the

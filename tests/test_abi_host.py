@@ -107,14 +107,19 @@ def test_arc_validation(fq):
     L = fq.lib()
     a = L.fp4q_arc_quantize
     P, O, G = 0x60000, 0x70000, 0x80000
-    assert a(X, 4, 128, 128, G, 1e-6, P, O, 24, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
-    assert a(X, 4, 128, 128, G, 1e-6, P, O, 144, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
-    assert a(X, 4, 32768, 32768, G, 1e-6, P, O, 16, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_UNSUPPORTED
-    assert a(X, 4, 128, 128, G, -1.0, P, O, 16, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
-    assert a(X, 4, 128, 128, None, 1e-6, P, O, 16, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
-    assert a(X, 4, 128, 128, G, 1e-6, P, None, 16, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
-    assert a(X, 4, 128, 128, G, 1e-6, P, O, 16, CODES, SCALES, SF, 0, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
-    assert a(X, 4, 128, 128, G + 1, 1e-6, P, O, 16, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_ALIGNMENT
+    assert a(X, 4, 128, 128, G, 1e-6, P, O, 24, 0, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert a(X, 4, 128, 128, G, 1e-6, P, O, 144, 0, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert a(X, 4, 32768, 32768, G, 1e-6, P, O, 16, 0, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_UNSUPPORTED
+    assert a(X, 4, 128, 128, G, -1.0, P, O, 16, 0, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert a(X, 4, 128, 128, None, 1e-6, P, O, 16, 0, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert a(X, 4, 128, 128, G, 1e-6, P, None, 16, 0, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert a(X, 4, 128, 128, G, 1e-6, P, O, 16, 0, CODES, SCALES, SF, 0, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert a(X, 4, 128, 128, G + 1, 1e-6, P, O, 16, 0, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_ALIGNMENT
+    # format: NVFP4 or MXFP4 only; MXFP4 needs S and K multiples of 32, no tensor scale
+    assert a(X, 4, 128, 128, G, 1e-6, P, O, 16, 2, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert a(X, 4, 128, 128, G, 1e-6, P, O, 16, 1, CODES, SCALES, None, 0, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert a(X, 4, 144, 144, G, 1e-6, P, O, 32, 1, CODES, SCALES, None, 0, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert a(X, 0, 128, 128, G, 1e-6, P, O, 32, 1, CODES, SCALES, None, 0, 0, None, 0, None) == fq.FP4Q_OK
 
 
 def test_dequantize_validation(fq):

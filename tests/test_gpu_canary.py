@@ -138,28 +138,41 @@ def test_canary_hadamard_quantize(fq, M, case, layout):
         _same("fp32 scales", sf.t, f)
 
 
+ARC_CASES = [  # (format name, K, S)
+    ("nvfp4", 1040, 16), ("nvfp4", 1056, 32), ("nvfp4", 1088, 64), ("nvfp4", 1152, 0),
+    ("mxfp4", 1056, 32), ("mxfp4", 1088, 64), ("mxfp4", 1152, 0),
+]
+
+
 @pytest.mark.parametrize("M", MS)
-@pytest.mark.parametrize("K,S", [(1040, 16), (1056, 32), (1088, 64), (1152, 0)])
+@pytest.mark.parametrize("case", ARC_CASES, ids=lambda c: f"{c[0]}-K{c[1]}-S{c[2]}")
 @pytest.mark.parametrize("layout", [0, 1])
 @pytest.mark.parametrize("mode", [0, 1])
-def test_canary_arc(fq, M, K, S, layout, mode):
+def test_canary_arc(fq, M, case, layout, mode):
+    fmt_name, K, S = case
+    mx = fmt_name == "mxfp4"
+    if mx and mode == 1:
+        pytest.skip("MXFP4 has no tensor-scale mode")
+    fmt = fq.FP4Q_MXFP4 if mx else fq.FP4Q_NVFP4
     x_bits, gamma, perm, outl = workloads.arc_activations(M, K, seed=M + K, S=S, calib_rows=64)
     x = bits_to_torch_cuda(x_bits)
     g = bits_to_torch_cuda(gamma)
     p = torch.from_numpy(perm).cuda()
     o = torch.from_numpy(outl).cuda() if S else None
     fill = torch.tensor([0.01], device="cuda")
-    codes, scales, sf = _outs(fq, M, (K + S) // 2, (K + S) // 16, layout, (1,), fill)
+    B = 32 if mx else 16
+    codes, scales, sf = _outs(fq, M, (K + S) // 2, (K + S) // B, layout, None if mx else (1,), fill)
     ws = Guarded((fq.FP4Q_WORKSPACE_BYTES,), torch.uint8)
-    fq.fp4q_arc_quantize(x, g, 1e-6, p, o, codes.t, scales.t, sf.t, mode, layout,
-                         ws.t if mode == 0 else None)
+    fq.fp4q_arc_quantize(x, g, 1e-6, p, o, fmt, codes.t, scales.t, None if mx else sf.t, mode, layout,
+                         ws.t if mode == 0 and not mx else None)
     torch.cuda.synchronize()
-    _check_all(f"arc M{M} K{K} S{S}", codes, scales, sf, ws)
-    c, s, f = fq.arc_quantize(x, g, p, o, 1e-6, fill if mode == 1 else None, layout)
+    _check_all(f"arc {fmt_name} M{M} K{K} S{S}", codes, scales, sf, ws)
+    c, s, f = fq.arc_quantize(x, g, p, o, 1e-6, fill if mode == 1 else None, layout, fmt=fmt)
     torch.cuda.synchronize()
     _same("codes", codes.t, c)
     _same("scales", scales.t, s)
-    _same("tensor scale", sf.t, f)
+    if not mx:
+        _same("tensor scale", sf.t, f)
 
 
 DQ_CASES = [  # (format name, n, K)

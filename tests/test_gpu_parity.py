@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import workloads
-from parity import (add_counts, assert_bitexact, assert_roundtrip, assert_tolerant, bf16_torch_to_bits,
+from parity import (add_counts, arc_counts, assert_bitexact, assert_roundtrip, assert_tolerant, bf16_torch_to_bits,
                     bits_to_torch_cuda, block_l2_identity, check_fractions, to_np,
                     tolerant_counts, unswizzle)
 
@@ -362,12 +362,9 @@ def test_arc_tolerance(fq, shape, layout):
     c_o, s_o, sc_o, y_o = oracle.arc(x_bits, gamma, perm, outl)
     assert abs(float(to_np(sf)[0]) - float(sc_o)) <= 4e-7 * float(sc_o)
     s_g = linear_scales(fq, scales, M, (K + S) // 16, layout)
-    # y for the comparator: primary columns then the oracle's residuals
-    dq_o = oracle.nvfp4_dequantize(c_o, s_o, sc_o)
-    res_o = y_o[:, outl] - dq_o[:, outl] if S else np.zeros((M, 0), np.float32)
-    y_full = np.concatenate([y_o, res_o], axis=1)
-    assert_tolerant("nvfp4", K + S, (to_np(codes), s_g, to_np(sf)), (c_o, s_o, sc_o), y_full,
-                    name="arc", frac=2e-4)
+    c = arc_counts("nvfp4", K, outl[:S], (to_np(codes), s_g, to_np(sf)),
+                   (c_o[:, :K // 2], s_o[:, :K // 16], sc_o), y_o, name="arc")
+    check_fractions(c, 2e-4, "arc")
 
 
 def test_arc_general_outlier_list(fq):
@@ -380,10 +377,49 @@ def test_arc_general_outlier_list(fq):
         torch.from_numpy(outl).cuda(), 1e-6, torch.tensor([0.01], device="cuda"))
     torch.cuda.synchronize()
     c_o, s_o, sc_o, y_o = oracle.arc(x_bits, gamma, perm, outl, s_t=0.01)
-    dq_o = oracle.nvfp4_dequantize(c_o, s_o, sc_o)
-    y_full = np.concatenate([y_o, y_o[:, outl] - dq_o[:, outl]], axis=1)
-    assert_tolerant("nvfp4", K + S, (to_np(codes), to_np(scales), to_np(sf)), (c_o, s_o, sc_o),
-                    y_full, name="arc-general", frac=2e-4)
+    c = arc_counts("nvfp4", K, outl, (to_np(codes), to_np(scales), to_np(sf)),
+                   (c_o[:, :K // 2], s_o[:, :K // 16], sc_o), y_o, name="arc-general")
+    check_fractions(c, 2e-4, "arc-general")
+
+
+# ----------------------------------------------------------------------------- ARC, MXFP4
+
+def _arc_mx_check(codes, scales_lin, x_bits, gamma, perm, outl, name):
+    """Counts of an MXFP4 ARC output against the oracle (primary, and residual
+    of the kernel's own primary codes)."""
+    c_o, s_o, _, y_o = oracle.arc(x_bits, gamma, perm, outl, fmt="mxfp4")
+    K = y_o.shape[1]
+    return arc_counts("mxfp4", K, outl, (codes, scales_lin, None), (c_o[:, :K // 2], s_o[:, :K // 32], None),
+                      y_o, name=name)
+
+
+@pytest.mark.parametrize("shape", [(64, 1024, 64), (37, 4096, 256), (20, 512, 0), (16, 8192, 128),
+                                   (131, 1056, 32)])
+@pytest.mark.parametrize("layout", [0, 1])
+def test_arc_mxfp4_tolerance(fq, shape, layout):
+    M, K, S = shape
+    x_bits, gamma, perm, outl = workloads.arc_activations(M, K, seed=K + S + 1, S=S)
+    codes, scales, sf = fq.arc_quantize(
+        bits_to_torch_cuda(x_bits), bits_to_torch_cuda(gamma), torch.from_numpy(perm).cuda(),
+        torch.from_numpy(outl).cuda() if S else None, 1e-6, None, layout, fmt=fq.FP4Q_MXFP4)
+    torch.cuda.synchronize()
+    assert sf is None
+    s_g = linear_scales(fq, scales, M, (K + S) // 32, layout)
+    check_fractions(_arc_mx_check(to_np(codes), s_g, x_bits, gamma, perm, outl[:S], "arc-mxfp4"), 2e-4,
+                    "arc-mxfp4")
+
+
+def test_arc_mxfp4_general_outlier_list(fq):
+    """Outlier positions in arbitrary order, some in the same 32-block."""
+    M, K, S = 24, 1024, 64
+    x_bits, gamma, perm, _ = workloads.arc_activations(M, K, seed=5, S=S)
+    outl = np.random.default_rng(6).choice(K, S, replace=False).astype(np.int32)
+    codes, scales, _ = fq.arc_quantize(
+        bits_to_torch_cuda(x_bits), bits_to_torch_cuda(gamma), torch.from_numpy(perm).cuda(),
+        torch.from_numpy(outl).cuda(), 1e-6, fmt=fq.FP4Q_MXFP4)
+    torch.cuda.synchronize()
+    check_fractions(_arc_mx_check(to_np(codes), to_np(scales), x_bits, gamma, perm, outl,
+                                  "arc-mxfp4-general"), 2e-4, "arc-mxfp4-general")
 
 
 # ----------------------------------------------------------------------------- full sizes
@@ -486,11 +522,9 @@ def test_full_arc_8192x4096(fq, mode):
     tot = None
     for r0 in range(0, M, CHUNK):
         yc = y[r0:r0 + CHUNK]
-        c_o, s_o = oracle.arc_quantize(yc, outl, st_o)
-        dq_o = oracle.nvfp4_dequantize(c_o[:, :K // 2], s_o[:, :K // 16], st_o)
-        y_full = np.concatenate([yc, yc[:, outl] - dq_o[:, outl]], axis=1)
-        c = tolerant_counts("nvfp4", K + S, (codes[r0:r0 + CHUNK], scales[r0:r0 + CHUNK], sf_g),
-                            (c_o, s_o, np.float32(st_o)), y_full, name="full-arc")
+        c_o, s_o = oracle.nvfp4_quantize(yc, st_o)
+        c = arc_counts("nvfp4", K, outl, (codes[r0:r0 + CHUNK], scales[r0:r0 + CHUNK], sf_g),
+                       (c_o, s_o, np.float32(st_o)), yc, name="full-arc")
         tot = add_counts(tot, c)
     check_fractions(tot, 2e-4, "full-arc")
 
@@ -526,3 +560,21 @@ def test_full_dual_fwht512_round_trip_32768x4096(fq):
     xh = bf16_torch_to_bits(y)[rows]
     assert_roundtrip(xh, w, 512, name="full-dual-roundtrip")
     block_l2_identity(x_bits[rows], xh, dq, y_o, w, 512, name="full-dual-l2")
+
+
+@pytest.mark.slow
+def test_full_arc_mxfp4_8192x4096(fq):
+    """MXFP4 ARC at the ARC workload's full size, every row."""
+    M, K, S = 8192, 4096, 256
+    x_bits, gamma, perm, outl = workloads.arc_activations(M, K, seed=4, S=S)
+    codes, scales, _ = fq.arc_quantize(
+        bits_to_torch_cuda(x_bits), bits_to_torch_cuda(gamma), torch.from_numpy(perm).cuda(),
+        torch.from_numpy(outl).cuda(), 1e-6, fmt=fq.FP4Q_MXFP4)
+    torch.cuda.synchronize()
+    codes, scales = to_np(codes), to_np(scales)
+    tot = None
+    for r0 in range(0, M, CHUNK):
+        c = _arc_mx_check(codes[r0:r0 + CHUNK], scales[r0:r0 + CHUNK], x_bits[r0:r0 + CHUNK], gamma, perm,
+                          outl, "full-arc-mxfp4")
+        tot = add_counts(tot, c)
+    check_fractions(tot, 2e-4, "full-arc-mxfp4")
