@@ -34,7 +34,8 @@ FP4Q_WORKSPACE_BYTES = 16384
 EXPORTED = [
     "fp4q_quantize_nvfp4", "fp4q_quantize_nvfp4_noalloc", "fp4q_quantize_mxfp4", "fp4q_hadamard_quantize", "fp4q_arc_quantize",
     "fp4q_dequantize", "fp4q_workspace_bytes", "fp4q_scales_bytes", "fp4q_status_string",
-    "fp4q_device_error", "fp4q_selftest_div", "fp4q_gemm_nvfp4",
+    "fp4q_device_error", "fp4q_selftest_div", "fp4q_gemm_nvfp4", "fp4q_hadamard_quantize_signed",
+    "fp4q_dequantize_signed",
 ]
 
 
@@ -66,6 +67,8 @@ def declare(L: C.CDLL) -> C.CDLL:
         "fp4q_device_error": (i32, []),
         "fp4q_selftest_div": (i32, [p, p, i64, p, p, p]),
         "fp4q_gemm_nvfp4": (i32, [p, p, p, p, p, p, i64, i64, i64, p, i32, p]),
+        "fp4q_hadamard_quantize_signed": (i32, [p, i64, i64, i64, i32, p, i32, p, p, p, i32, i32, p, sz, p]),
+        "fp4q_dequantize_signed": (i32, [i32, p, p, p, i64, i64, i32, i32, p, p, p]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -199,6 +202,33 @@ def fp4q_gemm_nvfp4(a_codes, a_scales, a_scale, b_codes, b_scales, b_scale, K, d
                   "fp4q_gemm_nvfp4")
 
 
+def _host_words(signs):
+    """A host uint32 pattern (numpy array or sequence) as a ctypes pointer, kept alive by the caller."""
+    import numpy as np
+    arr = np.ascontiguousarray(np.asarray(signs, dtype=np.uint32))
+    return arr, arr.ctypes.data
+
+
+def fp4q_hadamard_quantize_signed(x, had_size, signs, fmt, codes, scales, scale_fp32,
+                                  mode=FP4Q_TSCALE_DYNAMIC, layout=FP4Q_SCALES_LINEAR,
+                                  workspace=None, stream=None):
+    M, K = x.shape
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    keep, sp = _host_words(signs)
+    return _check(_lib.fp4q_hadamard_quantize_signed(_ptr(x), M, K, _ld(x), int(had_size), sp, int(fmt),
+                                                     _ptr(codes), _ptr(scales), _ptr(scale_fp32), mode,
+                                                     layout, _ptr(workspace), ws_bytes, _stream(stream)),
+                  "fp4q_hadamard_quantize_signed")
+
+
+def fp4q_dequantize_signed(fmt, codes, scales, scale_fp32, M, K, y, signs, layout=FP4Q_SCALES_LINEAR,
+                           inv_had_size=0, stream=None):
+    keep, sp = _host_words(signs)
+    return _check(_lib.fp4q_dequantize_signed(int(fmt), _ptr(codes), _ptr(scales), _ptr(scale_fp32), M, K,
+                                              layout, int(inv_had_size), sp, _ptr(y), _stream(stream)),
+                  "fp4q_dequantize_signed")
+
+
 def fp4q_device_error() -> int:
     return int(_lib.fp4q_device_error())
 
@@ -258,7 +288,8 @@ def quantize_mxfp4(x, layout=FP4Q_SCALES_LINEAR):
 
 
 def hadamard_quantize(x, had_size, fmt=FP4Q_NVFP4, tensor_scale=None, layout=FP4Q_SCALES_LINEAR,
-                      ws=None):
+                      ws=None, signs=None):
+    """Block Hadamard (with `signs`: the random-sign rotation) + quantization."""
     M, K = x.shape
     codes, scales, sf = alloc_outputs(M, K, fmt, layout, x.device)
     mode = FP4Q_TSCALE_DYNAMIC
@@ -267,7 +298,10 @@ def hadamard_quantize(x, had_size, fmt=FP4Q_NVFP4, tensor_scale=None, layout=FP4
         mode = FP4Q_TSCALE_STATIC
     if fmt == FP4Q_NVFP4 and mode == FP4Q_TSCALE_DYNAMIC and ws is None:
         ws = workspace(x.device)
-    fp4q_hadamard_quantize(x, had_size, fmt, codes, scales, sf, mode, layout, ws)
+    if signs is None:
+        fp4q_hadamard_quantize(x, had_size, fmt, codes, scales, sf, mode, layout, ws)
+    else:
+        fp4q_hadamard_quantize_signed(x, had_size, signs, fmt, codes, scales, sf, mode, layout, ws)
     return codes, scales, sf
 
 
@@ -287,10 +321,13 @@ def arc_quantize(x, gamma, perm, outliers, eps=1e-6, tensor_scale=None,
     return codes, scales, sf
 
 
-def dequantize(fmt, codes, scales, scale_fp32, K, layout=FP4Q_SCALES_LINEAR, inv_had_size=0):
+def dequantize(fmt, codes, scales, scale_fp32, K, layout=FP4Q_SCALES_LINEAR, inv_had_size=0, signs=None):
     M = codes.shape[0]
     y = torch.empty((M, K), dtype=torch.bfloat16, device=codes.device)
-    fp4q_dequantize(fmt, codes, scales, scale_fp32, M, K, y, layout, inv_had_size)
+    if signs is None:
+        fp4q_dequantize(fmt, codes, scales, scale_fp32, M, K, y, layout, inv_had_size)
+    else:
+        fp4q_dequantize_signed(fmt, codes, scales, scale_fp32, M, K, y, signs, layout, inv_had_size)
     return y
 
 

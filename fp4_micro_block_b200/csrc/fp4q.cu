@@ -253,13 +253,17 @@ fp4q_status launch_mma_h(int had, const CUtensorMap& map, const MmaParams& p, in
 }
 
 
+// signs (host, may be NULL): the random-sign pattern of a rotation, bit j for
+// input channel j of every min(had, 128) channels; tensor-core paths only.
 fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, int had,
                             int fmt, uint8_t* codes, uint8_t* scales, float* scale_fp32,
                             fp4q_tscale_mode mode, fp4q_scale_layout layout, void* ws,
-                            size_t ws_bytes, cudaStream_t stream) {
+                            size_t ws_bytes, cudaStream_t stream, const uint32_t* signs = nullptr) {
     fp4q_status st = check_x(x, M, K, ldx);
     if (st != FP4Q_OK) return st;
     if (!valid_had(had)) return FP4Q_ERR_INVALID_ARG;
+    if (signs && had == 0) return FP4Q_ERR_INVALID_ARG;
+    if (signs && !use_mma(had, K)) return FP4Q_ERR_UNSUPPORTED;  // K % 128 != 0: register path
     if (layout != FP4Q_SCALES_LINEAR && layout != FP4Q_SCALES_SWIZZLED) return FP4Q_ERR_INVALID_ARG;
     const int B = fmt == FMT_MXFP4 ? 32 : 16;
     if (K % B != 0 || (had && K % had != 0)) return FP4Q_ERR_INVALID_ARG;
@@ -318,6 +322,8 @@ fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, in
         q.partials = static_cast<float*>(ws);
         q.swizzled = p.swizzled;
         q.dynamic = dynamic;
+        if (signs)
+            for (int w = 0; w < (std::min(had, kMmaTile) + 31) / 32; ++w) q.signs[w] = signs[w];
         const int grid = (int)std::min<int64_t>({q.n_tiles, (int64_t)sms, (int64_t)kMaxGrid});
         if (dynamic) {
             if ((st = launch_mma_h<FMT_NVFP4, true>(had, map, q, grid, stream)) != FP4Q_OK) return st;
@@ -345,9 +351,9 @@ fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, in
 }
 
 // ---------------------------------------------------------------- dequantizer launch
-template <int FMT, int HAD>
+template <int FMT, int HAD, bool SIGNED>
 fp4q_status launch_dequant_t(const DequantParams& p, int sms, cudaStream_t s) {
-    auto kern = dequant_warp_kernel<FMT, HAD>;
+    auto kern = dequant_warp_kernel<FMT, HAD, SIGNED>;
     constexpr int kWarps = kThreads / 32;
     constexpr int smem = kWarps * kDqWarpSmem;
     const int64_t units = ((p.M + 1) / 2) * p.n_col_tiles;  // (row pair, 512 columns)
@@ -360,25 +366,27 @@ fp4q_status launch_dequant_t(const DequantParams& p, int sms, cudaStream_t s) {
 }
 
 // Rotation sizes 0, 16, 32: the streaming kernel, 4 CTAs of 256 threads per SM.
-template <int FMT, int HAD>
+template <int FMT, int HAD, bool SIGNED>
 fp4q_status launch_dequant_stream(const DequantParams& p, int sms, cudaStream_t s) {
     const int64_t units = p.M * ((p.K + 31) / 32);
     const int grid = (int)std::min<int64_t>({(units + kThreads - 1) / kThreads, (int64_t)3 * sms,
                                             (int64_t)kMaxGrid});
     const int w32 = ((reinterpret_cast<uintptr_t>(p.y) & 31) == 0 && (p.K & 15) == 0) ? 1 : 0;
-    return launch(dequant_stream_kernel<FMT, HAD>, grid, kThreads, 0, s, p, w32);
+    return launch(dequant_stream_kernel<FMT, HAD, SIGNED>, grid, kThreads, 0, s, p, w32);
 }
 
-template <int FMT>
+template <int FMT, bool SIGNED>
 fp4q_status launch_dequant_h(int had, const DequantParams& p, int sms, cudaStream_t s) {
     switch (had) {
-        case 0: return launch_dequant_stream<FMT, 0>(p, sms, s);
-        case 16: return launch_dequant_stream<FMT, 16>(p, sms, s);
-        case 32: return launch_dequant_stream<FMT, 32>(p, sms, s);
-        case 64: return launch_dequant_t<FMT, 64>(p, sms, s);
-        case 128: return launch_dequant_t<FMT, 128>(p, sms, s);
-        case 256: return launch_dequant_t<FMT, 256>(p, sms, s);
-        case 512: return launch_dequant_t<FMT, 512>(p, sms, s);
+        case 0:
+            if constexpr (SIGNED) return FP4Q_ERR_INVALID_ARG;
+            else return launch_dequant_stream<FMT, 0, false>(p, sms, s);
+        case 16: return launch_dequant_stream<FMT, 16, SIGNED>(p, sms, s);
+        case 32: return launch_dequant_stream<FMT, 32, SIGNED>(p, sms, s);
+        case 64: return launch_dequant_t<FMT, 64, SIGNED>(p, sms, s);
+        case 128: return launch_dequant_t<FMT, 128, SIGNED>(p, sms, s);
+        case 256: return launch_dequant_t<FMT, 256, SIGNED>(p, sms, s);
+        case 512: return launch_dequant_t<FMT, 512, SIGNED>(p, sms, s);
         default: return FP4Q_ERR_INVALID_ARG;
     }
 }
@@ -516,6 +524,24 @@ FP4Q_API fp4q_status fp4q_hadamard_quantize(const void* x, int64_t M, int64_t K,
                            workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
+FP4Q_API fp4q_status fp4q_hadamard_quantize_signed(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                                   int had_size, const uint32_t* signs,
+                                                   fp4q_format format, uint8_t* codes, uint8_t* scales,
+                                                   float* scale_fp32, fp4q_tscale_mode mode,
+                                                   fp4q_scale_layout layout, void* workspace,
+                                                   size_t workspace_bytes, fp4q_stream_t stream) {
+    if (!signs) return FP4Q_ERR_INVALID_ARG;
+    int fmt;
+    switch (format) {
+        case FP4Q_NVFP4: fmt = FMT_NVFP4; break;
+        case FP4Q_MXFP4: fmt = FMT_MXFP4; break;
+        case FP4Q_NVFP4_DUAL: fmt = FMT_DUAL; break;
+        default: return FP4Q_ERR_INVALID_ARG;
+    }
+    return quantize_common(x, M, K, ldx, had_size, fmt, codes, scales, scale_fp32, mode, layout,
+                           workspace, workspace_bytes, (cudaStream_t)stream, signs);
+}
+
 FP4Q_API fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int64_t ldx,
                                        const void* gamma, float eps, const int32_t* perm,
                                        const int32_t* outliers, int64_t S, fp4q_format format,
@@ -599,14 +625,15 @@ FP4Q_API fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int6
     return run(ArcKern<FMT_NVFP4, false>{}, W);
 }
 
-FP4Q_API fp4q_status fp4q_dequantize(fp4q_format format, const uint8_t* codes,
-                                     const uint8_t* scales, const float* scale_fp32, int64_t M,
-                                     int64_t K, fp4q_scale_layout layout, int inv_had_size,
-                                     void* y, fp4q_stream_t stream) {
+namespace {
+fp4q_status dequantize_common(fp4q_format format, const uint8_t* codes, const uint8_t* scales,
+                              const float* scale_fp32, int64_t M, int64_t K, fp4q_scale_layout layout,
+                              int inv_had_size, const uint32_t* signs, void* y, fp4q_stream_t stream) {
     if (M < 0 || K <= 0) return FP4Q_ERR_INVALID_ARG;
     if (M >= kMaxDim || K >= kMaxDim) return FP4Q_ERR_UNSUPPORTED;
     if (K < 64) return FP4Q_ERR_UNSUPPORTED;
     if (!valid_had(inv_had_size)) return FP4Q_ERR_INVALID_ARG;
+    if (signs && inv_had_size == 0) return FP4Q_ERR_INVALID_ARG;
     if (layout != FP4Q_SCALES_LINEAR && layout != FP4Q_SCALES_SWIZZLED) return FP4Q_ERR_INVALID_ARG;
     int fmt;
     switch (format) {
@@ -636,11 +663,37 @@ FP4Q_API fp4q_status fp4q_dequantize(fp4q_format format, const uint8_t* codes,
     p.swizzled = layout == FP4Q_SCALES_SWIZZLED;
     p.had_norm = had_norm(inv_had_size);
     cudaStream_t s = (cudaStream_t)stream;
-    switch (fmt) {
-        case FMT_NVFP4: return launch_dequant_h<FMT_NVFP4>(inv_had_size, p, sms, s);
-        case FMT_MXFP4: return launch_dequant_h<FMT_MXFP4>(inv_had_size, p, sms, s);
-        default: return launch_dequant_h<FMT_DUAL>(inv_had_size, p, sms, s);
+    if (signs) {
+        for (int w = 0; w < (std::min(inv_had_size, kMmaTile) + 31) / 32; ++w) p.signs[w] = signs[w];
+        switch (fmt) {
+            case FMT_NVFP4: return launch_dequant_h<FMT_NVFP4, true>(inv_had_size, p, sms, s);
+            case FMT_MXFP4: return launch_dequant_h<FMT_MXFP4, true>(inv_had_size, p, sms, s);
+            default: return launch_dequant_h<FMT_DUAL, true>(inv_had_size, p, sms, s);
+        }
     }
+    switch (fmt) {
+        case FMT_NVFP4: return launch_dequant_h<FMT_NVFP4, false>(inv_had_size, p, sms, s);
+        case FMT_MXFP4: return launch_dequant_h<FMT_MXFP4, false>(inv_had_size, p, sms, s);
+        default: return launch_dequant_h<FMT_DUAL, false>(inv_had_size, p, sms, s);
+    }
+}
+}  // namespace
+
+FP4Q_API fp4q_status fp4q_dequantize(fp4q_format format, const uint8_t* codes,
+                                     const uint8_t* scales, const float* scale_fp32, int64_t M,
+                                     int64_t K, fp4q_scale_layout layout, int inv_had_size,
+                                     void* y, fp4q_stream_t stream) {
+    return dequantize_common(format, codes, scales, scale_fp32, M, K, layout, inv_had_size, nullptr, y,
+                             stream);
+}
+
+FP4Q_API fp4q_status fp4q_dequantize_signed(fp4q_format format, const uint8_t* codes,
+                                            const uint8_t* scales, const float* scale_fp32, int64_t M,
+                                            int64_t K, fp4q_scale_layout layout, int inv_had_size,
+                                            const uint32_t* signs, void* y, fp4q_stream_t stream) {
+    if (!signs) return FP4Q_ERR_INVALID_ARG;
+    return dequantize_common(format, codes, scales, scale_fp32, M, K, layout, inv_had_size, signs, y,
+                             stream);
 }
 
 FP4Q_API fp4q_status fp4q_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales,

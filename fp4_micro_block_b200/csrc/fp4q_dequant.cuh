@@ -78,7 +78,16 @@ struct DequantParams {
     uint16_t* y;
     int swizzled;
     float had_norm;
+    uint32_t signs[4];  // random-sign rotation: bit j negates output channel j of every min(n, 128)
 };
+
+// x^ = D H y for a random-sign rotation: flips the sign of v where bit (sh + i)
+// of the pattern word w is set, i = 0..N-1 (all within one 32-bit word).
+template <int N>
+__device__ __forceinline__ void apply_signs(float* v, uint32_t w) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] = __uint_as_float(__float_as_uint(v[i]) ^ ((w << (31 - i)) & 0x80000000u));
+}
 
 // Raw bytes of one 32-column unit: packed codes, its scale byte(s) and the fp32
 // scale, loaded ahead of their use (software pipelining).
@@ -185,7 +194,7 @@ __device__ __forceinline__ void store_bf16x32(uint16_t* dst, const uint32_t* o, 
     }
 }
 
-template <int FMT, int HAD>
+template <int FMT, int HAD, bool SIGNED = false>
 __global__ void __launch_bounds__(kThreads, 3) dequant_stream_kernel(const DequantParams p, int w32) {
     pdl_wait();
     pdl_trigger();
@@ -232,6 +241,10 @@ __global__ void __launch_bounds__(kThreads, 3) dequant_stream_kernel(const Dequa
             if constexpr (HAD > 0) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] *= p.had_norm;
+            }
+            if constexpr (SIGNED) {  // period n (16 or 32): columns col + i, col % 32 == 0
+                const uint32_t w = HAD == 16 ? (p.signs[0] & 0xffffu) * 0x10001u : p.signs[0];
+                apply_signs<32>(v, w);
             }
             uint32_t o[16];
 #pragma unroll
@@ -284,7 +297,7 @@ __device__ __forceinline__ void decode_raw_scaled(const RawUnit& u, float c, flo
     }
 }
 
-template <int FMT, int HAD>
+template <int FMT, int HAD, bool SIGNED = false>
 __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_warp_kernel(const DequantParams p) {
     pdl_wait();
     pdl_trigger();
@@ -388,6 +401,13 @@ __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_warp_kern
                     }
                 }
             }
+        }
+        if constexpr (SIGNED) {
+            // output column cb + 32 k2 + i has pattern index (k1 + 32 k2 + i) mod
+            // min(n, 128): word k2 mod (period / 32), bit k1 + i
+            constexpr int kWords = (HAD < 128 ? HAD : 128) / 32;
+#pragma unroll
+            for (int k2 = 0; k2 < n2; ++k2) apply_signs<k1w>(a[k2], p.signs[k2 % kWords] >> k1);
         }
         // the block's columns exist when its first one does (K % n == 0)
         if (row < p.M && cb < p.K) {

@@ -3,7 +3,8 @@
 //
 // For rotation sizes n <= 128 the rotated tile is a dense product: a tile X of
 // 128 rows x 128 columns times B = -2^-f * blockdiag(H_n, ..., H_n) (128 x 128,
-// Sylvester order, f = floor(log2(n) / 2)).  Every product of a bf16 input with
+// Sylvester order, f = floor(log2(n) / 2); with a random-sign pattern D the
+// rows of B change sign, B = -2^-f * D * blockdiag(H_n)).  Every product of a bf16 input with
 // +-2^-f is exact and the sums accumulate in fp32 in tensor memory, so the tile
 // arrives in TMEM as the negated, (partly) normalised rotation; odd log2(n)
 // leaves a factor RN(1/sqrt(2)) for the epilogue.  B's columns come in the
@@ -160,8 +161,15 @@ __host__ __device__ constexpr int acc_col(int j) { return (j & ~31) | ((j & 1) <
 // tile: element (row nn, column k) of half h = k / 64 lives at byte
 // h * 16 KiB + nn * 128 + ((k % 64) / 8 ^ nn % 8) * 16 + (k % 8) * 2; row nn
 // holds the Hadamard entries of output column acc_col(nn).
+// Sign bit of tile column k (0..127) for a sign pattern of period min(n, 128).
+__device__ __forceinline__ uint32_t sign_bit(const uint32_t (&signs)[4], int k) {
+    return (signs[(k >> 5) & 3] >> (k & 31)) & 1u;
+}
+
+// With signs, B = -2^-f * D * blockdiag(H_n) (D = diag of the +-1 pattern):
+// entry (k, oc) changes sign where channel k of the period is negated.
 template <int HAD>
-__device__ __forceinline__ void build_hadamard_b(uint8_t* b) {
+__device__ __forceinline__ void build_hadamard_b(uint8_t* b, const uint32_t (&signs)[4]) {
     constexpr int lg = HAD == 16 ? 4 : HAD == 32 ? 5 : HAD == 64 ? 6 : 7;
     const uint32_t mag = 0x3f80u - (uint32_t)(lg / 2) * 0x80u;  // bf16 bits of 2^-f
     for (int chunk = threadIdx.x; chunk < kTileBytes / 16; chunk += blockDim.x) {
@@ -179,6 +187,7 @@ __device__ __forceinline__ void build_hadamard_b(uint8_t* b) {
                 if (k / HAD == oc / HAD) {
                     const int par = __popc((uint32_t)((k % HAD) & (oc % HAD))) & 1;
                     bits = mag | (par ? 0u : 0x8000u);  // -(+-1) * 2^-f
+                    bits ^= sign_bit(signs, k % HAD) << 15;
                 }
                 pair |= bits << (16 * t);
             }
@@ -198,6 +207,8 @@ struct MmaParams {
     int n_partials;
     int swizzled;
     int dynamic;
+    uint32_t signs[4];           // random-sign rotation: bit j negates input channel j of every
+                                 // min(n, 128) channels (all zero: the plain rotation)
 };
 
 // Quantize the 32 values of one chunk (negated pairs n): codes into w, returns
@@ -269,7 +280,7 @@ __global__ void __launch_bounds__(MmaGeo<FMT>::threads, 1)
         tmem_alloc(smem_u32(tmem_slot), Geo::tmem_cols);
         tmem_relinquish();
     }
-    build_hadamard_b<HAD>(smem + kMmaBOff);
+    build_hadamard_b<HAD>(smem + kMmaBOff, p.signs);
     fence_proxy_async_smem();  // B is read by the tensor cores (async proxy)
     pdl_wait();
     pdl_trigger();

@@ -95,9 +95,11 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// B = -2^-4 * H_128 (K-major, 128-byte swizzle) for n = 256 and 512, its rows
-// (accumulator columns) in the acc_col order of the 128-column kernel.
-__device__ __forceinline__ void build_h128_b(uint8_t* b) {
+// B = -2^-4 * D * H_128 (K-major, 128-byte swizzle) for n = 256 and 512, its
+// rows (accumulator columns) in the acc_col order of the 128-column kernel; D
+// is the random-sign pattern of period 128 (identity when all signs are zero),
+// so that H_n D_n = H_(n/128) (x) (H_128 D_128) with D_n = I (x) D_128.
+__device__ __forceinline__ void build_h128_b(uint8_t* b, const uint32_t (&signs)[4]) {
     const uint32_t mag = 0x3f80u - 4u * 0x80u;  // bf16 bits of 2^-4
     for (int chunk = threadIdx.x; chunk < kTileBytes / 16; chunk += blockDim.x) {
         const int h = chunk / 1024, nn = (chunk / 8) % 128, cp = chunk % 8;
@@ -110,7 +112,7 @@ __device__ __forceinline__ void build_h128_b(uint8_t* b) {
             for (int t = 0; t < 2; ++t) {
                 const int k = h * 64 + c * 8 + e + t;
                 const int par = __popc((uint32_t)(k & oc)) & 1;
-                pair |= (mag | (par ? 0u : 0x8000u)) << (16 * t);
+                pair |= ((mag | (par ? 0u : 0x8000u)) ^ (sign_bit(signs, k) << 15)) << (16 * t);
             }
             w[e / 2] = pair;
         }
@@ -153,7 +155,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         tmem_alloc(smem_u32(tmem_slot), 512u);
         tmem_relinquish();
     }
-    build_h128_b(smem);
+    build_h128_b(smem, p.signs);
     fence_proxy_async_smem();
     pdl_wait();
     pdl_trigger();

@@ -178,6 +178,24 @@ fp4q_status fp4q_hadamard_quantize(const void* x, int64_t M, int64_t K, int64_t 
                                    void* workspace, size_t workspace_bytes,
                                    fp4q_stream_t stream);
 
+/* fp4q_hadamard_quantize_signed -- fp4q_hadamard_quantize with a random-sign
+ * rotation: y = (1/sqrt(n)) H_n D x per contiguous n-block, D = diag(+-1), the
+ * randomized Hadamard transform that NVFP4 training recipes apply before
+ * quantizing (named as such in the nGPT abstract, "Normalized Architectures
+ * are Natively 4-Bit").
+ *   signs  HOST pointer to ceil(p/32) uint32 words, p = min(had_size, 128):
+ *          bit j (word j/32, bit j%32) set negates input channel j of every
+ *          p consecutive channels (D repeats with period p; for n = 256, 512 the
+ *          rotation is H_(n/128) (x) (H_128 D_128)).  Read during the call.
+ * Other arguments as for fp4q_hadamard_quantize; had_size in {16..512}.
+ * Requires K % 128 == 0 (the tensor-core rotation), else FP4Q_ERR_UNSUPPORTED. */
+fp4q_status fp4q_hadamard_quantize_signed(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                          int had_size, const uint32_t* signs, fp4q_format format,
+                                          uint8_t* codes, uint8_t* scales, float* scale_fp32,
+                                          fp4q_tscale_mode mode, fp4q_scale_layout layout,
+                                          void* workspace, size_t workspace_bytes,
+                                          fp4q_stream_t stream);
+
 /* fp4q_arc_quantize -- ARCQuant fused reorder + RMSNorm + primary quantization
  * + residual quantization of the outlier channels, in NVFP4 or MXFP4.
  *   For each row: y[p] = x[perm[p]] / sqrt(mean_k x[k]^2 + eps) * gamma[perm[p]]
@@ -254,6 +272,16 @@ fp4q_status fp4q_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales, con
                             const uint8_t* b_codes, const uint8_t* b_scales, const float* b_scale,
                             int64_t M, int64_t N, int64_t K, void* d, int d_bf16,
                             fp4q_stream_t stream);
+
+/* fp4q_dequantize_signed -- fp4q_dequantize followed by the inverse of a
+ * random-sign rotation: x = D (1/sqrt(n)) H_n y (the normalised H is its own
+ * inverse and D = D^-1).  signs: HOST pointer, the pattern given to
+ * fp4q_hadamard_quantize_signed (period min(inv_had_size, 128)).  inv_had_size
+ * must be non-zero; other arguments as for fp4q_dequantize. */
+fp4q_status fp4q_dequantize_signed(fp4q_format format, const uint8_t* codes, const uint8_t* scales,
+                                   const float* scale_fp32, int64_t M, int64_t K,
+                                   fp4q_scale_layout layout, int inv_had_size, const uint32_t* signs,
+                                   void* y, fp4q_stream_t stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fp4q_status_string(fp4q_status status);

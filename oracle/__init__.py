@@ -238,10 +238,23 @@ def hadamard_entry(i: int, j: int) -> int:
     return int(lib().orc_hadamard_entry(i, j))
 
 
-def hadamard(x: np.ndarray, n: int) -> np.ndarray:
+def sign_vector(signs, n: int, K: int) -> np.ndarray:
+    """The +-1 diagonal of a random-sign rotation over K channels: bit j of the
+    pattern (period p = min(n, 128)) negates channel j of every p channels."""
+    p = min(n, 128)
+    w = np.asarray(signs, np.uint32)
+    bits = np.array([(int(w[j // 32]) >> (j % 32)) & 1 for j in range(p)])
+    return np.tile(np.where(bits == 1, -1.0, 1.0), K // p).astype(np.float32)
+
+
+def hadamard(x: np.ndarray, n: int, signs=None) -> np.ndarray:
+    """Normalised block Hadamard of every contiguous n-block; with a sign
+    pattern, H_n D x (the randomised transform; D = diag(+-1), applied exactly)."""
     x = _f32(x)
     M, K = x.shape
     assert K % n == 0
+    if signs is not None:
+        x = x * sign_vector(signs, n, K)[None, :]
     y = np.empty((M, K), np.float32)
     lib().orc_hadamard(_ptr(x), M, K, K, int(n), _ptr(y))
     return y
@@ -295,11 +308,13 @@ def quantize_mxfp4(x_bits: np.ndarray):
     return mxfp4_quantize(bf16_to_f32(x_bits))
 
 
-def hadamard_quantize(x_bits: np.ndarray, n: int, fmt: str = "nvfp4", s_t: float | None = None):
-    """Block-Hadamard (size n, normalised) then NVFP4 / MXFP4 / dual quantization.
+def hadamard_quantize(x_bits: np.ndarray, n: int, fmt: str = "nvfp4", s_t: float | None = None,
+                      signs=None):
+    """Block-Hadamard (size n, normalised; with `signs` the random-sign H D)
+    then NVFP4 / MXFP4 / dual quantization.
 
     Returns (codes, scales, s_t_or_gscales, y) with y the rotated fp32 matrix."""
-    y = hadamard(bf16_to_f32(x_bits), n)
+    y = hadamard(bf16_to_f32(x_bits), n, signs)
     if fmt == "nvfp4":
         if s_t is None:
             s_t = tensor_scale(amax(y))
@@ -333,8 +348,9 @@ def arc(x_bits, gamma_bits, perm, outliers, eps: float = 1e-6, s_t: float | None
     return c, s, np.float32(s_t), y
 
 
-def dequantize(fmt: str, codes, scales, scale=None, inv_had: int = 0) -> np.ndarray:
-    """Dequantize to fp32 (then optionally inverse block Hadamard); returns fp32."""
+def dequantize(fmt: str, codes, scales, scale=None, inv_had: int = 0, signs=None) -> np.ndarray:
+    """Dequantize to fp32 (then optionally inverse block Hadamard, and with a
+    sign pattern the inverse D H of the random-sign rotation); returns fp32."""
     if fmt == "nvfp4":
         y = nvfp4_dequantize(codes, scales, float(scale))
     elif fmt == "mxfp4":
@@ -345,11 +361,13 @@ def dequantize(fmt: str, codes, scales, scale=None, inv_had: int = 0) -> np.ndar
         raise ValueError(fmt)
     if inv_had:
         y = hadamard(y, inv_had)  # the normalised Sylvester matrix is its own inverse
+        if signs is not None:
+            y = y * sign_vector(signs, inv_had, y.shape[1])[None, :]  # D = D^-1
     return y
 
 
-def dequantize_bf16(fmt: str, codes, scales, scale=None, inv_had: int = 0) -> np.ndarray:
-    return f32_to_bf16(dequantize(fmt, codes, scales, scale, inv_had))
+def dequantize_bf16(fmt: str, codes, scales, scale=None, inv_had: int = 0, signs=None) -> np.ndarray:
+    return f32_to_bf16(dequantize(fmt, codes, scales, scale, inv_had, signs))
 
 
 # --------------------------------------------------------------------------- consumer GEMM

@@ -140,3 +140,19 @@ def test_selftest_validation(fq):
     L = fq.lib()
     assert L.fp4q_selftest_div(X, X, -1, X, X, None) == fq.FP4Q_ERR_INVALID_ARG
     assert L.fp4q_selftest_div(None, X, 0, X, X, None) == fq.FP4Q_OK
+
+
+def test_signed_rotation_validation(fq):
+    """The random-sign variants: no pattern, no rotation or a register-path K
+    (not a multiple of 128) are rejected before any launch."""
+    import ctypes as C
+    L = fq.lib()
+    words = (C.c_uint32 * 4)(1, 2, 3, 4)
+    h = L.fp4q_hadamard_quantize_signed
+    assert h(X, 4, 256, 256, 128, None, 0, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert h(X, 4, 256, 256, 0, words, 0, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert h(X, 4, 1040, 1040, 16, words, 0, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_UNSUPPORTED
+    d = L.fp4q_dequantize_signed
+    Y = 0x90000
+    assert d(0, CODES, SCALES, SF, 4, 256, 0, 128, None, Y, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert d(0, CODES, SCALES, SF, 4, 256, 0, 0, words, Y, None) == fq.FP4Q_ERR_INVALID_ARG

@@ -76,6 +76,14 @@ def test_format_error_table(fq):
             assert abs(gpu_rows - orc_rows) <= 0.03 * orc_rows, (name, n, gpu_rows, orc_rows)
             table[f"{name}_had{n}"] = {"rel_mse": gpu, "rel_mse_oracle_rows": orc_rows,
                                        "rel_mse_rows": gpu_rows}
+    # the random-sign rotation (H_128 D with a seeded +-1 pattern)
+    signs = workloads.random_signs(128, seed=9)
+    for name, f in (("nvfp4", fq.FP4Q_NVFP4), ("mxfp4", fq.FP4Q_MXFP4)):
+        codes, scales, sf = fq.hadamard_quantize(x, 128, f, signs=signs)
+        y = fq.dequantize(f, codes, scales, sf, K, 0, 128, signs=signs)
+        torch.cuda.synchronize()
+        d = (y.float() - xf).double()
+        table[f"{name}_rht128"] = {"rel_mse": float((d * d).sum() / (xf.double() ** 2).sum())}
     for n in SIZES:
         assert table[f"mxfp4_had{n}"]["rel_mse"] > table[f"nvfp4_had{n}"]["rel_mse"], n
     out = os.environ.get("FP4Q_ERROR_TABLE")

@@ -275,6 +275,47 @@ def test_hadamard_static_scale(fq):
 
 
 @pytest.mark.parametrize("n", [16, 32, 64, 128, 256, 512])
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4", "dual"])
+def test_random_sign_hadamard_quantize_tolerance(fq, n, fmt):
+    """The random-sign rotation H_n D (pattern of period min(n, 128)) on the
+    tensor cores, against the oracle's H_n D, under the tolerance rule."""
+    M, K = 40, 2048
+    x_bits = workloads.hadamard_channels(M, K, seed=n + 3)
+    signs = workloads.random_signs(min(n, 128), seed=n)
+    fcode = {"nvfp4": fq.FP4Q_NVFP4, "mxfp4": fq.FP4Q_MXFP4, "dual": fq.FP4Q_NVFP4_DUAL}[fmt]
+    codes, scales, sf = fq.hadamard_quantize(bits_to_torch_cuda(x_bits), n, fcode, signs=signs)
+    torch.cuda.synchronize()
+    c_o, s_o, sc_o, y_o = oracle.hadamard_quantize(x_bits, n, fmt, signs=signs)
+    if fmt == "nvfp4":
+        assert abs(float(to_np(sf)[0]) - float(sc_o)) <= 4e-7 * float(sc_o)
+        gpu = (to_np(codes), to_np(scales), to_np(sf))
+    elif fmt == "dual":
+        np.testing.assert_allclose(to_np(sf), sc_o, rtol=4e-7)
+        gpu = (to_np(codes), to_np(scales), to_np(sf))
+    else:
+        gpu = (to_np(codes), to_np(scales), None)
+    assert_tolerant(fmt, K, gpu, (c_o, s_o, sc_o), y_o, name=f"rs-had{n}-{fmt}")
+
+
+@pytest.mark.parametrize("n", [16, 32, 64, 128, 256, 512])
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4", "dual"])
+def test_dequantize_random_sign_inverse(fq, n, fmt):
+    """Dequantize + inverse random-sign rotation D H_n of random payloads,
+    exact outside the bf16 rounding window of the oracle's D H_n."""
+    M, K = 33, 1024
+    codes, scales, sc = workloads.random_payload(M, K, fmt, seed=n + 7)
+    signs = workloads.random_signs(min(n, 128), seed=n + 1)
+    f = {"nvfp4": fq.FP4Q_NVFP4, "mxfp4": fq.FP4Q_MXFP4, "dual": fq.FP4Q_NVFP4_DUAL}[fmt]
+    sct = (None if sc is None else
+           torch.tensor([sc], device="cuda") if fmt == "nvfp4" else torch.from_numpy(sc).cuda())
+    y = fq.dequantize(f, torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(), sct, K, 0, n,
+                      signs=signs)
+    torch.cuda.synchronize()
+    want = oracle.dequantize(fmt, codes, scales, sc, inv_had=n, signs=signs)
+    assert_roundtrip(bf16_torch_to_bits(y), want, n, name=f"rs-inv-had{n}-{fmt}")
+
+
+@pytest.mark.parametrize("n", [16, 32, 64, 128, 256, 512])
 @pytest.mark.parametrize("fmt", ["nvfp4", "dual", "mxfp4"])
 def test_dequantize_inverse_hadamard(fq, n, fmt):
     M, K = 33, 1024

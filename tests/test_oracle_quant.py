@@ -460,3 +460,31 @@ def test_swizzle_matches_the_block_scaled_gemm_library_layout():
             ref = swizzle_blockscale(torch.from_numpy(lin).view(torch.float8_e4m3fn))
             want = ref.contiguous().view(torch.uint8).numpy().reshape(-1)
             assert np.array_equal(oracle.swizzle_scales(lin), want), (M, n)
+
+
+# ----------------------------------------------------------------------------- random-sign rotation
+
+def _pattern(words, p):
+    """+-1 per channel of the period from the bit mask (independent of the oracle's helper)."""
+    bits = np.unpackbits(np.asarray(words, np.uint32).view(np.uint8), bitorder="little")[:p]
+    return 1.0 - 2.0 * bits.astype(np.float64)
+
+
+@pytest.mark.parametrize("n", [16, 32, 128, 512])
+def test_random_sign_hadamard_matches_scipy(n):
+    """H_n D per block against scipy's Hadamard matrix times the sign diagonal
+    (period min(n, 128)); orthonormal (norms kept) and inverted by D H."""
+    rng = np.random.default_rng(40 + n)
+    K = 2 * n
+    x = rng.standard_normal((3, K)).astype(np.float32)
+    words = workloads.random_signs(min(n, 128), seed=n)
+    d = np.tile(_pattern(words, min(n, 128)), K // min(n, 128))
+    H = scipy.linalg.hadamard(n).astype(np.float64) / np.sqrt(n)
+    ref = ((x.astype(np.float64) * d).reshape(3, K // n, n) @ H.T).reshape(3, K)
+    y = oracle.hadamard(x, n, words)
+    np.testing.assert_allclose(y, ref.astype(np.float32), rtol=2 ** -23, atol=1e-30)
+    np.testing.assert_allclose(np.linalg.norm(y.reshape(3, -1, n), axis=2),
+                               np.linalg.norm(x.reshape(3, -1, n).astype(np.float64), axis=2), rtol=1e-6)
+    # the inverse through the dequantizer's path: D H y = x
+    back = oracle.hadamard(y, n) * d.astype(np.float32)
+    np.testing.assert_allclose(back, x, rtol=0, atol=4e-6 * np.abs(x).max())

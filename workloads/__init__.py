@@ -23,6 +23,7 @@ ARCQuant page).  No dataset is involved.
   dual_gain        : N(0,1) x per-token gain exp(N(0,1)) (LogNormal(0,1))
   random_payload   : uniform random code bytes and scale bytes (a dequantizer
                      input that needs no quantizer run to produce)
+  random_signs     : a seeded +-1 pattern (bit mask) for a random-sign rotation
 """
 from __future__ import annotations
 
@@ -38,6 +39,7 @@ __all__ = [
     "arc_activations",
     "dual_gain",
     "random_payload",
+    "random_signs",
     "WORKLOADS",
 ]
 
@@ -155,3 +157,14 @@ def random_payload(M: int, K: int, fmt: str, seed: int = 6):
     if fmt == "dual":
         return codes, scales, rng.uniform(1e-3, 1.0, size=(M, K // 128)).astype(np.float32)
     raise ValueError(fmt)
+
+
+def random_signs(period: int, seed: int = 8) -> np.ndarray:
+    """A uniformly random sign pattern of `period` channels as uint32 words:
+    bit j (word j // 32, bit j % 32) set means channel j is negated."""
+    rng = np.random.default_rng(seed)
+    bits = rng.integers(0, 2, size=period).astype(np.uint64)
+    words = np.zeros((period + 31) // 32, np.uint32)
+    for j in range(period):
+        words[j // 32] |= np.uint32(int(bits[j]) << (j % 32))
+    return words
