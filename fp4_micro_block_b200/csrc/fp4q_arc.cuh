@@ -174,15 +174,6 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return __byte_perm(a, b, sel);
 }
 
-// 32-bit shared-memory load that the compiler keeps in program order (so that a
-// block's loads are all issued before their first use) and does not move across
-// the pair loop (the buffer is rewritten for every pair).
-__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
-}
-
 // Store one scale byte of (row, col).
 __device__ __forceinline__ void put_scale(const ArcParams& p, int64_t row, int64_t col, int64_t nsc,
                                           int64_t nC, uint32_t byte) {
@@ -410,32 +401,19 @@ __global__ void __launch_bounds__(arc_max_warps<AMAX_ONLY>() * 32, 1) arc_kernel
             const int64_t r1 = r0 + 1;
             uint8_t* cp0 = p.codes + r0 * kcs;
             uint8_t* cp1 = p.codes + r1 * kcs;
-            const uint32_t lbase = smem_u32(l0);
-            // The table words and the interleaved words of block b: every shared
-            // load of the block is issued before any of its values is used.
-            auto gather_words = [&](int b, uint32_t* tw, uint32_t* xw) {
+            // (-z row 0, -z row 1) of the B positions of block b
+            auto gather = [&](int b, float2* v) {
 #pragma unroll
                 for (int k = 0; k < Q; ++k) {
-                    const uint4 t4 = *reinterpret_cast<const uint4*>(tab + 4 * (k * nbB + b));
-                    tw[4 * k] = t4.x;
-                    tw[4 * k + 1] = t4.y;
-                    tw[4 * k + 2] = t4.z;
-                    tw[4 * k + 3] = t4.w;
+                    const uint4 tw = *reinterpret_cast<const uint4*>(tab + 4 * (k * nbB + b));
+                    const uint32_t wv[4] = {tw.x, tw.y, tw.z, tw.w};
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const uint32_t xw = *reinterpret_cast<const uint32_t*>(l0 + (wv[t] & 0xffffu));
+                        const float ng_ = -__uint_as_float(wv[t] & 0xffff0000u);
+                        v[4 * k + t] = fmul2(make_float2(bf16lo(xw), bf16hi(xw)), dup2(ng_));
+                    }
                 }
-#pragma unroll
-                for (int i = 0; i < B; ++i) xw[i] = ld_shared_u32(lbase + (tw[i] & 0xffffu));
-            };
-            // (-z row 0, -z row 1) of the B positions from their words
-            auto unpack = [&](const uint32_t* tw, const uint32_t* xw, float2* v) {
-#pragma unroll
-                for (int i = 0; i < B; ++i)
-                    v[i] = fmul2(make_float2(bf16lo(xw[i]), bf16hi(xw[i])),
-                                 dup2(-__uint_as_float(tw[i] & 0xffff0000u)));
-            };
-            auto gather = [&](int b, float2* v) {
-                uint32_t tw[B], xw[B];
-                gather_words(b, tw, xw);
-                unpack(tw, xw, v);
             };
             // quantize + store block b of both rows, and its outlier residuals
             auto emit = [&](int b, const float2* v) {
@@ -519,15 +497,12 @@ __global__ void __launch_bounds__(arc_max_warps<AMAX_ONLY>() * 32, 1) arc_kernel
                 }
             };
             if constexpr (FMT == FMT_NVFP4) {
-                // two blocks per step: all 32 gathers in flight together
+                // two blocks per step (their gathers in flight together)
                 for (int b = lane; b < nbB; b += 64) {
-                    const bool second = b + 32 < nbB;
-                    uint32_t twa[B], xwa[B], twb[B], xwb[B];
-                    gather_words(b, twa, xwa);
-                    gather_words(second ? b + 32 : b, twb, xwb);
                     float2 va[B], vb[B];
-                    unpack(twa, xwa, va);
-                    unpack(twb, xwb, vb);
+                    const bool second = b + 32 < nbB;
+                    gather(b, va);
+                    if (second) gather(b + 32, vb);
                     emit(b, va);
                     if (second) emit(b + 32, vb);
                 }
