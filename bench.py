@@ -207,7 +207,7 @@ def peaks_tensor():
 _COMMON = ["fp4q_device.cuh", "fp4q_unit.cuh", "fp4q_quant.cuh"]
 KERNEL_SOURCES = {
     ("dual", "quantize"): _COMMON + ["fp4q_mma.cuh", "fp4q_mma_wide.cuh"],
-    ("dual", "dequantize"): _COMMON + ["fp4q_dequant.cuh"],
+    ("dual", "dequantize"): _COMMON + ["fp4q_mma.cuh", "fp4q_gemm.cuh", "fp4q_dqmma.cuh"],
     ("mxfp4", "quantize"): _COMMON,
     ("mxfp4", "dequantize"): _COMMON + ["fp4q_dequant.cuh"],
     ("arc", "arc"): _COMMON + ["fp4q_arc.cuh"],

@@ -15,6 +15,7 @@
 #include "../../include/fp4q.h"
 #include "fp4q_arc.cuh"
 #include "fp4q_dequant.cuh"
+#include "fp4q_dqmma.cuh"
 #include "fp4q_device.cuh"
 #include "fp4q_gemm.cuh"
 #include "fp4q_mma.cuh"
@@ -109,6 +110,23 @@ fp4q_status make_codes_map(CUtensorMap* map, const void* codes, int64_t rows, in
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box,
                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FP4Q_OK : FP4Q_ERR_CUDA;
+}
+
+// Row-major [rows, cols] of 1-byte or 4-byte elements (row stride row_bytes, a
+// multiple of 16), boxes of box_cols x box_rows, no swizzle, zero fill outside.
+fp4q_status make_plain_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, int64_t rows, int64_t cols,
+                           int64_t row_bytes, uint32_t box_cols, uint32_t box_rows) {
+    EncodeTiledFn enc;
+    fp4q_status st = encode_fn(&enc);
+    if (st != FP4Q_OK) return st;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FP4Q_OK : FP4Q_ERR_CUDA;
 }
 
@@ -351,17 +369,94 @@ fp4q_status quantize_common(const void* x, int64_t M, int64_t K, int64_t ldx, in
 }
 
 // ---------------------------------------------------------------- dequantizer launch
+// The tensor-core dequantizer (NVFP4 and dual, n >= 16): K % 512 == 0, linear
+// scales, scale arrays 16-byte aligned (the TMA boxes' bases and row strides).
+bool dqm_applies(int fmt, int had, const DequantParams& p) {
+    return fmt != FMT_MXFP4 && had >= 16 && p.K % 512 == 0 && !p.swizzled && aligned(p.scales, 16) &&
+           (fmt != FMT_DUAL || aligned(p.scale_fp32, 16));
+}
+
+template <int FMT, int HAD>
+fp4q_status launch_dqm_t(const DequantParams& d, int sms, cudaStream_t s) {
+    CUtensorMap codes_map, scales_map, g_map;
+    fp4q_status st;
+    if ((st = make_codes_map(&codes_map, d.codes, d.M, d.K / 2, 128)) != FP4Q_OK ||
+        (st = make_plain_map(&scales_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, d.scales, d.M, d.K / 16, d.K / 16, 32,
+                             128)) != FP4Q_OK)
+        return st;
+    if constexpr (FMT == FMT_DUAL) {
+        if ((st = make_plain_map(&g_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d.scale_fp32, d.M, d.K / 128,
+                                 d.K / 128 * 4, 4, 128)) != FP4Q_OK)
+            return st;
+    } else {
+        g_map = scales_map;  // not read
+    }
+    DqmParams p{};
+    p.M = d.M;
+    p.K = d.K;
+    p.n_ct = d.K / 512;
+    p.n_tiles = ((d.M + 127) / 128) * p.n_ct;
+    p.scale_fp32 = d.scale_fp32;
+    p.y = d.y;
+    p.had_norm = d.had_norm;
+    for (int w = 0; w < 4; ++w) p.signs[w] = d.signs[w];
+    p.w32 = (reinterpret_cast<uintptr_t>(d.y) & 31) == 0 ? 1 : 0;
+    auto kern = dequant_mma_kernel<FMT, HAD>;
+    static std::atomic<uint64_t> done{0};
+    if ((st = ensure_smem(kern, kDqmSmem, done)) != FP4Q_OK) return st;
+    const int grid = (int)std::min<int64_t>({p.n_tiles, (int64_t)sms, (int64_t)kMaxGrid});
+    return launch(kern, grid, kDqmThreads, kDqmSmem, s, codes_map, scales_map, g_map, p);
+}
+
+template <int FMT>
+fp4q_status launch_dqm(int had, const DequantParams& p, int sms, cudaStream_t s) {
+    switch (had) {
+        case 16: return launch_dqm_t<FMT, 16>(p, sms, s);
+        case 32: return launch_dqm_t<FMT, 32>(p, sms, s);
+        case 64: return launch_dqm_t<FMT, 64>(p, sms, s);
+        case 128: return launch_dqm_t<FMT, 128>(p, sms, s);
+        case 256: return launch_dqm_t<FMT, 256>(p, sms, s);
+        case 512: return launch_dqm_t<FMT, 512>(p, sms, s);
+        default: return FP4Q_ERR_INVALID_ARG;
+    }
+}
+
+// Rotation sizes 64..512: the TMA-fed kernel when K % 512 == 0, the scales are
+// linear and the scale arrays 16-byte aligned (the copies' bases and row
+// strides must be), else the kernel that loads codes and scales itself.
 template <int FMT, int HAD, bool SIGNED>
 fp4q_status launch_dequant_t(const DequantParams& p, int sms, cudaStream_t s) {
-    auto kern = dequant_warp_kernel<FMT, HAD, SIGNED>;
     constexpr int kWarps = kThreads / 32;
-    constexpr int smem = kWarps * kDqWarpSmem;
     const int64_t units = ((p.M + 1) / 2) * p.n_col_tiles;  // (row pair, 512 columns)
     const int grid = (int)std::min<int64_t>({(units + kWarps - 1) / kWarps, (int64_t)kDequantCtasPerSm * sms,
                                             (int64_t)kMaxGrid});
+    fp4q_status st;
+    if (p.K % kTileCols == 0 && !p.swizzled && aligned(p.scales, 16) &&
+        (FMT != FMT_DUAL || aligned(p.scale_fp32, 16))) {
+        constexpr int B = FMT == FMT_MXFP4 ? 32 : 16;
+        CUtensorMap codes_map, scales_map, g_map;
+        if ((st = make_plain_map(&codes_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.codes, p.M, p.K / 2, p.K / 2,
+                                 kTileCols / 2, 2)) != FP4Q_OK ||
+            (st = make_plain_map(&scales_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.scales, p.M, p.K / B, p.K / B,
+                                 kTileCols / B, 2)) != FP4Q_OK)
+            return st;
+        if constexpr (FMT == FMT_DUAL) {
+            if ((st = make_plain_map(&g_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.scale_fp32, p.M, p.K / 128,
+                                     p.K / 128 * 4, kTileCols / 128, 2)) != FP4Q_OK)
+                return st;
+        } else {
+            g_map = scales_map;  // not read
+        }
+        auto kern = dequant_tma_kernel<FMT, HAD, SIGNED>;
+        constexpr int smem = kWarps * kDqRingSmem;
+        static std::atomic<uint64_t> done{0};
+        if ((st = ensure_smem(kern, smem, done)) != FP4Q_OK) return st;
+        return launch(kern, grid, kThreads, smem, s, p, codes_map, scales_map, g_map);
+    }
+    auto kern = dequant_warp_kernel<FMT, HAD, SIGNED>;
+    constexpr int smem = kWarps * kDqWarpSmem;
     static std::atomic<uint64_t> done{0};
-    fp4q_status st = ensure_smem(kern, smem, done);
-    if (st != FP4Q_OK) return st;
+    if ((st = ensure_smem(kern, smem, done)) != FP4Q_OK) return st;
     return launch(kern, grid, kThreads, smem, s, p);
 }
 
@@ -663,8 +758,12 @@ fp4q_status dequantize_common(fp4q_format format, const uint8_t* codes, const ui
     p.swizzled = layout == FP4Q_SCALES_SWIZZLED;
     p.had_norm = had_norm(inv_had_size);
     cudaStream_t s = (cudaStream_t)stream;
-    if (signs) {
+    if (signs)
         for (int w = 0; w < (std::min(inv_had_size, kMmaTile) + 31) / 32; ++w) p.signs[w] = signs[w];
+    if (dqm_applies(fmt, inv_had_size, p))
+        return fmt == FMT_DUAL ? launch_dqm<FMT_DUAL>(inv_had_size, p, sms, s)
+                               : launch_dqm<FMT_NVFP4>(inv_had_size, p, sms, s);
+    if (signs) {
         switch (fmt) {
             case FMT_NVFP4: return launch_dequant_h<FMT_NVFP4, true>(inv_had_size, p, sms, s);
             case FMT_MXFP4: return launch_dequant_h<FMT_MXFP4, true>(inv_had_size, p, sms, s);

@@ -297,6 +297,108 @@ __device__ __forceinline__ void decode_raw_scaled(const RawUnit& u, float c, flo
     }
 }
 
+// Phase A, the exchange and phase B of one unit: the raw unit of lane (r2, l)
+// in, the lane's phase-B outputs out (a[k2][i] is column 32 k2 + i of the
+// lane's k1w-column slice of block b).  ws is the lane's row in the warp's
+// scratch; the caller has synchronised the warp since the scratch was last read.
+template <int FMT, int HAD, bool SIGNED>
+__device__ __forceinline__ void dq_unit(const DequantParams& p, const RawUnit& cur, bool live, uint8_t* ws,
+                                        uint32_t l, uint32_t b, uint32_t k1,
+                                        float (&a)[HadShape<HAD>::n2][HadShape<HAD>::k1w]) {
+    constexpr int n2 = HadShape<HAD>::n2, k1w = HadShape<HAD>::k1w;
+    // phase-B read offset of sub-row sl = b n2 + k2 within the lane's row
+    // (swizzled chunk); for n2 >= 8, b n2 is a multiple of 8 and the swizzle
+    // depends on k2 alone, a constant of the unrolled loop
+    auto rd_off = [&](uint32_t sl, int h) -> uint32_t {
+        const uint32_t z = n2 >= 8 ? dq_swz(sl % n2) : dq_swz(sl);
+        if constexpr (k1w == 2) return sl * 128u + (((k1 >> 2) ^ z) << 4) + (k1 & 3u) * 4u;
+        else return sl * 128u + ((((k1 >> 2) + (uint32_t)h) ^ z) << 4);
+    };
+    float v[32];
+    if (live) {
+        decode_raw_scaled<FMT>(cur, p.had_norm, v);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+    }
+    fwht_reg<32, true>(v);
+    {
+        uint8_t* rowp = ws + l * 128u;
+        const uint32_t z = dq_swz(l);
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+            *reinterpret_cast<float4*>(rowp + ((ch ^ z) << 4)) =
+                make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int k2 = 0; k2 < n2; ++k2) {
+        const uint32_t sl = b * n2 + (uint32_t)k2;  // sub-row of this block
+        if constexpr (k1w == 2) {
+            const float2 q = *reinterpret_cast<const float2*>(ws + rd_off(sl, 0));
+            a[k2][0] = q.x;
+            a[k2][1] = q.y;
+        } else {
+#pragma unroll
+            for (int h = 0; h < k1w / 4; ++h) {
+                const float4 q = *reinterpret_cast<const float4*>(ws + rd_off(sl, h));
+                a[k2][4 * h] = q.x;
+                a[k2][4 * h + 1] = q.y;
+                a[k2][4 * h + 2] = q.z;
+                a[k2][4 * h + 3] = q.w;
+            }
+        }
+    }
+    const float2 m1 = make_float2(-1.0f, -1.0f);
+#pragma unroll
+    for (int st = 1; st < n2; st <<= 1) {
+#pragma unroll
+        for (int k2 = 0; k2 < n2; ++k2) {
+            if ((k2 & st) == 0) {
+#pragma unroll
+                for (int i = 0; i < k1w; i += 2) {
+                    const float2 x0 = make_float2(a[k2][i], a[k2][i + 1]);
+                    const float2 x1 = make_float2(a[k2 + st][i], a[k2 + st][i + 1]);
+                    const float2 sm = __fadd2_rn(x0, x1), df = __ffma2_rn(x1, m1, x0);
+                    a[k2][i] = sm.x;
+                    a[k2][i + 1] = sm.y;
+                    a[k2 + st][i] = df.x;
+                    a[k2 + st][i + 1] = df.y;
+                }
+            }
+        }
+    }
+    if constexpr (SIGNED) {
+        // output column cb + 32 k2 + i has pattern index (k1 + 32 k2 + i) mod
+        // min(n, 128): word k2 mod (period / 32), bit k1 + i
+        constexpr int kWords = (HAD < 128 ? HAD : 128) / 32;
+#pragma unroll
+        for (int k2 = 0; k2 < n2; ++k2) apply_signs<k1w>(a[k2], p.signs[k2 % kWords] >> k1);
+    }
+}
+
+// bf16 of the lane's phase-B outputs, k1w consecutive columns per k2 (32 columns apart).
+template <int HAD>
+__device__ __forceinline__ void dq_store_slices(uint16_t* dst0, const float (&a)[HadShape<HAD>::n2][HadShape<HAD>::k1w]) {
+    constexpr int n2 = HadShape<HAD>::n2, k1w = HadShape<HAD>::k1w;
+#pragma unroll
+    for (int k2 = 0; k2 < n2; ++k2) {
+        uint16_t* dst = dst0 + 32 * k2;
+        if constexpr (k1w == 2) {
+            *reinterpret_cast<uint32_t*>(dst) = bf16x2_pack(a[k2][0], a[k2][1]);
+        } else if constexpr (k1w == 4) {
+            *reinterpret_cast<uint2*>(dst) =
+                make_uint2(bf16x2_pack(a[k2][0], a[k2][1]), bf16x2_pack(a[k2][2], a[k2][3]));
+        } else {
+#pragma unroll
+            for (int h = 0; h < k1w / 8; ++h)
+                reinterpret_cast<uint4*>(dst)[h] = make_uint4(
+                    bf16x2_pack(a[k2][8 * h + 0], a[k2][8 * h + 1]), bf16x2_pack(a[k2][8 * h + 2], a[k2][8 * h + 3]),
+                    bf16x2_pack(a[k2][8 * h + 4], a[k2][8 * h + 5]), bf16x2_pack(a[k2][8 * h + 6], a[k2][8 * h + 7]));
+        }
+    }
+}
+
 template <int FMT, int HAD, bool SIGNED = false>
 __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_warp_kernel(const DequantParams p) {
     pdl_wait();
@@ -327,14 +429,6 @@ __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_warp_kern
     auto in_range = [&](int32_t r, int32_t c) {  // K % 64 == 0: whole 32-column pieces
         return (int64_t)r * 2 + r2 < p.M && (int64_t)c * kTileCols + 32 * l < p.K;
     };
-    // phase-B read offset of sub-row sl = b n2 + k2 within the lane's row
-    // (swizzled chunk); for n2 >= 8, b n2 is a multiple of 8 and the swizzle
-    // depends on k2 alone, a constant of the unrolled loop
-    auto rd_off = [&](uint32_t sl, int h) -> uint32_t {
-        const uint32_t z = n2 >= 8 ? dq_swz(sl % n2) : dq_swz(sl);
-        if constexpr (k1w == 2) return sl * 128u + (((k1 >> 2) ^ z) << 4) + (k1 & 3u) * 4u;
-        else return sl * 128u + ((((k1 >> 2) + (uint32_t)h) ^ z) << 4);
-    };
     RawUnit cur{};
     if (rp < n_rp && in_range(rp, ct)) load_raw<FMT>(p, (int64_t)rp * 2 + r2, (int64_t)ct * kTileCols + 32 * l, 32, cur);
     while (rp < n_rp) {
@@ -345,92 +439,135 @@ __global__ void __launch_bounds__(kThreads, kDequantCtasPerSm) dequant_warp_kern
         advance(rn, cn);
         RawUnit nxt{};
         if (rn < n_rp && in_range(rn, cn)) load_raw<FMT>(p, (int64_t)rn * 2 + r2, (int64_t)cn * kTileCols + 32 * l, 32, nxt);
-        float v[32];
-        if (live) {
-            decode_raw_scaled<FMT>(cur, p.had_norm, v);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
-        }
-        cur = nxt;
-        fwht_reg<32, true>(v);
         __syncwarp();  // the previous unit's reads of this warp's scratch are done
-        {
-            uint8_t* rowp = ws + l * 128u;
-            const uint32_t z = dq_swz(l);
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-                *reinterpret_cast<float4*>(rowp + ((ch ^ z) << 4)) =
-                    make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
-        }
-        __syncwarp();
         float a[n2][k1w];
-#pragma unroll
-        for (int k2 = 0; k2 < n2; ++k2) {
-            const uint32_t sl = b * n2 + (uint32_t)k2;  // sub-row of this block
-            if constexpr (k1w == 2) {
-                const float2 q = *reinterpret_cast<const float2*>(ws + rd_off(sl, 0));
-                a[k2][0] = q.x;
-                a[k2][1] = q.y;
-            } else {
-#pragma unroll
-                for (int h = 0; h < k1w / 4; ++h) {
-                    const float4 q = *reinterpret_cast<const float4*>(ws + rd_off(sl, h));
-                    a[k2][4 * h] = q.x;
-                    a[k2][4 * h + 1] = q.y;
-                    a[k2][4 * h + 2] = q.z;
-                    a[k2][4 * h + 3] = q.w;
-                }
-            }
-        }
-        const float2 m1 = make_float2(-1.0f, -1.0f);
-#pragma unroll
-        for (int st = 1; st < n2; st <<= 1) {
-#pragma unroll
-            for (int k2 = 0; k2 < n2; ++k2) {
-                if ((k2 & st) == 0) {
-#pragma unroll
-                    for (int i = 0; i < k1w; i += 2) {
-                        const float2 x0 = make_float2(a[k2][i], a[k2][i + 1]);
-                        const float2 x1 = make_float2(a[k2 + st][i], a[k2 + st][i + 1]);
-                        const float2 sm = __fadd2_rn(x0, x1), df = __ffma2_rn(x1, m1, x0);
-                        a[k2][i] = sm.x;
-                        a[k2][i + 1] = sm.y;
-                        a[k2 + st][i] = df.x;
-                        a[k2 + st][i + 1] = df.y;
-                    }
-                }
-            }
-        }
-        if constexpr (SIGNED) {
-            // output column cb + 32 k2 + i has pattern index (k1 + 32 k2 + i) mod
-            // min(n, 128): word k2 mod (period / 32), bit k1 + i
-            constexpr int kWords = (HAD < 128 ? HAD : 128) / 32;
-#pragma unroll
-            for (int k2 = 0; k2 < n2; ++k2) apply_signs<k1w>(a[k2], p.signs[k2 % kWords] >> k1);
-        }
+        dq_unit<FMT, HAD, SIGNED>(p, cur, live, ws, l, b, k1, a);
         // the block's columns exist when its first one does (K % n == 0)
-        if (row < p.M && cb < p.K) {
-            uint16_t* dst0 = p.y + row * p.K + cb;
-#pragma unroll
-            for (int k2 = 0; k2 < n2; ++k2) {
-                uint16_t* dst = dst0 + 32 * k2;
-                if constexpr (k1w == 2) {
-                    *reinterpret_cast<uint32_t*>(dst) = bf16x2_pack(a[k2][0], a[k2][1]);
-                } else if constexpr (k1w == 4) {
-                    *reinterpret_cast<uint2*>(dst) =
-                        make_uint2(bf16x2_pack(a[k2][0], a[k2][1]), bf16x2_pack(a[k2][2], a[k2][3]));
-                } else {
-#pragma unroll
-                    for (int h = 0; h < k1w / 8; ++h)
-                        reinterpret_cast<uint4*>(dst)[h] = make_uint4(
-                            bf16x2_pack(a[k2][8 * h + 0], a[k2][8 * h + 1]), bf16x2_pack(a[k2][8 * h + 2], a[k2][8 * h + 3]),
-                            bf16x2_pack(a[k2][8 * h + 4], a[k2][8 * h + 5]), bf16x2_pack(a[k2][8 * h + 6], a[k2][8 * h + 7]));
-                }
-            }
-        }
+        if (row < p.M && cb < p.K) dq_store_slices<HAD>(p.y + row * p.K + cb, a);
+        cur = nxt;
         rp = rn;
         ct = cn;
+    }
+}
+
+// ---------------------------------------------------------------- TMA-fed dequantizer
+// The same unit walk and arithmetic as dequant_warp_kernel, for K % 512 == 0
+// and the linear scale layout.  Each warp keeps its next units' codes, scale
+// bytes and group scales in a private ring of kDqStages shared-memory stages
+// filled by 2-D TMA copies (boxes of 2 rows: 256 code bytes, 32 or 16 scale
+// bytes, 4 group scales), so the decode never waits on HBM; lane 0 refills a
+// stage as soon as every lane has decoded it.
+constexpr int kDqStages = 3;
+constexpr uint32_t kDqStageBytes = 768;  // codes 2 x 256 | scale bytes 2 x 32 | group scales 2 x 16
+constexpr uint32_t kDqRingSmem = kDqWarpSmem + kDqStages * kDqStageBytes + 128;  // + the stage barriers
+
+template <int FMT, int HAD, bool SIGNED = false>
+__global__ void __launch_bounds__(kThreads, kDequantCtasPerSm)
+    dequant_tma_kernel(const DequantParams p, const __grid_constant__ CUtensorMap codes_map,
+                       const __grid_constant__ CUtensorMap scales_map, const __grid_constant__ CUtensorMap g_map) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    constexpr int n2 = HadShape<HAD>::n2, k1w = HadShape<HAD>::k1w;
+    static_assert(HAD >= 64 && n2 * k1w == 32, "block sizes 64..512");
+    constexpr int kWarps = kThreads / 32;
+    constexpr uint32_t kScaleBytes = FMT == FMT_MXFP4 ? 32u : 64u;  // both rows' scale bytes
+    constexpr uint32_t kTx = 512u + kScaleBytes + (FMT == FMT_DUAL ? 32u : 0u);
+    const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint8_t* const wbase = smem_raw + warp * kDqRingSmem;
+    uint8_t* const ws = wbase + (lane >> 4) * 2048u;  // this lane's row of the exchange
+    uint8_t* const ring = wbase + kDqWarpSmem;
+    const uint32_t bar0 = smem_u32(ring + kDqStages * kDqStageBytes);
+    const uint32_t r2 = lane >> 4, l = lane & 15;
+    const uint32_t b = n2 == 16 ? 0u : l / n2, tau = l % n2, k1 = k1w * tau;
+    if (lane == 0) {
+        for (int s = 0; s < kDqStages; ++s) mbar_init(bar0 + 8 * s, 1);
+        fence_barrier_init();
+        prefetch_tmap(&codes_map);
+        prefetch_tmap(&scales_map);
+        if constexpr (FMT == FMT_DUAL) prefetch_tmap(&g_map);
+    }
+    __syncwarp();
+    pdl_wait();
+    pdl_trigger();
+    const int32_t n_ct = (int32_t)p.n_col_tiles, n_rp = (int32_t)((p.M + 1) / 2);
+    const int32_t stride = (int32_t)gridDim.x * kWarps;
+    const int32_t drp = stride / n_ct, dct = stride % n_ct;
+    const int32_t u0 = (int32_t)blockIdx.x * kWarps + (int32_t)warp;
+    int32_t rp = u0 / n_ct, ct = u0 % n_ct;
+    auto advance = [&](int32_t& r, int32_t& c) {
+        c += dct;
+        r += drp;
+        if (c >= n_ct) {
+            c -= n_ct;
+            ++r;
+        }
+    };
+    // unit (r, c) into stage s (lane 0); rows past M read as zeros
+    auto issue = [&](int s, int32_t r, int32_t c) {
+        uint8_t* st = ring + s * kDqStageBytes;
+        const uint32_t bar = bar0 + 8 * s;
+        mbar_arrive_expect_tx(bar, kTx);
+        tma_load_2d(smem_u32(st), &codes_map, c * (kTileCols / 2), 2 * r, bar);
+        tma_load_2d(smem_u32(st + 512), &scales_map, c * (int32_t)(kScaleBytes / 2), 2 * r, bar);
+        if constexpr (FMT == FMT_DUAL) tma_load_2d(smem_u32(st + 640), &g_map, c * 4, 2 * r, bar);
+    };
+    int32_t irp = rp, ict = ct;  // the next unit to issue
+    if (lane == 0) {
+        for (int s = 0; s < kDqStages && irp < n_rp; ++s) {
+            issue(s, irp, ict);
+            advance(irp, ict);
+        }
+    } else {
+        for (int s = 0; s < kDqStages && irp < n_rp; ++s) advance(irp, ict);
+    }
+    const float s_t = FMT == FMT_NVFP4 ? __ldg(p.scale_fp32) : 0.0f;
+    uint32_t it = 0;
+    while (rp < n_rp) {
+        const int s = (int)(it % kDqStages);
+        const bool ok = mbar_wait(bar0 + 8 * s, (it / kDqStages) & 1u);
+        if (!__all_sync(0xffffffffu, ok)) {
+            if (lane == 0) {
+                atomicOr(&g_device_error, kErrWaitTimeout);
+                // every copy issued into the ring lands before the CTA may exit
+                int32_t r = rp, c = ct;
+                for (uint32_t k = it; k < it + kDqStages && r < n_rp; ++k, advance(r, c))
+                    (void)mbar_wait(bar0 + 8 * (k % kDqStages), (k / kDqStages) & 1u);
+            }
+            break;
+        }
+        const uint8_t* st = ring + s * kDqStageBytes;
+        RawUnit cur;
+        {
+            const uint4 q = *reinterpret_cast<const uint4*>(st + 256 * r2 + 16 * l);
+            cur.w[0] = q.x;
+            cur.w[1] = q.y;
+            cur.w[2] = q.z;
+            cur.w[3] = q.w;
+            if constexpr (FMT == FMT_MXFP4) {
+                cur.e0 = st[512 + 16 * r2 + l];
+                cur.e1 = 0u;
+                cur.s = 0.0f;
+            } else {
+                const uint32_t e = *reinterpret_cast<const uint16_t*>(st + 512 + 32 * r2 + 2 * l);
+                cur.e0 = e & 0xffu;
+                cur.e1 = e >> 8;
+                cur.s = FMT == FMT_DUAL ? *reinterpret_cast<const float*>(st + 640 + 16 * r2 + 4 * (l >> 2)) : s_t;
+            }
+        }
+        const int64_t row = (int64_t)rp * 2 + r2;
+        const bool live = row < p.M;
+        __syncwarp();  // the previous unit's reads of the scratch are done
+        float a[n2][k1w];
+        dq_unit<FMT, HAD, SIGNED>(p, cur, live, ws, l, b, k1, a);
+        // Every lane has used all it loaded from stage s (dq_unit consumed the
+        // codes and scales before its first warp barrier): lane 0 refills it.
+        if (lane == 0 && irp < n_rp) {
+            fence_proxy_async_smem();
+            issue(s, irp, ict);
+        }
+        if (irp < n_rp) advance(irp, ict);
+        if (live) dq_store_slices<HAD>(p.y + row * p.K + (int64_t)ct * kTileCols + (int64_t)b * HAD + k1, a);
+        advance(rp, ct);
+        ++it;
     }
 }
 

@@ -354,6 +354,26 @@ def test_dequantize_inverse_hadamard_grid_stride(fq, n, fmt):
     assert_roundtrip(bf16_torch_to_bits(y)[rows], want, n, name=f"inv-had{n}-{fmt}-grid")
 
 
+@pytest.mark.parametrize("n,fmt,K,layout", [
+    (512, "dual", 4096, 1), (128, "nvfp4", 1024, 1), (64, "mxfp4", 1024, 1),  # tiled scale layout
+    (128, "dual", 1152, 0), (64, "nvfp4", 1088, 0), (256, "mxfp4", 1280, 0),  # K not a multiple of 512
+])
+def test_dequantize_inverse_hadamard_other_layouts(fq, n, fmt, K, layout):
+    """n >= 64 with the tiled scale layout or K % 512 != 0: the dequantizer that
+    loads codes and scales itself (the TMA-fed one needs linear scales and
+    K % 512 == 0).  Random payloads, odd row count."""
+    M = 301
+    codes, scales, sc = workloads.random_payload(M, K, fmt, seed=n + K)
+    s_dev = oracle.swizzle_scales(scales) if layout == 1 else scales
+    f = {"nvfp4": fq.FP4Q_NVFP4, "mxfp4": fq.FP4Q_MXFP4, "dual": fq.FP4Q_NVFP4_DUAL}[fmt]
+    sct = (None if sc is None else
+           torch.tensor([sc], device="cuda") if fmt == "nvfp4" else torch.from_numpy(sc).cuda())
+    y = fq.dequantize(f, torch.from_numpy(codes).cuda(), torch.from_numpy(s_dev).cuda(), sct, K, layout, n)
+    torch.cuda.synchronize()
+    want = oracle.dequantize(fmt, codes, scales, sc, inv_had=n)
+    assert_roundtrip(bf16_torch_to_bits(y), want, n, name=f"inv-had{n}-{fmt}-K{K}-layout{layout}")
+
+
 @pytest.mark.parametrize("layout", [0, 1])
 def test_empty_inputs(fq, layout):
     """M = 0 through every entry point: no launch, no error, empty outputs."""
