@@ -93,6 +93,13 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
                  "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
                  : "memory");
 }
+// The dual format's group scale of a group maximum gm: gm / 2688, correctly
+// rounded (the IEEE division for gm < 2^-90, out of line).
+__device__ __noinline__ float group_scale_tiny(float gm) { return __fdiv_rn(gm, 2688.0f); }
+__device__ __forceinline__ float group_scale(float gm) {
+    return gm >= 0x1p-90f ? div_split(-gm, 2688.0f, rcp2688()) : group_scale_tiny(gm);
+}
+
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // B = -2^-4 * D * H_128 (K-major, 128-byte swizzle) for n = 256 and 512, its
@@ -177,6 +184,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 
     const int64_t n_my = p.n_tiles > (int64_t)blockIdx.x ? (p.n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     float my_amax = 0.0f;
+
 
     if (warp == 0 || warp == 2) {
         // ------------------------------------------------ TMA producers: G sub-tiles per tile,
@@ -298,10 +306,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                 }
 #pragma unroll
                 for (int a = 0; a < G; ++a) {
-                    float mm = fmaxf(fabsf(z[a][0]), fabsf(z[a][1]));
+                    float mm = m[a];
 #pragma unroll
-                    for (int i = 2; i < 8; i += 2) mm = max3(mm, fabsf(z[a][i]), fabsf(z[a][i + 1]));
-                    m[a] = fmaxf(m[a], mm);
+                    for (int i = 0; i < 8; i += 2) mm = max3(mm, fabsf(z[a][i]), fabsf(z[a][i + 1]));
+                    m[a] = mm;
                     if constexpr (!AMAX_ONLY) tmem_st8(tbuf + a * kMmaTile + pos, z[a]);
                 }
             }
@@ -323,7 +331,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                 // the tcgen05 fences that order their TMEM stores before our loads.
                 // The dual format also exchanges its group maxima here.
                 tmem_wait_st();
-                float gs[G];
+                float gs[G / 2];
                 float* rp = red2 + (j & 1) * (4 * 4 * kMmaTile);
                 if constexpr (FMT == FMT_DUAL) {
 #pragma unroll
@@ -340,12 +348,11 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                 tc_fence_after();
                 if constexpr (FMT == FMT_DUAL) {  // group maxima over the four warpgroups
 #pragma unroll
-                    for (int a = 0; a < G; ++a) {
-                        float gm = rp[a * kMmaTile + rowt];
-#pragma unroll
-                        for (int w = 1; w < 4; ++w) gm = fmaxf(gm, rp[(w * 4 + a) * kMmaTile + rowt]);
-                        gm *= fold;
-                        gs[a] = (gm >= 0x1p-90f) ? div_split(-gm, 2688.0f, rcp2688()) : __fdiv_rn(gm, 2688.0f);
+                    for (int h = 0; h < G / 2; ++h) {  // the groups this warpgroup quantizes (pass 2)
+                        const int a = G == 4 ? 2 * h + (int)(wg / 2) : (int)(wg % 2);
+                        const float* rg = rp + a * kMmaTile + rowt;
+                        const float gm = fmaxf(fmaxf(rg[0], rg[4 * kMmaTile]), fmaxf(rg[8 * kMmaTile], rg[12 * kMmaTile]));
+                        gs[h] = group_scale(gm * fold);
                     }
                 }
                 // ---- pass 2: two warpgroups per output group, each quantizing two
@@ -366,8 +373,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                     float g = 0.0f;
                     if constexpr (FMT == FMT_DUAL) {
                         g = gs[0];
-#pragma unroll
-                        for (int q = 1; q < G; ++q) g = a == q ? gs[q] : g;
+                        if constexpr (G == 4) g = h ? gs[G / 2 - 1] : g;  // no indexed (local) array
                         if (live && c == 0) p.scale_fp32[row * (p.K / 128) + ct * G + a] = g;
                     }
                     const ScaleCtx ctx = FMT == FMT_DUAL ? make_ctx(g) : ctx_t;
