@@ -93,6 +93,26 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
                  "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
                  : "memory");
 }
+// The G consecutive group scales of a row and tile: one 16- or 8-byte store
+// when the address allows it.
+template <int G>
+__device__ __forceinline__ void store_group_scales(float* dst, const float (&g)[G]) {
+    const uintptr_t al = reinterpret_cast<uintptr_t>(dst);
+    if constexpr (G == 4) {
+        if ((al & 15) == 0) {
+            *reinterpret_cast<float4*>(dst) = make_float4(g[0], g[1], g[2], g[3]);
+            return;
+        }
+    }
+    if ((al & 7) == 0) {
+#pragma unroll
+        for (int a = 0; a < G; a += 2) *reinterpret_cast<float2*>(dst + a) = make_float2(g[a], g[a + 1]);
+        return;
+    }
+#pragma unroll
+    for (int a = 0; a < G; ++a) dst[a] = g[a];
+}
+
 // The dual format's group scale of a group maximum gm: gm / 2688, correctly
 // rounded (the IEEE division for gm < 2^-90, out of line).
 __device__ __noinline__ float group_scale_tiny(float gm) { return __fdiv_rn(gm, 2688.0f); }
@@ -184,7 +204,6 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 
     const int64_t n_my = p.n_tiles > (int64_t)blockIdx.x ? (p.n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     float my_amax = 0.0f;
-
 
     if (warp == 0 || warp == 2) {
         // ------------------------------------------------ TMA producers: G sub-tiles per tile,
@@ -347,12 +366,25 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                 }
                 tc_fence_after();
                 if constexpr (FMT == FMT_DUAL) {  // group maxima over the four warpgroups
-#pragma unroll
-                    for (int h = 0; h < G / 2; ++h) {  // the groups this warpgroup quantizes (pass 2)
-                        const int a = G == 4 ? 2 * h + (int)(wg / 2) : (int)(wg % 2);
+                    auto gscale = [&](int a) {
                         const float* rg = rp + a * kMmaTile + rowt;
                         const float gm = fmaxf(fmaxf(rg[0], rg[4 * kMmaTile]), fmaxf(rg[8 * kMmaTile], rg[12 * kMmaTile]));
-                        gs[h] = group_scale(gm * fold);
+                        return group_scale(gm * fold);
+                    };
+                    if (wg == 0) {
+                        // the first warpgroup writes the row's G group scales of the
+                        // tile with one store (a 4-byte store per group from two
+                        // warpgroups per round cost 2.5 us on the C5 quantizer)
+                        float ga[G];
+#pragma unroll
+                        for (int a = 0; a < G; ++a) ga[a] = gscale(a);
+                        if (live) store_group_scales<G>(p.scale_fp32 + row * (p.K / 128) + ct * G, ga);
+#pragma unroll
+                        for (int h = 0; h < G / 2; ++h) gs[h] = ga[G == 4 ? 2 * h : 0];
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < G / 2; ++h)  // the groups this warpgroup quantizes (pass 2)
+                            gs[h] = gscale(G == 4 ? 2 * h + (int)(wg / 2) : (int)(wg % 2));
                     }
                 }
                 // ---- pass 2: two warpgroups per output group, each quantizing two
@@ -374,7 +406,6 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                     if constexpr (FMT == FMT_DUAL) {
                         g = gs[0];
                         if constexpr (G == 4) g = h ? gs[G / 2 - 1] : g;  // no indexed (local) array
-                        if (live && c == 0) p.scale_fp32[row * (p.K / 128) + ct * G + a] = g;
                     }
                     const ScaleCtx ctx = FMT == FMT_DUAL ? make_ctx(g) : ctx_t;
                     const int64_t col = ct * HAD + a * kMmaTile + 32 * c;  // first column of the pair
