@@ -348,6 +348,56 @@ def arc(x_bits, gamma_bits, perm, outliers, eps: float = 1e-6, s_t: float | None
     return c, s, np.float32(s_t), y
 
 
+def arc_alignment(y, outliers, s_t, codes, scales, fmt: str = "nvfp4"):
+    """Block alignment factors of the ARCQuant two-stage path (ARCQuant summary,
+    "Analyse de la Borne d'Erreur Theorique": the alignment overhead of the two
+    stages, about 1.266, against under 2 for MXFP8).  Reading: a block's grid is
+    aligned to its content when the decoded block scale d equals amax / 6 (the
+    block maximum on the top E2M1 value); the factor phi = d / (amax / 6) is
+    how far the stored scale moved it.  One E4M3 step is 2^-3 of the value, and
+    (1 + 2^-3)^2 = 1.265625 is the page's figure for two stages; round to
+    nearest keeps phi within 1 +- 2^-4 while the scale is a normal E4M3 number
+    (MXFP4's power-of-two scale, chosen from the exponent of amax: phi in
+    (0.75, 1.5]).
+
+    ``y`` [M, K] is the prepared fp32 matrix and ``codes`` / ``scales`` its
+    oracle quantization (``arc``).  The residuals are recomputed the way the
+    quantizer forms them (fp32).  Returns ``(phi_primary [M, K/B],
+    phi_residual [M, S/B], normal_primary, normal_residual)``: the factors
+    (NaN for all-zero blocks) and masks of the blocks whose scale byte is a
+    normal E4M3 value (NVFP4; all True for MXFP4)."""
+    y = _f32(y)
+    M, K = y.shape
+    o = np.asarray(outliers, np.int64)
+    S = o.size
+    B = 16 if fmt == "nvfp4" else 32
+    cv = e2m1_decode(unpack_codes(np.asarray(codes)))  # [M, K + S] E2M1 values
+    sb = np.asarray(scales, np.uint8).reshape(M, (K + S) // B)
+    if fmt == "nvfp4":
+        d = (e4m3_decode(sb).astype(np.float32) * np.float32(s_t)).astype(np.float32)
+        unit = e4m3_decode(sb).astype(np.float32)
+        normal = (sb & 0x78) != 0  # exponent field non-zero
+    else:
+        d = e8m0_decode(sb).astype(np.float32)
+        unit = d
+        normal = np.ones(sb.shape, bool)
+    # residual of outlier position p: y[p] - dq(p), dq as the dequantizer forms it
+    cp = cv[:, o].astype(np.float32)
+    up = unit[:, o // B]
+    dq = (cp * up).astype(np.float32)
+    if fmt == "nvfp4":
+        dq = (dq * np.float32(s_t)).astype(np.float32)
+    res = (y[:, o] - dq).astype(np.float32)
+
+    def phi(vals, dd):
+        am = np.abs(vals.astype(np.float64)).reshape(M, -1, B).max(axis=2)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            return np.where(am > 0, dd.astype(np.float64) / (am / 6.0), np.nan)
+
+    nb = K // B
+    return phi(y, d[:, :nb]), phi(res, d[:, nb:]), normal[:, :nb], normal[:, nb:]
+
+
 def dequantize(fmt: str, codes, scales, scale=None, inv_had: int = 0, signs=None) -> np.ndarray:
     """Dequantize to fp32 (then optionally inverse block Hadamard, and with a
     sign pattern the inverse D H of the random-sign rotation); returns fp32."""
