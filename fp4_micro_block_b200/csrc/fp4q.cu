@@ -491,7 +491,9 @@ fp4q_status launch_dequant_h(int had, const DequantParams& p, int sms, cudaStrea
 template <int FMT, bool AMAX_ONLY>
 struct ArcKern {
     static constexpr void (*fn)(const ArcParams) = arc_kernel<FMT, AMAX_ONLY>;
-    static int total(int64_t K, int64_t S, int warps) { return arc_layout<AMAX_ONLY>(K, S, warps).total; }
+    static constexpr int wpp = arc_warps_per_pair<FMT, AMAX_ONLY>();
+    static constexpr int max_warps = arc_max_warps<FMT, AMAX_ONLY>();
+    static int total(int64_t K, int64_t S, int warps) { return arc_layout<AMAX_ONLY>(K, S, warps / wpp).total; }
 };
 
 // ---------------------------------------------------------------- self-test kernel
@@ -682,17 +684,17 @@ FP4Q_API fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int6
     p.partials = static_cast<float*>(workspace);
     p.swizzled = layout == FP4Q_SCALES_SWIZZLED;
     p.dynamic = dynamic;
-    // Warps per CTA (a row pair each): as many as the shared memory holds, up
-    // to the kernel's launch bound.
+    // Warps per CTA (the kernel's warps per row pair times the pairs): as many pairs as the
+    // shared memory holds, up to the kernel's launch bound.
     constexpr int kSmemMax = 227 * 1024;
-    auto warps_for = [&](auto amax_only) -> int {
-        constexpr bool A = decltype(amax_only)::value;
-        for (int w = arc_max_warps<A>(); w >= 1; --w)
-            if (arc_layout<A>(K, S, w).total <= kSmemMax) return w;
+    auto warps_for = [&](auto kern) -> int {
+        using Kn = decltype(kern);
+        for (int slots = Kn::max_warps / Kn::wpp; slots >= 1; --slots)
+            if (Kn::total(K, S, slots * Kn::wpp) <= kSmemMax) return slots * Kn::wpp;
         return 0;
     };
-    const int W = warps_for(std::false_type{});
-    const int Wa = dynamic ? warps_for(std::true_type{}) : 1;
+    const int W = mx ? warps_for(ArcKern<FMT_MXFP4, false>{}) : warps_for(ArcKern<FMT_NVFP4, false>{});
+    const int Wa = dynamic ? warps_for(ArcKern<FMT_NVFP4, true>{}) : 1;
     if (W == 0 || Wa == 0) return FP4Q_ERR_UNSUPPORTED;
     const int64_t pairs = (M + 1) / 2;
     if (p.swizzled) {
@@ -703,7 +705,8 @@ FP4Q_API fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int6
     }
     // The shared-memory size depends on K and S, so the attribute is set on every call.
     auto run = [&](auto kern, int warps) -> fp4q_status {
-        const int grid = (int)std::min<int64_t>({(pairs + warps - 1) / warps, (int64_t)sms, (int64_t)kMaxGrid});
+        const int slots = warps / decltype(kern)::wpp;
+        const int grid = (int)std::min<int64_t>({(pairs + slots - 1) / slots, (int64_t)sms, (int64_t)kMaxGrid});
         p.warps = warps;
         const int smem = decltype(kern)::total(K, S, warps);
         if (smem > 48 * 1024 &&

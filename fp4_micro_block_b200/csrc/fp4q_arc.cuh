@@ -4,10 +4,13 @@
 // summary, "Methodologie" items 1-5), in NVFP4 or MXFP4 ("Generalisabilite":
 // the scheme carries over to MXFP4).
 //
-// One warp owns a PAIR of rows at a time: there is no CTA-wide barrier on the
-// path.  Each warp streams its row pairs through its own 4K-byte buffer, filled
-// by two 1-D bulk copies (row 0 in the first half, row 1 in the second).  Per
-// pair:
+// Two warps own a PAIR of rows at a time (the amax pre-pass: one warp): there
+// is no CTA-wide barrier on the path, only a 64-thread named barrier between
+// the two warps of a pair.  They stream their row pairs through a shared 4K-byte
+// buffer, filled by two 1-D bulk copies (row 0 in the first half, row 1 in the
+// second), and split every step of a pair between them (alternate 16-byte
+// chunks in step 1, alternate 32-block groups in steps 2 and 3), which halves
+// the registers a warp holds and doubles the warps an SM runs.  Per pair:
 //   1. natural order (conflict-free 16-byte reads of both rows): the sum of
 //      squares of each row, and one 32-bit word per channel holding the bf16 of
 //      row 0 (low half) and of row 1 (high half), written IN PLACE: lane l
@@ -27,8 +30,8 @@
 //      y - dequant(primary) goes to a per-warp buffer in position order; after
 //      a warp barrier the lanes quantize the residual blocks (residual column j
 //      reads the slot of outlier j); then the buffer takes the next pair.
-// A warp waits for each pair's copies; the other warps of the SM (up to 12,
-// one buffer each) hide that latency.
+// The two warps wait for each pair's copies; the other pairs of the SM (up to
+// 11, one buffer each) hide that latency.
 // Per CTA (built once): for every position q a 32-bit word (byte offset of the
 // word of channel perm[q] | bf16 gamma of that channel << 16), laid out so that
 // the 16-byte loads of 32 lanes (blocks b = lane + 32 i) are consecutive; per
@@ -42,15 +45,15 @@
 
 namespace fp4q {
 
-#ifndef FP4Q_ARC_MAX_WARPS
-#define FP4Q_ARC_MAX_WARPS 12
-#endif
-// Launch bounds (warps per CTA, one CTA per SM): the quantizer keeps two
-// blocks of both rows in registers; the amax pre-pass is a light streaming loop.
-constexpr int kArcMaxWarps = FP4Q_ARC_MAX_WARPS;
-constexpr int kArcAmaxMaxWarps = 16;
-template <bool AMAX_ONLY>
-constexpr int arc_max_warps() { return AMAX_ONLY ? kArcAmaxMaxWarps : kArcMaxWarps; }
+// Launch bounds (warps per CTA, one CTA per SM).  The NVFP4 quantizer runs up to
+// 10 row pairs of two warps (one 16-block of both rows in registers at a time,
+// at most 102 registers a thread); the MXFP4 quantizer, whose 32-blocks hold
+// twice the values, one warp per pair (12 pairs); the amax pre-pass is a light
+// streaming loop with one warp per pair.
+template <int FMT, bool AMAX_ONLY>
+__host__ __device__ constexpr int arc_max_warps() { return AMAX_ONLY ? 16 : FMT == FMT_MXFP4 ? 12 : 20; }
+template <int FMT, bool AMAX_ONLY>
+__host__ __device__ constexpr int arc_warps_per_pair() { return (AMAX_ONLY || FMT == FMT_MXFP4) ? 1 : 2; }
 
 struct ArcParams {
     int64_t M, K, S;
@@ -67,13 +70,14 @@ struct ArcParams {
     int n_partials;
     int swizzled;
     int dynamic;
-    int warps;                // warps per CTA (one row pair each at a time)
+    int warps;                // warps per CTA (arc_warps_per_pair per row pair)
 };
 
 // Shared-memory layout (byte offsets).  CTA part: tab (u32 [K]), om (u32 per
 // 16-position group), rslot (u16 [S]), red (f32 [32]), stab (float2 [128]);
-// then per warp: the pair buffer (2 rows of bf16, then the interleaved words;
-// the pre-pass: two stages of 2 rows), residuals (f32 [2][S]), mbarriers.
+// then per pair slot: the pair buffer (2 rows of bf16, then the interleaved
+// words; the pre-pass: two stages of 2 rows), residuals (f32 [2][S]), the two
+// warps' partial sums of squares, mbarriers.
 struct ArcLayout {
     int tab, om, rslot, red, stab, warp0, warp_bytes, land, res, bar, total;
 };
@@ -81,7 +85,7 @@ struct ArcLayout {
 __host__ __device__ inline int arc_al(int64_t v) { return (int)((v + 127) / 128 * 128); }
 
 template <bool AMAX_ONLY>
-__host__ __device__ inline ArcLayout arc_layout(int64_t K, int64_t S, int warps) {
+__host__ __device__ inline ArcLayout arc_layout(int64_t K, int64_t S, int slots) {
     ArcLayout l;
     int off = 0;
     l.tab = off;
@@ -101,10 +105,10 @@ __host__ __device__ inline ArcLayout arc_layout(int64_t K, int64_t S, int warps)
     w += arc_al(stages * 2 * K * 2);
     l.res = w;
     w += AMAX_ONLY ? 0 : arc_al(2 * S * 4);
-    l.bar = w;
+    l.bar = w;  // mbarriers, then the two warps' partial sums (2 x float2) at +64
     w += 128;
     l.warp_bytes = w;
-    l.total = off + warps * w + 128;  // + alignment slack of the dynamic buffer
+    l.total = off + slots * w + 128;  // + alignment slack of the dynamic buffer
     return l;
 }
 
@@ -182,7 +186,7 @@ __device__ __forceinline__ void put_scale(const ArcParams& p, int64_t row, int64
 }
 
 template <int FMT, bool AMAX_ONLY>
-__global__ void __launch_bounds__(arc_max_warps<AMAX_ONLY>() * 32, 1) arc_kernel(const ArcParams p) {
+__global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_kernel(const ArcParams p) {
     static_assert(FMT == FMT_NVFP4 || (FMT == FMT_MXFP4 && !AMAX_ONLY), "formats of the ARC path");
     constexpr int B = FMT == FMT_MXFP4 ? 32 : 16;  // block size
     constexpr int Q = B / 4;                       // 16-byte table quads per block
@@ -192,8 +196,9 @@ __global__ void __launch_bounds__(arc_max_warps<AMAX_ONLY>() * 32, 1) arc_kernel
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                                ~uintptr_t(127));
-    const int K = (int)p.K, S = (int)p.S, nbB = K / B, ng = K / 16, W = p.warps;
-    const ArcLayout L = arc_layout<AMAX_ONLY>(p.K, p.S, W);
+    constexpr int WPP = arc_warps_per_pair<FMT, AMAX_ONLY>();
+    const int K = (int)p.K, S = (int)p.S, nbB = K / B, ng = K / 16, W = p.warps, NP = W / WPP;
+    const ArcLayout L = arc_layout<AMAX_ONLY>(p.K, p.S, NP);
     const uint32_t row_bytes = (uint32_t)K * 2u;
     uint32_t* tab = reinterpret_cast<uint32_t*>(smem + L.tab);
     uint32_t* om = reinterpret_cast<uint32_t*>(smem + L.om);
@@ -202,15 +207,28 @@ __global__ void __launch_bounds__(arc_max_warps<AMAX_ONLY>() * 32, 1) arc_kernel
     float2* stab = reinterpret_cast<float2*>(smem + L.stab);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nthreads = blockDim.x;
 
-    // ---- this warp's buffer and barriers; its first pairs' copies overlap the
-    // building of the CTA tables below
-    uint8_t* const wb = smem + L.warp0 + (size_t)warp * L.warp_bytes;
+    // ---- this pair slot's buffer and barriers (warps WPP ps .. WPP ps + WPP - 1);
+    // its first pairs' copies overlap the building of the CTA tables below
+    const int ps = warp / WPP, sub = warp % WPP;
+    uint8_t* const wb = smem + L.warp0 + (size_t)ps * L.warp_bytes;
     uint64_t* const bars = reinterpret_cast<uint64_t*>(wb + L.bar);
+    float2* const part = reinterpret_cast<float2*>(wb + L.bar + 64);  // the warps' partial sums
+    // The warps of a pair meet at a 64-thread named barrier (id 1 + ps; 0 is the
+    // CTA's); a vote on it makes every early exit a joint decision.
+    auto pair_sync = [&]() {
+        if constexpr (WPP > 1) bar_sync(1 + ps, 32 * WPP);
+        else __syncwarp();
+    };
+    auto pair_all = [&](bool v) -> bool {
+        v = __all_sync(0xffffffffu, v);
+        if constexpr (WPP > 1) v = bar_and(1 + ps, 32 * WPP, v);
+        return v;
+    };
     const int64_t P = (p.M + 1) / 2;  // row pairs
-    const int64_t gw = (int64_t)blockIdx.x * W + warp, nw = (int64_t)gridDim.x * W;
+    const int64_t gw = (int64_t)blockIdx.x * NP + ps, nw = (int64_t)gridDim.x * NP;
     const int64_t n_my = P > gw ? (P - 1 - gw) / nw + 1 : 0;
     uint8_t* const land = wb + L.land;
-    auto issue = [&](int64_t i) {  // lane 0: pair i of this warp into stage i % SR
+    auto issue = [&](int64_t i) {  // lane 0 of the first warp: pair i of the slot into stage i % SR
         const int64_t r0 = 2 * (gw + i * nw);
         const bool two = r0 + 1 < p.M;
         const uint32_t bar = smem_u32(&bars[i % SR]);
@@ -222,7 +240,7 @@ __global__ void __launch_bounds__(arc_max_warps<AMAX_ONLY>() * 32, 1) arc_kernel
         bulk_load_1d(smem_u32(dst), p.x + r0 * p.ldx_bytes, row_bytes, bar);
         if (two) bulk_load_1d(smem_u32(dst + row_bytes), p.x + (r0 + 1) * p.ldx_bytes, row_bytes, bar);
     };
-    if (lane == 0) {
+    if (sub == 0 && lane == 0) {  // (the CTA barriers below publish the initialisation)
         for (int k = 0; k < SR; ++k) mbar_init(smem_u32(&bars[k]), 1);
         fence_barrier_init();
         for (int64_t i = 0; i < min64(SR, n_my); ++i) issue(i);
@@ -315,8 +333,8 @@ __global__ void __launch_bounds__(arc_max_warps<AMAX_ONLY>() * 32, 1) arc_kernel
 
     for (int64_t i = 0; i < n_my; ++i) {
         const bool ok = mbar_wait(smem_u32(&bars[i % SR]), (uint32_t)((i / SR) & 1));
-        if (!__all_sync(0xffffffffu, ok)) {
-            if (lane == 0) {
+        if (!pair_all(ok)) {
+            if (sub == 0 && lane == 0) {
                 atomicOr(&g_device_error, kErrWaitTimeout);
                 for (int64_t k = i; k < min64(n_my, i + SR); ++k)
                     (void)mbar_wait(smem_u32(&bars[k % SR]), (uint32_t)((k / SR) & 1));
@@ -361,14 +379,14 @@ __global__ void __launch_bounds__(arc_max_warps<AMAX_ONLY>() * 32, 1) arc_kernel
             const float2 rs = make_float2(__frcp_rn(__fsqrt_rn(__fdiv_rn(ss.x, rK) + p.eps)),
                                           __frcp_rn(__fsqrt_rn(__fdiv_rn(ss.y, rK) + p.eps)));
             // every value read from the stage is consumed above: refill it
-            __syncwarp();
-            if (lane == 0 && i + SR < n_my) issue(i + SR);
+            pair_sync();
+            if (sub == 0 && lane == 0 && i + SR < n_my) issue(i + SR);
             my_amax = fmaxf(my_amax, zmax.x * rs.x);
             if (two) my_amax = fmaxf(my_amax, zmax.y * rs.y);
         } else {
             // 1. natural order, in place: sums of squares and the interleaved words
 #pragma unroll 2
-            for (int j = lane; 8 * j < K; j += 32) {
+            for (int j = lane + 32 * sub; 8 * j < K; j += 32 * WPP) {
                 const uint4 a = *reinterpret_cast<const uint4*>(l0 + 16 * j);
                 const uint4 b = two ? *reinterpret_cast<const uint4*>(l1 + 16 * j) : make_uint4(0u, 0u, 0u, 0u);
                 const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
@@ -392,10 +410,17 @@ __global__ void __launch_bounds__(arc_max_warps<AMAX_ONLY>() * 32, 1) arc_kernel
                 ss.x += __shfl_xor_sync(0xffffffffu, ss.x, o);
                 ss.y += __shfl_xor_sync(0xffffffffu, ss.y, o);
             }
+            if constexpr (WPP > 1) {
+                if (lane == 0) part[sub] = ss;
+                pair_sync();  // both warps' interleaved words and partial sums are written
+                const float2 o = part[sub ^ 1];
+                ss = make_float2(ss.x + o.x, ss.y + o.y);  // the same sum in both warps
+            } else {
+                __syncwarp();  // every lane's interleaved words are written
+            }
             const float rK = (float)K;
             const float2 rs = make_float2(__frcp_rn(__fsqrt_rn(__fdiv_rn(ss.x, rK) + p.eps)),
                                           __frcp_rn(__fsqrt_rn(__fdiv_rn(ss.y, rK) + p.eps)));
-            __syncwarp();  // every lane's interleaved words are written
 
             // 2. reordered positions: gather both rows, quantize, store
             const int64_t r1 = r0 + 1;
@@ -496,26 +521,16 @@ __global__ void __launch_bounds__(arc_max_warps<AMAX_ONLY>() * 32, 1) arc_kernel
                     }
                 }
             };
-            if constexpr (FMT == FMT_NVFP4) {
-                // two blocks per step (their gathers in flight together)
-                for (int b = lane; b < nbB; b += 64) {
-                    float2 va[B], vb[B];
-                    const bool second = b + 32 < nbB;
-                    gather(b, va);
-                    if (second) gather(b + 32, vb);
-                    emit(b, va);
-                    if (second) emit(b + 32, vb);
-                }
-            } else {  // a 32-block already has 32 gathers in flight
-                for (int b = lane; b < nbB; b += 32) {
-                    float2 va[B];
-                    gather(b, va);
-                    emit(b, va);
-                }
+            // one block of both rows per step; the warps of the pair take
+            // alternate groups of 32 blocks
+            for (int b = lane + 32 * sub; b < nbB; b += 32 * WPP) {
+                float2 va[B];
+                gather(b, va);
+                emit(b, va);
             }
-            __syncwarp();
+            pair_sync();  // every residual slot is written
             // residual blocks: slots of columns B j .. B j + B - 1 -> columns K + B j
-            for (int j = lane; B * j < S; j += 32) {
+            for (int j = lane + 32 * sub; B * j < S; j += 32 * WPP) {
                 const int64_t col = nbB + j;
                 if constexpr (FMT == FMT_NVFP4) {
                     float2 n[16];
@@ -552,10 +567,10 @@ __global__ void __launch_bounds__(arc_max_warps<AMAX_ONLY>() * 32, 1) arc_kernel
                 }
             }
             // Every value read from the buffer (the gathers) and from the
-            // residual slots has been consumed by the stores above: the buffer
-            // takes the next pair.
-            __syncwarp();
-            if (lane == 0 && i + SR < n_my) issue(i + SR);
+            // residual slots has been consumed by the stores above, in both
+            // warps: the buffer takes the next pair.
+            pair_sync();
+            if (sub == 0 && lane == 0 && i + SR < n_my) issue(i + SR);
         }
     }
 
