@@ -174,6 +174,19 @@ __device__ __forceinline__ float2 amax_pair_tree(const float2* n) {
                        fmaxf(max3(b[0], b[1], b[2]), max3(b[3], b[4], b[5])));
 }
 
+// Shared-memory loads by 32-bit shared address (the gather's table words and
+// pair words).
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint4 lds_v4(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return __byte_perm(a, b, sel);
 }
@@ -426,15 +439,16 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
             const int64_t r1 = r0 + 1;
             uint8_t* cp0 = p.codes + r0 * kcs;
             uint8_t* cp1 = p.codes + r1 * kcs;
+            const uint32_t tab_s = smem_u32(tab), l0_s = smem_u32(l0);
             // (-z row 0, -z row 1) of the B positions of block b
             auto gather = [&](int b, float2* v) {
 #pragma unroll
                 for (int k = 0; k < Q; ++k) {
-                    const uint4 tw = *reinterpret_cast<const uint4*>(tab + 4 * (k * nbB + b));
+                    const uint4 tw = lds_v4(tab_s + 16u * (uint32_t)(k * nbB + b));
                     const uint32_t wv[4] = {tw.x, tw.y, tw.z, tw.w};
 #pragma unroll
                     for (int t = 0; t < 4; ++t) {
-                        const uint32_t xw = *reinterpret_cast<const uint32_t*>(l0 + (wv[t] & 0xffffu));
+                        const uint32_t xw = lds_u32(l0_s + (wv[t] & 0xffffu));
                         const float ng_ = -__uint_as_float(wv[t] & 0xffff0000u);
                         v[4 * k + t] = fmul2(make_float2(bf16lo(xw), bf16hi(xw)), dup2(ng_));
                     }
