@@ -542,9 +542,16 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
                 gather(b, va);
                 emit(b, va);
             }
-            pair_sync();  // every residual slot is written
-            // residual blocks: slots of columns B j .. B j + B - 1 -> columns K + B j
-            for (int j = lane + 32 * sub; B * j < S; j += 32 * WPP) {
+            // Every residual slot is written, and every value gathered from the
+            // buffer has been consumed by the stores above, in both warps: the
+            // buffer takes the next pair now, its copy overlapping the residual
+            // blocks (which read only the slots; the next pair's first barrier
+            // orders them before its residuals are written).
+            pair_sync();
+            if (sub == 0 && lane == 0 && i + SR < n_my) issue(i + SR);
+            // residual blocks: slots of columns B j .. B j + B - 1 -> columns K + B j,
+            // alternate blocks to the two warps
+            for (int j = sub + WPP * lane; B * j < S; j += 32 * WPP) {
                 const int64_t col = nbB + j;
                 if constexpr (FMT == FMT_NVFP4) {
                     float2 n[16];
@@ -580,11 +587,6 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
                     }
                 }
             }
-            // Every value read from the buffer (the gathers) and from the
-            // residual slots has been consumed by the stores above, in both
-            // warps: the buffer takes the next pair.
-            pair_sync();
-            if (sub == 0 && lane == 0 && i + SR < n_my) issue(i + SR);
         }
     }
 
