@@ -207,8 +207,7 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
     pdl_wait();
     pdl_trigger();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
-                                               ~uintptr_t(127));
+    uint8_t* smem = align_shared<128>(smem_raw);
     constexpr int WPP = arc_warps_per_pair<FMT, AMAX_ONLY>();
     const int K = (int)p.K, S = (int)p.S, nbB = K / B, ng = K / 16, W = p.warps, NP = W / WPP;
     const ArcLayout L = arc_layout<AMAX_ONLY>(p.K, p.S, NP);

@@ -199,6 +199,17 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return (uint32_t)__cvta_generic_to_shared(p);
 }
 
+// The first byte of the dynamic shared buffer `base` aligned to A bytes, by
+// pointer arithmetic on the shared array: the compiler keeps the result (and
+// every pointer derived from it) in the shared address space.  Rounding the
+// address through an integer instead loses that, and every load and store
+// through the pointer becomes a generic one (slower, and waited for on the
+// long scoreboard).
+template <uint32_t A>
+__device__ __forceinline__ uint8_t* align_shared(uint8_t* base) {
+    return base + ((A - (smem_u32(base) & (A - 1))) & (A - 1));
+}
+
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
 }

@@ -168,8 +168,7 @@ __global__ void __launch_bounds__(kDqmThreads, 1)
                        const __grid_constant__ CUtensorMap g_map, const DqmParams p) {
     static_assert(FMT == FMT_NVFP4 || FMT == FMT_DUAL, "16-element E4M3 block scales");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~uintptr_t(1023));
+    uint8_t* smem = align_shared<1024>(smem_raw);
     const uint32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t full0 = smem_u32(smem + kDqmBarOff), empty0 = full0 + 8 * kDqmStages;
     const uint32_t sfr0 = empty0 + 8 * kDqmStages, sfe0 = sfr0 + 16;  // [2] repacked / copied out

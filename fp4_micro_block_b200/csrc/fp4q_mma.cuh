@@ -251,8 +251,7 @@ __global__ void __launch_bounds__(MmaGeo<FMT>::threads, 1)
     using Geo = MmaGeo<FMT>;
     constexpr int kGroups = Geo::groups;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~uintptr_t(1023));
+    uint8_t* smem = align_shared<1024>(smem_raw);
     const uint32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kMmaBarOff);
     const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * kMmaStages;

@@ -153,8 +153,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     using W = Wide<HAD>;
     constexpr int G = W::G, NBUF = W::NBUF;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~uintptr_t(1023));
+    uint8_t* smem = align_shared<1024>(smem_raw);
     const uint32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t full0 = smem_u32(smem + W::bar_off), empty0 = full0 + 8 * kMmaStages;
     const uint32_t accf0 = empty0 + 8 * kMmaStages, relg0 = accf0 + 8 * NBUF;

@@ -130,8 +130,7 @@ __global__ void __launch_bounds__(QGeo<FMT, HAD>::threads, kQCtas)
     static_assert(HAD == 0 || HAD == 16 || HAD == 32 || HAD == 64, "register-path rotation sizes");
     constexpr int S = G::stages, U = G::units, NG = G::groups;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~uintptr_t(1023));
+    uint8_t* smem = align_shared<1024>(smem_raw);
     const uint32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t full0 = smem_u32(smem + G::bar_off), empty0 = full0 + 8 * S;
     float* red = reinterpret_cast<float*>(smem + G::red_off);
