@@ -58,6 +58,14 @@ def lib() -> C.CDLL:
             "orc_e4m3_encode_array": (None, [p, i64, p]),
             "orc_e4m3_decode_array": (None, [p, i64, p]),
             "orc_e8m0_encode_array": (None, [p, i64, p]),
+            "orc_int4_encode": (C.c_uint8, [f32]),
+            "orc_int4_decode": (f32, [C.c_uint8]),
+            "orc_int4_tensor_scale": (f32, [f32]),
+            "orc_int4_quantize": (None, [p, i64, i64, i64, f32, p, p]),
+            "orc_int4_dequantize": (None, [p, p, f32, i64, i64, p]),
+            "orc_arc_quantize_int4": (None, [p, i64, i64, i64, p, f32, p, p]),
+            "orc_int4_encode_array": (None, [p, i64, p]),
+            "orc_int4_decode_array": (None, [p, i64, p]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -225,6 +233,45 @@ def dual_dequantize(codes, scales, gscales) -> np.ndarray:
     return out
 
 
+def int4_encode(v) -> np.ndarray:
+    """Nibbles of clamp(RNE(v), -7, 7) (4-bit two's complement)."""
+    v = _f32(np.atleast_1d(v))
+    out = np.empty(v.shape, np.uint8)
+    lib().orc_int4_encode_array(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def int4_decode(codes) -> np.ndarray:
+    """Two's complement values of 4-bit codes (one per byte)."""
+    c = np.ascontiguousarray(codes, np.uint8)
+    out = np.empty(c.shape, np.float32)
+    lib().orc_int4_decode_array(_ptr(c), c.size, _ptr(out))
+    return out
+
+
+def int4_tensor_scale(a: float) -> float:
+    return float(lib().orc_int4_tensor_scale(float(a)))
+
+
+def int4_quantize(y: np.ndarray, s_t: float):
+    y = _f32(y)
+    M, K = y.shape
+    assert K % 16 == 0
+    codes = np.empty((M, K // 2), np.uint8)
+    scales = np.empty((M, K // 16), np.uint8)
+    lib().orc_int4_quantize(_ptr(y), M, K, K, float(s_t), _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def int4_dequantize(codes, scales, s_t: float) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    M, K = codes.shape[0], codes.shape[1] * 2
+    out = np.empty((M, K), np.float32)
+    lib().orc_int4_dequantize(_ptr(codes), _ptr(scales), float(s_t), M, K, _ptr(out))
+    return out
+
+
 def mxfp4_dequantize(codes, scales) -> np.ndarray:
     codes = np.ascontiguousarray(codes, np.uint8)
     scales = np.ascontiguousarray(scales, np.uint8)
@@ -272,13 +319,13 @@ def rmsnorm_permute(x: np.ndarray, gamma: np.ndarray, perm, eps: float) -> np.nd
 
 
 def arc_quantize(y: np.ndarray, outliers, s_t: float | None, fmt: str = "nvfp4"):
-    """Primary + residual quantization of the prepared matrix y; NVFP4 (block
-    16, tensor scale s_t) or MXFP4 (block 32, s_t unused)."""
+    """Primary + residual quantization of the prepared matrix y; NVFP4 or INT4
+    (block 16, tensor scale s_t) or MXFP4 (block 32, s_t unused)."""
     y = _f32(y)
     M, K = y.shape
     o = np.ascontiguousarray(outliers, np.int32)
     S = o.size
-    B = 16 if fmt == "nvfp4" else 32
+    B = 32 if fmt == "mxfp4" else 16
     assert K % B == 0 and S % B == 0
     codes = np.empty((M, (K + S) // 2), np.uint8)
     scales = np.empty((M, (K + S) // B), np.uint8)
@@ -288,6 +335,9 @@ def arc_quantize(y: np.ndarray, outliers, s_t: float | None, fmt: str = "nvfp4")
     elif fmt == "mxfp4":
         lib().orc_arc_quantize_mxfp4(_ptr(y), M, K, S, _ptr(o) if S else None, _ptr(codes),
                                      _ptr(scales))
+    elif fmt == "int4":
+        lib().orc_arc_quantize_int4(_ptr(y), M, K, S, _ptr(o) if S else None, float(s_t),
+                                    _ptr(codes), _ptr(scales))
     else:
         raise ValueError(fmt)
     return codes, scales
@@ -337,14 +387,14 @@ def arc_prepare(x_bits, gamma_bits, perm, eps: float = 1e-6) -> np.ndarray:
 def arc(x_bits, gamma_bits, perm, outliers, eps: float = 1e-6, s_t: float | None = None,
         fmt: str = "nvfp4"):
     """ARCQuant path: reorder + RMSNorm, primary + residual quantization.
-    Returns (codes, scales, s_t (NVFP4) or None (MXFP4), y)."""
+    Returns (codes, scales, s_t (NVFP4, INT4) or None (MXFP4), y)."""
     y = arc_prepare(x_bits, gamma_bits, perm, eps)
     if fmt == "mxfp4":
         c, s = arc_quantize(y, outliers, None, "mxfp4")
         return c, s, None, y
     if s_t is None:
-        s_t = tensor_scale(amax(y))
-    c, s = arc_quantize(y, outliers, s_t)
+        s_t = int4_tensor_scale(amax(y)) if fmt == "int4" else tensor_scale(amax(y))
+    c, s = arc_quantize(y, outliers, s_t, fmt)
     return c, s, np.float32(s_t), y
 
 
@@ -354,7 +404,8 @@ def arc_alignment(y, outliers, s_t, codes, scales, fmt: str = "nvfp4"):
     stages, about 1.266, against under 2 for MXFP8).  Reading: a block's grid is
     aligned to its content when the decoded block scale d equals amax / 6 (the
     block maximum on the top E2M1 value); the factor phi = d / (amax / 6) is
-    how far the stored scale moved it.  One E4M3 step is 2^-3 of the value, and
+    how far the stored scale moved it (INT4: amax / 7, its largest integer).
+    One E4M3 step is 2^-3 of the value, and
     (1 + 2^-3)^2 = 1.265625 is the page's figure for two stages; round to
     nearest keeps phi within 1 +- 2^-4 while the scale is a normal E4M3 number
     (MXFP4's power-of-two scale, chosen from the exponent of amax: phi in
@@ -370,10 +421,12 @@ def arc_alignment(y, outliers, s_t, codes, scales, fmt: str = "nvfp4"):
     M, K = y.shape
     o = np.asarray(outliers, np.int64)
     S = o.size
-    B = 16 if fmt == "nvfp4" else 32
-    cv = e2m1_decode(unpack_codes(np.asarray(codes)))  # [M, K + S] E2M1 values
+    B = 32 if fmt == "mxfp4" else 16
+    top = 7.0 if fmt == "int4" else 6.0  # the largest grid value
+    u = unpack_codes(np.asarray(codes))
+    cv = int4_decode(u) if fmt == "int4" else e2m1_decode(u)  # [M, K + S] grid values
     sb = np.asarray(scales, np.uint8).reshape(M, (K + S) // B)
-    if fmt == "nvfp4":
+    if fmt in ("nvfp4", "int4"):
         d = (e4m3_decode(sb).astype(np.float32) * np.float32(s_t)).astype(np.float32)
         unit = e4m3_decode(sb).astype(np.float32)
         normal = (sb & 0x78) != 0  # exponent field non-zero
@@ -385,14 +438,14 @@ def arc_alignment(y, outliers, s_t, codes, scales, fmt: str = "nvfp4"):
     cp = cv[:, o].astype(np.float32)
     up = unit[:, o // B]
     dq = (cp * up).astype(np.float32)
-    if fmt == "nvfp4":
+    if fmt in ("nvfp4", "int4"):
         dq = (dq * np.float32(s_t)).astype(np.float32)
     res = (y[:, o] - dq).astype(np.float32)
 
     def phi(vals, dd):
         am = np.abs(vals.astype(np.float64)).reshape(M, -1, B).max(axis=2)
         with np.errstate(divide="ignore", invalid="ignore"):
-            return np.where(am > 0, dd.astype(np.float64) / (am / 6.0), np.nan)
+            return np.where(am > 0, dd.astype(np.float64) / (am / top), np.nan)
 
     nb = K // B
     return phi(y, d[:, :nb]), phi(res, d[:, nb:]), normal[:, :nb], normal[:, nb:]
@@ -407,6 +460,8 @@ def dequantize(fmt: str, codes, scales, scale=None, inv_had: int = 0, signs=None
         y = mxfp4_dequantize(codes, scales)
     elif fmt == "dual":
         y = dual_dequantize(codes, scales, scale)
+    elif fmt == "int4":
+        y = int4_dequantize(codes, scales, float(scale))
     else:
         raise ValueError(fmt)
     if inv_had:

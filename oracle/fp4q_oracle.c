@@ -24,7 +24,8 @@
  *     abstract: two-level FWHT).  The oracle applies the dense Sylvester matrix.
  *   - ARCQuant fused path: reorder -> RMSNorm -> primary NVFP4 quantization ->
  *     residual NVFP4 quantization of the outlier channels, appended along K
- *     (ARCQuant, "Methodologie" items 1, 2, 3 and 5).
+ *     (ARCQuant, "Methodologie" items 1, 2, 3 and 5); the same in MXFP4 and
+ *     INT4 ("Generalisabilite": the scheme extends to both formats).
  *
  * Numeric rules (where the pages only name the formats, these are the plain
  * readings of them, each taken where the pages leave the step open):
@@ -42,6 +43,13 @@
  *            b = 0 and all codes 0.
  *   Dual   : G = amax_128 / 2688 per 128-element group, then the NVFP4 rule per
  *            16-block with G in place of s_t.
+ *   INT4   : (ARCQuant summary, "Generalisabilite": the residual scheme extends
+ *            to INT4; the pages give no INT4 scale rule, so this is the NVFP4
+ *            container with the integer grid in place of E2M1) elements are the
+ *            integers -7..7 in 4-bit two's complement; s_t = amax_tensor / 3136
+ *            (3136 = 7*448); per 16-block r = (amax_b / 7) / s_t, e = E4M3(r),
+ *            d = E4M3val(e) * s_t, code_i = clamp(RNE(fl32(y_i / d)), -7, 7)
+ *            (nearest integer, ties to even); d == 0 gives all codes 0.
  */
 #include <math.h>
 #include <stdint.h>
@@ -431,6 +439,111 @@ ORC_EXPORT void orc_arc_quantize(const float* y, int64_t M, int64_t K, int64_t S
 }
 
 /* ------------------------------------------------------------------------ */
+/* INT4 in the micro-block container (ARCQuant summary, "Generalisabilite")   */
+/* ------------------------------------------------------------------------ */
+
+/* Nearest integer to q, ties to the even integer, written out with floor so
+ * that it does not depend on the floating-point rounding mode; then clamped to
+ * the symmetric range -7..7 and stored as a 4-bit two's complement nibble. */
+ORC_EXPORT uint8_t orc_int4_encode(float q) {
+    double a = (double)q; /* exact */
+    double f = floor(a);
+    double frac = a - f;  /* exact: a and f are within 1 of each other */
+    double n = f;
+    if (a != a) return 0; /* NaN (not produced by finite inputs): code 0 */
+    if (frac > 0.5 || (frac == 0.5 && fmod(f, 2.0) != 0.0)) n = f + 1.0;
+    if (n > 7.0) n = 7.0;
+    if (n < -7.0) n = -7.0;
+    return (uint8_t)(((int)n) & 15);
+}
+
+/* Two's complement value of a nibble (-8..7; the encoder never writes -8). */
+ORC_EXPORT float orc_int4_decode(uint8_t c) {
+    int v = c & 15;
+    return (float)(v >= 8 ? v - 16 : v);
+}
+
+/* s_t = amax / (7 * 448), one binary32 division. */
+ORC_EXPORT float orc_int4_tensor_scale(float amax) { return amax / 3136.0f; }
+
+/* One 16-element block against the FP32 scale s: 8 bytes of codes (low nibble
+ * = even index) and the E4M3 scale byte, as nvfp4_block with the largest grid
+ * value 7 and the integer grid. */
+static uint8_t int4_block(const float* y, float s, uint8_t* codes8) {
+    float amax = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+        float a = fabsf(y[i]);
+        if (a > amax) amax = a;
+    }
+    uint8_t e = 0;
+    float d = 0.0f;
+    if (s > 0.0f) {
+        float bs = amax / 7.0f;
+        float r = bs / s;
+        e = orc_e4m3_encode(r);
+        d = orc_e4m3_decode(e) * s;
+    }
+    for (int i = 0; i < 8; ++i) {
+        uint8_t lo = 0, hi = 0;
+        if (d != 0.0f) {
+            lo = orc_int4_encode(y[2 * i] / d);
+            hi = orc_int4_encode(y[2 * i + 1] / d);
+        }
+        codes8[i] = (uint8_t)(lo | (hi << 4));
+    }
+    return e;
+}
+
+/* INT4 quantization of y[M, K] (row stride ld) with tensor scale s_t:
+ * codes [M, K/2], scales [M, K/16] E4M3 bytes (linear). */
+ORC_EXPORT void orc_int4_quantize(const float* y, int64_t M, int64_t K, int64_t ld, float s_t,
+                                  uint8_t* codes, uint8_t* scales) {
+    for (int64_t r = 0; r < M; ++r)
+        for (int64_t b = 0; b < K / 16; ++b)
+            scales[r * (K / 16) + b] = int4_block(y + r * ld + 16 * b, s_t, codes + r * (K / 2) + 8 * b);
+}
+
+/* value = (integer * E4M3val) * s_t: the first product is exact, the second
+ * one binary32 rounding. */
+ORC_EXPORT void orc_int4_dequantize(const uint8_t* codes, const uint8_t* scales, float s_t,
+                                    int64_t M, int64_t K, float* out) {
+    for (int64_t r = 0; r < M; ++r)
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t byte = codes[r * (K / 2) + k / 2];
+            uint8_t c = (k & 1) ? (byte >> 4) : (byte & 15);
+            float p = orc_int4_decode(c) * orc_e4m3_decode(scales[r * (K / 16) + k / 16]);
+            out[r * K + k] = p * s_t;
+        }
+}
+
+/* ARCQuant two-stage path in INT4: primary INT4 of all K columns with s_t;
+ * residual of outlier position p: y[p] - (integer * E4M3val) * s_t, quantized
+ * in 16-blocks with the same s_t and appended along K (codes [M, (K+S)/2],
+ * scales [M, (K+S)/16]). */
+ORC_EXPORT void orc_arc_quantize_int4(const float* y, int64_t M, int64_t K, int64_t S,
+                                      const int32_t* outliers, float s_t, uint8_t* codes,
+                                      uint8_t* scales) {
+    int64_t KS = K + S;
+    float* res = (float*)malloc(sizeof(float) * (size_t)(S > 0 ? S : 1));
+    for (int64_t r = 0; r < M; ++r) {
+        const float* yr = y + r * K;
+        uint8_t* cr = codes + r * (KS / 2);
+        uint8_t* sr = scales + r * (KS / 16);
+        for (int64_t b = 0; b < K / 16; ++b) sr[b] = int4_block(yr + 16 * b, s_t, cr + 8 * b);
+        for (int64_t j = 0; j < S; ++j) {
+            int64_t p = outliers[j];
+            uint8_t byte = cr[p / 2];
+            uint8_t c = (p & 1) ? (byte >> 4) : (byte & 15);
+            float dq = (orc_int4_decode(c) * orc_e4m3_decode(sr[p / 16])) * s_t;
+            res[j] = yr[p] - dq;
+        }
+        for (int64_t b = 0; b < S / 16; ++b)
+            sr[K / 16 + b] = int4_block(res + 16 * b, s_t, cr + K / 2 + 8 * b);
+    }
+    free(res);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Array forms of the scalar encoders (for the Python binding)                */
 /* ------------------------------------------------------------------------ */
 
@@ -478,4 +591,12 @@ ORC_EXPORT void orc_e4m3_decode_array(const uint8_t* b, int64_t n, float* out) {
 
 ORC_EXPORT void orc_e8m0_encode_array(const float* v, int64_t n, uint8_t* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = orc_e8m0_encode(v[i]);
+}
+
+ORC_EXPORT void orc_int4_encode_array(const float* v, int64_t n, uint8_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_int4_encode(v[i]);
+}
+
+ORC_EXPORT void orc_int4_decode_array(const uint8_t* c, int64_t n, float* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_int4_decode(c[i]);
 }
