@@ -105,6 +105,12 @@ def _make_workload(name: str, rows: int = 0):
                     desc="arc_mxfp4_8192x4096 reorder+RMSNorm+MXFP4+residual(S=256)",
                     x=lambda: workloads.arc_activations(M, K, seed=4, S=S),
                     kernels=[("arc", M * K * 2 + M * (K + S) // 2 + M * (K + S) // 32)])
+    if name == "arc_int4":
+        M, K, S = rows or 8192, 4096, 256
+        return dict(name=name, M=M, K=K, S=S, fmt="INT4", had=0,
+                    desc="arc_int4_8192x4096 reorder+RMSNorm+INT4+residual(S=256), static tensor scale",
+                    x=lambda: workloads.arc_activations(M, K, seed=4, S=S),
+                    kernels=[("arc", M * K * 2 + M * (K + S) // 2 + M * (K + S) // 16)])
     if name == "dual":
         M, K = rows or 32768, 4096
         return dict(name=name, M=M, K=K, fmt="DUAL", had=512,
@@ -212,6 +218,7 @@ KERNEL_SOURCES = {
     ("mxfp4", "dequantize"): _COMMON + ["fp4q_dequant.cuh"],
     ("arc", "arc"): _COMMON + ["fp4q_arc.cuh"],
     ("arc_mxfp4", "arc"): _COMMON + ["fp4q_arc.cuh"],
+    ("arc_int4", "arc"): _COMMON + ["fp4q_arc.cuh"],
 }
 
 
@@ -264,7 +271,8 @@ def run_ours(args, rank, world, local_rank):
 
     S = wl.get("S", 0)
     KS = K + S
-    fmt = {"MXFP4": fq.FP4Q_MXFP4, "NVFP4": fq.FP4Q_NVFP4, "DUAL": fq.FP4Q_NVFP4_DUAL}[wl["fmt"]]
+    fmt = {"MXFP4": fq.FP4Q_MXFP4, "NVFP4": fq.FP4Q_NVFP4, "DUAL": fq.FP4Q_NVFP4_DUAL,
+           "INT4": fq.FP4Q_INT4}[wl["fmt"]]
     B = 32 if fmt == fq.FP4Q_MXFP4 else 16
     labels = [k for k, _ in wl["kernels"]]
     alg = dict(wl["kernels"])
@@ -279,7 +287,7 @@ def run_ours(args, rank, world, local_rank):
         xi = x_host.to(dev)
         codes = torch.empty((M, KS // 2), dtype=torch.uint8, device=dev)
         scales = torch.empty((M, KS // B), dtype=torch.uint8, device=dev)
-        if fmt == fq.FP4Q_NVFP4:
+        if fmt in (fq.FP4Q_NVFP4, fq.FP4Q_INT4):
             sf = torch.zeros(1, dtype=torch.float32, device=dev)
         elif fmt == fq.FP4Q_NVFP4_DUAL:
             sf = torch.empty((M, K // 128), dtype=torch.float32, device=dev)
@@ -294,7 +302,7 @@ def run_ours(args, rank, world, local_rank):
     L = fq.lib()
 
     # static tensor scale for the Hadamard / ARC workloads: the dynamic value of a first call
-    if wl["name"].startswith("hadamard") or wl["name"] == "arc":  # NVFP4 tensor scale
+    if wl["name"].startswith("hadamard") or wl["name"] in ("arc", "arc_int4"):  # tensor scale
         for i in range(R):
             codes, scales, sf, _ = outs[i]
             if wl["name"].startswith("arc"):
@@ -709,7 +717,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dual",
-                    help="dual (default) | mxfp4 | nvfp4 | hadamard128 | hadamard16 | hadamard32 | arc | arc_mxfp4 | arc_gemm")
+                    help="dual (default) | mxfp4 | nvfp4 | hadamard128 | hadamard16 | hadamard32 | arc | "
+                         "arc_mxfp4 | arc_int4 | arc_gemm")
     ap.add_argument("--rows", type=int, default=0,
                     help="override the workload's row count (small cases for profiler captures)")
     ap.add_argument("--units", type=int, default=0,

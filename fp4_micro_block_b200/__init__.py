@@ -26,7 +26,7 @@ LIB_PATH = os.environ.get("FP4Q_LIBRARY") or os.path.join(_HERE, "libfp4q.so")
 # enum values of include/fp4q.h
 FP4Q_OK, FP4Q_ERR_INVALID_ARG, FP4Q_ERR_UNSUPPORTED, FP4Q_ERR_ALIGNMENT, FP4Q_ERR_CUDA, \
     FP4Q_ERR_DEVICE = range(6)
-FP4Q_NVFP4, FP4Q_MXFP4, FP4Q_NVFP4_DUAL = 0, 1, 2
+FP4Q_NVFP4, FP4Q_MXFP4, FP4Q_NVFP4_DUAL, FP4Q_INT4 = 0, 1, 2, 3
 FP4Q_SCALES_LINEAR, FP4Q_SCALES_SWIZZLED = 0, 1
 FP4Q_TSCALE_DYNAMIC, FP4Q_TSCALE_STATIC = 0, 1
 FP4Q_WORKSPACE_BYTES = 16384
@@ -247,14 +247,14 @@ def _block(fmt: int) -> int:
 def alloc_outputs(M: int, K: int, fmt: int, layout: int = FP4Q_SCALES_LINEAR, device="cuda",
                   ncols: int | None = None):
     """codes [M, K/2] u8, scales (linear [M, ncols] or the padded tiled buffer),
-    and the fp32 scale(s): 1 float (NVFP4), [M, K/128] (dual) or None (MXFP4)."""
+    and the fp32 scale(s): 1 float (NVFP4, INT4), [M, K/128] (dual) or None (MXFP4)."""
     ncols = K // _block(fmt) if ncols is None else ncols
     codes = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
     if layout == FP4Q_SCALES_LINEAR:
         scales = torch.empty((M, ncols), dtype=torch.uint8, device=device)
     else:
         scales = torch.empty(fp4q_scales_bytes(M, ncols, layout), dtype=torch.uint8, device=device)
-    if fmt == FP4Q_NVFP4:
+    if fmt in (FP4Q_NVFP4, FP4Q_INT4):
         sf = torch.zeros(1, dtype=torch.float32, device=device)
     elif fmt == FP4Q_NVFP4_DUAL:
         sf = torch.empty((M, K // 128), dtype=torch.float32, device=device)
@@ -307,12 +307,12 @@ def hadamard_quantize(x, had_size, fmt=FP4Q_NVFP4, tensor_scale=None, layout=FP4
 
 def arc_quantize(x, gamma, perm, outliers, eps=1e-6, tensor_scale=None,
                  layout=FP4Q_SCALES_LINEAR, ws=None, fmt=FP4Q_NVFP4):
-    """ARCQuant path; returns (codes, scales, tensor scale (NVFP4) or None (MXFP4))."""
+    """ARCQuant path; returns (codes, scales, tensor scale (NVFP4, INT4) or None (MXFP4))."""
     M, K = x.shape
     S = 0 if outliers is None else outliers.numel()
     codes, scales, sf = alloc_outputs(M, K + S, fmt, layout, x.device)
     mode = FP4Q_TSCALE_DYNAMIC
-    if fmt == FP4Q_NVFP4:
+    if fmt in (FP4Q_NVFP4, FP4Q_INT4):
         if tensor_scale is not None:
             sf.copy_(tensor_scale.reshape(1))
             mode = FP4Q_TSCALE_STATIC

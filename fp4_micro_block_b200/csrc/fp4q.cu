@@ -648,8 +648,8 @@ FP4Q_API fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int6
                                        fp4q_stream_t stream) {
     fp4q_status st = check_x(x, M, K, ldx);
     if (st != FP4Q_OK) return st;
-    if (format != FP4Q_NVFP4 && format != FP4Q_MXFP4) return FP4Q_ERR_INVALID_ARG;
-    const bool mx = format == FP4Q_MXFP4;
+    if (format != FP4Q_NVFP4 && format != FP4Q_MXFP4 && format != FP4Q_INT4) return FP4Q_ERR_INVALID_ARG;
+    const bool mx = format == FP4Q_MXFP4, i4 = format == FP4Q_INT4;
     const int B = mx ? 32 : 16;
     if (K % B != 0 || S < 0 || S % B != 0 || S > K) return FP4Q_ERR_INVALID_ARG;
     if (K > 16384) return FP4Q_ERR_UNSUPPORTED;
@@ -693,7 +693,8 @@ FP4Q_API fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int6
             if (Kn::total(K, S, slots * Kn::wpp) <= kSmemMax) return slots * Kn::wpp;
         return 0;
     };
-    const int W = mx ? warps_for(ArcKern<FMT_MXFP4, false>{}) : warps_for(ArcKern<FMT_NVFP4, false>{});
+    const int W = mx ? warps_for(ArcKern<FMT_MXFP4, false>{})
+                     : i4 ? warps_for(ArcKern<FMT_INT4, false>{}) : warps_for(ArcKern<FMT_NVFP4, false>{});
     const int Wa = dynamic ? warps_for(ArcKern<FMT_NVFP4, true>{}) : 1;
     if (W == 0 || Wa == 0) return FP4Q_ERR_UNSUPPORTED;
     const int64_t pairs = (M + 1) / 2;
@@ -720,6 +721,7 @@ FP4Q_API fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int6
         p.n_partials = grid_a;
     }
     if (mx) return run(ArcKern<FMT_MXFP4, false>{}, W);
+    if (i4) return run(ArcKern<FMT_INT4, false>{}, W);
     return run(ArcKern<FMT_NVFP4, false>{}, W);
 }
 
@@ -738,10 +740,12 @@ fp4q_status dequantize_common(fp4q_format format, const uint8_t* codes, const ui
         case FP4Q_NVFP4: fmt = FMT_NVFP4; break;
         case FP4Q_MXFP4: fmt = FMT_MXFP4; break;
         case FP4Q_NVFP4_DUAL: fmt = FMT_DUAL; break;
+        case FP4Q_INT4: fmt = FMT_INT4; break;
         default: return FP4Q_ERR_INVALID_ARG;
     }
     const int B = fmt == FMT_MXFP4 ? 32 : 16;
     if (K % B != 0 || (inv_had_size && K % inv_had_size != 0)) return FP4Q_ERR_INVALID_ARG;
+    if (fmt == FMT_INT4 && inv_had_size != 0) return FP4Q_ERR_UNSUPPORTED;  // no rotated INT4 path
     if (fmt == FMT_DUAL && K % 128 != 0) return FP4Q_ERR_INVALID_ARG;
     if (M == 0) return FP4Q_OK;
     if (!codes || !scales || !y || (fmt != FMT_MXFP4 && !scale_fp32)) return FP4Q_ERR_INVALID_ARG;
@@ -763,6 +767,7 @@ fp4q_status dequantize_common(fp4q_format format, const uint8_t* codes, const ui
     cudaStream_t s = (cudaStream_t)stream;
     if (signs)
         for (int w = 0; w < (std::min(inv_had_size, kMmaTile) + 31) / 32; ++w) p.signs[w] = signs[w];
+    if (fmt == FMT_INT4) return launch_dequant_stream<FMT_INT4, 0, false>(p, sms, s);
     if (dqm_applies(fmt, inv_had_size, p))
         return fmt == FMT_DUAL ? launch_dqm<FMT_DUAL>(inv_had_size, p, sms, s)
                                : launch_dqm<FMT_NVFP4>(inv_had_size, p, sms, s);

@@ -1,8 +1,9 @@
 // fp4q_arc.cuh -- ARCQuant fused kernel for sm_100a: channel reorder + RMSNorm
 // + primary quantization + quantization of the residual of the outlier
 // channels, written as one [primary K | residual S] GEMM operand (ARCQuant
-// summary, "Methodologie" items 1-5), in NVFP4 or MXFP4 ("Generalisabilite":
-// the scheme carries over to MXFP4).
+// summary, "Methodologie" items 1-5), in NVFP4, MXFP4 or INT4
+// ("Generalisabilite": the scheme carries over to MXFP4 and INT4; INT4 is the
+// NVFP4 container with the integers -7..7 as the grid).
 //
 // Two warps own a PAIR of rows at a time (the amax pre-pass: one warp): there
 // is no CTA-wide barrier on the path, only a 64-thread named barrier between
@@ -125,6 +126,8 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return _
 // fold per component: the unit holds -z and v = z * fold.  Scale bytes from
 // RN(RN(amax(v) * RN(1/6)) * RN(1/s)) and quotients z * RN(RN(1/d) * fold), as
 // in nvfp4_unit's table path.  stab[e] = (d, RN(1/d)) for the tensor scale s.
+// INT4: the same with RN(1/7) and the integer grid.
+template <bool INT4>
 __device__ __forceinline__ uint32_t arc_nvfp4_unit(const float2* n, float2 am, const ScaleCtx& c,
                                                    const float2* stab, float2 fold, uint32_t (&w)[4]) {
     am.x *= fold.x;
@@ -134,12 +137,12 @@ __device__ __forceinline__ uint32_t arc_nvfp4_unit(const float2* n, float2 am, c
     const bool in_range = c.fast && (b0 - 1u) >= tiny - 1u && (b1 - 1u) >= tiny - 1u &&
                           fmaxf(am.x, am.y) <= c.am_max;
     if (!in_range) {
-        const uint32_t e0 = nvfp4_block_ieee<false>(n, am.x, c.s, fold.x, w[0], w[1]);
-        const uint32_t e1 = nvfp4_block_ieee<true>(n, am.y, c.s, fold.y, w[2], w[3]);
+        const uint32_t e0 = nvfp4_block_ieee<false, INT4>(n, am.x, c.s, fold.x, w[0], w[1]);
+        const uint32_t e1 = nvfp4_block_ieee<true, INT4>(n, am.y, c.s, fold.y, w[2], w[3]);
         return e0 | (e1 << 8);
     }
-    const float k6 = __uint_as_float(0x3e2aaaabu);  // RN(1/6)
-    const uint32_t e2 = e4m3x2_encode(make_float2((am.x * k6) * c.rs.rn, (am.y * k6) * c.rs.rn));
+    const float k = __uint_as_float(INT4 ? 0x3e124925u : 0x3e2aaaabu);  // RN(1/7), RN(1/6)
+    const uint32_t e2 = e4m3x2_encode(make_float2((am.x * k) * c.rs.rn, (am.y * k) * c.rs.rn));
     const float2 t0 = stab[e2 & 0xffu], t1 = stab[e2 >> 8];
     const float2 m = make_float2(-(t0.y * fold.x), -(t1.y * fold.y));  // n holds -z
     float q0[16], q1[16];
@@ -149,10 +152,17 @@ __device__ __forceinline__ uint32_t arc_nvfp4_unit(const float2* n, float2 am, c
         q0[i] = q.x;
         q1[i] = q.y;
     }
-    w[0] = e2m1_pack8(q0);
-    w[1] = e2m1_pack8(q0 + 8);
-    w[2] = e2m1_pack8(q1);
-    w[3] = e2m1_pack8(q1 + 8);
+    if constexpr (INT4) {
+        w[0] = int4_pack8(q0);
+        w[1] = int4_pack8(q0 + 8);
+        w[2] = int4_pack8(q1);
+        w[3] = int4_pack8(q1 + 8);
+    } else {
+        w[0] = e2m1_pack8(q0);
+        w[1] = e2m1_pack8(q0 + 8);
+        w[2] = e2m1_pack8(q1);
+        w[3] = e2m1_pack8(q1 + 8);
+    }
     if (t0.x == 0.0f) w[0] = w[1] = 0u;  // zero block scale: all codes +0
     if (t1.x == 0.0f) w[2] = w[3] = 0u;
     return e2;
@@ -200,7 +210,9 @@ __device__ __forceinline__ void put_scale(const ArcParams& p, int64_t row, int64
 
 template <int FMT, bool AMAX_ONLY>
 __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_kernel(const ArcParams p) {
-    static_assert(FMT == FMT_NVFP4 || (FMT == FMT_MXFP4 && !AMAX_ONLY), "formats of the ARC path");
+    static_assert(FMT == FMT_NVFP4 || ((FMT == FMT_MXFP4 || FMT == FMT_INT4) && !AMAX_ONLY),
+                  "formats of the ARC path");
+    constexpr bool I4 = FMT == FMT_INT4;
     constexpr int B = FMT == FMT_MXFP4 ? 32 : 16;  // block size
     constexpr int Q = B / 4;                       // 16-byte table quads per block
     constexpr int SR = AMAX_ONLY ? 2 : 1;          // landing stages per warp
@@ -322,9 +334,9 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
             rslot[i] = (uint16_t)((w >> 16) + __popc(w & ((1u << (q & 15)) - 1u)));
         }
         if (bad_index) atomicOr(&g_device_error, kErrBadIndex);
-        if constexpr (FMT == FMT_NVFP4) {
+        if constexpr (FMT == FMT_NVFP4 || I4) {
             if (p.dynamic) {
-                s_t = tensor_scale_from_partials(p.partials, p.n_partials, red);
+                s_t = tensor_scale_from_partials(p.partials, p.n_partials, red, I4 ? 3136.0f : 2688.0f);
                 if (blockIdx.x == 0 && tid == 0) *p.tensor_scale = s_t;
             } else {
                 s_t = *p.tensor_scale;
@@ -455,9 +467,9 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
             };
             // quantize + store block b of both rows, and its outlier residuals
             auto emit = [&](int b, const float2* v) {
-                if constexpr (FMT == FMT_NVFP4) {
+                if constexpr (FMT == FMT_NVFP4 || I4) {
                     uint32_t w[4];
-                    const uint32_t e2 = arc_nvfp4_unit(v, amax_pair_tree(v), ctx, stab, rs, w);
+                    const uint32_t e2 = arc_nvfp4_unit<I4>(v, amax_pair_tree(v), ctx, stab, rs, w);
                     *reinterpret_cast<uint2*>(cp0 + 8 * b) = make_uint2(w[0], w[1]);
                     put_scale(p, r0, b, nsc, nC, e2 & 0xffu);
                     if (two) {
@@ -473,10 +485,11 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
                             const uint32_t m2 = (o >> k) & 3u;
                             if (m2 == 0u) continue;
                             const uint32_t sh = 4 * (k & 7);
-                            const float2 c0 = e2m1x2_decode((w[k >> 3] >> sh) & 0xffu);      // row 0, k, k+1
-                            const float2 c1 = e2m1x2_decode((w[2 + (k >> 3)] >> sh) & 0xffu);  // row 1
+                            const uint32_t b0 = (w[k >> 3] >> sh) & 0xffu, b1 = (w[2 + (k >> 3)] >> sh) & 0xffu;
+                            const float2 c0 = I4 ? int4x2_decode(b0) : e2m1x2_decode(b0);  // row 0, k, k+1
+                            const float2 c1 = I4 ? int4x2_decode(b1) : e2m1x2_decode(b1);  // row 1
                             const int base = (int)(o >> 16) + __popc(o & ((1u << k) - 1u));
-                            // residual y - (E2M1 value * E4M3 value) * s_t, y = z * rs
+                            // residual y - (grid value * E4M3 value) * s_t, y = z * rs
                             if (m2 & 1u) {
                                 res[base] = -v[k].x * rs.x - (c0.x * es0) * s_t;
                                 res[S + base] = -v[k].y * rs.y - (c1.x * es1) * s_t;
@@ -552,7 +565,7 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
             // alternate blocks to the two warps
             for (int j = sub + WPP * lane; B * j < S; j += 32 * WPP) {
                 const int64_t col = nbB + j;
-                if constexpr (FMT == FMT_NVFP4) {
+                if constexpr (FMT == FMT_NVFP4 || I4) {
                     float2 n[16];
 #pragma unroll
                     for (int k = 0; k < 16; ++k) {
@@ -560,7 +573,7 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
                         n[k] = make_float2(-res[sl], -res[S + sl]);
                     }
                     uint32_t w[4];
-                    const uint32_t e2 = arc_nvfp4_unit(n, amax_pair_tree(n), ctx, stab, make_float2(1.0f, 1.0f), w);
+                    const uint32_t e2 = arc_nvfp4_unit<I4>(n, amax_pair_tree(n), ctx, stab, make_float2(1.0f, 1.0f), w);
                     *reinterpret_cast<uint2*>(cp0 + p.K / 2 + 8 * j) = make_uint2(w[0], w[1]);
                     put_scale(p, r0, col, nsc, nC, e2 & 0xffu);
                     if (two) {

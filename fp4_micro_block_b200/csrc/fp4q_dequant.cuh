@@ -140,7 +140,8 @@ template <int FMT>
 __device__ __forceinline__ void decode_raw(const RawUnit& u, float* v) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-        float2 c = e2m1x2_decode((u.w[i >> 2] >> (8 * (i & 3))) & 0xffu);
+        const uint32_t byte = (u.w[i >> 2] >> (8 * (i & 3))) & 0xffu;
+        float2 c = FMT == FMT_INT4 ? int4x2_decode(byte) : e2m1x2_decode(byte);
         v[2 * i] = c.x;
         v[2 * i + 1] = c.y;
     }

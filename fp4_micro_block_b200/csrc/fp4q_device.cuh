@@ -82,6 +82,32 @@ __device__ __forceinline__ float2 e2m1x2_decode(uint32_t byte) {
     return r;
 }
 
+// INT4 (4-bit two's complement, the symmetric range -7..7): four bytes of
+// codes from eight quotients q (q[0] -> low nibble of byte 0).  Each q is
+// clamped to [-7, 7] and rounded to the nearest integer, ties to even, by one
+// IEEE addition of 1.5 * 2^23 (whose ulp is 1); the integer is then the low
+// bits of the sum's significand (2^22 + k for k in -7..7), its low nibble the
+// two's complement code.
+__device__ __forceinline__ uint32_t int4_pack8(const float* q) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float c = fminf(fmaxf(q[i], -7.0f), 7.0f);
+        const uint32_t k = __float_as_uint(__fadd_rn(c, 12582912.0f));
+        asm("bfi.b32 %0, %1, %2, %3, 4;" : "=r"(w) : "r"(k), "r"(w), "r"(4 * i));
+    }
+    return w;
+}
+
+// Two INT4 codes (one byte, low nibble first) -> two binary32 (exact): a
+// nibble n holds k = (n ^ 8) - 8; n ^ 8 goes into the low significand bits of
+// 1.5 * 2^23 (whose ulp is 1), and 1.5 * 2^23 + 8 is subtracted.
+__device__ __forceinline__ float2 int4x2_decode(uint32_t byte) {
+    const float lo = __uint_as_float((byte & 0xfu) ^ 0x4b400008u) - 12582920.0f;
+    const float hi = __uint_as_float(((byte >> 4) & 0xfu) ^ 0x4b400008u) - 12582920.0f;
+    return make_float2(lo, hi);
+}
+
 // Binary32 -> bf16 bits, round to nearest even (finite values).
 __device__ __forceinline__ uint32_t bf16x2_pack(float lo, float hi) {
     uint32_t r;

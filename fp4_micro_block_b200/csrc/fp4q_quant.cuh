@@ -42,7 +42,7 @@ constexpr int kQProducers = FP4Q_QPRODUCERS;
 constexpr int kQCtas = FP4Q_QCTAS;             // CTAs per SM
 constexpr int kQRingBytes = 192 * 1024 / kQCtas;
 
-enum : int { FMT_NVFP4 = 0, FMT_MXFP4 = 1, FMT_DUAL = 2 };
+enum : int { FMT_NVFP4 = 0, FMT_MXFP4 = 1, FMT_DUAL = 2, FMT_INT4 = 3 };
 
 struct QuantParams {
     int64_t M, K;
@@ -80,9 +80,10 @@ struct QGeo {
     static_assert(smem <= 227 * 1024, "shared memory");
 };
 
-// Tensor scale of the dynamic NVFP4 mode: amax over the per-CTA partials / 2688.
+// Tensor scale of the dynamic mode: amax over the per-CTA partials / top (the
+// largest grid value times 448: 2688 for NVFP4, 3136 for INT4).
 __device__ __forceinline__ float tensor_scale_from_partials(const float* partials, int n,
-                                                            float* red) {
+                                                            float* red, float top = 2688.0f) {
     float m = 0.0f;
     for (int i = threadIdx.x; i < n; i += blockDim.x) m = fmaxf(m, partials[i]);
 #pragma unroll
@@ -92,7 +93,7 @@ __device__ __forceinline__ float tensor_scale_from_partials(const float* partial
     m = 0.0f;
     for (int i = 0; i < (int)(blockDim.x >> 5); ++i) m = fmaxf(m, red[i]);
     __syncthreads();
-    return __fdiv_rn(m, 2688.0f);
+    return __fdiv_rn(m, top);
 }
 
 // Orders the computation of x before any later volatile asm.

@@ -185,14 +185,15 @@ __device__ __forceinline__ void build_table(float4* t, float s) {
 
 // The NVFP4 rule with IEEE divisions for one block of a unit (component Y of
 // the pairs), for units outside the fast range.  Writes two code words and
-// returns the scale byte.
-template <bool Y>
+// returns the scale byte.  INT4: the same rule with the largest grid value 7
+// and integer codes.
+template <bool Y, bool INT4 = false>
 __device__ __forceinline__ uint32_t nvfp4_block_ieee(const float2* n, float a, float s, float fold,
                                                      uint32_t& w0, uint32_t& w1) {
     float d = 0.0f;
     uint32_t e = 0;
     if (s > 0.0f) {
-        const float r = __fdiv_rn(__fdiv_rn(a, 6.0f), s);  // a already folded
+        const float r = __fdiv_rn(__fdiv_rn(a, INT4 ? 7.0f : 6.0f), s);  // a already folded
         e = e4m3_encode(r);
         d = e4m3_decode(e) * s;
     }
@@ -202,8 +203,13 @@ __device__ __forceinline__ uint32_t nvfp4_block_ieee(const float2* n, float a, f
         const float x = -(Y ? n[i].y : n[i].x) * fold;
         q[i] = d != 0.0f ? __fdiv_rn(x, d) : 0.0f;
     }
-    w0 = d != 0.0f ? e2m1_pack8(q) : 0u;
-    w1 = d != 0.0f ? e2m1_pack8(q + 8) : 0u;
+    if constexpr (INT4) {
+        w0 = d != 0.0f ? int4_pack8(q) : 0u;
+        w1 = d != 0.0f ? int4_pack8(q + 8) : 0u;
+    } else {
+        w0 = d != 0.0f ? e2m1_pack8(q) : 0u;
+        w1 = d != 0.0f ? e2m1_pack8(q + 8) : 0u;
+    }
     return e;
 }
 

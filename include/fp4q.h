@@ -46,6 +46,14 @@
  *  - Dual scale (FP4Quant abstract, "micro-grouped dual-scale FP4"): an FP32
  *    group scale G = amax_128/2688 per 128 contiguous elements, then the NVFP4
  *    rule per 16-block with G in place of s_t.
+ *  - INT4 (ARCQuant summary, "Generalisabilite": the ARCQuant scheme extends
+ *    to INT4; the pages give no INT4 rule, so this is the NVFP4 container with
+ *    the integer grid): codes are the integers -7..7 as 4-bit two's complement
+ *    (low nibble = even column; -8 is never written); s_t = amax/3136
+ *    (3136 = 7*448); per 16-block r = (amax_b/7)/s_t, e = E4M3(r),
+ *    d = E4M3(e)*s_t, code = y/d rounded to the nearest integer (ties to even)
+ *    and clamped to +-7.  Produced by fp4q_arc_quantize, read by
+ *    fp4q_dequantize.
  */
 #ifndef FP4Q_H
 #define FP4Q_H
@@ -72,7 +80,9 @@ typedef enum fp4q_status {
 typedef enum fp4q_format {
     FP4Q_NVFP4 = 0,      /* B = 16, E4M3 block scale, FP32 tensor scale          */
     FP4Q_MXFP4 = 1,      /* B = 32, E8M0 shared exponent                          */
-    FP4Q_NVFP4_DUAL = 2  /* B = 16, E4M3 micro-scale, FP32 scale per 128 elements */
+    FP4Q_NVFP4_DUAL = 2, /* B = 16, E4M3 micro-scale, FP32 scale per 128 elements */
+    FP4Q_INT4 = 3        /* B = 16, integers -7..7, E4M3 block scale, FP32 tensor
+                            scale (fp4q_arc_quantize and fp4q_dequantize only)   */
 } fp4q_format;
 
 typedef enum fp4q_scale_layout {
@@ -83,8 +93,9 @@ typedef enum fp4q_scale_layout {
 } fp4q_scale_layout;
 
 typedef enum fp4q_tscale_mode {
-    FP4Q_TSCALE_DYNAMIC = 0, /* compute s_t = amax/2688 of the quantized tensor and
-                                WRITE it to *tensor_scale (two passes over x)        */
+    FP4Q_TSCALE_DYNAMIC = 0, /* compute s_t = amax/2688 (INT4: amax/3136) of the
+                                quantized tensor and WRITE it to *tensor_scale (two
+                                passes over x)                                       */
     FP4Q_TSCALE_STATIC = 1   /* READ s_t from *tensor_scale (a calibrated scale;
                                 one pass).  s_t <= 0 gives zero scales and codes.    */
 } fp4q_tscale_mode;
@@ -197,7 +208,7 @@ fp4q_status fp4q_hadamard_quantize_signed(const void* x, int64_t M, int64_t K, i
                                           fp4q_stream_t stream);
 
 /* fp4q_arc_quantize -- ARCQuant fused reorder + RMSNorm + primary quantization
- * + residual quantization of the outlier channels, in NVFP4 or MXFP4.
+ * + residual quantization of the outlier channels, in NVFP4, MXFP4 or INT4.
  *   For each row: y[p] = x[perm[p]] / sqrt(mean_k x[k]^2 + eps) * gamma[perm[p]]
  *   (p = 0..K-1), primary = Q(y); for j < S, the residual
  *   res[j] = y[outliers[j]] - dq(outliers[j]), quantized in the same format.
@@ -205,6 +216,8 @@ fp4q_status fp4q_hadamard_quantize_signed(const void* x, int64_t M, int64_t K, i
  *       halves; dq = (E2M1 value * E4M3 value) * s_t.
  *     FP4Q_MXFP4: blocks of 32, E8M0 scales; dq = E2M1 value * 2^(b - 127).
  *       tensor_scale, mode and workspace are unused (may be NULL / 0).
+ *     FP4Q_INT4: blocks of 16, E4M3 scales, one tensor scale s_t (amax/3136
+ *       in DYNAMIC mode); dq = (integer * E4M3 value) * s_t.
  *   Output row = [primary K columns | residual S columns]:
  *   codes uint8 [M, (K+S)/2], scales [M, (K+S)/B] (or swizzled).
  *   gamma     bf16 [K], indexed by ORIGINAL channel.
@@ -215,8 +228,8 @@ fp4q_status fp4q_hadamard_quantize_signed(const void* x, int64_t M, int64_t K, i
  *             out-of-range handling as perm); the
  *             calibrated choice is 0..S-1 (channels sorted by descending
  *             calibration absmax).  May be NULL when S == 0.
- *   tensor_scale / mode / workspace as for fp4q_quantize_nvfp4 (NVFP4 only);
- *   DYNAMIC uses the amax of y.
+ *   tensor_scale / mode / workspace as for fp4q_quantize_nvfp4 (NVFP4 and
+ *   INT4); DYNAMIC uses the amax of y.
  * Requires K % B == 0, S % B == 0, 0 <= S <= K, K <= 16384, eps >= 0, and that
  * one warp's buffers fit in shared memory (12 K + 8 S bytes plus the CTA's
  * 4 K + S/8 + 1.3 KiB, within 227 KiB), else FP4Q_ERR_UNSUPPORTED.
@@ -224,7 +237,7 @@ fp4q_status fp4q_hadamard_quantize_signed(const void* x, int64_t M, int64_t K, i
  * maximum, subset S), 2 (two-stage quantization), 3 (residual channels
  * concatenated along K) and 5 (one fused kernel: reorder, RMSNorm, primary and
  * residual quantization, GEMM-ready channel layout); "Generalisabilite" (the
- * scheme extends to MXFP4). */
+ * scheme extends to MXFP4 and INT4). */
 fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int64_t ldx,
                               const void* gamma, float eps, const int32_t* perm,
                               const int32_t* outliers, int64_t S, fp4q_format format,
@@ -236,13 +249,14 @@ fp4q_status fp4q_arc_quantize(const void* x, int64_t M, int64_t K, int64_t ldx,
 /* fp4q_dequantize -- codes + scales back to bf16, optionally followed by the
  * inverse block Hadamard (the normalised Sylvester matrix is its own inverse).
  *   value = (E2M1 value * E4M3 value) * s (s = *scale_fp32 for NVFP4, the
- *   group scale for the dual format) or E2M1 value * 2^(b-127) for MXFP4,
- *   computed in FP32, then (if inv_had_size) rotated, then rounded to bf16
- *   (nearest even).
+ *   group scale for the dual format), E2M1 value * 2^(b-127) for MXFP4, or
+ *   (integer * E4M3 value) * *scale_fp32 for INT4, computed in FP32, then (if
+ *   inv_had_size) rotated, then rounded to bf16 (nearest even).
  *   codes      uint8 [M, K/2]; scales [M, K/B] or swizzled, per `layout`.
- *   scale_fp32 NVFP4: 1 float; dual: float [M, K/128]; MXFP4: unused.
+ *   scale_fp32 NVFP4, INT4: 1 float; dual: float [M, K/128]; MXFP4: unused.
  *   y          bf16 [M, K] (row stride K).  (written)
- *   inv_had_size 0 or n in {16, 32, 64, 128, 256, 512}, K % n == 0.
+ *   inv_had_size 0 or n in {16, 32, 64, 128, 256, 512}, K % n == 0 (INT4: 0
+ *              only, else FP4Q_ERR_UNSUPPORTED).
  * Requires K % B == 0 (K % 128 for dual), K >= 64, 16-byte aligned codes and y.
  * Defined by: FP4Quant abstract (the receiving side of FP4-compressed
  * activations: unpack, rescale, inverse FWHT). */

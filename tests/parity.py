@@ -36,8 +36,10 @@ def bits_to_torch_cuda(bits: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-def code_values(codes_packed: np.ndarray) -> np.ndarray:
+def code_values(codes_packed: np.ndarray, fmt: str = "nvfp4") -> np.ndarray:
     u = oracle.unpack_codes(codes_packed)
+    if fmt == "int4":  # 4-bit two's complement integers
+        return oracle.int4_decode(u).astype(np.float64)
     mag = E2M1_MAG[u & 7]
     return np.where(u & 8, -mag, mag)
 
@@ -83,8 +85,8 @@ def tolerant_counts(fmt: str, K: int, gpu, orc, y_orc: np.ndarray, name: str = "
     co, so, fo = orc
     dg = block_scale(fmt, sg, fg, K)
     do = block_scale(fmt, so, fo, K)
-    vg = code_values(cg) * dg
-    vo = code_values(co) * do
+    vg = code_values(cg, fmt) * dg
+    vo = code_values(co, fmt) * do
     scale_diff = np.repeat(sg != so, 16 if fmt != "mxfp4" else 32, axis=1)[:, :K]
     n_blocks_diff = int((sg != so).sum())
     if n_blocks_diff:
@@ -95,19 +97,26 @@ def tolerant_counts(fmt: str, K: int, gpu, orc, y_orc: np.ndarray, name: str = "
     bad = ~close & ~scale_diff
     nbad = int(bad.sum())
     if nbad:
-        ug = oracle.unpack_codes(cg)[bad]
-        uo = oracle.unpack_codes(co)[bad]
-        # position on the signed grid: -7..-1, 0, 1..7
-        pg = np.where(ug & 8, -(ug & 7).astype(np.int64), (ug & 7).astype(np.int64))
-        po = np.where(uo & 8, -(uo & 7).astype(np.int64), (uo & 7).astype(np.int64))
+        if fmt == "int4":  # the integer is its own grid position
+            pg = code_values(cg, fmt)[bad].astype(np.int64)
+            po = code_values(co, fmt)[bad].astype(np.int64)
+        else:
+            ug = oracle.unpack_codes(cg)[bad]
+            uo = oracle.unpack_codes(co)[bad]
+            # position on the signed grid: -7..-1, 0, 1..7
+            pg = np.where(ug & 8, -(ug & 7).astype(np.int64), (ug & 7).astype(np.int64))
+            po = np.where(uo & 8, -(uo & 7).astype(np.int64), (uo & 7).astype(np.int64))
         assert np.all(np.abs(pg - po) <= 1), f"{name}: codes more than one grid step apart"
     # elements of blocks whose scale differs: round-to-nearest bound against y_orc
     if n_blocks_diff:
         y = y_orc.astype(np.float64)[scale_diff]
         v = np.abs(y) / np.maximum(dg[scale_diff], 1e-300)
-        step = np.where(v <= 2, 0.5, np.where(v <= 4, 1.0, 2.0))
         err = np.abs(vg[scale_diff] - y)
-        bound = np.where(v > 6, (v - 6 + 1e-3) * dg[scale_diff], (step / 2 + 1e-3) * dg[scale_diff])
+        if fmt == "int4":  # unit steps, clamp at 7
+            bound = np.where(v > 7, (v - 7 + 1e-3) * dg[scale_diff], (0.5 + 1e-3) * dg[scale_diff])
+        else:
+            step = np.where(v <= 2, 0.5, np.where(v <= 4, 1.0, 2.0))
+            bound = np.where(v > 6, (v - 6 + 1e-3) * dg[scale_diff], (step / 2 + 1e-3) * dg[scale_diff])
         assert np.all(err <= bound * (1 + 1e-6)), f"{name}: error bound violated in rescaled blocks"
     return {"codes_off": nbad, "blocks_rescaled": n_blocks_diff, "n": int(vg.size),
             "n_blocks": int(sg.size)}
@@ -152,11 +161,15 @@ def arc_counts(fmt: str, K: int, outl, gpu, orc_primary, y_orc: np.ndarray, name
         return c
     if fmt == "mxfp4":
         dq = oracle.mxfp4_dequantize(cg[:, :K // 2], sg[:, :K // B])
+    elif fmt == "int4":
+        dq = oracle.int4_dequantize(cg[:, :K // 2], sg[:, :K // B], float(np.asarray(fg).reshape(-1)[0]))
     else:
         dq = oracle.nvfp4_dequantize(cg[:, :K // 2], sg[:, :K // B], float(np.asarray(fg).reshape(-1)[0]))
     r = (np.asarray(y_orc, np.float32)[:, outl] - dq[:, outl]).astype(np.float32)
     if fmt == "mxfp4":
         cr, sr = oracle.mxfp4_quantize(r)
+    elif fmt == "int4":
+        cr, sr = oracle.int4_quantize(r, fo)
     else:
         cr, sr = oracle.nvfp4_quantize(r, fo)
     c2 = tolerant_counts(fmt, S, (cg[:, K // 2:], sg[:, K // B:], fg), (cr, sr, fo), r, name + "-residual")

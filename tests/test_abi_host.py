@@ -101,6 +101,8 @@ def test_quantize_mxfp4_and_hadamard_validation(fq):
     assert h(X, 4, 192, 192, 64, 2, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
     assert h(X, 4, 128, 128, 64, 9, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
     assert h(X, 4, 128, 128, 64, 2, CODES, SCALES, None, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
+    # INT4 is an ARC / dequantize format only
+    assert h(X, 4, 128, 128, 64, fq.FP4Q_INT4, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
 
 
 def test_arc_validation(fq):
@@ -120,6 +122,13 @@ def test_arc_validation(fq):
     assert a(X, 4, 128, 128, G, 1e-6, P, O, 16, 1, CODES, SCALES, None, 0, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
     assert a(X, 4, 144, 144, G, 1e-6, P, O, 32, 1, CODES, SCALES, None, 0, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
     assert a(X, 0, 128, 128, G, 1e-6, P, O, 32, 1, CODES, SCALES, None, 0, 0, None, 0, None) == fq.FP4Q_OK
+    # INT4: blocks of 16 under a tensor scale, like NVFP4; unknown formats are rejected
+    i4 = fq.FP4Q_INT4
+    assert a(X, 4, 128, 128, G, 1e-6, P, O, 16, i4, CODES, SCALES, None, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert a(X, 4, 128, 128, G, 1e-6, P, O, 24, i4, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert a(X, 4, 128, 128, G, 1e-6, P, O, 16, i4, CODES, SCALES, SF, 0, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert a(X, 4, 128, 128, G, 1e-6, P, O, 16, 4, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert a(X, 0, 128, 128, G, 1e-6, P, O, 16, i4, CODES, SCALES, SF, 1, 0, None, 0, None) == fq.FP4Q_OK
 
 
 def test_dequantize_validation(fq):
@@ -128,7 +137,12 @@ def test_dequantize_validation(fq):
     Y = 0x90000
     assert d(0, CODES, SCALES, SF, 4, 72, 0, 0, Y, None) == fq.FP4Q_ERR_INVALID_ARG
     assert d(1, CODES, SCALES, None, 4, 80, 0, 0, Y, None) == fq.FP4Q_ERR_INVALID_ARG
-    assert d(3, CODES, SCALES, SF, 4, 128, 0, 0, Y, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert d(4, CODES, SCALES, SF, 4, 128, 0, 0, Y, None) == fq.FP4Q_ERR_INVALID_ARG
+    # INT4: a tensor scale is required, and there is no rotated INT4 path
+    assert d(fq.FP4Q_INT4, CODES, SCALES, None, 4, 128, 0, 0, Y, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert d(fq.FP4Q_INT4, CODES, SCALES, SF, 4, 128, 0, 16, Y, None) == fq.FP4Q_ERR_UNSUPPORTED
+    assert d(fq.FP4Q_INT4, CODES, SCALES, SF, 4, 72, 0, 0, Y, None) == fq.FP4Q_ERR_INVALID_ARG
+    assert d(fq.FP4Q_INT4, CODES, SCALES, SF, 0, 128, 0, 0, Y, None) == fq.FP4Q_OK
     assert d(0, CODES, SCALES, SF, 4, 128, 0, 48, Y, None) == fq.FP4Q_ERR_INVALID_ARG
     assert d(0, CODES, SCALES, None, 4, 128, 0, 0, Y, None) == fq.FP4Q_ERR_INVALID_ARG
     assert d(0, CODES + 8, SCALES, SF, 4, 128, 0, 0, Y, None) == fq.FP4Q_ERR_ALIGNMENT

@@ -141,6 +141,7 @@ def test_canary_hadamard_quantize(fq, M, case, layout):
 ARC_CASES = [  # (format name, K, S)
     ("nvfp4", 1040, 16), ("nvfp4", 1056, 32), ("nvfp4", 1088, 64), ("nvfp4", 1152, 0),
     ("mxfp4", 1056, 32), ("mxfp4", 1088, 64), ("mxfp4", 1152, 0),
+    ("int4", 1040, 16), ("int4", 1088, 64),
 ]
 
 
@@ -153,7 +154,7 @@ def test_canary_arc(fq, M, case, layout, mode):
     mx = fmt_name == "mxfp4"
     if mx and mode == 1:
         pytest.skip("MXFP4 has no tensor-scale mode")
-    fmt = fq.FP4Q_MXFP4 if mx else fq.FP4Q_NVFP4
+    fmt = {"nvfp4": fq.FP4Q_NVFP4, "mxfp4": fq.FP4Q_MXFP4, "int4": fq.FP4Q_INT4}[fmt_name]
     x_bits, gamma, perm, outl = workloads.arc_activations(M, K, seed=M + K, S=S, calib_rows=64)
     x = bits_to_torch_cuda(x_bits)
     g = bits_to_torch_cuda(gamma)
@@ -180,6 +181,7 @@ DQ_CASES = [  # (format name, n, K)
     ("nvfp4", 128, 1152), ("nvfp4", 512, 1536),
     ("mxfp4", 0, 1056), ("mxfp4", 32, 1056), ("mxfp4", 64, 1088), ("mxfp4", 256, 1536),
     ("dual", 0, 1152), ("dual", 16, 1152), ("dual", 128, 1152), ("dual", 512, 1536),
+    ("int4", 0, 1040), ("int4", 0, 1088),
 ]
 
 
@@ -188,12 +190,13 @@ DQ_CASES = [  # (format name, n, K)
 @pytest.mark.parametrize("layout", [0, 1])
 def test_canary_dequantize(fq, M, case, layout):
     fmt_name, n, K = case
-    fmt = {"nvfp4": fq.FP4Q_NVFP4, "mxfp4": fq.FP4Q_MXFP4, "dual": fq.FP4Q_NVFP4_DUAL}[fmt_name]
+    fmt = {"nvfp4": fq.FP4Q_NVFP4, "mxfp4": fq.FP4Q_MXFP4, "dual": fq.FP4Q_NVFP4_DUAL,
+           "int4": fq.FP4Q_INT4}[fmt_name]
     codes, scales, sc = workloads.random_payload(M, K, fmt_name, seed=M + K + n)
     if layout == 1:
         import oracle  # test infrastructure: lays the scale bytes out in the tiled layout
         scales = oracle.swizzle_scales(scales)
-    sct = (None if sc is None else torch.tensor([sc], device="cuda") if fmt_name == "nvfp4"
+    sct = (None if sc is None else torch.tensor([sc], device="cuda") if fmt_name in ("nvfp4", "int4")
            else torch.from_numpy(sc).cuda())
     ct, st = torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda()
     y = Guarded((M, K), torch.bfloat16)

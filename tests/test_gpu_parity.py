@@ -201,6 +201,21 @@ def test_dequantize_bitexact(fq, fmt, layout):
     assert_bitexact("dequant", bf16_torch_to_bits(y), want)
 
 
+@pytest.mark.parametrize("shape", [(70, 2048), (131, 1040), (1, 64)])
+@pytest.mark.parametrize("layout", [0, 1])
+def test_dequantize_int4_random_payload_bitexact(fq, shape, layout):
+    """INT4 dequantization of uniformly random code and scale bytes (every
+    nibble, -8 included): (integer * E4M3) * s_t to bf16, bit-exact."""
+    M, K = shape
+    c, s, sc = workloads.random_payload(M, K, "int4", seed=M + K)
+    want = oracle.dequantize_bf16("int4", c, s, sc)
+    s_dev = s if layout == 0 else oracle.swizzle_scales(s)
+    y = fq.dequantize(fq.FP4Q_INT4, torch.from_numpy(c).cuda(), torch.from_numpy(s_dev).cuda(),
+                      torch.tensor([sc], device="cuda"), K, layout)
+    torch.cuda.synchronize()
+    assert_bitexact("dequant-int4-random", bf16_torch_to_bits(y), want)
+
+
 # ----------------------------------------------------------------------------- Hadamard
 
 @pytest.mark.parametrize("n", [16, 32, 64, 128, 256, 512])
@@ -483,6 +498,70 @@ def test_arc_mxfp4_general_outlier_list(fq):
                                   "arc-mxfp4-general"), 2e-4, "arc-mxfp4-general")
 
 
+# ----------------------------------------------------------------------------- ARC, INT4
+
+def _arc_int4(fq, x_bits, gamma, perm, outl, ts=None, layout=0):
+    """The INT4 ARC path through the C ABI (ts: a static tensor scale)."""
+    codes, scales, sf = fq.arc_quantize(
+        bits_to_torch_cuda(x_bits), bits_to_torch_cuda(gamma), torch.from_numpy(perm).cuda(),
+        torch.from_numpy(outl).cuda() if len(outl) else None, 1e-6,
+        None if ts is None else torch.tensor([np.float32(ts)], device="cuda"), layout, fmt=fq.FP4Q_INT4)
+    torch.cuda.synchronize()
+    return codes, scales, sf
+
+
+@pytest.mark.parametrize("shape", [(64, 1024, 64), (37, 4096, 256), (20, 512, 0), (16, 8192, 128),
+                                   (131, 1056, 32)])
+@pytest.mark.parametrize("layout", [0, 1])
+def test_arc_int4_tolerance(fq, shape, layout):
+    """INT4 variant of the two-stage path (ARCQuant summary, Generalisabilite),
+    dynamic tensor scale amax / 3136: primary columns against the oracle's
+    INT4 of y, residual columns against the oracle's INT4 of the residual of
+    the kernel's own primary codes."""
+    M, K, S = shape
+    x_bits, gamma, perm, outl = workloads.arc_activations(M, K, seed=K + S + 2, S=S)
+    outl = outl[:S]
+    codes, scales, sf = _arc_int4(fq, x_bits, gamma, perm, outl, layout=layout)
+    c_o, s_o, sc_o, y_o = oracle.arc(x_bits, gamma, perm, outl, fmt="int4")
+    assert abs(float(to_np(sf)[0]) - float(sc_o)) <= 4e-7 * float(sc_o)
+    s_g = linear_scales(fq, scales, M, (K + S) // 16, layout)
+    c = arc_counts("int4", K, outl, (to_np(codes), s_g, to_np(sf)),
+                   (c_o[:, :K // 2], s_o[:, :K // 16], sc_o), y_o, name="arc-int4")
+    check_fractions(c, 2e-4, "arc-int4")
+
+
+def test_arc_int4_static_and_general_outlier_list(fq):
+    """Static tensor scale (read, not written) and outlier positions in
+    arbitrary order, two of them in one 16-block."""
+    M, K, S = 24, 1024, 32
+    x_bits, gamma, perm, _ = workloads.arc_activations(M, K, seed=7, S=S)
+    outl = np.random.default_rng(8).choice(K, S, replace=False).astype(np.int32)
+    outl[1] = outl[0] ^ 1
+    assert len(set(outl.tolist())) == S
+    codes, scales, sf = _arc_int4(fq, x_bits, gamma, perm, outl, ts=0.004)
+    assert to_np(sf)[0] == np.float32(0.004)
+    c_o, s_o, sc_o, y_o = oracle.arc(x_bits, gamma, perm, outl, s_t=np.float32(0.004), fmt="int4")
+    c = arc_counts("int4", K, outl, (to_np(codes), to_np(scales), to_np(sf)),
+                   (c_o[:, :K // 2], s_o[:, :K // 16], sc_o), y_o, name="arc-int4-static")
+    check_fractions(c, 2e-4, "arc-int4-static")
+
+
+@pytest.mark.parametrize("layout", [0, 1])
+def test_dequantize_int4_bitexact(fq, layout):
+    """INT4 dequantization of the ARC operand [K | S]: value = (integer * E4M3)
+    * s_t rounded to bf16, bit-exact against the oracle on the kernel's own
+    codes and scales."""
+    M, K, S = 131, 1056, 32
+    x_bits, gamma, perm, outl = workloads.arc_activations(M, K, seed=9, S=S)
+    codes, scales, sf = _arc_int4(fq, x_bits, gamma, perm, outl[:S], layout=layout)
+    y = fq.dequantize(fq.FP4Q_INT4, codes, scales, sf, K + S, layout)
+    torch.cuda.synchronize()
+    s_lin = linear_scales(fq, scales, M, (K + S) // 16, layout)
+    want = oracle.f32_to_bf16(oracle.int4_dequantize(to_np(codes), s_lin, float(to_np(sf)[0])))
+    assert_bitexact("dequant-int4", bf16_torch_to_bits(y), want)
+    assert fq.fp4q_device_error() == 0
+
+
 # ----------------------------------------------------------------------------- full sizes
 
 CHUNK = 1024  # oracle rows per chunk (bounded host memory for the comparisons)
@@ -621,6 +700,28 @@ def test_full_dual_fwht512_round_trip_32768x4096(fq):
     xh = bf16_torch_to_bits(y)[rows]
     assert_roundtrip(xh, w, 512, name="full-dual-roundtrip")
     block_l2_identity(x_bits[rows], xh, dq, y_o, w, 512, name="full-dual-l2")
+
+
+@pytest.mark.slow
+def test_full_arc_int4_8192x4096(fq):
+    """INT4 ARC at the ARC workload's full size, dynamic tensor scale, every row."""
+    M, K, S = 8192, 4096, 256
+    x_bits, gamma, perm, outl = workloads.arc_activations(M, K, seed=4, S=S)
+    y = np.empty((M, K), np.float32)
+    for r0 in range(0, M, CHUNK):
+        y[r0:r0 + CHUNK] = oracle.arc_prepare(x_bits[r0:r0 + CHUNK], gamma, perm)
+    st_o = np.float32(oracle.int4_tensor_scale(oracle.amax(y)))
+    codes, scales, sf = _arc_int4(fq, x_bits, gamma, perm, outl)
+    assert abs(float(to_np(sf)[0]) - float(st_o)) <= 4e-7 * float(st_o)
+    sf_g, codes, scales = to_np(sf), to_np(codes), to_np(scales)
+    tot = None
+    for r0 in range(0, M, CHUNK):
+        yc = y[r0:r0 + CHUNK]
+        c_o, s_o = oracle.int4_quantize(yc, st_o)
+        c = arc_counts("int4", K, outl, (codes[r0:r0 + CHUNK], scales[r0:r0 + CHUNK], sf_g),
+                       (c_o, s_o, st_o), yc, name="full-arc-int4")
+        tot = add_counts(tot, c)
+    check_fractions(tot, 2e-4, "full-arc-int4")
 
 
 @pytest.mark.slow

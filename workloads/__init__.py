@@ -145,14 +145,16 @@ def random_payload(M: int, K: int, fmt: str, seed: int = 6):
 
     Returns ``(codes [M, K/2] uint8, scales uint8, scale)``: every code byte in
     0..255 (two E2M1 codes); scale bytes E4M3 in 0x08..0x6f (NVFP4 / dual) or
-    E8M0 in 100..139 (MXFP4); ``scale`` a float32 tensor scale (NVFP4), a
-    [M, K/128] float32 array drawn from U(1e-3, 1) (dual) or None (MXFP4)."""
+    E8M0 in 100..139 (MXFP4); ``scale`` a float32 tensor scale (NVFP4, INT4),
+    a [M, K/128] float32 array drawn from U(1e-3, 1) (dual) or None (MXFP4).
+    INT4 code bytes hold two 4-bit two's complement integers (every nibble,
+    -8 included, is a valid input to a dequantizer)."""
     rng = np.random.default_rng(seed)
     codes = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
     if fmt == "mxfp4":
         return codes, rng.integers(100, 140, size=(M, K // 32), dtype=np.uint8), None
     scales = rng.integers(0x08, 0x70, size=(M, K // 16), dtype=np.uint8)
-    if fmt == "nvfp4":
+    if fmt in ("nvfp4", "int4"):
         return codes, scales, np.float32(rng.uniform(1e-3, 1.0))
     if fmt == "dual":
         return codes, scales, rng.uniform(1e-3, 1.0, size=(M, K // 128)).astype(np.float32)
