@@ -90,3 +90,54 @@ def test_format_error_table(fq):
     if out:
         with open(out, "w") as fh:
             json.dump({"workload": f"hadamard_channels {M}x{K} seed 3", "table": table}, fh, indent=1)
+
+
+def _arc_dequant_two_stage(fmt: str, codes, scales, s_t, K: int, outl) -> tuple:
+    """(primary values, primary + residual correction) of an ARC operand, from
+    the oracle's dequantizer (fp32)."""
+    prim = oracle.dequantize(fmt, codes[:, :K // 2], scales[:, :K // (32 if fmt == "mxfp4" else 16)], s_t)
+    res = oracle.dequantize(fmt, codes[:, K // 2:], scales[:, K // (32 if fmt == "mxfp4" else 16):], s_t)
+    two = prim.astype(np.float64).copy()
+    two[:, outl] += res
+    return prim.astype(np.float64), two
+
+
+@pytest.mark.slow
+def test_arc_format_error_table(fq):
+    """Error of the ARCQuant two-stage path in NVFP4, MXFP4 and INT4 on the ARC
+    workload's recipe (1024 rows x 4096, S = 256): relative MSE against the
+    prepared matrix y of the primary stage alone and of primary + residual
+    (ARCQuant summary, Methodologie item 2: the residual corrects the outlier
+    channels; Generalisabilite: the scheme carries over to MXFP4 and INT4).
+    The kernels' codes are decoded by the oracle; the oracle's own codes on the
+    same rows must give the same errors to 3 %, and for every format the
+    residual stage must lower the error.  With FP4Q_ARC_ERROR_TABLE=<path> the
+    table is written there as JSON."""
+    M, K, S = 1024, 4096, 256
+    x_bits, gamma, perm, outl = workloads.arc_activations(M, K, seed=4, S=S)
+    y = oracle.arc_prepare(x_bits, gamma, perm).astype(np.float64)
+    ny = float(np.square(y).sum())
+    table = {}
+    for name, f in (("nvfp4", fq.FP4Q_NVFP4), ("mxfp4", fq.FP4Q_MXFP4), ("int4", fq.FP4Q_INT4)):
+        codes, scales, sf = fq.arc_quantize(
+            bits_to_torch_cuda(x_bits), bits_to_torch_cuda(gamma), torch.from_numpy(perm).cuda(),
+            torch.from_numpy(outl).cuda(), 1e-6, fmt=f)
+        torch.cuda.synchronize()
+        s_t = None if sf is None else float(sf.item())
+        prim, two = _arc_dequant_two_stage(name, codes.cpu().numpy(), scales.cpu().numpy(), s_t, K, outl)
+        c_o, s_o, st_o, _ = oracle.arc(x_bits, gamma, perm, outl, fmt=name)
+        prim_o, two_o = _arc_dequant_two_stage(name, c_o, s_o, None if st_o is None else float(st_o), K, outl)
+        e1, e2 = float(np.square(prim - y).sum() / ny), float(np.square(two - y).sum() / ny)
+        o1, o2 = float(np.square(prim_o - y).sum() / ny), float(np.square(two_o - y).sum() / ny)
+        assert abs(e1 - o1) <= 0.03 * o1 and abs(e2 - o2) <= 0.03 * o2, (name, e1, o1, e2, o2)
+        assert e2 < e1, (name, e1, e2)
+        yo = y[:, outl]
+        out1 = float(np.square(prim[:, outl] - yo).sum() / np.square(yo).sum())
+        out2 = float(np.square(two[:, outl] - yo).sum() / np.square(yo).sum())
+        table[name] = {"rel_mse_primary": e1, "rel_mse_two_stage": e2,
+                       "rel_mse_outlier_channels_primary": out1, "rel_mse_outlier_channels_two_stage": out2}
+    assert table["mxfp4"]["rel_mse_two_stage"] > table["nvfp4"]["rel_mse_two_stage"]
+    out = os.environ.get("FP4Q_ARC_ERROR_TABLE")
+    if out:
+        with open(out, "w") as fh:
+            json.dump({"workload": f"arc_activations {M}x{K} S={S} seed 4", "table": table}, fh, indent=1)
