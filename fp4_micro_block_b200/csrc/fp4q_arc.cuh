@@ -249,8 +249,12 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
         return v;
     };
     const int64_t P = (p.M + 1) / 2;  // row pairs
-    const int64_t gw = (int64_t)blockIdx.x * NP + ps, nw = (int64_t)gridDim.x * NP;
-    const int64_t n_my = P > gw ? (P - 1 - gw) / nw + 1 : 0;
+    // Each CTA takes a contiguous range of P / gridDim.x pairs (the ranges differ
+    // by at most one pair), dealt round-robin to its slots: per-CTA loads stay
+    // balanced even when there are only two or three pairs per slot.
+    const int64_t p_lo = (int64_t)blockIdx.x * P / gridDim.x, p_hi = ((int64_t)blockIdx.x + 1) * P / gridDim.x;
+    const int64_t gw = p_lo + ps, nw = NP;
+    const int64_t n_my = p_hi > gw ? (p_hi - 1 - gw) / nw + 1 : 0;
     uint8_t* const land = wb + L.land;
     auto issue = [&](int64_t i) {  // lane 0 of the first warp: pair i of the slot into stage i % SR
         const int64_t r0 = 2 * (gw + i * nw);
