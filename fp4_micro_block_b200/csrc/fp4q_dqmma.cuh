@@ -24,7 +24,7 @@
 // N = 32 per group), three slices in flight in TMEM, so the tensor cores work
 // on the next slices while the epilogue drains one.
 //
-// CTA roles (persistent, one CTA per SM, 3 + 4 kDqmEpiWg warps):
+// CTA roles (persistent, one CTA per SM, 3 + 8 warps):
 //   warp 0 lane 0  TMA: per tile the codes (two 128-byte-swizzled boxes of
 //                  128 rows x 256 codes), the linear scale bytes (128 x 32) and
 //                  the group scales (128 x 4, dual) into a ring of stages;
@@ -33,10 +33,9 @@
 //   warp 2         rewrites a tile's linear scale bytes into the 128 x 4 tiled
 //                  layout that tcgen05.cp reads (eight 512-byte tiles, one per
 //                  64-column K step);
-//   warps 3..      epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 (one row
-//                  each) and 16 of the 32 columns of a slice (half wg % 2 of
-//                  warpgroup wg = (w - 3) / 4); with four warpgroups, warpgroups
-//                  0-1 take the even slices and 2-3 the odd ones.
+//   warps 3..10    epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 (one row
+//                  each) and 16 of the 32 columns of every slice (half wg of
+//                  warpgroup wg = (w - 3) / 4).
 // Every wait is bounded: a wait that runs out sets g_device_error, the role
 // stops, and the CTA drains its copies and MMAs before it frees TMEM and exits.
 #pragma once
@@ -59,12 +58,13 @@ constexpr int kDqmBarOff = kDqmOneOff + 512;
 constexpr int kDqmNumBars = 2 * kDqmStages + 2 * 2 + 2 * kDqmSlots + 1;
 constexpr int kDqmSlotOff = kDqmBarOff + kDqmNumBars * 8;
 constexpr int kDqmSmem = 1024 + kDqmSlotOff + 16;
-#ifndef FP4Q_DQM_EPI_WG
-#define FP4Q_DQM_EPI_WG 2
-#endif
-constexpr int kDqmEpiWg = FP4Q_DQM_EPI_WG;             // epilogue warpgroups: 2 or 4
+// Two epilogue warpgroups, both reading every slice (one half of its columns
+// each).  The slice barriers are waited on by phase parity, which is exact only
+// while every waiter takes every phase of a slot in turn: a warpgroup that
+// skipped the uses of a slot by other warpgroups (slots are reused by slices of
+// alternating parity) could see a phase two ahead as complete.
+constexpr int kDqmEpiWg = 2;
 constexpr int kDqmThreads = 96 + 128 * kDqmEpiWg;      // 3 role warps + the epilogue
-static_assert(kDqmEpiWg == 2 || kDqmEpiWg == 4, "two warpgroups per slice, one or two slice parities");
 constexpr uint32_t kDqmTmemCols = 512;
 constexpr uint32_t kDqmSfaCol = 384, kDqmSfbCol = 416;  // after the three 128-column slices
 static_assert(kDqmStageBytes % 1024 == 0, "stages keep the 1024-byte alignment of the swizzle");
@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(kDqmThreads, 1)
     } else {
         // ------------------------------------------------ epilogue
         constexpr int G = HAD >= 256 ? HAD / 128 : 1;  // groups per Hadamard block
-        const uint32_t wg = (warp - 3) >> 2, quarter = warp & 3, half = wg & 1, parity = wg >> 1;
+        const uint32_t wg = (warp - 3) >> 2, quarter = warp & 3, half = wg & 1;
         const uint32_t lane_base = (quarter * 32u) << 16;
         const float st_scale = FMT == FMT_NVFP4 ? *p.scale_fp32 : 0.0f;
 #pragma unroll 1
@@ -355,7 +355,6 @@ __global__ void __launch_bounds__(kDqmThreads, 1)
 #pragma unroll 1
             for (int q = 0; q < 4; ++q) {
                 const int64_t j = 4 * i + q;
-                if (kDqmEpiWg == 4 && (uint32_t)(j & 1) != parity) continue;
                 const int slot = (int)(j % kDqmSlots);
                 const bool a = mbar_wait(accf0 + 8 * slot, (uint32_t)((j / kDqmSlots) & 1));
                 if (!__all_sync(0xffffffffu, a)) {

@@ -65,13 +65,18 @@ struct QGeo {
     static constexpr int tc = FMT == FMT_DUAL ? 128 : 64;      // tile columns
     static constexpr int boxes = tc / 64;
     static constexpr int stage_bytes = boxes * kQBoxBytes;
-    static constexpr int stages = kQRingBytes / stage_bytes;    // 12 or 6
+    static constexpr int stages = kQRingBytes / stage_bytes;    // 24 or 12 (one CTA per SM)
     static constexpr int units = tc / 32;                       // units per lane per tile
     // consumer warpgroups: three where a lane holds 64 values at once (n = 64)
     // or reduces a dual-scale group, so that 128 registers per thread fit
     static constexpr int cwarps = ((HAD == 64 || FMT == FMT_DUAL) ? 12 : 16) / kQCtas;
     static_assert(cwarps % kQWarpsPerTile == 0, "consumer warps form whole tile groups");
     static constexpr int groups = cwarps / kQWarpsPerTile;
+    // Tile j lands in stage j % stages and goes to consumer group j % groups.
+    // The stages' full barriers are waited on by phase parity, which is exact
+    // only while one group takes every use of a stage: a group that skipped
+    // another group's use of its stage could see a phase two ahead as complete.
+    static_assert(stages % groups == 0, "each stage is consumed by one consumer group");
     static constexpr int threads = 32 * (kQProducers + cwarps);
     static constexpr int bar_off = kQRingBytes;
     static constexpr int red_off = bar_off + 2 * stages * 8;
