@@ -26,10 +26,11 @@ step).
 The JSON line adds: the roofline of the dominant kernel (algorithmic bytes per
 launch / its mean back-to-back duration in the timed steps, against the
 measured HBM copy bandwidth), every kernel's mean duration, an end-to-end
-figure through the public API with host buffers (pinned host -> device copy of
-one batch, the path, device -> host copy of its outputs, all inside the timed
-region), the SM clocks sampled during the timed region, and the CPU oracle
-timed on the host as a baseline (rank 0, N = 1).
+figure through the public API with host buffers (per step: pinned host ->
+device copy of one batch, the path, device -> host copy of its outputs, all
+inside the timed region; consecutive batches overlap on three streams), the SM
+clocks sampled during the timed region, and the CPU oracle timed on the host
+as a baseline (rank 0, N = 1).
 """
 from __future__ import annotations
 
