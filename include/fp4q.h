@@ -4,7 +4,8 @@
  * The library turns bf16 activations [M tokens x K channels] into 4-bit E2M1
  * codes plus block scales, in the two hardware micro-scaling formats and a
  * dual-scale variant, optionally after a block Hadamard rotation or the
- * ARCQuant reorder + RMSNorm + residual path, and back again.
+ * ARCQuant reorder + RMSNorm + residual path (which also writes 4-bit integer
+ * codes, FP4Q_INT4), and back again.
  *
  * Common conventions
  * ------------------
@@ -15,7 +16,8 @@
  *  - bf16 matrices are row-major with a row stride `ld*` given in ELEMENTS.
  *  - Packed codes are row-major uint8 [M, K/2]: two E2M1 codes per byte, the
  *    code of the even column in the LOW nibble.  E2M1 code c: bit 3 = sign,
- *    magnitude (c & 7) -> {0, 0.5, 1, 1.5, 2, 3, 4, 6}.
+ *    magnitude (c & 7) -> {0, 0.5, 1, 1.5, 2, 3, 4, 6}.  FP4Q_INT4 packs
+ *    4-bit two's complement integers the same way.
  *  - Scale matrices are uint8 [M, K/B] row-major (FP4Q_SCALES_LINEAR) or the
  *    128x4-tiled layout of block-scaled tensor-core GEMMs
  *    (FP4Q_SCALES_SWIZZLED, see fp4q_scales_bytes): rows padded to a multiple
