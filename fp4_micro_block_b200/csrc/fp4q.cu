@@ -130,6 +130,23 @@ fp4q_status make_plain_map(CUtensorMap* map, CUtensorMapDataType dt, const void*
     return r == CUDA_SUCCESS ? FP4Q_OK : FP4Q_ERR_CUDA;
 }
 
+// bf16 [rows, cols] output (row stride cols * 2 bytes, a multiple of 16) stored
+// by the TMA in boxes of 32 columns x 128 rows with the 64-byte swizzle; rows
+// past `rows` are not written.
+fp4q_status make_bf16_store_map(CUtensorMap* map, void* base, int64_t rows, int64_t cols) {
+    EncodeTiledFn enc;
+    fp4q_status st = encode_fn(&enc);
+    if (st != FP4Q_OK) return st;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(cols * 2)};
+    cuuint32_t box[2] = {32u, 128u};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FP4Q_OK : FP4Q_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------- validation
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -378,8 +395,9 @@ bool dqm_applies(int fmt, int had, const DequantParams& p) {
 
 template <int FMT, int HAD>
 fp4q_status launch_dqm_t(const DequantParams& d, int sms, cudaStream_t s) {
-    CUtensorMap codes_map, scales_map, g_map;
+    CUtensorMap codes_map, scales_map, g_map, y_map;
     fp4q_status st;
+    if ((st = make_bf16_store_map(&y_map, d.y, d.M, d.K)) != FP4Q_OK) return st;
     if ((st = make_codes_map(&codes_map, d.codes, d.M, d.K / 2, 128)) != FP4Q_OK ||
         (st = make_plain_map(&scales_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, d.scales, d.M, d.K / 16, d.K / 16, 32,
                              128)) != FP4Q_OK)
@@ -397,15 +415,13 @@ fp4q_status launch_dqm_t(const DequantParams& d, int sms, cudaStream_t s) {
     p.n_ct = d.K / 512;
     p.n_tiles = ((d.M + 127) / 128) * p.n_ct;
     p.scale_fp32 = d.scale_fp32;
-    p.y = d.y;
     p.had_norm = d.had_norm;
     for (int w = 0; w < 4; ++w) p.signs[w] = d.signs[w];
-    p.w32 = (reinterpret_cast<uintptr_t>(d.y) & 31) == 0 ? 1 : 0;
     auto kern = dequant_mma_kernel<FMT, HAD>;
     static std::atomic<uint64_t> done{0};
     if ((st = ensure_smem(kern, kDqmSmem, done)) != FP4Q_OK) return st;
     const int grid = (int)std::min<int64_t>({p.n_tiles, (int64_t)sms, (int64_t)kMaxGrid});
-    return launch(kern, grid, kDqmThreads, kDqmSmem, s, codes_map, scales_map, g_map, p);
+    return launch(kern, grid, kDqmThreads, kDqmSmem, s, codes_map, scales_map, g_map, y_map, p);
 }
 
 template <int FMT>

@@ -57,7 +57,12 @@ constexpr int kDqmOneOff = kDqmSfOff + 2 * kDqmSfBytes;  // 512 bytes of E4M3 1.
 constexpr int kDqmBarOff = kDqmOneOff + 512;
 constexpr int kDqmNumBars = 2 * kDqmStages + 2 * 2 + 2 * kDqmSlots + 1;
 constexpr int kDqmSlotOff = kDqmBarOff + kDqmNumBars * 8;
-constexpr int kDqmSmem = 1024 + kDqmSlotOff + 16;
+// bf16 output staging for the TMA stores: two buffers of one slice each, four
+// boxes (one per group) of 128 rows x 32 columns with the 64-byte swizzle
+constexpr int kDqmBoxBytes = 128 * 64;
+constexpr int kDqmStgBytes = 4 * kDqmBoxBytes;
+constexpr int kDqmStgOff = (kDqmSlotOff + 16 + 1023) / 1024 * 1024;
+constexpr int kDqmSmem = 1024 + kDqmStgOff + 2 * kDqmStgBytes;
 // Two epilogue warpgroups, both reading every slice (one half of its columns
 // each).  The slice barriers are waited on by phase parity, which is exact only
 // while every waiter takes every phase of a slot in turn: a warpgroup that
@@ -77,24 +82,9 @@ struct DqmParams {
     int64_t M, K;
     int64_t n_ct, n_tiles;  // 512-column tiles per row; tiles (column tile fastest)
     const float* scale_fp32;  // NVFP4: the tensor scale (the dual format's come by TMA)
-    uint16_t* y;
     float had_norm;
     uint32_t signs[4];
-    int w32;  // y is 32-byte aligned: one 256-bit store per 16 columns
 };
-
-// 16 bf16 (32 bytes, one sector) at dst: one 256-bit store when w32, else two 128-bit.
-__device__ __forceinline__ void store_bf16x16(uint16_t* dst, const uint32_t (&o)[8], bool w32) {
-    if (w32) {
-        asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst), "r"(o[0]), "r"(o[1]),
-                     "r"(o[2]), "r"(o[3]), "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7])
-                     : "memory");
-    } else {
-        uint4* d4 = reinterpret_cast<uint4*>(dst);
-        d4[0] = make_uint4(o[0], o[1], o[2], o[3]);
-        d4[1] = make_uint4(o[4], o[5], o[6], o[7]);
-    }
-}
 
 // B = D_s * blockdiag(H_n) (n <= 128) or D_s * H_128 (n >= 128) as E2M1 codes
 // (+1 = 0x2, -1 = 0xA, 0 off the diagonal blocks), in the K-major 128-byte
@@ -165,7 +155,8 @@ __device__ __forceinline__ void tmem_wait_ld16x4(uint32_t (&r)[4][16]) {
 template <int FMT, int HAD>
 __global__ void __launch_bounds__(kDqmThreads, 1)
     dequant_mma_kernel(const __grid_constant__ CUtensorMap codes_map, const __grid_constant__ CUtensorMap scales_map,
-                       const __grid_constant__ CUtensorMap g_map, const DqmParams p) {
+                       const __grid_constant__ CUtensorMap g_map, const __grid_constant__ CUtensorMap y_map,
+                       const DqmParams p) {
     static_assert(FMT == FMT_NVFP4 || FMT == FMT_DUAL, "16-element E4M3 block scales");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = align_shared<1024>(smem_raw);
@@ -180,6 +171,7 @@ __global__ void __launch_bounds__(kDqmThreads, 1)
         prefetch_tmap(&codes_map);
         prefetch_tmap(&scales_map);
         if constexpr (FMT == FMT_DUAL) prefetch_tmap(&g_map);
+        prefetch_tmap(&y_map);
         for (int s = 0; s < kDqmStages; ++s) {
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, 2 + 4 * kDqmEpiWg);  // the MMAs' commit, the repack warp, the epilogue warps
@@ -321,22 +313,32 @@ __global__ void __launch_bounds__(kDqmThreads, 1)
         }
     } else {
         // ------------------------------------------------ epilogue
+        // The eight epilogue warps vote at every wait on a named barrier (id 1),
+        // so that an exit is always a joint decision, and meet once per slice
+        // after writing it into a staging buffer; one thread then stores the
+        // slice's four boxes with the TMA (bulk group per slice, two buffers).
         constexpr int G = HAD >= 256 ? HAD / 128 : 1;  // groups per Hadamard block
+        constexpr int kEpiThreads = 128 * kDqmEpiWg;
         const uint32_t wg = (warp - 3) >> 2, quarter = warp & 3, half = wg & 1;
         const uint32_t lane_base = (quarter * 32u) << 16;
         const float st_scale = FMT == FMT_NVFP4 ? *p.scale_fp32 : 0.0f;
+        const bool issuer = warp == 3 && lane == 0;
+        // this thread's row of the tile and its two 16-byte chunks (columns
+        // 16 half .. + 15 of the box's 32) after the 64-byte swizzle
+        const uint32_t rt = quarter * 32u + lane, sw = (rt >> 1) & 3u;
+        const uint32_t off0 = rt * 64u + (((2u * half) ^ sw) << 4), off1 = rt * 64u + (((2u * half + 1u) ^ sw) << 4);
+        const uint32_t stg0 = smem_u32(smem + kDqmStgOff);
 #pragma unroll 1
         for (int64_t i = 0; i < n_my; ++i) {
             const int s = (int)(i % kDqmStages);
             const bool ok = mbar_wait(full0 + 8 * s, (uint32_t)((i / kDqmStages) & 1));
-            if (!__all_sync(0xffffffffu, ok)) {
+            if (!bar_and(1, kEpiThreads, ok)) {
                 if (lane == 0) atomicOr(&g_device_error, kErrWaitTimeout);
                 break;
             }
             const int64_t t = blockIdx.x + i * gridDim.x;
             const int64_t ct = t % p.n_ct;
-            const int64_t row = (t / p.n_ct) * 128 + quarter * 32 + lane;
-            const bool live = row < p.M;
+            const int32_t y0 = (int32_t)((t / p.n_ct) * 128);
             float gm[4];
             if constexpr (FMT == FMT_DUAL) {
                 const float4 g4 = *reinterpret_cast<const float4*>(smem + s * kDqmStageBytes + kDqmCodeBytes +
@@ -356,8 +358,12 @@ __global__ void __launch_bounds__(kDqmThreads, 1)
             for (int q = 0; q < 4; ++q) {
                 const int64_t j = 4 * i + q;
                 const int slot = (int)(j % kDqmSlots);
+                const uint32_t box0 = stg0 + (uint32_t)(j & 1) * kDqmStgBytes;
+                // the store issued from this buffer two slices ago has read it
+                // before the issuer joins the vote below
+                if (issuer) bulk_wait_read1();
                 const bool a = mbar_wait(accf0 + 8 * slot, (uint32_t)((j / kDqmSlots) & 1));
-                if (!__all_sync(0xffffffffu, a)) {
+                if (!bar_and(1, kEpiThreads, a)) {
                     aok = false;
                     break;
                 }
@@ -398,15 +404,24 @@ __global__ void __launch_bounds__(kDqmThreads, 1)
                                     v[g + st][e + 1] = df.y;
                                 }
                 }
-                if (live) {  // 16 columns = one whole 32-byte sector of the row per group
-                    uint16_t* dst0 = p.y + row * p.K + ct * 512 + 32 * q + 16 * half;
+                // bf16 into the staging boxes: 16 columns of the row per group
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        uint32_t o[8];
+                for (int g = 0; g < 4; ++g) {
+                    uint32_t o[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) o[e] = bf16x2_pack(v[g][2 * e], v[g][2 * e + 1]);
-                        store_bf16x16(dst0 + 128 * g, o, p.w32 != 0);
-                    }
+                    for (int e = 0; e < 8; ++e) o[e] = bf16x2_pack(v[g][2 * e], v[g][2 * e + 1]);
+                    const uint32_t bx = box0 + (uint32_t)g * kDqmBoxBytes;
+                    sts_v4(bx + off0, o[0], o[1], o[2], o[3]);
+                    sts_v4(bx + off1, o[4], o[5], o[6], o[7]);
+                }
+                fence_proxy_async_smem();  // visible to the TMA store
+                bar_sync(1, kEpiThreads);
+                if (issuer) {  // rows past M are not written (the map ends at row M)
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        tma_store_2d(&y_map, (int32_t)(ct * 512 + 128 * g + 32 * q), y0,
+                                     box0 + (uint32_t)g * kDqmBoxBytes);
+                    bulk_commit();
                 }
             }
             if (!aok) {
@@ -414,6 +429,7 @@ __global__ void __launch_bounds__(kDqmThreads, 1)
                 break;
             }
         }
+        if (issuer) bulk_wait0();  // every store has completed before the CTA exits
     }
 
     tc_fence_before();
