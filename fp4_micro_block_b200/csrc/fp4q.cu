@@ -270,7 +270,12 @@ fp4q_status launch_mma_t(const CUtensorMap& map, const MmaParams& p, int grid, c
         constexpr int smem = Wide<HAD>::smem;
         fp4q_status st = ensure_smem(kern, smem, done);
         if (st != FP4Q_OK) return st;
-        return launch(kern, grid, kWideThreads, smem, s, map, p);
+        // the codes are written by TMA stores of 128-row x 128-byte boxes (the
+        // amax pre-pass writes none: it gets the input's map as a placeholder)
+        CUtensorMap codes_map = map;
+        if constexpr (!AMAX)
+            if ((st = make_codes_map(&codes_map, p.codes, p.M, p.K / 2, 128)) != FP4Q_OK) return st;
+        return launch(kern, grid, kWideThreads, smem, s, map, codes_map, p);
     }
 }
 

@@ -19,15 +19,21 @@
 //   pass 1  reads z in steps of 8 columns of every group, applies H_G, takes
 //           the per-group maxima and writes y back into TMEM in place (the
 //           remaining RN(1/sqrt 2) of n = 512 is folded into the quantizer);
-//   (sync)  the epilogue warps meet (their pass-2 columns were written by
-//           other warpgroups), and the dual format's group maxima of the four
-//           warpgroups meet in shared memory;
+//   (sync)  the epilogue warps meet at a named barrier (their pass-2 columns
+//           were written by other warpgroups), and the dual format's group
+//           maxima of the four warpgroups meet in shared memory;
 //   pass 2  two warpgroups per output group, each quantizing two adjacent
-//           32-column chunks (64 consecutive columns, whole 32-byte sectors of
-//           a lane's row); for n = 512 in two rounds, groups 0-1 then 2-3.  A
-//           group's TMEM columns go back to the MMA warp as soon as its two
-//           warpgroups have read them, so the next tile's UMMAs overlap the
-//           rest of pass 2 (n = 512: groups 0 and 1 during the second round).
+//           32-column chunks (64 consecutive columns of a lane's row); for
+//           n = 512 in two rounds, groups 0-1 then 2-3.  A group's TMEM columns
+//           go back to the MMA warp as soon as its two warpgroups have read
+//           them, so the next tile's UMMAs overlap the rest of pass 2 (n = 512:
+//           groups 0 and 1 during the second round).  The codes of a round
+//           (128 rows x 128 bytes) are written into a shared-memory box with the
+//           128-byte swizzle and stored by one thread with the TMA; the scale
+//           bytes go out directly.
+// The sixteen epilogue warps vote on the accumulator wait of every tile
+// (bar.red.and), so an early exit is joint and no warp is left at the named
+// barriers that follow.
 #pragma once
 
 #include "fp4q_mma.cuh"
@@ -37,19 +43,23 @@ namespace fp4q {
 constexpr int kWideEpiWarps = 16;                    // four warpgroups
 constexpr int kWideThreads = 96 + 32 * kWideEpiWarps;  // 2 producer warps, the MMA warp, epilogue
 constexpr int kWideRedBytes = 2 * 4 * 4 * kMmaTile * 4;  // [parity][warpgroup][group][row] fp32
+constexpr int kWideBoxBytes = kMmaTile * 128;            // codes of 256 columns x 128 rows
 
 template <int HAD>
 struct Wide {
     static constexpr int G = HAD / kMmaTile;           // 128-column groups per block
     static constexpr int NBUF = 4 / G;                 // tiles in TMEM
-    static constexpr int bars = 2 * kMmaStages + NBUF + NBUF * G + 2 + 1;
+    static constexpr int bars = 2 * kMmaStages + NBUF + NBUF * G + 1;
     static constexpr int ring_off = kTileBytes;
     static constexpr int red_off = ring_off + kMmaStages * kTileBytes;
     static constexpr int bar_off = red_off + kWideRedBytes;
     static constexpr int slot_off = bar_off + bars * 8;
     static constexpr int tab_off = (slot_off + 4 + 15) / 16 * 16;
     static constexpr int misc_off = tab_off + 128 * 16;
-    static constexpr int smem = 1024 + misc_off + (kWideThreads / 32) * 4;
+    // codes staging for the TMA stores: one 128-row x 128-byte box per pass-2
+    // round (128-byte swizzle), two buffers
+    static constexpr int stg_off = (misc_off + (kWideThreads / 32) * 4 + 1023) / 1024 * 1024;
+    static constexpr int smem = 1024 + stg_off + 2 * kWideBoxBytes;
     static_assert(smem <= 227 * 1024, "shared memory");
 };
 
@@ -149,7 +159,8 @@ __device__ __forceinline__ void build_h128_b(uint8_t* b, const uint32_t (&signs)
 
 template <int FMT, int HAD, bool AMAX_ONLY>
 __global__ void __launch_bounds__(kWideThreads, 1)
-    had_mma_wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const MmaParams p) {
+    had_mma_wide_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap codes_map,
+                        const MmaParams p) {
     using W = Wide<HAD>;
     constexpr int G = W::G, NBUF = W::NBUF;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -157,8 +168,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     const uint32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t full0 = smem_u32(smem + W::bar_off), empty0 = full0 + 8 * kMmaStages;
     const uint32_t accf0 = empty0 + 8 * kMmaStages, relg0 = accf0 + 8 * NBUF;
-    const uint32_t redb0 = relg0 + 8 * NBUF * G;  // [2] all epilogue warps between the two passes
-    const uint32_t done_bar = redb0 + 16;
+    const uint32_t done_bar = relg0 + 8 * NBUF * G;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + W::slot_off);
     float4* tab = reinterpret_cast<float4*>(smem + W::tab_off);
     float* red = reinterpret_cast<float*>(smem + W::misc_off);
@@ -167,13 +177,13 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 
     if (tid == 0) {
         prefetch_tmap(&tmap_x);
+        if constexpr (!AMAX_ONLY) prefetch_tmap(&codes_map);
         for (int s = 0; s < kMmaStages; ++s) {
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, 1);
         }
         for (int b = 0; b < NBUF; ++b) mbar_init(accf0 + 8 * b, 1);
         for (int k = 0; k < NBUF * G; ++k) mbar_init(relg0 + 8 * k, 8);  // two warpgroups read a group
-        for (int k = 0; k < 2; ++k) mbar_init(redb0 + 8 * k, kWideEpiWarps);
         mbar_init(done_bar, 1);
         fence_barrier_init();
     }
@@ -269,12 +279,15 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         // n = 512: the remaining RN(1/sqrt 2) is applied per block by the quantizer
         const float fold = kOddLog ? __uint_as_float(0x3f3504f3u) : 1.0f;
         const ScaleCtx ctx_t = make_ctx(s_t);
-        const int64_t kc = p.K / 2;
+        const bool issuer = ew == 0 && lane == 0;
+        const uint32_t stg0 = smem_u32(smem + W::stg_off);
 #pragma unroll 1
         for (int64_t j = 0; j < n_my; ++j) {
             const int b = (int)(j % NBUF);
             const bool ok = mbar_wait(accf0 + 8 * b, (uint32_t)((j / NBUF) & 1));
-            if (!__all_sync(0xffffffffu, ok)) {
+            // a joint decision of the sixteen epilogue warps (named barrier 1),
+            // so that none is left at the barriers below
+            if (!bar_and(1, 32 * kWideEpiWarps, ok)) {
                 if (lane == 0) atomicOr(&g_device_error, kErrWaitTimeout);
                 break;
             }
@@ -356,13 +369,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                     for (int a = 0; a < G; ++a) rp[(wg * 4 + a) * kMmaTile + rowt] = m[a];
                 }
                 tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(redb0 + 8 * (uint32_t)(j & 1));
-                const bool rok = mbar_wait(redb0 + 8 * (uint32_t)(j & 1), (uint32_t)((j >> 1) & 1));
-                if (!__all_sync(0xffffffffu, rok)) {
-                    if (lane == 0) atomicOr(&g_device_error, kErrWaitTimeout);
-                    break;
-                }
+                // both codes staging buffers are free once the previous tile's
+                // stores have read them: the issuer waits before it joins
+                if (issuer) bulk_wait_read0();
+                bar_sync(1, 32 * kWideEpiWarps);
                 tc_fence_after();
                 if constexpr (FMT == FMT_DUAL) {  // group maxima over the four warpgroups
                     auto gscale = [&](int a) {
@@ -395,8 +405,6 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                 // TMEM columns go back to the MMA warp as soon as its two
                 // warpgroups have read them, so the next tile's UMMAs for groups
                 // 0 and 1 overlap the second round.
-                const int64_t row_even = row - (lane & 1u);
-                const bool live_even = row_even < p.M, live_odd = row_even + 1 < p.M;
 #pragma unroll 1
                 for (int h = 0; h < G / 2; ++h) {
                     const int a = G == 4 ? 2 * h + (int)(wg / 2) : (int)(wg % 2);
@@ -422,7 +430,14 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 16; ++i) n[i] = make_float2(v[2 * i], v[2 * i + 1]);
                     const uint32_t eb = quant_chunk<FMT>(n, ctx, tab, fold, wb);
-                    store_chunk_pair(p.codes + row * kc + col / 2, kc, live_even, live_odd, lane, wa, wb);
+                    // this row's 32 bytes of the round's box: 16-byte chunks
+                    // 4 (a - 2h) + c and + 1, at their 128-byte-swizzle places
+                    {
+                        const uint32_t k0 = 4u * (uint32_t)(a - 2 * h) + (uint32_t)c, rs = rowt & 7u;
+                        const uint32_t bx = stg0 + (uint32_t)h * kWideBoxBytes + rowt * 128u;
+                        sts_v4(bx + ((k0 ^ rs) << 4), wa[0], wa[1], wa[2], wa[3]);
+                        sts_v4(bx + (((k0 + 1u) ^ rs) << 4), wb[0], wb[1], wb[2], wb[3]);
+                    }
                     if (live) {
                         if constexpr (FMT == FMT_MXFP4) {  // two E8M0 bytes, 2-byte aligned
                             const int64_t nsc = p.K / 32, cb = col / 32;
@@ -436,9 +451,19 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                             *reinterpret_cast<uint32_t*>(sp) = ea | (eb << 16);
                         }
                     }
+                    // the round's box is written: one thread stores it (rows past
+                    // M are clipped by the map)
+                    fence_proxy_async_smem();
+                    bar_sync(1, 32 * kWideEpiWarps);
+                    if (issuer) {
+                        tma_store_2d(&codes_map, (int32_t)(ct * (HAD / 2) + 128 * h), (int32_t)(rt * kMmaTile),
+                                     stg0 + (uint32_t)h * kWideBoxBytes);
+                        bulk_commit();
+                    }
                 }
             }
         }
+        if (issuer) bulk_wait0();  // every store has completed before the CTA exits
     }
 
     if constexpr (AMAX_ONLY) {
