@@ -130,6 +130,25 @@ fp4q_status make_plain_map(CUtensorMap* map, CUtensorMapDataType dt, const void*
     return r == CUDA_SUCCESS ? FP4Q_OK : FP4Q_ERR_CUDA;
 }
 
+// Packed codes [rows, row_bytes] written by TMA stores of box_bytes x 128 rows
+// (64-byte boxes with the 64-byte swizzle, 128-byte boxes with the 128-byte
+// one); rows past `rows` are not written.
+fp4q_status make_codes_store_map(CUtensorMap* map, void* codes, int64_t rows, int64_t row_bytes,
+                                 uint32_t box_bytes) {
+    EncodeTiledFn enc;
+    fp4q_status st = encode_fn(&enc);
+    if (st != FP4Q_OK) return st;
+    cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {box_bytes, 128u};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, codes, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     box_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FP4Q_OK : FP4Q_ERR_CUDA;
+}
+
 // bf16 [rows, cols] output (row stride cols * 2 bytes, a multiple of 16) stored
 // by the TMA in boxes of 32 columns x 128 rows with the 64-byte swizzle; rows
 // past `rows` are not written.
@@ -264,7 +283,12 @@ fp4q_status launch_mma_t(const CUtensorMap& map, const MmaParams& p, int grid, c
         auto kern = had_mma_kernel<FMT, HAD, AMAX>;
         fp4q_status st = ensure_smem(kern, MmaGeo<FMT>::smem, done);
         if (st != FP4Q_OK) return st;
-        return launch(kern, grid, MmaGeo<FMT>::threads, MmaGeo<FMT>::smem, s, map, p);
+        // the codes go out by TMA stores of 128-row x 64-byte boxes (the amax
+        // pre-pass writes none: it gets the input's map as a placeholder)
+        CUtensorMap codes_map = map;
+        if constexpr (!AMAX)
+            if ((st = make_codes_store_map(&codes_map, p.codes, p.M, p.K / 2, 64)) != FP4Q_OK) return st;
+        return launch(kern, grid, MmaGeo<FMT>::threads, MmaGeo<FMT>::smem, s, map, codes_map, p);
     } else {
         auto kern = had_mma_wide_kernel<FMT, HAD, AMAX>;
         constexpr int smem = Wide<HAD>::smem;
@@ -274,7 +298,7 @@ fp4q_status launch_mma_t(const CUtensorMap& map, const MmaParams& p, int grid, c
         // amax pre-pass writes none: it gets the input's map as a placeholder)
         CUtensorMap codes_map = map;
         if constexpr (!AMAX)
-            if ((st = make_codes_map(&codes_map, p.codes, p.M, p.K / 2, 128)) != FP4Q_OK) return st;
+            if ((st = make_codes_store_map(&codes_map, p.codes, p.M, p.K / 2, 128)) != FP4Q_OK) return st;
         return launch(kern, grid, kWideThreads, smem, s, map, codes_map, p);
     }
 }

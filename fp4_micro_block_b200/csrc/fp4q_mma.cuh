@@ -149,7 +149,11 @@ struct MmaGeo {
     static constexpr int slot_off = kMmaBarOff + num_bars * 8;
     static constexpr int tab_off = (slot_off + 4 + 15) / 16 * 16;
     static constexpr int red_off = tab_off + 128 * 16;
-    static constexpr int smem = 1024 + red_off + (threads / 32) * 4;
+    // codes staging for the TMA stores: per epilogue warpgroup two boxes of
+    // 128 rows x 64 bytes (one tile's codes, 64-byte swizzle)
+    static constexpr int box_bytes = kMmaTile * 64;
+    static constexpr int stg_off = (red_off + (threads / 32) * 4 + 1023) / 1024 * 1024;
+    static constexpr int smem = 1024 + stg_off + groups * 2 * box_bytes;
     static_assert(groups * kMmaTile <= 512, "accumulators exceed TMEM");
     static_assert(smem <= 227 * 1024, "shared memory");
 };
@@ -250,7 +254,8 @@ __device__ __forceinline__ void store_chunk_pair(uint8_t* mine, int64_t stride, 
 
 template <int FMT, int HAD, bool AMAX_ONLY>
 __global__ void __launch_bounds__(MmaGeo<FMT>::threads, 1)
-    had_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, const MmaParams p) {
+    had_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap codes_map,
+                   const MmaParams p) {
     using Geo = MmaGeo<FMT>;
     constexpr int kGroups = Geo::groups;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -267,6 +272,7 @@ __global__ void __launch_bounds__(MmaGeo<FMT>::threads, 1)
 
     if (tid == 0) {
         prefetch_tmap(&tmap_x);
+        if constexpr (!AMAX_ONLY) prefetch_tmap(&codes_map);
         for (int s = 0; s < kMmaStages; ++s) {
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, 1);
@@ -369,11 +375,21 @@ __global__ void __launch_bounds__(MmaGeo<FMT>::threads, 1)
         ScaleCtx ctx = make_ctx(s_t);
         // odd log2 n: the remaining RN(1/sqrt 2) is applied per block by the quantizer
         const float fold = kOddLog ? __uint_as_float(0x3f3504f3u) : 1.0f;
-        const int64_t kc = p.K / 2;
+        // The warpgroup's four warps vote at every accumulator wait (named
+        // barrier 1 + g), so an exit is joint; each tile's codes go through one
+        // of the warpgroup's two staging boxes and a TMA store by its first thread.
+        const bool issuer = (ew & 3u) == 0 && lane == 0;
+        const uint32_t bar_id = 1u + g;
+        const uint32_t stg_g = smem_u32(smem + Geo::stg_off) + g * 2u * Geo::box_bytes;
+        const uint32_t rt_ = quarter * 32u + lane, sw = (rt_ >> 1) & 3u;  // row of the tile, its swizzle
 #pragma unroll 1
         for (int64_t j = g; j < n_my; j += kGroups) {
+            // the store issued from this box two tiles ago has read it
+            if constexpr (!AMAX_ONLY) {
+                if (issuer) bulk_wait_read1();
+            }
             const bool ok = mbar_wait(accf0 + 8 * g, (uint32_t)((j / kGroups) & 1));
-            if (!__all_sync(0xffffffffu, ok)) {
+            if (!bar_and((int)bar_id, 128, ok)) {
                 if (lane == 0) atomicOr(&g_device_error, kErrWaitTimeout);
                 break;
             }
@@ -426,9 +442,7 @@ __global__ void __launch_bounds__(MmaGeo<FMT>::threads, 1)
                     ctx = make_ctx(Gs);
                     if (live) p.scale_fp32[row * (p.K / 128) + ct] = Gs;
                 }
-                uint8_t* cp = p.codes + row * kc + ct * (kMmaTile / 2);
-                const int64_t row_even = row - (lane & 1u);
-                const bool live_even = row_even < p.M, live_odd = row_even + 1 < p.M;
+                const uint32_t box = stg_g + (uint32_t)((j / kGroups) & 1) * Geo::box_bytes + rt_ * 64u;
                 uint32_t sc0 = 0u, sc1 = 0u;  // scale bytes of blocks 0-3 / 4-7 (MXFP4: sc0)
 #pragma unroll 1
                 for (int c = 0; c < 4; c += 2) {
@@ -439,7 +453,9 @@ __global__ void __launch_bounds__(MmaGeo<FMT>::threads, 1)
                     load_chunk(c + 1, n);
                     if (c + 1 == 3) release();
                     const uint32_t eb = quant_chunk<FMT>(n, ctx, tab, fold, wb);
-                    store_chunk_pair(cp + 16 * c, kc, live_even, live_odd, lane, wa, wb);
+                    // 16-byte chunks c and c + 1 of the row's 64 bytes, swizzled
+                    sts_v4(box + (((uint32_t)c ^ sw) << 4), wa[0], wa[1], wa[2], wa[3]);
+                    sts_v4(box + (((uint32_t)(c + 1) ^ sw) << 4), wb[0], wb[1], wb[2], wb[3]);
                     if constexpr (FMT == FMT_MXFP4) {
                         sc0 |= (ea | (eb << 8)) << (8 * c);
                     } else {
@@ -466,7 +482,19 @@ __global__ void __launch_bounds__(MmaGeo<FMT>::threads, 1)
                         }
                     }
                 }
+                // the tile's codes are in the box: its first thread stores them
+                // (rows past M are clipped by the map)
+                fence_proxy_async_smem();
+                bar_sync((int)bar_id, 128);
+                if (issuer) {
+                    tma_store_2d(&codes_map, (int32_t)(ct * (kMmaTile / 2)), (int32_t)(rt * kMmaTile),
+                                 stg_g + (uint32_t)((j / kGroups) & 1) * Geo::box_bytes);
+                    bulk_commit();
+                }
             }
+        }
+        if constexpr (!AMAX_ONLY) {
+            if (issuer) bulk_wait0();  // every store has completed before the CTA exits
         }
     }
 
