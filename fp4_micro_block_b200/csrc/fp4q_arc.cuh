@@ -201,11 +201,10 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return __byte_perm(a, b, sel);
 }
 
-// Store one scale byte of (row, col).
-__device__ __forceinline__ void put_scale(const ArcParams& p, int64_t row, int64_t col, int64_t nsc,
-                                          int64_t nC, uint32_t byte) {
-    if (p.swizzled) p.scales[swizzle_offset(row, col, nC)] = (uint8_t)byte;
-    else p.scales[row * nsc + col] = (uint8_t)byte;
+// Offset of row `row`'s scales: linear, the row's start; tiled (128 x 4 tiles),
+// the part of the tile offset that depends on the row only.
+__device__ __forceinline__ int64_t scale_row_base(const ArcParams& p, int64_t row, int64_t nsc, int64_t nC) {
+    return p.swizzled ? (row >> 7) * nC * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 : row * nsc;
 }
 
 template <int FMT, bool AMAX_ONLY>
@@ -454,6 +453,11 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
             const int64_t r1 = r0 + 1;
             uint8_t* cp0 = p.codes + r0 * kcs;
             uint8_t* cp1 = p.codes + r1 * kcs;
+            // the two rows' scale bases (linear: the row; tiled: the row's part of
+            // the 128 x 4 tile offset) and the column part of a scale's offset
+            uint8_t* const sb0 = p.scales + scale_row_base(p, r0, nsc, nC);
+            uint8_t* const sb1 = p.scales + scale_row_base(p, r1, nsc, nC);
+            auto scol = [&](int64_t c) -> int64_t { return p.swizzled ? ((c >> 2) << 9) + (c & 3) : c; };
             const uint32_t tab_s = smem_u32(tab), l0_s = smem_u32(l0);
             // (-z row 0, -z row 1) of the B positions of block b
             auto gather = [&](int b, float2* v) {
@@ -475,10 +479,10 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
                     uint32_t w[4];
                     const uint32_t e2 = arc_nvfp4_unit<I4>(v, amax_pair_tree(v), ctx, stab, rs, w);
                     *reinterpret_cast<uint2*>(cp0 + 8 * b) = make_uint2(w[0], w[1]);
-                    put_scale(p, r0, b, nsc, nC, e2 & 0xffu);
+                    sb0[scol(b)] = (uint8_t)(e2 & 0xffu);
                     if (two) {
                         *reinterpret_cast<uint2*>(cp1 + 8 * b) = make_uint2(w[2], w[3]);
-                        put_scale(p, r1, b, nsc, nC, e2 >> 8);
+                        sb1[scol(b)] = (uint8_t)(e2 >> 8);
                     }
                     // 3. residuals of the outlier positions of the block
                     const uint32_t o = om[b];
@@ -516,10 +520,10 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
                     const uint32_t e0 = mxfp4_unit(u0, rs.x, w0);
                     const uint32_t e1 = mxfp4_unit(u1, rs.y, w1);
                     *reinterpret_cast<uint4*>(cp0 + 16 * b) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
-                    put_scale(p, r0, b, nsc, nC, e0);
+                    sb0[scol(b)] = (uint8_t)(e0);
                     if (two) {
                         *reinterpret_cast<uint4*>(cp1 + 16 * b) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-                        put_scale(p, r1, b, nsc, nC, e1);
+                        sb1[scol(b)] = (uint8_t)(e1);
                     }
                     const uint32_t oa = om[2 * b], ob = om[2 * b + 1];
                     if ((oa | ob) & 0xffffu) {
@@ -579,10 +583,10 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
                     uint32_t w[4];
                     const uint32_t e2 = arc_nvfp4_unit<I4>(n, amax_pair_tree(n), ctx, stab, make_float2(1.0f, 1.0f), w);
                     *reinterpret_cast<uint2*>(cp0 + p.K / 2 + 8 * j) = make_uint2(w[0], w[1]);
-                    put_scale(p, r0, col, nsc, nC, e2 & 0xffu);
+                    sb0[scol(col)] = (uint8_t)(e2 & 0xffu);
                     if (two) {
                         *reinterpret_cast<uint2*>(cp1 + p.K / 2 + 8 * j) = make_uint2(w[2], w[3]);
-                        put_scale(p, r1, col, nsc, nC, e2 >> 8);
+                        sb1[scol(col)] = (uint8_t)(e2 >> 8);
                     }
                 } else {
                     float2 u0[16], u1[16];
@@ -596,10 +600,10 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
                     const uint32_t e0 = mxfp4_unit(u0, 1.0f, w0);
                     const uint32_t e1 = mxfp4_unit(u1, 1.0f, w1);
                     *reinterpret_cast<uint4*>(cp0 + p.K / 2 + 16 * j) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
-                    put_scale(p, r0, col, nsc, nC, e0);
+                    sb0[scol(col)] = (uint8_t)(e0);
                     if (two) {
                         *reinterpret_cast<uint4*>(cp1 + p.K / 2 + 16 * j) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-                        put_scale(p, r1, col, nsc, nC, e1);
+                        sb1[scol(col)] = (uint8_t)(e1);
                     }
                 }
             }
