@@ -276,6 +276,7 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
 
     // ---- per-CTA tables
     float s_t = 0.0f;
+    int slots_in_order = 1;  // residual column i takes slot i (outlier list in position order)
     if constexpr (!AMAX_ONLY) {
         bool bad_index = false;
         // word of position q = B b + 4 k + t at index 4 (k nbB + b) + t; four
@@ -334,7 +335,9 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
         for (int i = tid; i < S; i += nthreads) {  // slot (position rank) of residual column i
             const unsigned q0 = (unsigned)p.outliers[i], q = q0 < (unsigned)K ? q0 : 0u;
             const uint32_t w = om[q >> 4];
-            rslot[i] = (uint16_t)((w >> 16) + __popc(w & ((1u << (q & 15)) - 1u)));
+            const uint32_t sl = (w >> 16) + __popc(w & ((1u << (q & 15)) - 1u));
+            rslot[i] = (uint16_t)sl;
+            slots_in_order &= (int)(sl == (uint32_t)i);
         }
         if (bad_index) atomicOr(&g_device_error, kErrBadIndex);
         if constexpr (FMT == FMT_NVFP4 || I4) {
@@ -351,7 +354,7 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
             }
         }
     }
-    __syncthreads();
+    const bool in_order = __syncthreads_and(slots_in_order) != 0;
 
     const ScaleCtx ctx = make_ctx(s_t);
     const int64_t KS = p.K + p.S, kcs = KS / 2, nsc = KS / B, nC = (nsc + 3) / 4;
@@ -484,28 +487,50 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
                         *reinterpret_cast<uint2*>(cp1 + 8 * b) = make_uint2(w[2], w[3]);
                         sb1[scol(b)] = (uint8_t)(e2 >> 8);
                     }
-                    // 3. residuals of the outlier positions of the block
+                    // 3. residuals of the outlier positions of the block:
+                    // y - (grid value * E4M3 value) * s_t, y = z * rs
                     const uint32_t o = om[b];
                     if (o & 0xffffu) {
                         const float es0 = e4m3_decode(e2 & 0xffu), es1 = e4m3_decode(e2 >> 8);
-#pragma unroll
-                        for (int k = 0; k < 16; k += 2) {
-                            const uint32_t m2 = (o >> k) & 3u;
-                            if (m2 == 0u) continue;
+                        auto resid = [&](float nz, float r, float c, float es) { return -nz * r - (c * es) * s_t; };
+                        auto pair_at = [&](int k, float2& c0, float2& c1) {  // grid values of k, k + 1 (rows 0, 1)
                             const uint32_t sh = 4 * (k & 7);
                             const uint32_t b0 = (w[k >> 3] >> sh) & 0xffu, b1 = (w[2 + (k >> 3)] >> sh) & 0xffu;
-                            const float2 c0 = I4 ? int4x2_decode(b0) : e2m1x2_decode(b0);  // row 0, k, k+1
-                            const float2 c1 = I4 ? int4x2_decode(b1) : e2m1x2_decode(b1);  // row 1
-                            const int base = (int)(o >> 16) + __popc(o & ((1u << k) - 1u));
-                            // residual y - (grid value * E4M3 value) * s_t, y = z * rs
-                            if (m2 & 1u) {
-                                res[base] = -v[k].x * rs.x - (c0.x * es0) * s_t;
-                                res[S + base] = -v[k].y * rs.y - (c1.x * es1) * s_t;
+                            c0 = I4 ? int4x2_decode(b0) : e2m1x2_decode(b0);
+                            c1 = I4 ? int4x2_decode(b1) : e2m1x2_decode(b1);
+                        };
+                        const int base = (int)(o >> 16);
+                        if ((o & 0xffffu) == 0xffffu && (base & 3) == 0) {
+                            // every position of the block is an outlier: slots base .. base + 15
+#pragma unroll
+                            for (int k = 0; k < 16; k += 4) {
+                                float2 c0, c1, d0, d1;
+                                pair_at(k, c0, c1);
+                                pair_at(k + 2, d0, d1);
+                                *reinterpret_cast<float4*>(res + base + k) =
+                                    make_float4(resid(v[k].x, rs.x, c0.x, es0), resid(v[k + 1].x, rs.x, c0.y, es0),
+                                                resid(v[k + 2].x, rs.x, d0.x, es0), resid(v[k + 3].x, rs.x, d0.y, es0));
+                                *reinterpret_cast<float4*>(res + S + base + k) =
+                                    make_float4(resid(v[k].y, rs.y, c1.x, es1), resid(v[k + 1].y, rs.y, c1.y, es1),
+                                                resid(v[k + 2].y, rs.y, d1.x, es1), resid(v[k + 3].y, rs.y, d1.y, es1));
                             }
-                            if (m2 & 2u) {
-                                const int s1 = base + (int)(m2 & 1u);
-                                res[s1] = -v[k + 1].x * rs.x - (c0.y * es0) * s_t;
-                                res[S + s1] = -v[k + 1].y * rs.y - (c1.y * es1) * s_t;
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < 16; k += 2) {
+                                const uint32_t m2 = (o >> k) & 3u;
+                                if (m2 == 0u) continue;
+                                float2 c0, c1;
+                                pair_at(k, c0, c1);
+                                const int s0 = base + __popc(o & ((1u << k) - 1u));
+                                if (m2 & 1u) {
+                                    res[s0] = resid(v[k].x, rs.x, c0.x, es0);
+                                    res[S + s0] = resid(v[k].y, rs.y, c1.x, es1);
+                                }
+                                if (m2 & 2u) {
+                                    const int s1 = s0 + (int)(m2 & 1u);
+                                    res[s1] = resid(v[k + 1].x, rs.x, c0.y, es0);
+                                    res[S + s1] = resid(v[k + 1].y, rs.y, c1.y, es1);
+                                }
                             }
                         }
                     }
@@ -529,26 +554,48 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
                     if ((oa | ob) & 0xffffu) {
                         const float es0 = e0 ? __uint_as_float(e0 << 23) : __uint_as_float(0x00400000u);
                         const float es1 = e1 ? __uint_as_float(e1 << 23) : __uint_as_float(0x00400000u);
+                        auto resid = [&](float nz, float r, float c, float es) { return -nz * r - c * es; };
+                        auto pair_at = [&](int kk, float2& c0, float2& c1) {  // grid values of kk, kk + 1
+                            const uint32_t sh = 4 * (kk & 7);
+                            c0 = e2m1x2_decode((w0[kk >> 3] >> sh) & 0xffu);
+                            c1 = e2m1x2_decode((w1[kk >> 3] >> sh) & 0xffu);
+                        };
+                        const int base = (int)(oa >> 16);
+                        if ((oa & ob & 0xffffu) == 0xffffu && (base & 3) == 0) {
+                            // every position of the block is an outlier: slots base .. base + 31
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const uint32_t o = h ? ob : oa;
+                            for (int k = 0; k < 32; k += 4) {
+                                float2 c0, c1, d0, d1;
+                                pair_at(k, c0, c1);
+                                pair_at(k + 2, d0, d1);
+                                *reinterpret_cast<float4*>(res + base + k) =
+                                    make_float4(resid(v[k].x, rs.x, c0.x, es0), resid(v[k + 1].x, rs.x, c0.y, es0),
+                                                resid(v[k + 2].x, rs.x, d0.x, es0), resid(v[k + 3].x, rs.x, d0.y, es0));
+                                *reinterpret_cast<float4*>(res + S + base + k) =
+                                    make_float4(resid(v[k].y, rs.y, c1.x, es1), resid(v[k + 1].y, rs.y, c1.y, es1),
+                                                resid(v[k + 2].y, rs.y, d1.x, es1), resid(v[k + 3].y, rs.y, d1.y, es1));
+                            }
+                        } else {
 #pragma unroll
-                            for (int k = 0; k < 16; k += 2) {
-                                const uint32_t m2 = (o >> k) & 3u;
-                                if (m2 == 0u) continue;
-                                const int kk = 16 * h + k;  // position within the block
-                                const uint32_t sh = 4 * (kk & 7);
-                                const float2 c0 = e2m1x2_decode((w0[kk >> 3] >> sh) & 0xffu);
-                                const float2 c1 = e2m1x2_decode((w1[kk >> 3] >> sh) & 0xffu);
-                                const int base = (int)(o >> 16) + __popc(o & ((1u << k) - 1u));
-                                if (m2 & 1u) {
-                                    res[base] = -v[kk].x * rs.x - c0.x * es0;
-                                    res[S + base] = -v[kk].y * rs.y - c1.x * es1;
-                                }
-                                if (m2 & 2u) {
-                                    const int s1 = base + (int)(m2 & 1u);
-                                    res[s1] = -v[kk + 1].x * rs.x - c0.y * es0;
-                                    res[S + s1] = -v[kk + 1].y * rs.y - c1.y * es1;
+                            for (int h = 0; h < 2; ++h) {
+                                const uint32_t o = h ? ob : oa;
+#pragma unroll
+                                for (int k = 0; k < 16; k += 2) {
+                                    const uint32_t m2 = (o >> k) & 3u;
+                                    if (m2 == 0u) continue;
+                                    const int kk = 16 * h + k;  // position within the block
+                                    float2 c0, c1;
+                                    pair_at(kk, c0, c1);
+                                    const int s0 = (int)(o >> 16) + __popc(o & ((1u << k) - 1u));
+                                    if (m2 & 1u) {
+                                        res[s0] = resid(v[kk].x, rs.x, c0.x, es0);
+                                        res[S + s0] = resid(v[kk].y, rs.y, c1.x, es1);
+                                    }
+                                    if (m2 & 2u) {
+                                        const int s1 = s0 + (int)(m2 & 1u);
+                                        res[s1] = resid(v[kk + 1].x, rs.x, c0.y, es0);
+                                        res[S + s1] = resid(v[kk + 1].y, rs.y, c1.y, es1);
+                                    }
                                 }
                             }
                         }
@@ -575,10 +622,22 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
                 const int64_t col = nbB + j;
                 if constexpr (FMT == FMT_NVFP4 || I4) {
                     float2 n[16];
+                    if (in_order) {  // slots 16 j .. 16 j + 15
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const int sl = rslot[16 * j + k];
-                        n[k] = make_float2(-res[sl], -res[S + sl]);
+                        for (int k = 0; k < 16; k += 4) {
+                            const float4 a = *reinterpret_cast<const float4*>(res + 16 * j + k);
+                            const float4 c = *reinterpret_cast<const float4*>(res + S + 16 * j + k);
+                            n[k] = make_float2(-a.x, -c.x);
+                            n[k + 1] = make_float2(-a.y, -c.y);
+                            n[k + 2] = make_float2(-a.z, -c.z);
+                            n[k + 3] = make_float2(-a.w, -c.w);
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            const int sl = rslot[16 * j + k];
+                            n[k] = make_float2(-res[sl], -res[S + sl]);
+                        }
                     }
                     uint32_t w[4];
                     const uint32_t e2 = arc_nvfp4_unit<I4>(n, amax_pair_tree(n), ctx, stab, make_float2(1.0f, 1.0f), w);
@@ -590,11 +649,29 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
                     }
                 } else {
                     float2 u0[16], u1[16];
+                    if (in_order) {  // slots 32 j .. 32 j + 31
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const int sa = rslot[32 * j + k], sb = rslot[32 * j + 16 + k];
-                        u0[k] = make_float2(-res[sa], -res[sb]);
-                        u1[k] = make_float2(-res[S + sa], -res[S + sb]);
+                        for (int k = 0; k < 16; k += 4) {
+                            const float4 a = *reinterpret_cast<const float4*>(res + 32 * j + k);
+                            const float4 b = *reinterpret_cast<const float4*>(res + 32 * j + 16 + k);
+                            const float4 c = *reinterpret_cast<const float4*>(res + S + 32 * j + k);
+                            const float4 d = *reinterpret_cast<const float4*>(res + S + 32 * j + 16 + k);
+                            u0[k] = make_float2(-a.x, -b.x);
+                            u0[k + 1] = make_float2(-a.y, -b.y);
+                            u0[k + 2] = make_float2(-a.z, -b.z);
+                            u0[k + 3] = make_float2(-a.w, -b.w);
+                            u1[k] = make_float2(-c.x, -d.x);
+                            u1[k + 1] = make_float2(-c.y, -d.y);
+                            u1[k + 2] = make_float2(-c.z, -d.z);
+                            u1[k + 3] = make_float2(-c.w, -d.w);
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            const int sa = rslot[32 * j + k], sb = rslot[32 * j + 16 + k];
+                            u0[k] = make_float2(-res[sa], -res[sb]);
+                            u1[k] = make_float2(-res[S + sa], -res[S + sb]);
+                        }
                     }
                     uint32_t w0[4], w1[4];
                     const uint32_t e0 = mxfp4_unit(u0, 1.0f, w0);
