@@ -127,6 +127,33 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return _
 // RN(RN(amax(v) * RN(1/6)) * RN(1/s)) and quotients z * RN(RN(1/d) * fold), as
 // in nvfp4_unit's table path.  stab[e] = (d, RN(1/d)) for the tensor scale s.
 // INT4: the same with RN(1/7) and the integer grid.
+// INT4 codes of the quotients q = n[i] * m of 16 pairs (x: row 0 -> w[0..1],
+// y: row 1 -> w[2..3]), optionally clamped to [-7, 7] first: each q is rounded
+// to the nearest integer, ties to even, by one IEEE addition of 1.5 * 2^23
+// (whose ulp is 1), and the low nibble of the sum's significand is the two's
+// complement code.
+template <bool CLAMP>
+__device__ __forceinline__ void int4_pack_pairs(const float2* n, float2 m, uint32_t (&w)[4]) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t a = 0, b = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float2 q = fmul2(n[8 * h + i], m);
+            if constexpr (CLAMP) {
+                q.x = fminf(fmaxf(q.x, -7.0f), 7.0f);
+                q.y = fminf(fmaxf(q.y, -7.0f), 7.0f);
+            }
+            const uint32_t ka = __float_as_uint(__fadd_rn(q.x, 12582912.0f));
+            const uint32_t kb = __float_as_uint(__fadd_rn(q.y, 12582912.0f));
+            asm("bfi.b32 %0, %1, %2, %3, 4;" : "=r"(a) : "r"(ka), "r"(a), "r"(4 * i));
+            asm("bfi.b32 %0, %1, %2, %3, 4;" : "=r"(b) : "r"(kb), "r"(b), "r"(4 * i));
+        }
+        w[h] = a;
+        w[2 + h] = b;
+    }
+}
+
 template <bool INT4>
 __device__ __forceinline__ uint32_t arc_nvfp4_unit(const float2* n, float2 am, const ScaleCtx& c,
                                                    const float2* stab, float2 fold, uint32_t (&w)[4]) {
@@ -145,19 +172,21 @@ __device__ __forceinline__ uint32_t arc_nvfp4_unit(const float2* n, float2 am, c
     const uint32_t e2 = e4m3x2_encode(make_float2((am.x * k) * c.rs.rn, (am.y * k) * c.rs.rn));
     const float2 t0 = stab[e2 & 0xffu], t1 = stab[e2 >> 8];
     const float2 m = make_float2(-(t0.y * fold.x), -(t1.y * fold.y));  // n holds -z
-    float q0[16], q1[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float2 q = fmul2(n[i], m);
-        q0[i] = q.x;
-        q1[i] = q.y;
-    }
     if constexpr (INT4) {
-        w[0] = int4_pack8(q0);
-        w[1] = int4_pack8(q0 + 8);
-        w[2] = int4_pack8(q1);
-        w[3] = int4_pack8(q1 + 8);
+        // A scale byte in the normal range below 448 (8 .. 0x7d: no saturation,
+        // relative rounding error at most 2^-4) bounds every |q| by about
+        // 7 / (1 - 2^-4) < 7.47, which rounds into -7..7 by itself; other
+        // blocks are clamped to [-7, 7] first.
+        if ((e2 & 0xffu) - 8u < 0x76u && (e2 >> 8) - 8u < 0x76u) int4_pack_pairs<false>(n, m, w);
+        else int4_pack_pairs<true>(n, m, w);
     } else {
+        float q0[16], q1[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float2 q = fmul2(n[i], m);
+            q0[i] = q.x;
+            q1[i] = q.y;
+        }
         w[0] = e2m1_pack8(q0);
         w[1] = e2m1_pack8(q0 + 8);
         w[2] = e2m1_pack8(q1);
