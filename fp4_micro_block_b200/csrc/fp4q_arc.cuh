@@ -645,9 +645,14 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
             // orders them before its residuals are written).
             pair_sync();
             if (sub == 0 && lane == 0 && i + SR < n_my) issue(i + SR);
-            // residual blocks: slots of columns B j .. B j + B - 1 -> columns K + B j,
-            // alternate blocks to the two warps
-            for (int j = sub + WPP * lane; B * j < S; j += 32 * WPP) {
+            // residual blocks: slots of columns B j .. B j + B - 1 -> columns K + B j.
+            // Up to 32 blocks all go to the pair's last warp (one pass either way;
+            // its partner carried the outlier residuals of the primary blocks),
+            // more alternate between the warps.
+            const int nrb = S / B;
+            const bool last_only = nrb <= 32;
+            const int j0 = last_only ? (sub == WPP - 1 ? lane : nrb) : sub + WPP * lane;
+            for (int j = j0; j < nrb; j += last_only ? 32 : 32 * WPP) {
                 const int64_t col = nbB + j;
                 if constexpr (FMT == FMT_NVFP4 || I4) {
                     float2 n[16];
