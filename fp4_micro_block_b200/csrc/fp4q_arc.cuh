@@ -400,6 +400,13 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
             }
             break;
         }
+        // the slot's next pair into L2 now, so that its copy (issued once this
+        // pair's buffer is consumed) does not wait on DRAM
+        if (sub == 0 && lane == 0 && i + SR < n_my) {
+            const int64_t rn = 2 * (gw + (i + SR) * nw);
+            bulk_prefetch_l2(p.x + rn * p.ldx_bytes, row_bytes);
+            if (rn + 1 < p.M) bulk_prefetch_l2(p.x + (rn + 1) * p.ldx_bytes, row_bytes);
+        }
         const int64_t r0 = 2 * (gw + i * nw);
         const bool two = r0 + 1 < p.M;
         uint8_t* const l0 = land + (i % SR) * 2 * row_bytes;
