@@ -220,6 +220,7 @@ KERNEL_SOURCES = {
     ("dual", "dequantize"): _COMMON + ["fp4q_mma.cuh", "fp4q_gemm.cuh", "fp4q_dqmma.cuh"],
     ("mxfp4", "quantize"): _COMMON,
     ("mxfp4", "dequantize"): _COMMON + ["fp4q_dequant.cuh"],
+    ("hadamard128", "quantize"): _COMMON + ["fp4q_mma.cuh"],
     ("arc", "arc"): _COMMON + ["fp4q_arc.cuh"],
     ("arc_mxfp4", "arc"): _COMMON + ["fp4q_arc.cuh"],
     ("arc_int4", "arc"): _COMMON + ["fp4q_arc.cuh"],

@@ -230,6 +230,12 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return __byte_perm(a, b, sel);
 }
 
+// Hint: bring a 16-byte aligned range (size a multiple of 16) of global memory
+// into L2; no completion to wait for.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Offset of row `row`'s scales: linear, the row's start; tiled (128 x 4 tiles),
 // the part of the tile offset that depends on the row only.
 __device__ __forceinline__ int64_t scale_row_base(const ArcParams& p, int64_t row, int64_t nsc, int64_t nC) {
