@@ -144,8 +144,8 @@ __device__ __forceinline__ void int4_pack_pairs(const float2* n, float2 m, uint3
                 q.x = fminf(fmaxf(q.x, -7.0f), 7.0f);
                 q.y = fminf(fmaxf(q.y, -7.0f), 7.0f);
             }
-            const uint32_t ka = __float_as_uint(__fadd_rn(q.x, 12582912.0f));
-            const uint32_t kb = __float_as_uint(__fadd_rn(q.y, 12582912.0f));
+            const float2 k = __fadd2_rn(q, make_float2(12582912.0f, 12582912.0f));  // both rows at once
+            const uint32_t ka = __float_as_uint(k.x), kb = __float_as_uint(k.y);
             asm("bfi.b32 %0, %1, %2, %3, 4;" : "=r"(a) : "r"(ka), "r"(a), "r"(4 * i));
             asm("bfi.b32 %0, %1, %2, %3, 4;" : "=r"(b) : "r"(kb), "r"(b), "r"(4 * i));
         }
