@@ -34,7 +34,7 @@
 // The two warps wait for each pair's copies; the other pairs of the SM (up to
 // 11, one buffer each) hide that latency.
 // Per CTA (built once): for every position q a 32-bit word (byte offset of the
-// word of channel perm[q] | bf16 gamma of that channel << 16), laid out so that
+// word of channel perm[q] << 16 | bf16 gamma of that channel), laid out so that
 // the 16-byte loads of 32 lanes (blocks b = lane + 32 i) are consecutive; per
 // 16-position group the outlier bit mask and the number of outlier positions
 // before the group; the slot of every residual column; the NVFP4 scale table
@@ -157,8 +157,7 @@ __device__ __forceinline__ void int4_pack_pairs(const float2* n, float2 m, uint3
 template <bool INT4>
 __device__ __forceinline__ uint32_t arc_nvfp4_unit(const float2* n, float2 am, const ScaleCtx& c,
                                                    const float2* stab, float2 fold, uint32_t (&w)[4]) {
-    am.x *= fold.x;
-    am.y *= fold.y;
+    am = fmul2(am, fold);
     const uint32_t b0 = __float_as_uint(am.x), b1 = __float_as_uint(am.y);
     const uint32_t tiny = __float_as_uint(0x1p-90f);
     const bool in_range = c.fast && (b0 - 1u) >= tiny - 1u && (b1 - 1u) >= tiny - 1u &&
@@ -169,9 +168,9 @@ __device__ __forceinline__ uint32_t arc_nvfp4_unit(const float2* n, float2 am, c
         return e0 | (e1 << 8);
     }
     const float k = __uint_as_float(INT4 ? 0x3e124925u : 0x3e2aaaabu);  // RN(1/7), RN(1/6)
-    const uint32_t e2 = e4m3x2_encode(make_float2((am.x * k) * c.rs.rn, (am.y * k) * c.rs.rn));
+    const uint32_t e2 = e4m3x2_encode(fmul2(fmul2(am, make_float2(k, k)), make_float2(c.rs.rn, c.rs.rn)));
     const float2 t0 = stab[e2 & 0xffu], t1 = stab[e2 >> 8];
-    const float2 m = make_float2(-(t0.y * fold.x), -(t1.y * fold.y));  // n holds -z
+    const float2 m = fmul2(make_float2(-t0.y, -t1.y), fold);  // n holds -z
     if constexpr (INT4) {
         // A scale byte in the normal range below 448 (8 .. 0x7d: no saturation,
         // relative rounding error at most 2^-4) bounds every |q| by about
@@ -335,7 +334,7 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
                 const int q = q0 + u * nthreads;
                 if (q >= K) continue;
                 const int b = q / B, k = (q % B) >> 2, t = q & 3;
-                tab[4 * (k * nbB + b) + t] = arc_word_off((uint32_t)c[u], (uint32_t)K) | (g[u] << 16);
+                tab[4 * (k * nbB + b) + t] = (arc_word_off((uint32_t)c[u], (uint32_t)K) << 16) | g[u];
             }
         }
         for (int g = tid; g < ng; g += nthreads) om[g] = 0u;
@@ -512,8 +511,8 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
                     const uint32_t wv[4] = {tw.x, tw.y, tw.z, tw.w};
 #pragma unroll
                     for (int t = 0; t < 4; ++t) {
-                        const uint32_t xw = lds_u32(l0_s + (wv[t] & 0xffffu));
-                        const float ng_ = -__uint_as_float(wv[t] & 0xffff0000u);
+                        const uint32_t xw = lds_u32(l0_s + (wv[t] >> 16));
+                        const float ng_ = -__uint_as_float(wv[t] << 16);
                         v[4 * k + t] = fmul2(make_float2(bf16lo(xw), bf16hi(xw)), dup2(ng_));
                     }
                 }
