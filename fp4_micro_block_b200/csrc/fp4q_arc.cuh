@@ -5,13 +5,14 @@
 // ("Generalisabilite": the scheme carries over to MXFP4 and INT4; INT4 is the
 // NVFP4 container with the integers -7..7 as the grid).
 //
-// Two warps own a PAIR of rows at a time (the amax pre-pass: one warp): there
-// is no CTA-wide barrier on the path, only a 64-thread named barrier between
-// the two warps of a pair.  They stream their row pairs through a shared 4K-byte
-// buffer, filled by two 1-D bulk copies (row 0 in the first half, row 1 in the
-// second), and split every step of a pair between them (alternate 16-byte
-// chunks in step 1, alternate 32-block groups in steps 2 and 3), which halves
-// the registers a warp holds and doubles the warps an SM runs.  Per pair:
+// The warps of a pair slot own a PAIR of rows at a time (two warps for NVFP4
+// and INT4, one for MXFP4 and for the amax pre-pass): there is no CTA-wide
+// barrier on the path, only a named barrier between the warps of a pair.  They
+// stream their row pairs through a shared buffer of 4K bytes (K channels),
+// filled by two 1-D bulk copies (row 0 in the first half, row 1 in the second),
+// and split steps 1 and 2 of a pair between them (alternate 16-byte chunks,
+// alternate 32-block groups), which halves the registers a warp holds and
+// doubles the warps an SM runs.  Per pair:
 //   1. natural order (conflict-free 16-byte reads of both rows): the sum of
 //      squares of each row, and one 32-bit word per channel holding the bf16 of
 //      row 0 (low half) and of row 1 (high half), written IN PLACE: lane l
@@ -19,20 +20,27 @@
 //      and writes their 8 words back to the same 32 bytes, channels 8j..8j+3
 //      into the first half and 8j+4..8j+7 into the second, so the word of
 //      channel c sits at 16 (c >> 3) + 4 (c & 3) + ((c >> 2) & 1) * 2K;
-//   2. reordered order: lane l owns the output blocks b = l, l + 32, ... (two
-//      at a time); one shared-memory load per position gathers that position's
-//      channel for both rows, a packed multiply applies -gamma of the channel,
-//      and the two rows' blocks are quantized side by side (NVFP4: one unit of
-//      two 16-blocks; MXFP4: one 32-block unit per row).  The RMS factor rs of
-//      each row is not applied per element: it scales the block maximum and
-//      the quotient multiplier of its row (the "fold" of the unit quantizers),
-//      so y = z * rs with z = x * gamma;
-//   3. at the outlier positions (a bit mask per 16-block) the residual
-//      y - dequant(primary) goes to a per-warp buffer in position order; after
-//      a warp barrier the lanes quantize the residual blocks (residual column j
-//      reads the slot of outlier j); then the buffer takes the next pair.
-// The two warps wait for each pair's copies; the other pairs of the SM (up to
-// 11, one buffer each) hide that latency.
+//   2. reordered order: lane l of warp w owns the output blocks
+//      b = l + 32 w, l + 32 w + 64, ..., one per step; one shared-memory load
+//      per position gathers that position's channel for both rows, a packed
+//      multiply applies -gamma of the channel, and the two rows' blocks are
+//      quantized side by side (NVFP4 and INT4: one unit of two 16-blocks;
+//      MXFP4: one 32-block unit per row).  The RMS factor rs of each row is not
+//      applied per element: it scales the block maximum and the quotient
+//      multiplier of its row (the "fold" of the unit quantizers), so
+//      y = z * rs with z = x * gamma;
+//   3. at the outlier positions (a bit mask per 16-position group) the
+//      residual y - dequant(primary) goes to the pair's slot buffer in position
+//      order (a block whose positions are all outliers, as the reorder makes
+//      them, in straight-line code); after the pair barrier the buffer takes
+//      the next pair, and the residual blocks are quantized (residual column j
+//      reads the slot of outlier j; contiguously when the outlier list is in
+//      position order): up to 32 blocks all by the pair's last warp in one
+//      pass, more alternating between the warps.
+// Each warp waits for its pair's copies; the other pairs of the SM (10 for
+// NVFP4 and INT4, 12 for MXFP4, one buffer each) hide that latency, and each
+// slot's next pair is prefetched into L2 when the current one lands, so the
+// copy issued after step 2 reads L2.
 // Per CTA (built once): for every position q a 32-bit word (byte offset of the
 // word of channel perm[q] << 16 | bf16 gamma of that channel), laid out so that
 // the 16-byte loads of 32 lanes (blocks b = lane + 32 i) are consecutive; per
@@ -122,11 +130,6 @@ __host__ __device__ inline uint32_t arc_word_off(uint32_t c, uint32_t K) {
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
-// NVFP4 rule for the two blocks of a unit (component x: row 0, y: row 1) with a
-// fold per component: the unit holds -z and v = z * fold.  Scale bytes from
-// RN(RN(amax(v) * RN(1/6)) * RN(1/s)) and quotients z * RN(RN(1/d) * fold), as
-// in nvfp4_unit's table path.  stab[e] = (d, RN(1/d)) for the tensor scale s.
-// INT4: the same with RN(1/7) and the integer grid.
 // INT4 codes of the quotients q = n[i] * m of 16 pairs (x: row 0 -> w[0..1],
 // y: row 1 -> w[2..3]), optionally clamped to [-7, 7] first: each q is rounded
 // to the nearest integer, ties to even, by one IEEE addition of 1.5 * 2^23
@@ -154,6 +157,11 @@ __device__ __forceinline__ void int4_pack_pairs(const float2* n, float2 m, uint3
     }
 }
 
+// NVFP4 rule for the two blocks of a unit (component x: row 0, y: row 1) with a
+// fold per component: the unit holds -z and v = z * fold.  Scale bytes from
+// RN(RN(amax(v) * RN(1/6)) * RN(1/s)) and quotients z * RN(RN(1/d) * fold), as
+// in nvfp4_unit's table path.  stab[e] = (d, RN(1/d)) for the tensor scale s.
+// INT4: the same with RN(1/7) and the integer grid.
 template <bool INT4>
 __device__ __forceinline__ uint32_t arc_nvfp4_unit(const float2* n, float2 am, const ScaleCtx& c,
                                                    const float2* stab, float2 fold, uint32_t (&w)[4]) {
@@ -248,7 +256,7 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
     constexpr bool I4 = FMT == FMT_INT4;
     constexpr int B = FMT == FMT_MXFP4 ? 32 : 16;  // block size
     constexpr int Q = B / 4;                       // 16-byte table quads per block
-    constexpr int SR = AMAX_ONLY ? 2 : 1;          // landing stages per warp
+    constexpr int SR = AMAX_ONLY ? 2 : 1;          // landing stages per pair slot
     pdl_wait();
     pdl_trigger();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
