@@ -464,7 +464,7 @@ __global__ void __launch_bounds__(arc_max_warps<FMT, AMAX_ONLY>() * 32, 1) arc_k
             if (two) my_amax = fmaxf(my_amax, zmax.y * rs.y);
         } else {
             // 1. natural order, in place: sums of squares and the interleaved words
-#pragma unroll 2
+#pragma unroll 4
             for (int j = lane + 32 * sub; 8 * j < K; j += 32 * WPP) {
                 const uint4 a = *reinterpret_cast<const uint4*>(l0 + 16 * j);
                 const uint4 b = two ? *reinterpret_cast<const uint4*>(l1 + 16 * j) : make_uint4(0u, 0u, 0u, 0u);
