@@ -546,6 +546,58 @@ def test_arc_int4_static_and_general_outlier_list(fq):
     check_fractions(c, 2e-4, "arc-int4-static")
 
 
+def _mixed_outlier_lists(K, B):
+    """Outlier lists (S a multiple of the block B) that mix the fused kernel's
+    whole-block and general residual paths:
+      * the first 2B positions listed in reverse: whole outlier blocks, with
+        the residual columns not in position order;
+      * two positions of block 0, then all of block 1: a whole block whose
+        residual slots start at 2 (not a multiple of 4);
+      * four positions of block 0, then all of block 1: a whole block whose
+        slots start at 4;
+    the last two padded with scattered positions to a multiple of B."""
+    rng = np.random.default_rng(K + B)
+    lists = [np.arange(2 * B)[::-1].copy()]
+    for head in ([1, 2], [0, 1, 2, 3]):
+        base = list(head) + list(range(B, 2 * B))
+        rest = rng.choice(np.arange(4 * B, K), (-len(base)) % B + B, replace=False)
+        lists.append(np.array(base + sorted(rest.tolist())))
+    return [o.astype(np.int32) for o in lists]
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4", "int4"])
+@pytest.mark.parametrize("case", [0, 1, 2])
+def test_arc_mixed_outlier_paths(fq, fmt, case):
+    """Whole-block and general residual paths in one call, against the oracle."""
+    M, K = 37, 1024
+    B = 32 if fmt == "mxfp4" else 16
+    outl = _mixed_outlier_lists(K, B)[case]
+    S = len(outl)
+    assert S % B == 0 and len(set(outl.tolist())) == S
+    x_bits, gamma, perm, _ = workloads.arc_activations(M, K, seed=11 + case, S=S)
+    name = f"arc-{fmt}-mixed-{case}"
+    if fmt == "mxfp4":
+        codes, scales, _ = fq.arc_quantize(
+            bits_to_torch_cuda(x_bits), bits_to_torch_cuda(gamma), torch.from_numpy(perm).cuda(),
+            torch.from_numpy(outl).cuda(), 1e-6, fmt=fq.FP4Q_MXFP4)
+        torch.cuda.synchronize()
+        c = _arc_mx_check(to_np(codes), to_np(scales), x_bits, gamma, perm, outl, name)
+    elif fmt == "int4":
+        codes, scales, sf = _arc_int4(fq, x_bits, gamma, perm, outl, ts=0.004)
+        c_o, s_o, sc_o, y_o = oracle.arc(x_bits, gamma, perm, outl, s_t=np.float32(0.004), fmt="int4")
+        c = arc_counts("int4", K, outl, (to_np(codes), to_np(scales), to_np(sf)),
+                       (c_o[:, :K // 2], s_o[:, :K // 16], sc_o), y_o, name=name)
+    else:
+        codes, scales, sf = fq.arc_quantize(
+            bits_to_torch_cuda(x_bits), bits_to_torch_cuda(gamma), torch.from_numpy(perm).cuda(),
+            torch.from_numpy(outl).cuda(), 1e-6, torch.tensor([0.01], device="cuda"))
+        torch.cuda.synchronize()
+        c_o, s_o, sc_o, y_o = oracle.arc(x_bits, gamma, perm, outl, s_t=0.01)
+        c = arc_counts("nvfp4", K, outl, (to_np(codes), to_np(scales), to_np(sf)),
+                       (c_o[:, :K // 2], s_o[:, :K // 16], sc_o), y_o, name=name)
+    check_fractions(c, 2e-4, name)
+
+
 @pytest.mark.parametrize("layout", [0, 1])
 def test_dequantize_int4_bitexact(fq, layout):
     """INT4 dequantization of the ARC operand [K | S]: value = (integer * E4M3)
